@@ -1,0 +1,150 @@
+"""Window-attention oracle: plain fp64 CPU reference (ctypes over winattn_oracle.c).
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package.  It shares no code with
+the CUDA path and the CUDA path never calls it.
+
+What it computes is the plain definition of exact windowed softmax attention
+from "FLASHSWIN: Unlocking Large Windows and Dense Tokens in Swin Vision
+Transformers with Memory Efficient Attention" (section "어떻게 동작하나": window
+partition, cyclic shift with an additive wrap mask, window-local 2D RoPE) and
+the feature concatenation of "Rank-Factorized Implicit Neural Bias" (section
+2.1).  Steps are written out in ``winattn_oracle.c``.
+
+Inputs are numpy arrays in storage form: ``uint16`` arrays holding bf16 bits,
+or ``float32`` arrays.  ``theta`` is float32 ``[heads][d/4]``; ``bias`` is
+``[heads][2][M*M][rank]`` in the same storage dtype as q/k/v.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "winattn_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+_lib = None
+
+
+def build(src: str = _SRC, out: str = _LIB, extra_flags: tuple = ()) -> str:
+    """Compile the oracle with gcc into a shared library; returns its path."""
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-o", out, src,
+           "-lm", "-lpthread", *extra_flags]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+def load(path: str | None = None):
+    """Load (building if missing or stale) the oracle library."""
+    global _lib
+    if path is not None:
+        return _bind(ctypes.CDLL(path))
+    if _lib is None:
+        if (not os.path.exists(_LIB)) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+            build()
+        _lib = _bind(ctypes.CDLL(_LIB))
+    return _lib
+
+
+def _bind(lib):
+    vp, i32, i64, f64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double
+    lib.oracle_fwd.argtypes = [vp, vp, vp, i32, vp, vp] + [i32] * 8 + [vp, i32, f64]
+    lib.oracle_fwd.restype = i32
+    lib.oracle_fwd_units.argtypes = [vp, vp, vp, i32, vp, vp] + [i32] * 8 + [vp, i64, vp, i32, f64]
+    lib.oracle_fwd_units.restype = i32
+    lib.oracle_rope.argtypes = [vp, i32, f64, f64, vp, vp]
+    lib.oracle_rope.restype = i32
+    lib.oracle_token_origin.argtypes = [i32] * 7 + [vp, vp]
+    lib.oracle_token_origin.restype = i32
+    return lib
+
+
+def _dtype_code(a: np.ndarray) -> int:
+    if a.dtype == np.uint16:
+        return 0
+    if a.dtype == np.float32:
+        return 1
+    raise TypeError(f"oracle inputs must be uint16 (bf16 bits) or float32, got {a.dtype}")
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+class Oracle:
+    """A bound oracle library (the real one, or a test-built variant)."""
+
+    def __init__(self, lib=None):
+        self.lib = lib if lib is not None else load()
+
+    def _prep(self, q, k, v, theta, bias, M):
+        q, k, v = (np.ascontiguousarray(x) for x in (q, k, v))
+        if not (q.shape == k.shape == v.shape) or q.ndim != 5:
+            raise ValueError("q, k, v must share one [B, H, W, heads, d] shape")
+        code = _dtype_code(q)
+        if _dtype_code(k) != code or _dtype_code(v) != code:
+            raise TypeError("q, k, v must share one storage dtype")
+        B, H, W, heads, d = q.shape
+        if theta is not None:
+            theta = np.ascontiguousarray(theta, dtype=np.float32)
+            if theta.shape != (heads, d // 4):
+                raise ValueError(f"theta must be [heads, d/4] = {(heads, d // 4)}")
+        rank = 0
+        if bias is not None:
+            bias = np.ascontiguousarray(bias)
+            if _dtype_code(bias) != code:
+                raise TypeError("bias must share the q/k/v storage dtype")
+            if bias.ndim != 4 or bias.shape[:3] != (heads, 2, M * M):
+                raise ValueError("bias must be [heads, 2, M*M, rank]")
+            rank = bias.shape[3]
+        return q, k, v, theta, bias, code, (B, H, W, heads, d, rank)
+
+    def fwd(self, q, k, v, *, M, shift=0, theta=None, bias=None, nthreads=0,
+            mem_budget=8e9) -> np.ndarray:
+        """Whole output map [B, H, W, heads, d] in fp64."""
+        q, k, v, theta, bias, code, (B, H, W, heads, d, rank) = self._prep(q, k, v, theta, bias, M)
+        out = np.zeros((B, H, W, heads, d), dtype=np.float64)
+        rc = self.lib.oracle_fwd(_ptr(q), _ptr(k), _ptr(v), code, _ptr(theta), _ptr(bias),
+                                 B, H, W, M, shift, heads, d, rank, _ptr(out), nthreads,
+                                 float(mem_budget))
+        if rc < 0:
+            raise ValueError(f"oracle rejected the problem (code {rc})")
+        return out
+
+    def fwd_units(self, q, k, v, units, *, M, shift=0, theta=None, bias=None,
+                  nthreads=0, mem_budget=8e9) -> np.ndarray:
+        """Selected units u = ((b*nWy + wy)*nWx + wx)*heads + h -> [n, M*M, d] fp64,
+        each in window order p = i*M + j."""
+        q, k, v, theta, bias, code, (B, H, W, heads, d, rank) = self._prep(q, k, v, theta, bias, M)
+        units = np.ascontiguousarray(units, dtype=np.int64)
+        out = np.zeros((len(units), M * M, d), dtype=np.float64)
+        rc = self.lib.oracle_fwd_units(_ptr(q), _ptr(k), _ptr(v), code, _ptr(theta), _ptr(bias),
+                                       B, H, W, M, shift, heads, d, rank, _ptr(units),
+                                       len(units), _ptr(out), nthreads, float(mem_budget))
+        if rc < 0:
+            raise ValueError(f"oracle rejected the problem (code {rc})")
+        return out
+
+    def rope(self, vec, i, j, theta_h) -> np.ndarray:
+        """R(i, j) vec for one d-vector (window-local row i, column j)."""
+        vec = np.ascontiguousarray(vec, dtype=np.float64)
+        theta_h = np.ascontiguousarray(theta_h, dtype=np.float32)
+        out = np.empty_like(vec)
+        if self.lib.oracle_rope(_ptr(vec), vec.shape[0], float(i), float(j), _ptr(theta_h), _ptr(out)):
+            raise ValueError("bad rope arguments")
+        return out
+
+    def token_origin(self, H, W, M, shift, wy, wx, p):
+        """Original (row, col) of token p of rolled window (wy, wx)."""
+        y, x = ctypes.c_int(), ctypes.c_int()
+        if self.lib.oracle_token_origin(H, W, M, shift, wy, wx, p, ctypes.byref(y), ctypes.byref(x)):
+            raise ValueError("bad token arguments")
+        return y.value, x.value
+
+
+def oracle() -> Oracle:
+    return Oracle()

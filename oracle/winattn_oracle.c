@@ -1,0 +1,367 @@
+/*
+ * Window-attention oracle: a plain, slow, fp64 CPU statement of what the
+ * fused window-attention forward computes.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the CPU
+ * baseline of the benchmark may load this library.  It shares no code,
+ * header, table or helper with the CUDA path, and the CUDA path never
+ * calls it.
+ *
+ * What it follows (pages are cited by title and section):
+ *  - "FLASHSWIN: Unlocking Large Windows and Dense Tokens in Swin Vision
+ *    Transformers with Memory Efficient Attention", section "어떻게 동작하나"
+ *    (how it works): attention is exact softmax attention restricted to
+ *    non-overlapping M x M windows; shifted windows are a cyclic move of the
+ *    map followed by per-window recomputation; wrapped windows are masked by
+ *    an additive mask; window-local learned 2D RoPE splits the head dim in
+ *    half, the first half encoding the row y and the second half the column
+ *    x, both halves sharing one frequency set theta_i = exp(omega_i).
+ *  - same page, section "전제와 한계" (premises and limits), second
+ *    paragraph: bf16 Q/K/V in, RoPE in fp32, softmax accumulated in fp32
+ *    (the oracle does all of it in fp64 on the exact input values).
+ *  - "Rank-Factorized Implicit Neural Bias: Scaling Super-Resolution
+ *    Transformer with FlashAttention", section 2.1 (RIB): the position
+ *    features are concatenated to the content features so that
+ *    [Qc, Qp][Kc, Kp]^T = Qc Kc^T + Qp Kp^T.
+ *
+ * Readings where the pages are silent (each is listed in the design notes):
+ *  - d/4 shared frequencies per head (the page's "d/2 parameters per head"
+ *    cannot rotate d/2 dims with one angle per pair); pairs are adjacent
+ *    (2k, 2k+1) inside each half; counter-clockwise rotation;
+ *  - roll by -s (token (i, j) of the rolled map is original token
+ *    (i + s, j + s) mod (H, W)), inverse roll on write-back;
+ *  - wrap label L = 2*[row in last s rows] + [col in last s cols] of the
+ *    rolled map, mask value -inf where labels differ;
+ *  - scale d^-1/2 applies to the content dot product only, the bias dot
+ *    product u.w is added unscaled.
+ *
+ * Parity of every function here is pinned by the not-gpu tests (closed
+ * forms, the displacement identity of the rotation, brute-force masked
+ * global attention, Swin's slice-based region labels, planted mistakes).
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+#define ORACLE_DTYPE_BF16 0
+#define ORACLE_DTYPE_FP32 1
+
+typedef struct {
+    const void *q, *k, *v;   /* [B][H][W][heads][d], storage dtype */
+    int dtype;
+    const float *theta;      /* [heads][d/4] or NULL */
+    const void *bias;        /* [heads][2][M*M][rank] storage dtype, or NULL */
+    int B, H, W, M, shift, heads, d, rank;
+} problem_t;
+
+/* Step 1: read one stored element as fp64 (bf16 -> fp64 and fp32 -> fp64 are exact). */
+static double read_elem(const void *base, int dtype, size_t idx)
+{
+    if (dtype == ORACLE_DTYPE_FP32)
+        return (double)((const float *)base)[idx];
+    uint32_t bits = (uint32_t)((const uint16_t *)base)[idx] << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+/* Step 2: the rolled map.  Rolled row yr, rolled column xr hold the original
+ * token at row (yr + s) mod H, column (xr + s) mod W. */
+static size_t rolled_token_offset(const problem_t *p, int b, int yr, int xr, int h)
+{
+    int y = (yr + p->shift) % p->H;
+    int x = (xr + p->shift) % p->W;
+    return ((((size_t)b * p->H + y) * p->W + x) * p->heads + h) * p->d;
+}
+
+/* Step 4: window-local 2D RoPE on one d-vector at window-local (row i, col j).
+ * Pair k of the first half turns by i*theta_k, pair k of the second half by
+ * j*theta_k; rot(a)(x0, x1) = (x0 cos a - x1 sin a, x0 sin a + x1 cos a). */
+static void rope_rotate(double *vec, int d, double i, double j, const float *theta_h)
+{
+    int half = d / 2;
+    for (int k = 0; k < d / 4; ++k) {
+        double th = (double)theta_h[k];
+        double ay = i * th, ax = j * th;
+        double x0 = vec[2 * k], x1 = vec[2 * k + 1];
+        vec[2 * k] = x0 * cos(ay) - x1 * sin(ay);
+        vec[2 * k + 1] = x0 * sin(ay) + x1 * cos(ay);
+        double y0 = vec[half + 2 * k], y1 = vec[half + 2 * k + 1];
+        vec[half + 2 * k] = y0 * cos(ax) - y1 * sin(ax);
+        vec[half + 2 * k + 1] = y0 * sin(ax) + y1 * cos(ax);
+    }
+}
+
+/* Step 6: wrap label of rolled-map row yr, column xr (0 when unshifted). */
+static int wrap_label(const problem_t *p, int yr, int xr)
+{
+    if (p->shift == 0)
+        return 0;
+    return 2 * (yr >= p->H - p->shift) + (xr >= p->W - p->shift);
+}
+
+typedef struct {
+    double *q, *k, *v, *s; /* N x d, N x d, N x d, N x N */
+} scratch_t;
+
+/* Steps 3-8 for one (batch b, window (wy, wx), head h): O = softmax(S) V in
+ * window order p = i*M + j, written to out[N][d]. */
+static void unit_forward(const problem_t *p, int b, int wy, int wx, int h,
+                         scratch_t *w, double *out)
+{
+    const int M = p->M, N = M * M, d = p->d, r = p->rank;
+    const double scale = 1.0 / sqrt((double)d);
+
+    /* Step 3: gather the window's N tokens from the rolled map. */
+    for (int i = 0; i < M; ++i)
+        for (int j = 0; j < M; ++j) {
+            int t = i * M + j;
+            size_t off = rolled_token_offset(p, b, wy * M + i, wx * M + j, h);
+            for (int c = 0; c < d; ++c) {
+                w->q[(size_t)t * d + c] = read_elem(p->q, p->dtype, off + c);
+                w->k[(size_t)t * d + c] = read_elem(p->k, p->dtype, off + c);
+                w->v[(size_t)t * d + c] = read_elem(p->v, p->dtype, off + c);
+            }
+        }
+
+    /* Step 4: RoPE with window-local coordinates. */
+    if (p->theta) {
+        const float *th = p->theta + (size_t)h * (d / 4);
+        for (int i = 0; i < M; ++i)
+            for (int j = 0; j < M; ++j) {
+                int t = i * M + j;
+                rope_rotate(w->q + (size_t)t * d, d, (double)i, (double)j, th);
+                rope_rotate(w->k + (size_t)t * d, d, (double)i, (double)j, th);
+            }
+    }
+
+    /* Step 5: the full N x N score matrix, content scaled, bias added. */
+    for (int a = 0; a < N; ++a)
+        for (int c = 0; c < N; ++c) {
+            double dot = 0.0;
+            for (int e = 0; e < d; ++e)
+                dot += w->q[(size_t)a * d + e] * w->k[(size_t)c * d + e];
+            double sc = scale * dot;
+            if (p->bias) {
+                size_t ub = (((size_t)h * 2 + 0) * N + a) * r;
+                size_t wb = (((size_t)h * 2 + 1) * N + c) * r;
+                double bd = 0.0;
+                for (int e = 0; e < r; ++e)
+                    bd += read_elem(p->bias, p->dtype, ub + e) * read_elem(p->bias, p->dtype, wb + e);
+                sc += bd;
+            }
+            w->s[(size_t)a * N + c] = sc;
+        }
+
+    /* Step 6: additive -inf mask between different wrap regions. */
+    for (int a = 0; a < N; ++a) {
+        int la = wrap_label(p, wy * M + a / M, wx * M + a % M);
+        for (int c = 0; c < N; ++c) {
+            int lc = wrap_label(p, wy * M + c / M, wx * M + c % M);
+            if (la != lc)
+                w->s[(size_t)a * N + c] = -INFINITY;
+        }
+    }
+
+    /* Step 7: row softmax (max subtracted, exp, divided by the sum). */
+    for (int a = 0; a < N; ++a) {
+        double *row = w->s + (size_t)a * N;
+        double mx = -INFINITY;
+        for (int c = 0; c < N; ++c)
+            if (row[c] > mx)
+                mx = row[c];
+        double sum = 0.0;
+        for (int c = 0; c < N; ++c) {
+            row[c] = exp(row[c] - mx);
+            sum += row[c];
+        }
+        for (int c = 0; c < N; ++c)
+            row[c] /= sum;
+    }
+
+    /* Step 8: O = P V. */
+    for (int a = 0; a < N; ++a)
+        for (int e = 0; e < d; ++e) {
+            double acc = 0.0;
+            for (int c = 0; c < N; ++c)
+                acc += w->s[(size_t)a * N + c] * w->v[(size_t)c * d + e];
+            out[(size_t)a * d + e] = acc;
+        }
+}
+
+/* Units are numbered u = ((b * nWy + wy) * nWx + wx) * heads + h. */
+static void unit_coords(const problem_t *p, int64_t u, int *b, int *wy, int *wx, int *h)
+{
+    int nWy = p->H / p->M, nWx = p->W / p->M;
+    *h = (int)(u % p->heads);
+    u /= p->heads;
+    *wx = (int)(u % nWx);
+    u /= nWx;
+    *wy = (int)(u % nWy);
+    *b = (int)(u / nWy);
+}
+
+typedef struct {
+    const problem_t *p;
+    const int64_t *units;  /* NULL = every unit in order */
+    int64_t n_units;
+    double *out_units;     /* [n_units][N][d] or NULL */
+    double *out_map;       /* [B][H][W][heads][d] or NULL (step 9 scatter) */
+    int64_t next;          /* shared work counter */
+    int failed;
+} job_t;
+
+static void *worker(void *arg)
+{
+    job_t *job = (job_t *)arg;
+    const problem_t *p = job->p;
+    const size_t N = (size_t)p->M * p->M, d = (size_t)p->d;
+    scratch_t w;
+    w.q = malloc(N * d * sizeof(double));
+    w.k = malloc(N * d * sizeof(double));
+    w.v = malloc(N * d * sizeof(double));
+    w.s = malloc(N * N * sizeof(double));
+    double *o = malloc(N * d * sizeof(double));
+    if (!w.q || !w.k || !w.v || !w.s || !o) {
+        __atomic_store_n(&job->failed, 1, __ATOMIC_RELAXED);
+        goto done;
+    }
+    for (;;) {
+        int64_t n = __atomic_fetch_add(&job->next, 1, __ATOMIC_RELAXED);
+        if (n >= job->n_units)
+            break;
+        int64_t u = job->units ? job->units[n] : n;
+        int b, wy, wx, h;
+        unit_coords(p, u, &b, &wy, &wx, &h);
+        double *dst = job->out_units ? job->out_units + (size_t)n * N * d : o;
+        unit_forward(p, b, wy, wx, h, &w, dst);
+        if (job->out_map) {
+            /* Step 9: write back through the inverse roll, i.e. to the same
+             * original position each token was gathered from. */
+            for (int i = 0; i < p->M; ++i)
+                for (int j = 0; j < p->M; ++j) {
+                    size_t off = rolled_token_offset(p, b, wy * p->M + i, wx * p->M + j, h);
+                    memcpy(job->out_map + off, dst + ((size_t)i * p->M + j) * d, d * sizeof(double));
+                }
+        }
+    }
+done:
+    free(w.q);
+    free(w.k);
+    free(w.v);
+    free(w.s);
+    free(o);
+    return NULL;
+}
+
+static int check_problem(const problem_t *p)
+{
+    if (!p->q || !p->k || !p->v)
+        return -1;
+    if (p->dtype != ORACLE_DTYPE_BF16 && p->dtype != ORACLE_DTYPE_FP32)
+        return -1;
+    if (p->B <= 0 || p->H <= 0 || p->W <= 0 || p->M <= 0 || p->heads <= 0)
+        return -1;
+    if (p->H % p->M || p->W % p->M || p->shift < 0 || p->shift >= p->M)
+        return -1;
+    if (p->d <= 0 || p->d % 4)
+        return -1;
+    if ((p->rank > 0) != (p->bias != NULL) || p->rank < 0)
+        return -1;
+    return 0;
+}
+
+static int run(const problem_t *p, const int64_t *units, int64_t n_units,
+               double *out_units, double *out_map, int nthreads, double mem_budget_bytes)
+{
+    if (check_problem(p))
+        return -1;
+    if (n_units <= 0)
+        return 0;
+    long ncpu = sysconf(_SC_NPROCESSORS_ONLN);
+    if (nthreads <= 0)
+        nthreads = ncpu > 0 ? (int)ncpu : 1;
+    double per_thread = ((double)p->M * p->M) * ((double)p->M * p->M + 4.0 * p->d) * sizeof(double);
+    if (mem_budget_bytes <= 0)
+        mem_budget_bytes = 8e9;
+    int cap = (int)(mem_budget_bytes / per_thread);
+    if (cap < 1)
+        cap = 1;
+    if (nthreads > cap)
+        nthreads = cap;
+    if (nthreads > n_units)
+        nthreads = (int)n_units;
+
+    job_t job = {p, units, n_units, out_units, out_map, 0, 0};
+    pthread_t *th = malloc(sizeof(pthread_t) * (size_t)nthreads);
+    if (!th)
+        return -2;
+    int started = 0;
+    for (int t = 0; t < nthreads; ++t) {
+        if (pthread_create(&th[t], NULL, worker, &job) != 0)
+            break;
+        ++started;
+    }
+    if (started == 0)
+        worker(&job);
+    for (int t = 0; t < started; ++t)
+        pthread_join(th[t], NULL);
+    free(th);
+    return job.failed ? -2 : (started == 0 ? 1 : started);
+}
+
+/* ---- exported entry points (called through ctypes by oracle/__init__.py) ---- */
+
+/* Every unit; output scattered to out_map [B][H][W][heads][d] fp64.
+ * Returns the number of threads used (> 0), or < 0 on bad arguments. */
+int oracle_fwd(const void *q, const void *k, const void *v, int dtype,
+               const float *theta, const void *bias,
+               int B, int H, int W, int M, int shift, int heads, int d, int rank,
+               double *out_map, int nthreads, double mem_budget_bytes)
+{
+    problem_t p = {q, k, v, dtype, theta, bias, B, H, W, M, shift, heads, d, rank};
+    if (check_problem(&p) || !out_map)
+        return -1;
+    int64_t n = (int64_t)B * (H / M) * (W / M) * heads;
+    return run(&p, NULL, n, NULL, out_map, nthreads, mem_budget_bytes);
+}
+
+/* Selected units; out_units [n_units][M*M][d] fp64 in window order p = i*M + j. */
+int oracle_fwd_units(const void *q, const void *k, const void *v, int dtype,
+                     const float *theta, const void *bias,
+                     int B, int H, int W, int M, int shift, int heads, int d, int rank,
+                     const int64_t *units, int64_t n_units,
+                     double *out_units, int nthreads, double mem_budget_bytes)
+{
+    problem_t p = {q, k, v, dtype, theta, bias, B, H, W, M, shift, heads, d, rank};
+    if (check_problem(&p) || !units || !out_units)
+        return -1;
+    int64_t total = (int64_t)B * (H / M) * (W / M) * heads;
+    for (int64_t n = 0; n < n_units; ++n)
+        if (units[n] < 0 || units[n] >= total)
+            return -1;
+    return run(&p, units, n_units, out_units, NULL, nthreads, mem_budget_bytes);
+}
+
+/* The rotation alone, for the displacement-identity checks: out = R(i, j) vec. */
+int oracle_rope(const double *vec, int d, double i, double j, const float *theta_h, double *out)
+{
+    if (!vec || !theta_h || !out || d <= 0 || d % 4)
+        return -1;
+    memcpy(out, vec, (size_t)d * sizeof(double));
+    rope_rotate(out, d, i, j, theta_h);
+    return 0;
+}
+
+/* Original (row, col) of rolled-window token p of window (wy, wx). */
+int oracle_token_origin(int H, int W, int M, int shift, int wy, int wx, int p, int *y, int *x)
+{
+    if (M <= 0 || p < 0 || p >= M * M || !y || !x)
+        return -1;
+    *y = (wy * M + p / M + shift) % H;
+    *x = (wx * M + p % M + shift) % W;
+    return 0;
+}

@@ -1,0 +1,67 @@
+"""Planted mistakes: each builds a copy of the oracle with one plausible error
+(a wrong sign, index, operand or dropped term) and checks that some pin fails.
+This is what makes the pins worth trusting: none of these errors slips by."""
+import os
+
+import pytest
+
+import oracle
+from tests import pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "winattn_oracle.c")
+
+MUTANTS = {
+    "clockwise_rotation": [
+        ("vec[2 * k] = x0 * cos(ay) - x1 * sin(ay);", "vec[2 * k] = x0 * cos(ay) + x1 * sin(ay);"),
+        ("vec[2 * k + 1] = x0 * sin(ay) + x1 * cos(ay);", "vec[2 * k + 1] = -x0 * sin(ay) + x1 * cos(ay);"),
+    ],
+    "halves_swapped": [("double ay = i * th, ax = j * th;", "double ay = j * th, ax = i * th;")],
+    "pair_members_swapped": [("double x0 = vec[2 * k], x1 = vec[2 * k + 1];",
+                              "double x0 = vec[2 * k + 1], x1 = vec[2 * k];")],
+    "mask_dropped": [("if (la != lc)", "if (0)")],
+    "mask_inverted": [("if (la != lc)", "if (la == lc && a != c)")],
+    "label_off_by_one": [("yr >= p->H - p->shift", "yr > p->H - p->shift")],
+    "scale_dropped": [("const double scale = 1.0 / sqrt((double)d);", "const double scale = 1.0;")],
+    "roll_reversed": [
+        ("int y = (yr + p->shift) % p->H;", "int y = (yr - p->shift + p->H) % p->H;"),
+        ("int x = (xr + p->shift) % p->W;", "int x = (xr - p->shift + p->W) % p->W;"),
+    ],
+    "scores_transposed": [("dot += w->q[(size_t)a * d + e] * w->k[(size_t)c * d + e];",
+                           "dot += w->q[(size_t)c * d + e] * w->k[(size_t)a * d + e];")],
+    "sum_not_divided": [("row[c] /= sum;", "row[c] /= 1.0;")],
+    "value_index": [("acc += w->s[(size_t)a * N + c] * w->v[(size_t)c * d + e];",
+                     "acc += w->s[(size_t)a * N + c] * w->v[(size_t)a * d + e];")],
+    "bias_sides_swapped": [
+        ("size_t ub = (((size_t)h * 2 + 0) * N + a) * r;", "size_t ub = (((size_t)h * 2 + 1) * N + a) * r;"),
+        ("size_t wb = (((size_t)h * 2 + 1) * N + c) * r;", "size_t wb = (((size_t)h * 2 + 0) * N + c) * r;"),
+    ],
+    "bias_scaled": [("sc += bd;", "sc += scale * bd;")],
+    "bias_dropped": [("sc += bd;", "sc += 0.0 * bd;")],
+    "scatter_unrolled": [(
+        "size_t off = rolled_token_offset(p, b, wy * p->M + i, wx * p->M + j, h);",
+        "size_t off = rolled_token_offset(p, b, (wy * p->M + i + p->H - p->shift) % p->H, "
+        "(wx * p->M + j + p->W - p->shift) % p->W, h);")],
+    "query_coords_global": [(
+        "rope_rotate(w->q + (size_t)t * d, d, (double)i, (double)j, th);",
+        "rope_rotate(w->q + (size_t)t * d, d, (double)(i + wy * M), (double)j, th);")],
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_fails_a_pin(name, tmp_path):
+    with open(SRC) as f:
+        src = f.read()
+    for old, new in MUTANTS[name]:
+        assert src.count(old) == 1, f"mutation site for {name!r} not found exactly once"
+        src = src.replace(old, new)
+    path = tmp_path / "mutant.c"
+    path.write_text(src)
+    lib = oracle.build(str(path), str(tmp_path / "libmutant.so"))
+    orc = oracle.Oracle(oracle.load(lib))
+    failed = []
+    for pin in pins.ALL_PINS:
+        try:
+            pin(orc)
+        except AssertionError:
+            failed.append(pin.__name__)
+    assert failed, f"mutant {name!r} passed every pin"
