@@ -1,0 +1,396 @@
+"""Benchmark of the fused window-attention forward on B200.
+
+One step = one pass of the whole hot path over one batch: the workload's
+winattn_fwd call(s) (two calls, unshifted then shifted, for workloads that
+alternate).  Default workload: the Swin-T stage-1 shape (B=64, 56x56 tokens,
+3 heads of d=32, M=8 windows shifted by 4, bf16, learned 2D RoPE).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...      # the fp64 CPU oracle, bounded sample
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own batch (weak
+scaling, no collective on the data path); the timed region is bracketed by a
+barrier and the time is the max over ranks.  Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "window-attn fwd TFLOP/s & tokens/s on 1 B200 vs M; % of roofline"
+L2_BYTES = 126 * 2**20
+KERNEL_SOURCES = ["windowed_attention_vision_b200/csrc/fwd_tc.cuh", "windowed_attention_vision_b200/csrc/ptx.cuh",
+                  "windowed_attention_vision_b200/csrc/geometry.cuh"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="swin")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def read_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), bf16_tflops=float(p["bf16_tflops"]),
+                    bf16_tflops_sustained=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                    source="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch of the attention kernel from the committed ncu
+    summary for this workload, if it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", f"winattn_fwd_tc_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    m_hash = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
+    if not m_bytes or not m_hash or m_hash.group(1) != kernel_source_hash():
+        return None
+    return float(m_bytes.group(1))
+
+
+# ----------------------------------------------------------------- clocks (NVML)
+
+class ClockSampler:
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks_setting"}
+
+    def __init__(self, torch_device_index: int, period_s: float = 0.002):
+        self.ok = False
+        self.samples = []
+        self.period = period_s
+        self.marks = {}
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(torch_device_index)
+            handle = None
+            uuid = getattr(props, "uuid", None)
+            if uuid is not None:
+                try:
+                    handle = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + str(uuid)).encode())
+                except Exception:
+                    handle = None
+            if handle is None:
+                handle = pynvml.nvmlDeviceGetHandleByIndex(torch_device_index)
+            self.nvml, self.h = pynvml, handle
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # pragma: no cover - no NVML
+            self.err = str(e)
+
+    def _reasons(self):
+        try:
+            return self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            return self.nvml.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append((time.perf_counter(),
+                                     self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM),
+                                     self._reasons()))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._stop = threading.Event()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def mark(self, name):
+        self.marks[name] = time.perf_counter()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "note": "NVML unavailable"}
+        t0, t1 = self.marks.get("timed_start", 0), self.marks.get("timed_end", 1e30)
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        used = inside if inside else self.samples
+        reasons = set()
+        for _, _, r in used:
+            for bit, name in self.REASONS.items():
+                if r & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median([s[1] for s in used]) if used else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons),
+                "samples": len(inside), "samples_window": "timed region" if inside else "warm-up + timed region"}
+
+
+# ----------------------------------------------------------------- helpers
+
+def workload_calls(w):
+    """(shift) per call of one step."""
+    return list(w.shifts)
+
+
+def roofline(w, kernel_s, peaks, traffic):
+    flops, nbytes = w.flops(), w.bytes()
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if flops / nbytes < ridge:
+        achieved = nbytes / kernel_s / 1e9
+        peak = peaks["hbm_gbs"]
+        r = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s"}
+    else:
+        achieved = flops / kernel_s / 1e12
+        peak = peaks["bf16_tflops"]
+        r = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+             "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"]}
+    r["frac"] = r["achieved"] / r["peak"]
+    r["traffic"] = traffic
+    r["peak_source"] = peaks["source"]
+    r["algorithmic_bytes_per_launch"] = nbytes
+    r["algorithmic_flops_per_launch"] = flops
+    return r
+
+
+def oracle_sample_rate(w, target_s, base=0):
+    """Time the fp64 oracle on a bounded sample of the workload's units on all
+    host cores; returns (tokens/s extrapolated to the whole workload, sample
+    description, cores)."""
+    import numpy as np
+
+    import oracle
+    from windowed_attention_vision_b200 import inputs as I
+    cores = cpu_cores()
+    (qkv,), theta, bias = I.make_inputs(w, "cpu", base)
+    args = [I.to_storage_numpy(t) for t in qkv]
+    th = None if theta is None else theta.numpy()
+    bs = I.to_storage_numpy(bias)
+    orc = oracle.oracle()
+    total_units = w.B * (w.H // w.M) * (w.W // w.M) * w.heads
+    rng = np.random.default_rng(base)
+    shift = w.shifts[-1]
+    probe = min(total_units, cores)
+    t0 = time.perf_counter()
+    orc.fwd_units(*args, rng.choice(total_units, probe, replace=False), M=w.M, shift=shift, theta=th, bias=bs,
+                  nthreads=cores)
+    per_batch = time.perf_counter() - t0
+    n = int(min(total_units, max(probe, probe * max(1.0, target_s / max(per_batch, 1e-6)))))
+    units = rng.choice(total_units, n, replace=False)
+    t0 = time.perf_counter()
+    orc.fwd_units(*args, units, M=w.M, shift=shift, theta=th, bias=bs, nthreads=cores)
+    dt = time.perf_counter() - t0
+    calls = len(workload_calls(w))
+    tokens_per_s = w.tokens * (n / total_units) / dt
+    sample = (f"{n} of {total_units} (window, head) units of one {w.name} call (shift {shift}), "
+              f"{dt:.1f} s on {cores} threads, extrapolated by unit count")
+    return tokens_per_s, sample, cores, calls
+
+
+# ----------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from windowed_attention_vision_b200 import inputs as I
+    w = I.WORKLOADS[args.workload]
+    per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    rates = []
+    for s in range(args.warmup + args.steps):
+        rate, sample, cores, _ = oracle_sample_rate(w, per_step, base=s)
+        if s >= args.warmup:
+            rates.append(rate)
+    value = statistics.median(rates)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": w.tokens / value * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_of(w, args.gpus),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def config_of(w, n):
+    return {"workload": w.name, "B_per_gpu": w.B, "H": w.H, "W": w.W, "M": w.M, "shifts": list(w.shifts),
+            "heads": w.heads, "d": w.d, "rank": w.rank, "rope": w.rope, "global_batch": w.B * n,
+            "parallelism": f"replicas x{n} (independent batches)"}
+
+
+# ----------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import windowed_attention_vision_b200 as wa
+    from windowed_attention_vision_b200 import _lib
+    from windowed_attention_vision_b200 import inputs as I
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    w = I.WORKLOADS[args.workload]
+    calls = workload_calls(w)
+    map_bytes = w.tokens * w.heads * w.d * w.elt
+    # rotate over enough input sets that one pass over them exceeds 2x L2
+    copies = max(2, int((2 * L2_BYTES) // (4 * map_bytes)) + 1)
+    sets, theta, bias = I.make_inputs(w, dev, base=rank, copies=copies)
+    outs = [torch.empty_like(s[0]) for s in sets]
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        q, k, v = sets[i % copies]
+        for s in calls:
+            wa.window_attention(q, k, v, w.M, s, theta=theta, bias_feats=bias, out=outs[i % copies])
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.01)
+    # per-launch events around every call give the kernel's average duration
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps * len(calls))]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    clocks.mark("timed_start")
+    start.record(stream)
+    n = 0
+    for i in range(args.steps):
+        q, k, v = sets[i % copies]
+        for s in calls:
+            ev[n][0].record(stream)
+            wa.window_attention(q, k, v, w.M, s, theta=theta, bias_feats=bias, out=outs[i % copies])
+            ev[n][1].record(stream)
+            n += 1
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.mark("timed_end")
+    if world > 1:
+        dist.barrier()
+    time.sleep(0.01)
+    clocks.stop()
+    status = wa.device_status(dev)
+    elapsed_ms = start.elapsed_time(end)
+    kernel_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    if world > 1:
+        t = torch.tensor([elapsed_ms, kernel_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms, kernel_ms = t.tolist()
+
+    tokens_all = w.tokens * len(calls) * args.steps * world
+    value = tokens_all / (elapsed_ms / 1e3)
+    tflops = w.flops() * len(calls) * args.steps * world / (elapsed_ms / 1e3) / 1e12
+
+    # end to end through the C ABI on host buffers (pinned), copies inside the region
+    e2e = None
+    if args.e2e_steps > 0:
+        hq, hk, hv = (t.cpu().pin_memory() for t in sets[0])
+        hout = torch.empty_like(hq).pin_memory()
+        need = _lib.host_workspace_bytes(w.B, w.H, w.W, w.heads, w.d, _lib.BF16 if w.dtype == "bf16" else _lib.FP32)
+        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+        for s in calls:
+            wa.window_attention_host(hq, hk, hv, w.M, s, theta=theta, bias_feats=bias, out=hout, workspace=ws,
+                                     device=dev, synchronize=False)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            for s in calls:
+                wa.window_attention_host(hq, hk, hv, w.M, s, theta=theta, bias_feats=bias, out=hout,
+                                         workspace=ws, device=dev, synchronize=False)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = t.item()
+        e2e = {"value": w.tokens * len(calls) * args.e2e_steps * world / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": 3 * map_bytes * len(calls), "d2h_bytes_per_step": map_bytes * len(calls),
+               "steps": args.e2e_steps, "api": "winattn_fwd_host (C ABI, pinned host buffers)"}
+
+    if rank == 0:
+        peaks = read_peaks()
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+                "config": dict(config_of(w, world),
+                               l2=f"inputs larger than L2: {copies} rotating input sets of "
+                                  f"{4 * map_bytes / 1e6:.0f} MB (q, k, v, out)"),
+                "tflops": tflops, "kernel_ms_per_launch": kernel_ms, "gpu_launches": args.steps * len(calls),
+                "roofline": roofline(w, kernel_ms / 1e3, peaks, recorded_traffic(w.name)),
+                "clocks": clocks.summary(), "e2e": e2e, "device_status": status}
+        if world == 1 and not args.no_cpu_baseline:
+            rate, sample, cores, _ = oracle_sample_rate(w, args.cpu_seconds)
+            line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                    "sample": sample}
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,155 @@
+/*
+ * winattn — fused, exact windowed softmax attention (forward) for vision
+ * transformers on NVIDIA B200 (sm_100a).
+ *
+ * The operation (from "FLASHSWIN: Unlocking Large Windows and Dense Tokens
+ * in Swin Vision Transformers with Memory Efficient Attention", section
+ * "어떻게 동작하나", and "Rank-Factorized Implicit Neural Bias: Scaling
+ * Super-Resolution Transformer with FlashAttention", section 2.1):
+ *
+ *   For every image b, head h and M x M window (wy, wx) of the map rolled by
+ *   -shift (rolled token (yr, xr) is original token ((yr + shift) mod H,
+ *   (xr + shift) mod W)), with window-local token p = i*M + j:
+ *
+ *     q~_p = [ R(i, j) q_p , u_h(p) ]        k~_p = [ R(i, j) k_p , w_h(p) ]
+ *     z(p, p') = d^-1/2 <R q_p, R k_p'> + <u_h(p), w_h(p')>
+ *                + ( -inf if shift > 0 and L(p) != L(p') else 0 )
+ *     o_p = sum_p' softmax_p'(z(p, .)) v_p'
+ *
+ *   and o_p is written back to the original position of token p.  R(i, j)
+ *   is window-local 2D RoPE: pair (2k, 2k+1) of the first half of the head
+ *   dim turns counter-clockwise by i * theta_h[k], pair (d/2 + 2k,
+ *   d/2 + 2k + 1) of the second half by j * theta_h[k], k < d/4.  L is the
+ *   wrap label 2*[yr >= H - shift] + [xr >= W - shift] of the rolled map.
+ *   The u/w bias terms are present only when bias_feats is given.
+ *
+ * The N x N score matrix of a window (N = M*M) is never stored: the kernel
+ * streams key tiles with an online softmax, so device memory beyond the
+ * caller's buffers does not grow with M.
+ *
+ * Threading: every call is asynchronous on the given CUDA stream.  Calls on
+ * different streams may run concurrently; they share only the per-device
+ * status word read by winattn_last_device_status().
+ */
+#ifndef WINATTN_H
+#define WINATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes.  0 is success; every error is negative. */
+#define WINATTN_OK                  0
+#define WINATTN_ERR_ARG            -1  /* null pointer, non-positive size, H % M or W % M != 0,
+                                          shift outside [0, M), unsupported head dim d          */
+#define WINATTN_ERR_RANK           -2  /* rank > 0 without bias_feats, bias_feats without rank,
+                                          or rank outside the supported set                    */
+#define WINATTN_ERR_ALIGN          -3  /* a device pointer is not 16-byte aligned              */
+#define WINATTN_ERR_DTYPE          -4  /* dtype is neither WINATTN_BF16 nor WINATTN_FP32       */
+#define WINATTN_ERR_ARCH           -5  /* the current device is not compute capability 10.0    */
+#define WINATTN_ERR_CUDA           -6  /* a CUDA runtime call or kernel launch failed          */
+#define WINATTN_ERR_DEVICE_TIMEOUT -7  /* a bounded wait inside a kernel gave up               */
+#define WINATTN_ERR_ALIAS          -8  /* out overlaps q, k or v                               */
+#define WINATTN_ERR_SIZE           -9  /* a size product overflows the kernel's index range,
+                                          or a host workspace is too small                     */
+
+/* Storage / arithmetic types of q, k, v, bias_feats and out. */
+#define WINATTN_BF16 0  /* bf16 storage; tensor-core QK^T and PV (bf16 in, fp32 accumulate),
+                           RoPE and softmax in fp32                                            */
+#define WINATTN_FP32 1  /* fp32 storage; fp32 arithmetic throughout                            */
+
+/*
+ * winattn_fwd — the fused forward pass.
+ *
+ *   q, k, v     device, [B][H_img][W_img][heads][d] row-major (channel-last,
+ *               C = heads*d contiguous per token), element type `dtype`.
+ *               16-byte aligned.  Read only.
+ *   theta       device, fp32 [heads][d/4] RoPE frequencies theta = exp(omega),
+ *               or NULL for no rotation.  Read only.
+ *   bias_feats  device, element type `dtype`, [heads][2][M*M][rank]: index 0
+ *               holds u(p) (query side), index 1 holds w(p) (key side), for
+ *               window-local p = i*M + j; or NULL when rank == 0.  16-byte
+ *               aligned.  Read only.
+ *   B, H_img, W_img, M, shift, heads, d, rank
+ *               sizes: H_img % M == 0, W_img % M == 0, 0 <= shift < M,
+ *               d in {32, 64} for WINATTN_BF16, d in {16, 32, 64} for
+ *               WINATTN_FP32; rank in {0, 16, 32}; M <= 256; the number of
+ *               128-row query tiles must fit in a 31-bit grid.
+ *   dtype       WINATTN_BF16 or WINATTN_FP32.
+ *   out         device, same layout and type as q; caller-allocated, must not
+ *               overlap q, k or v.  Every element is written.
+ *   stream      a cudaStream_t (NULL = the legacy default stream).
+ *
+ * Ownership: the caller owns every buffer; the library keeps no pointer past
+ * the call and allocates no device memory.  Errors found on the host return
+ * before anything is enqueued (out is untouched).  A kernel that gives up a
+ * bounded wait records WINATTN_ERR_DEVICE_TIMEOUT in the per-device status
+ * word (see winattn_last_device_status) and leaves `out` unspecified.
+ */
+int winattn_fwd(const void *q, const void *k, const void *v,
+                const float *theta, const void *bias_feats,
+                int B, int H_img, int W_img, int M, int shift,
+                int heads, int d, int rank, int dtype,
+                void *out, void *stream);
+
+/*
+ * winattn_check_args — the host-side argument checks of winattn_fwd alone:
+ * returns the code winattn_fwd would return before enqueuing anything
+ * (WINATTN_OK if the arguments are acceptable).  Touches no device and makes
+ * no CUDA call; pointers are only compared and checked for alignment.
+ */
+int winattn_check_args(const void *q, const void *k, const void *v,
+                       const float *theta, const void *bias_feats,
+                       int B, int H_img, int W_img, int M, int shift,
+                       int heads, int d, int rank, int dtype, const void *out);
+
+/*
+ * winattn_fwd_host — the same operation on HOST buffers q, k, v, out (pinned
+ * memory gives asynchronous copies; pageable memory works but the copies
+ * then block).  theta and bias_feats stay device pointers (resident
+ * parameters).  `workspace` is a caller-owned device buffer of at least
+ * winattn_host_workspace_bytes(...) bytes, 16-byte aligned, that holds the
+ * device copies of q, k, v and out.  Enqueues H2D copies, the kernel and the
+ * D2H copy of out on `stream` and returns; synchronise the stream before
+ * reading out.  Allocates nothing.
+ */
+int winattn_fwd_host(const void *q_host, const void *k_host, const void *v_host,
+                     const float *theta, const void *bias_feats,
+                     int B, int H_img, int W_img, int M, int shift,
+                     int heads, int d, int rank, int dtype,
+                     void *out_host, void *workspace, size_t workspace_bytes,
+                     void *stream);
+
+/* Bytes of device workspace winattn_fwd_host needs (4 maps, each rounded up to
+ * 256 bytes), or 0 for invalid sizes. */
+size_t winattn_host_workspace_bytes(int B, int H_img, int W_img, int heads, int d, int dtype);
+
+/* A static, human-readable description of a return code. */
+const char *winattn_strerror(int code);
+
+/*
+ * winattn_last_device_status — synchronises `stream`, then reads and clears
+ * the current device's status word.  Returns WINATTN_OK when no kernel has
+ * given up a bounded wait since the last read, WINATTN_ERR_DEVICE_TIMEOUT
+ * when one has, or WINATTN_ERR_CUDA if the synchronisation failed.
+ */
+int winattn_last_device_status(void *stream);
+
+/*
+ * winattn_launch_info — the launch plan winattn_fwd would use, for tests and
+ * benchmarks: work items (query tiles of 128 rows), grid size, threads per
+ * CTA, dynamic shared memory bytes and windows packed per tile.  Any output
+ * pointer may be NULL.  Makes no CUDA call.  Returns the winattn_check_args
+ * code for the sizes (pointers are not checked).
+ */
+int winattn_launch_info(int B, int H_img, int W_img, int M, int shift, int heads, int d,
+                        int rank, int dtype, int64_t *work_items, int *grid, int *threads,
+                        int *smem_bytes, int *windows_per_tile);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* WINATTN_H */

@@ -1,0 +1,108 @@
+"""The C ABI without a GPU: the library loads, exports every declared entry
+point, and its host-side checks and launch plan behave as documented."""
+import math
+import os
+import re
+
+import pytest
+
+from windowed_attention_vision_b200 import _lib, build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "winattn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_ ]*?\*?\s*\b(winattn_[a-z_]+)\s*\(",
+                                 text, re.M)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 7, names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in winattn.h but not exported"
+    assert set(names) == set(_lib.EXPORTS)
+
+
+A = 1 << 20  # fake, 16-byte aligned addresses: only compared, never dereferenced
+
+
+def chk(**kw):
+    a = dict(q=A, k=2 * A, v=3 * A, theta=None, bias=None, B=2, H=16, W=16, M=8, shift=4, heads=2, d=32,
+             rank=0, dtype=_lib.BF16, out=4 * A)
+    a.update(kw)
+    return _lib.check_args(a["q"], a["k"], a["v"], a["theta"], a["bias"], a["B"], a["H"], a["W"], a["M"],
+                           a["shift"], a["heads"], a["d"], a["rank"], a["dtype"], a["out"])
+
+
+def test_check_args_accepts_valid(lib):
+    assert chk() == _lib.OK
+    assert chk(theta=5 * A) == _lib.OK
+    assert chk(rank=16, bias=6 * A) == _lib.OK
+    assert chk(dtype=_lib.FP32, d=16) == _lib.OK
+    assert chk(M=1, shift=0) == _lib.OK
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), _lib.ERR_ARG),
+    (dict(out=None), _lib.ERR_ARG),
+    (dict(B=0), _lib.ERR_ARG),
+    (dict(heads=-1), _lib.ERR_ARG),
+    (dict(M=0), _lib.ERR_ARG),
+    (dict(M=3), _lib.ERR_ARG),            # 16 % 3 != 0
+    (dict(shift=8), _lib.ERR_ARG),        # shift must be < M
+    (dict(shift=-1), _lib.ERR_ARG),
+    (dict(d=48), _lib.ERR_ARG),           # bf16 head dims are 32 or 64
+    (dict(d=8, dtype=_lib.FP32), _lib.ERR_ARG),
+    (dict(M=512, H=512, W=512), _lib.ERR_ARG),
+    (dict(rank=16), _lib.ERR_RANK),       # rank without bias_feats
+    (dict(bias=6 * A), _lib.ERR_RANK),    # bias_feats without rank
+    (dict(rank=8, bias=6 * A), _lib.ERR_RANK),
+    (dict(q=A + 8), _lib.ERR_ALIGN),
+    (dict(out=4 * A + 2), _lib.ERR_ALIGN),
+    (dict(theta=5 * A + 2), _lib.ERR_ALIGN),
+    (dict(rank=16, bias=6 * A + 4), _lib.ERR_ALIGN),
+    (dict(dtype=7), _lib.ERR_DTYPE),
+    (dict(out=A + 4096), _lib.ERR_ALIAS),  # overlaps q
+])
+def test_check_args_rejects(lib, kw, code):
+    assert chk(**kw) == code
+
+
+def test_strerror_covers_codes(lib):
+    for code in range(-9, 1):
+        s = _lib.strerror(code)
+        assert s and s != "unknown error code"
+    assert _lib.strerror(-100) == "unknown error code"
+
+
+def test_host_workspace_bytes(lib):
+    n = 2 * 16 * 16 * 2 * 32 * 2
+    assert _lib.host_workspace_bytes(2, 16, 16, 2, 32, _lib.BF16) == 4 * ((n + 255) // 256 * 256)
+    assert _lib.host_workspace_bytes(0, 16, 16, 2, 32, _lib.BF16) == 0
+
+
+@pytest.mark.parametrize("B,H,W,M,heads,d,rank,U,tiles", [
+    (64, 56, 56, 8, 3, 32, 0, 2, 1),      # Swin stage 1: two 64-token windows per tile
+    (16, 128, 128, 32, 3, 32, 0, 1, 8),   # 1024-token windows: 8 query tiles each
+    (4, 192, 192, 96, 6, 32, 16, 1, 72),  # 9216-token windows
+    (1, 24, 24, 12, 1, 32, 0, 1, 2),      # 144 tokens: a ragged second tile
+    (1, 9, 9, 3, 2, 64, 0, 14, 1),        # 9-token windows: 14 per tile
+    (2, 5, 5, 1, 1, 32, 0, 128, 1),       # one-token windows
+    (1, 10, 10, 10, 1, 32, 0, 1, 1),      # 100 tokens: one ragged tile
+])
+def test_launch_plan(lib, B, H, W, M, heads, d, rank, U, tiles):
+    rc, info = _lib.launch_info(B, H, W, M, 0, heads, d, rank, _lib.BF16)
+    assert rc == _lib.OK
+    windows = B * (H // M) * (W // M)
+    assert info["windows_per_tile"] == U
+    assert info["work_items"] == heads * math.ceil(windows / U) * tiles
+    assert info["threads"] == 128
+    assert 0 < info["smem_bytes"] <= 227 * 1024

@@ -1,1 +1,107 @@
-"""winattn: fused window attention for vision transformers on B200 (sm_100a)."""
+"""winattn: fused, exact windowed softmax attention for vision transformers on
+B200 (sm_100a), behind a C ABI (include/winattn.h).
+
+``window_attention`` is the public call on device tensors; ``window_attention_host``
+runs the same call on host tensors (copies in, kernel, copy out, all enqueued by
+the library).  Both go through the CUDA library; nothing here computes.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import WinattnError
+
+__all__ = ["window_attention", "window_attention_host", "WinattnError", "device_status"]
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return _lib.BF16
+    if t.dtype == torch.float32:
+        return _lib.FP32
+    raise WinattnError(_lib.ERR_DTYPE, f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _shape(q, k, v, theta, bias, M):
+    if q.dim() != 5 or q.shape != k.shape or q.shape != v.shape:
+        raise WinattnError(_lib.ERR_ARG, "q, k, v must share one [B, H, W, heads, d] shape")
+    if q.dtype != k.dtype or q.dtype != v.dtype:
+        raise WinattnError(_lib.ERR_DTYPE, "q, k, v must share one dtype")
+    for t in (q, k, v, theta, bias):
+        if t is not None and not t.is_contiguous():
+            raise WinattnError(_lib.ERR_ARG, "tensors must be contiguous")
+    B, H, W, heads, d = q.shape
+    if theta is not None and (theta.dtype != torch.float32 or tuple(theta.shape) != (heads, d // 4)):
+        raise WinattnError(_lib.ERR_ARG, "theta must be fp32 [heads, d/4]")
+    rank = 0
+    if bias is not None:
+        if bias.dim() != 4 or tuple(bias.shape[:3]) != (heads, 2, M * M) or bias.dtype != q.dtype:
+            raise WinattnError(_lib.ERR_RANK, "bias_feats must be [heads, 2, M*M, rank] in q's dtype")
+        rank = bias.shape[3]
+    return B, H, W, heads, d, rank
+
+
+def window_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, M: int, shift: int = 0,
+                     theta: Optional[torch.Tensor] = None, bias_feats: Optional[torch.Tensor] = None,
+                     out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Fused window attention on CUDA tensors [B, H, W, heads, d] (bf16 or fp32),
+    enqueued on torch's current stream.  See include/winattn.h for the exact
+    operation."""
+    B, H, W, heads, d, rank = _shape(q, k, v, theta, bias_feats, M)
+    for t in (q, k, v, theta, bias_feats):
+        if t is not None and not t.is_cuda:
+            raise WinattnError(_lib.ERR_ARG, "window_attention takes CUDA tensors")
+    if out is None:
+        out = torch.empty_like(q)
+    stream = torch.cuda.current_stream(q.device).cuda_stream
+    with torch.cuda.device(q.device):
+        rc = _lib.fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(theta), _ptr(bias_feats), B, H, W, M, shift, heads, d,
+                      rank, _dtype_code(q), _ptr(out), stream)
+    if rc != _lib.OK:
+        raise WinattnError(rc, "winattn_fwd")
+    return out
+
+
+def window_attention_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, M: int, shift: int = 0,
+                          theta: Optional[torch.Tensor] = None, bias_feats: Optional[torch.Tensor] = None,
+                          out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+                          device=None, synchronize: bool = True) -> torch.Tensor:
+    """The same operation on host tensors (pinned for asynchronous copies);
+    theta / bias_feats are CUDA tensors.  ``workspace`` is a uint8 CUDA tensor of
+    at least ``host_workspace_bytes`` bytes (allocated here when omitted)."""
+    B, H, W, heads, d, rank = _shape(q, k, v, theta, bias_feats, M)
+    device = torch.device(device or (theta.device if theta is not None else "cuda"))
+    code = _dtype_code(q)
+    need = _lib.host_workspace_bytes(B, H, W, heads, d, code)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=device)
+    if out is None:
+        out = torch.empty_like(q, pin_memory=q.is_pinned())
+    stream = torch.cuda.current_stream(device).cuda_stream
+    with torch.cuda.device(device):
+        rc = _lib.fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(theta), _ptr(bias_feats), B, H, W, M, shift, heads,
+                           d, rank, code, _ptr(out), _ptr(workspace), workspace.numel(), stream)
+    if rc != _lib.OK:
+        raise WinattnError(rc, "winattn_fwd_host")
+    if synchronize:
+        torch.cuda.current_stream(device).synchronize()
+    return out
+
+
+def host_workspace_bytes(q: torch.Tensor) -> int:
+    B, H, W, heads, d = q.shape
+    return _lib.host_workspace_bytes(B, H, W, heads, d, _dtype_code(q))
+
+
+def device_status(device=None) -> int:
+    """Synchronise torch's current stream and read/clear the bounded-wait status."""
+    dev = torch.device(device or "cuda")
+    with torch.cuda.device(dev):
+        return _lib.last_device_status(torch.cuda.current_stream(dev).cuda_stream)

@@ -1,0 +1,99 @@
+"""ctypes binding of the C ABI in include/winattn.h (argument marshalling only).
+
+Every step of the attention runs inside the CUDA library; this module only
+passes pointers, sizes and the stream.  It raises ``WinattnError`` when the
+library is missing or a call fails: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libwinattn.so")
+
+OK = 0
+ERR_ARG, ERR_RANK, ERR_ALIGN, ERR_DTYPE, ERR_ARCH = -1, -2, -3, -4, -5
+ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_ALIAS, ERR_SIZE = -6, -7, -8, -9
+BF16, FP32 = 0, 1
+
+EXPORTS = ("winattn_fwd", "winattn_check_args", "winattn_fwd_host", "winattn_host_workspace_bytes",
+           "winattn_strerror", "winattn_last_device_status", "winattn_launch_info")
+
+
+class WinattnError(RuntimeError):
+    def __init__(self, code: int, what: str = ""):
+        self.code = code
+        msg = strerror(code) if _lib is not None else f"code {code}"
+        super().__init__(f"{what}: {msg} ({code})" if what else f"{msg} ({code})")
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load the in-tree CUDA library (built by ``build.build()``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise WinattnError(ERR_CUDA, f"CUDA library {path} is missing; run __graft_entry__.build()")
+    lib = ctypes.CDLL(path)
+    vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    lib.winattn_fwd.argtypes = [vp, vp, vp, vp, vp] + [i32] * 9 + [vp, vp]
+    lib.winattn_fwd.restype = i32
+    lib.winattn_check_args.argtypes = [vp, vp, vp, vp, vp] + [i32] * 9 + [vp]
+    lib.winattn_check_args.restype = i32
+    lib.winattn_fwd_host.argtypes = [vp, vp, vp, vp, vp] + [i32] * 9 + [vp, vp, sz, vp]
+    lib.winattn_fwd_host.restype = i32
+    lib.winattn_host_workspace_bytes.argtypes = [i32] * 6
+    lib.winattn_host_workspace_bytes.restype = sz
+    lib.winattn_strerror.argtypes = [i32]
+    lib.winattn_strerror.restype = ctypes.c_char_p
+    lib.winattn_last_device_status.argtypes = [vp]
+    lib.winattn_last_device_status.restype = i32
+    lib.winattn_launch_info.argtypes = [i32] * 9 + [ctypes.POINTER(i64)] + [ctypes.POINTER(i32)] * 4
+    lib.winattn_launch_info.restype = i32
+    _lib = lib
+    return lib
+
+
+def strerror(code: int) -> str:
+    return load().winattn_strerror(code).decode()
+
+
+def fwd(q_ptr, k_ptr, v_ptr, theta_ptr, bias_ptr, B, H, W, M, shift, heads, d, rank, dtype, out_ptr,
+        stream) -> int:
+    return load().winattn_fwd(q_ptr, k_ptr, v_ptr, theta_ptr, bias_ptr, B, H, W, M, shift, heads, d, rank,
+                              dtype, out_ptr, stream)
+
+
+def check_args(q_ptr, k_ptr, v_ptr, theta_ptr, bias_ptr, B, H, W, M, shift, heads, d, rank, dtype,
+               out_ptr) -> int:
+    return load().winattn_check_args(q_ptr, k_ptr, v_ptr, theta_ptr, bias_ptr, B, H, W, M, shift, heads, d,
+                                     rank, dtype, out_ptr)
+
+
+def fwd_host(q_ptr, k_ptr, v_ptr, theta_ptr, bias_ptr, B, H, W, M, shift, heads, d, rank, dtype, out_ptr,
+             ws_ptr, ws_bytes, stream) -> int:
+    return load().winattn_fwd_host(q_ptr, k_ptr, v_ptr, theta_ptr, bias_ptr, B, H, W, M, shift, heads, d,
+                                   rank, dtype, out_ptr, ws_ptr, ws_bytes, stream)
+
+
+def host_workspace_bytes(B, H, W, heads, d, dtype) -> int:
+    return load().winattn_host_workspace_bytes(B, H, W, heads, d, dtype)
+
+
+def last_device_status(stream) -> int:
+    return load().winattn_last_device_status(stream)
+
+
+def launch_info(B, H, W, M, shift, heads, d, rank, dtype):
+    """(rc, dict) with work_items, grid, threads, smem_bytes, windows_per_tile."""
+    i64, i32 = ctypes.c_int64, ctypes.c_int
+    items, grid, threads, smem, wpt = i64(), i32(), i32(), i32(), i32()
+    rc = load().winattn_launch_info(B, H, W, M, shift, heads, d, rank, dtype, ctypes.byref(items),
+                                    ctypes.byref(grid), ctypes.byref(threads), ctypes.byref(smem),
+                                    ctypes.byref(wpt))
+    return rc, dict(work_items=items.value, grid=grid.value, threads=threads.value, smem_bytes=smem.value,
+                    windows_per_tile=wpt.value)

@@ -1,0 +1,330 @@
+// bf16 window-attention forward on the sm_100a tensor cores (tcgen05 UMMA,
+// accumulators in TMEM).
+//
+// One CTA of 128 threads owns one 128-row query tile; thread t owns row t
+// (TMEM lane t).  Per key tile:
+//   1. gather: each thread loads one key token and one value token of the
+//      window straight from the B x H x W x (heads*d) map (cyclic shift by
+//      index), applies window-local 2D RoPE to the key in fp32 registers,
+//      rounds to bf16 and stores K, V (and the rank-r key factors w) into
+//      swizzled shared-memory operand tiles;
+//   2. S = Q~ K~^T: one thread issues d/16 (+ r/16) UMMAs 128x128x16 into TMEM;
+//   3. online softmax: each thread reads its S row from TMEM, masks
+//      (wrap labels, packed-window blocks, ragged tails), keeps the running
+//      max / sum in fp32 and writes P (bf16) into a swizzled tile;
+//   4. O_tile = P V: eight UMMAs 128 x d x 16 into TMEM (the S columns, now
+//      free), added to the fp32 register accumulator after rescaling.
+// The query tile is gathered and rotated the same way once per CTA, scaled by
+// d^-1/2 before rounding (the rank-r query factors u stay unscaled, so
+// S = d^-1/2 q.k + u.w in one dot product, as the RIB page's concatenation
+// [Qc, Qp][Kc, Kp]^T = Qc Kc^T + Qp Kp^T has it).
+//
+// Sources: "FLASHSWIN" page, section "어떻게 동작하나" (fused IO-aware kernel,
+// online softmax, N x N never stored, window-local RoPE, additive wrap mask)
+// and section "전제와 한계" (bf16 Q/K/V, RoPE in fp32, fp32 softmax);
+// "Rank-Factorized Implicit Neural Bias" page, section 2.1.
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "geometry.cuh"
+#include "ptx.cuh"
+
+namespace winattn {
+
+// Set (bit 0) by a kernel that gave up a bounded wait; read and cleared by
+// winattn_last_device_status.  One word per device (module-scope variable).
+__device__ unsigned int g_status_word = 0;
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D, int R>
+struct TcLayout {
+    static constexpr uint32_t QC = 0;                       // query content  [128][D]  bf16
+    static constexpr uint32_t QB = QC + 256 * D;            // query factors  [128][R]  bf16
+    static constexpr uint32_t KC = QB + 256 * R;            // key content    [128][D]
+    static constexpr uint32_t KB = KC + 256 * D;            // key factors    [128][R]
+    static constexpr uint32_t VO = KB + 256 * R;            // values         [128][D]
+    static constexpr uint32_t PO = VO + 256 * D;            // probabilities  2 x [128][64]
+    static constexpr uint32_t TB = PO + 32768;              // RoPE table     [M][D/4] float2
+    static __host__ __device__ uint32_t table_bytes(int M) { return (uint32_t)((M * (D / 4) * 8 + 15) & ~15); }
+    static __host__ __device__ uint32_t codes(int M) { return TB + table_bytes(M); }   // [128] u16
+    static __host__ __device__ uint32_t bar(int M) { return codes(M) + 256; }          // u64
+    static __host__ __device__ uint32_t tslot(int M) { return bar(M) + 8; }            // u32
+    static __host__ __device__ uint32_t bytes(int M) { return tslot(M) + 16 + 1024; }  // + alignment slack
+};
+
+// Gather one d-vector (bf16), rotate it by R(i, j) in fp32, multiply by `mul`,
+// round to bf16 and store it as row `row` of a swizzled K-major tile.
+template <int D>
+__device__ __forceinline__ void gather_rotate_store(const __nv_bfloat16 *__restrict__ src, const float2 *table,
+                                                   int i, int j, float mul, uint8_t *tile, int row)
+{
+    float x[D];
+    const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+        const uint4 u = __ldg(s4 + c);
+        x[8 * c + 0] = bf16lo(u.x); x[8 * c + 1] = bf16hi(u.x);
+        x[8 * c + 2] = bf16lo(u.y); x[8 * c + 3] = bf16hi(u.y);
+        x[8 * c + 4] = bf16lo(u.z); x[8 * c + 5] = bf16hi(u.z);
+        x[8 * c + 6] = bf16lo(u.w); x[8 * c + 7] = bf16hi(u.w);
+    }
+    if (table) {
+#pragma unroll
+        for (int k = 0; k < D / 4; ++k) {
+            const float2 ry = table[i * (D / 4) + k];   // (cos, sin) of i * theta_k
+            const float a0 = x[2 * k], a1 = x[2 * k + 1];
+            x[2 * k] = a0 * ry.x - a1 * ry.y;
+            x[2 * k + 1] = a0 * ry.y + a1 * ry.x;
+            const float2 rx = table[j * (D / 4) + k];   // (cos, sin) of j * theta_k
+            const float b0 = x[D / 2 + 2 * k], b1 = x[D / 2 + 2 * k + 1];
+            x[D / 2 + 2 * k] = b0 * rx.x - b1 * rx.y;
+            x[D / 2 + 2 * k + 1] = b0 * rx.y + b1 * rx.x;
+        }
+    }
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+        uint4 o;
+        o.x = pack_bf16x2(x[8 * c + 0] * mul, x[8 * c + 1] * mul);
+        o.y = pack_bf16x2(x[8 * c + 2] * mul, x[8 * c + 3] * mul);
+        o.z = pack_bf16x2(x[8 * c + 4] * mul, x[8 * c + 5] * mul);
+        o.w = pack_bf16x2(x[8 * c + 6] * mul, x[8 * c + 7] * mul);
+        *reinterpret_cast<uint4 *>(tile + swz_offset(row, c, 2 * D)) = o;
+    }
+}
+
+// Copy COLS bf16 values unchanged into row `row` of a swizzled tile.
+template <int COLS>
+__device__ __forceinline__ void copy_row(const __nv_bfloat16 *__restrict__ src, uint8_t *tile, int row)
+{
+    const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
+#pragma unroll
+    for (int c = 0; c < COLS / 8; ++c)
+        *reinterpret_cast<uint4 *>(tile + swz_offset(row, c, 2 * COLS)) = __ldg(s4 + c);
+}
+
+template <int COLS>
+__device__ __forceinline__ void zero_row(uint8_t *tile, int row)
+{
+#pragma unroll
+    for (int c = 0; c < COLS / 8; ++c)
+        *reinterpret_cast<uint4 *>(tile + swz_offset(row, c, 2 * COLS)) = make_uint4(0, 0, 0, 0);
+}
+
+template <int D, int R>
+__global__ void __launch_bounds__(128, 1)
+    winattn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                          const __nv_bfloat16 *__restrict__ v, const float *__restrict__ theta,
+                          const __nv_bfloat16 *__restrict__ bias, __nv_bfloat16 *__restrict__ out,
+                          const Geometry g, const float scale)
+{
+    using L = TcLayout<D, R>;
+    extern __shared__ uint8_t smem_raw[];
+    // Operand tiles need 1024-byte alignment of their shared-memory address.
+    uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(base);
+    float2 *table = reinterpret_cast<float2 *>(base + L::TB);
+    uint16_t *codes = reinterpret_cast<uint16_t *>(base + L::codes(g.M));
+    uint64_t *bar = reinterpret_cast<uint64_t *>(base + L::bar(g.M));
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(base + L::tslot(g.M));
+
+    const int t = threadIdx.x;
+    const int warp = t >> 5;
+    constexpr uint32_t kTmemCols = 128;
+
+    if (warp == 0) {
+        tmem_alloc(tslot, kTmemCols);
+        tmem_relinquish();
+    }
+    if (t == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    const Item it = decode_item(g, blockIdx.x);
+    if (theta) {
+        for (int idx = t; idx < g.M * (D / 4); idx += blockDim.x) {
+            const int c = idx / (D / 4), kk = idx - c * (D / 4);
+            float sn, cs;
+            sincosf((float)c * __ldg(theta + it.h * (D / 4) + kk), &sn, &cs);
+            table[idx] = make_float2(cs, sn);
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tslot;
+    const uint32_t tmem_row = tmem + ((uint32_t)(warp * 32) << 16);
+    const float2 *tab = theta ? table : nullptr;
+
+    // ---- query row t
+    const RowRef qr = tile_row(g, it.pack, it.tile, t);
+    int qcode = 0xFFFF;  // matches no key code
+    if (qr.valid) {
+        const TokenRef tk = token_ref(g, qr.w, qr.p, it.h);
+        qcode = (qr.slot << 2) | tk.label;
+        gather_rotate_store<D>(q + tk.offset, tab, tk.i, tk.j, scale, base + L::QC, t);
+        if constexpr (R > 0)
+            copy_row<R>(bias + (((int64_t)it.h * 2 + 0) * g.N + qr.p) * R, base + L::QB, t);
+    } else {
+        zero_row<D>(base + L::QC, t);
+        if constexpr (R > 0)
+            zero_row<R>(base + L::QB, t);
+    }
+
+    constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false);
+    constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
+
+    float m = -INFINITY, l = 0.f;
+    float o[D];
+#pragma unroll
+    for (int e = 0; e < D; ++e)
+        o[e] = 0.f;
+    uint32_t phase = 0;
+    bool ok = true;
+
+    for (int kv = 0; kv < g.n_tiles; ++kv) {
+        // ---- 1. gather K (rotated), w, V for key row t
+        const RowRef kr = tile_row(g, it.pack, kv, t);
+        uint16_t code = 0xFFFE;
+        if (kr.valid) {
+            const TokenRef tk = token_ref(g, kr.w, kr.p, it.h);
+            code = (uint16_t)((kr.slot << 2) | tk.label);
+            gather_rotate_store<D>(k + tk.offset, tab, tk.i, tk.j, 1.f, base + L::KC, t);
+            if constexpr (R > 0)
+                copy_row<R>(bias + (((int64_t)it.h * 2 + 1) * g.N + kr.p) * R, base + L::KB, t);
+            copy_row<D>(v + tk.offset, base + L::VO, t);
+        } else {
+            zero_row<D>(base + L::KC, t);
+            if constexpr (R > 0)
+                zero_row<R>(base + L::KB, t);
+            zero_row<D>(base + L::VO, t);
+        }
+        codes[t] = code;
+        fence_proxy_async_smem();
+        tc_fence_before_sync();
+        __syncthreads();
+
+        // ---- 2. S = Q~ K~^T
+        if (t == 0) {
+            tc_fence_after_sync();
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                const uint64_t a = smem_desc(sbase + L::QC + ks * 32, 16, 16 * D, swizzle_code(2 * D));
+                const uint64_t b = smem_desc(sbase + L::KC + ks * 32, 16, 16 * D, swizzle_code(2 * D));
+                umma_bf16_ss(tmem, a, b, kIdescS, ks > 0);
+            }
+#pragma unroll
+            for (int ks = 0; ks < R / 16; ++ks) {
+                const uint64_t a = smem_desc(sbase + L::QB + ks * 32, 16, 16 * R, swizzle_code(2 * R));
+                const uint64_t b = smem_desc(sbase + L::KB + ks * 32, 16, 16 * R, swizzle_code(2 * R));
+                umma_bf16_ss(tmem, a, b, kIdescS, 1);
+            }
+            umma_commit(bar);
+        }
+        const bool s_done = mbar_wait(bar, phase);
+        phase ^= 1;
+        if (__syncthreads_or(!s_done)) {
+            ok = false;
+            break;
+        }
+        tc_fence_after_sync();
+
+        // ---- 3. online softmax on row t
+        float s[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            tmem_ld32(tmem_row + c * 32, s + c * 32);
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+            if (codes[c] != qcode)
+                s[c] = -INFINITY;
+            mx = fmaxf(mx, s[c]);
+        }
+        const float m_new = fmaxf(m, mx * kLog2e);
+        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+        const float alpha = fast_exp2(m - m_use);
+        float rs = 0.f;
+#pragma unroll
+        for (int ch = 0; ch < 16; ++ch) {
+            float p[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                p[e] = fast_exp2(fmaf(s[8 * ch + e], kLog2e, -m_use));
+                rs += p[e];
+            }
+            uint4 pk;
+            pk.x = pack_bf16x2(p[0], p[1]);
+            pk.y = pack_bf16x2(p[2], p[3]);
+            pk.z = pack_bf16x2(p[4], p[5]);
+            pk.w = pack_bf16x2(p[6], p[7]);
+            *reinterpret_cast<uint4 *>(base + L::PO + (ch >> 3) * 16384 + swz_offset(t, ch & 7, 128)) = pk;
+        }
+        l = l * alpha + rs;
+        m = m_new;
+        fence_proxy_async_smem();
+        tc_fence_before_sync();
+        __syncthreads();
+
+        // ---- 4. O_tile = P V  (into the S columns)
+        if (t == 0) {
+            tc_fence_after_sync();
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint64_t a = smem_desc(sbase + L::PO + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, 2);
+                const uint64_t b = smem_desc(sbase + L::VO + ks * 32 * D, 8192, 16 * D, swizzle_code(2 * D));
+                umma_bf16_ss(tmem, a, b, kIdescPV, ks > 0);
+            }
+            umma_commit(bar);
+        }
+        const bool o_done = mbar_wait(bar, phase);
+        phase ^= 1;
+        if (__syncthreads_or(!o_done)) {
+            ok = false;
+            break;
+        }
+        tc_fence_after_sync();
+        float ot[D];
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c)
+            tmem_ld32(tmem_row + c * 32, ot + c * 32);
+#pragma unroll
+        for (int e = 0; e < D; ++e)
+            o[e] = fmaf(o[e], alpha, ot[e]);
+        tc_fence_before_sync();
+        __syncthreads();
+    }
+
+    // ---- normalise and write back to the original (un-shifted) position
+    if (ok && qr.valid) {
+        const TokenRef tk = token_ref(g, qr.w, qr.p, it.h);
+        const float inv = 1.f / l;
+        uint4 *dst = reinterpret_cast<uint4 *>(out + tk.offset);
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+            uint4 w;
+            w.x = pack_bf16x2(o[8 * c + 0] * inv, o[8 * c + 1] * inv);
+            w.y = pack_bf16x2(o[8 * c + 2] * inv, o[8 * c + 3] * inv);
+            w.z = pack_bf16x2(o[8 * c + 4] * inv, o[8 * c + 5] * inv);
+            w.w = pack_bf16x2(o[8 * c + 6] * inv, o[8 * c + 7] * inv);
+            dst[c] = w;
+        }
+    }
+    if (!ok) {
+        if (t == 0) {
+            atomicOr(&g_status_word, 1u);
+            // Give an MMA that may still be in flight one more bounded chance
+            // to land before its TMEM is released.
+            mbar_wait(bar, phase);
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace winattn

@@ -1,0 +1,296 @@
+// C ABI of the fused window-attention forward (declared in include/winattn.h):
+// argument checks, launch planning, kernel dispatch, the host-buffer variant
+// and the per-device status word of the bounded waits.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/winattn.h"
+#include "fwd_simt.cuh"
+#include "fwd_tc.cuh"
+#include "geometry.cuh"
+
+namespace winattn {
+
+namespace {
+
+constexpr int kMaxM = 256;      // RoPE table and window index limits
+constexpr int kThreads = 128;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb)
+{
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+int check_sizes(int B, int H, int W, int M, int shift, int heads, int d, int rank, int dtype)
+{
+    if (dtype != WINATTN_BF16 && dtype != WINATTN_FP32)
+        return WINATTN_ERR_DTYPE;
+    if (B <= 0 || H <= 0 || W <= 0 || M <= 0 || heads <= 0 || M > kMaxM)
+        return WINATTN_ERR_ARG;
+    if (H % M || W % M || shift < 0 || shift >= M)
+        return WINATTN_ERR_ARG;
+    if (dtype == WINATTN_BF16 && d != 32 && d != 64)
+        return WINATTN_ERR_ARG;
+    if (dtype == WINATTN_FP32 && d != 16 && d != 32 && d != 64)
+        return WINATTN_ERR_ARG;
+    if (rank != 0 && rank != 16 && rank != 32)
+        return WINATTN_ERR_RANK;
+    const Geometry g = Geometry::make(B, H, W, M, shift, heads, d, rank);
+    const double elems = (double)B * H * W * heads * d;
+    if (elems > 9.0e18 || g.items > 0x7FFFFFFFLL)
+        return WINATTN_ERR_SIZE;
+    return WINATTN_OK;
+}
+
+size_t map_bytes(int B, int H, int W, int heads, int d, int dtype)
+{
+    return (size_t)B * H * W * heads * d * (dtype == WINATTN_BF16 ? 2 : 4);
+}
+
+int smem_bytes_for(const Geometry &g, int dtype)
+{
+    if (dtype == WINATTN_BF16) {
+        switch (g.d * 100 + g.rank) {
+        case 3200: return (int)TcLayout<32, 0>::bytes(g.M);
+        case 3216: return (int)TcLayout<32, 16>::bytes(g.M);
+        case 3232: return (int)TcLayout<32, 32>::bytes(g.M);
+        case 6400: return (int)TcLayout<64, 0>::bytes(g.M);
+        case 6416: return (int)TcLayout<64, 16>::bytes(g.M);
+        case 6432: return (int)TcLayout<64, 32>::bytes(g.M);
+        }
+    } else {
+        switch (g.d * 100 + g.rank) {
+        case 1600: return (int)SimtLayout<16, 0>::bytes(g.M);
+        case 1616: return (int)SimtLayout<16, 16>::bytes(g.M);
+        case 1632: return (int)SimtLayout<16, 32>::bytes(g.M);
+        case 3200: return (int)SimtLayout<32, 0>::bytes(g.M);
+        case 3216: return (int)SimtLayout<32, 16>::bytes(g.M);
+        case 3232: return (int)SimtLayout<32, 32>::bytes(g.M);
+        case 6400: return (int)SimtLayout<64, 0>::bytes(g.M);
+        case 6416: return (int)SimtLayout<64, 16>::bytes(g.M);
+        case 6432: return (int)SimtLayout<64, 32>::bytes(g.M);
+        }
+    }
+    return -1;
+}
+
+// Compute capability check, cached per device.
+int check_device()
+{
+    static std::mutex mu;
+    static int cached[64];  // 0 unknown, 1 ok, 2 wrong arch
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return WINATTN_ERR_CUDA;
+    if (dev < 0 || dev >= 64)
+        return WINATTN_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cached[dev] == 0) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+            return WINATTN_ERR_CUDA;
+        cached[dev] = (major == 10 && minor == 0) ? 1 : 2;
+    }
+    return cached[dev] == 1 ? WINATTN_OK : WINATTN_ERR_ARCH;
+}
+
+template <typename Kernel>
+int launch(Kernel kernel, int smem, const Geometry &g, cudaStream_t stream, auto... args)
+{
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return WINATTN_ERR_CUDA;
+    kernel<<<(unsigned)g.items, kThreads, smem, stream>>>(args..., g, 1.0f / std::sqrt((float)g.d));
+    return cudaGetLastError() == cudaSuccess ? WINATTN_OK : WINATTN_ERR_CUDA;
+}
+
+template <int D, int R>
+int launch_tc(const void *q, const void *k, const void *v, const float *theta, const void *bias, void *out,
+              const Geometry &g, cudaStream_t stream)
+{
+    using T = __nv_bfloat16;
+    return launch(winattn_fwd_tc_kernel<D, R>, (int)TcLayout<D, R>::bytes(g.M), g, stream,
+                  static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), theta,
+                  static_cast<const T *>(bias), static_cast<T *>(out));
+}
+
+template <int D, int R>
+int launch_simt(const void *q, const void *k, const void *v, const float *theta, const void *bias, void *out,
+                const Geometry &g, cudaStream_t stream)
+{
+    return launch(winattn_fwd_simt_kernel<D, R>, (int)SimtLayout<D, R>::bytes(g.M), g, stream,
+                  static_cast<const float *>(q), static_cast<const float *>(k), static_cast<const float *>(v),
+                  theta, static_cast<const float *>(bias), static_cast<float *>(out));
+}
+
+int dispatch(const void *q, const void *k, const void *v, const float *theta, const void *bias, void *out,
+             const Geometry &g, int dtype, cudaStream_t s)
+{
+    if (dtype == WINATTN_BF16) {
+        switch (g.d * 100 + g.rank) {
+        case 3200: return launch_tc<32, 0>(q, k, v, theta, bias, out, g, s);
+        case 3216: return launch_tc<32, 16>(q, k, v, theta, bias, out, g, s);
+        case 3232: return launch_tc<32, 32>(q, k, v, theta, bias, out, g, s);
+        case 6400: return launch_tc<64, 0>(q, k, v, theta, bias, out, g, s);
+        case 6416: return launch_tc<64, 16>(q, k, v, theta, bias, out, g, s);
+        case 6432: return launch_tc<64, 32>(q, k, v, theta, bias, out, g, s);
+        }
+    } else {
+        switch (g.d * 100 + g.rank) {
+        case 1600: return launch_simt<16, 0>(q, k, v, theta, bias, out, g, s);
+        case 1616: return launch_simt<16, 16>(q, k, v, theta, bias, out, g, s);
+        case 1632: return launch_simt<16, 32>(q, k, v, theta, bias, out, g, s);
+        case 3200: return launch_simt<32, 0>(q, k, v, theta, bias, out, g, s);
+        case 3216: return launch_simt<32, 16>(q, k, v, theta, bias, out, g, s);
+        case 3232: return launch_simt<32, 32>(q, k, v, theta, bias, out, g, s);
+        case 6400: return launch_simt<64, 0>(q, k, v, theta, bias, out, g, s);
+        case 6416: return launch_simt<64, 16>(q, k, v, theta, bias, out, g, s);
+        case 6432: return launch_simt<64, 32>(q, k, v, theta, bias, out, g, s);
+        }
+    }
+    return WINATTN_ERR_ARG;
+}
+
+}  // namespace
+}  // namespace winattn
+
+using namespace winattn;
+
+extern "C" {
+
+int winattn_check_args(const void *q, const void *k, const void *v, const float *theta, const void *bias_feats,
+                       int B, int H_img, int W_img, int M, int shift, int heads, int d, int rank, int dtype,
+                       const void *out)
+{
+    const int rc = check_sizes(B, H_img, W_img, M, shift, heads, d, rank, dtype);
+    if (rc != WINATTN_OK)
+        return rc;
+    if (!q || !k || !v || !out)
+        return WINATTN_ERR_ARG;
+    if ((rank > 0) != (bias_feats != nullptr))
+        return WINATTN_ERR_RANK;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        (bias_feats && !aligned16(bias_feats)) || (reinterpret_cast<uintptr_t>(theta) & 3u))
+        return WINATTN_ERR_ALIGN;
+    const size_t n = map_bytes(B, H_img, W_img, heads, d, dtype);
+    if (overlaps(out, n, q, n) || overlaps(out, n, k, n) || overlaps(out, n, v, n))
+        return WINATTN_ERR_ALIAS;
+    return WINATTN_OK;
+}
+
+int winattn_fwd(const void *q, const void *k, const void *v, const float *theta, const void *bias_feats, int B,
+                int H_img, int W_img, int M, int shift, int heads, int d, int rank, int dtype, void *out,
+                void *stream)
+{
+    int rc = winattn_check_args(q, k, v, theta, bias_feats, B, H_img, W_img, M, shift, heads, d, rank, dtype, out);
+    if (rc != WINATTN_OK)
+        return rc;
+    rc = check_device();
+    if (rc != WINATTN_OK)
+        return rc;
+    const Geometry g = Geometry::make(B, H_img, W_img, M, shift, heads, d, rank);
+    return dispatch(q, k, v, theta, bias_feats, out, g, dtype, static_cast<cudaStream_t>(stream));
+}
+
+size_t winattn_host_workspace_bytes(int B, int H_img, int W_img, int heads, int d, int dtype)
+{
+    if (B <= 0 || H_img <= 0 || W_img <= 0 || heads <= 0 || d <= 0 ||
+        (dtype != WINATTN_BF16 && dtype != WINATTN_FP32))
+        return 0;
+    const size_t n = (map_bytes(B, H_img, W_img, heads, d, dtype) + 255) & ~size_t(255);
+    return 4 * n;
+}
+
+int winattn_fwd_host(const void *q_host, const void *k_host, const void *v_host, const float *theta,
+                     const void *bias_feats, int B, int H_img, int W_img, int M, int shift, int heads, int d,
+                     int rank, int dtype, void *out_host, void *workspace, size_t workspace_bytes, void *stream)
+{
+    int rc = check_sizes(B, H_img, W_img, M, shift, heads, d, rank, dtype);
+    if (rc != WINATTN_OK)
+        return rc;
+    if (!q_host || !k_host || !v_host || !out_host || !workspace)
+        return WINATTN_ERR_ARG;
+    if (workspace_bytes < winattn_host_workspace_bytes(B, H_img, W_img, heads, d, dtype))
+        return WINATTN_ERR_SIZE;
+    if (!aligned16(workspace))
+        return WINATTN_ERR_ALIGN;
+    const size_t n = map_bytes(B, H_img, W_img, heads, d, dtype);
+    const size_t stride = (n + 255) & ~size_t(255);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    void *dq = ws, *dk = ws + stride, *dv = ws + 2 * stride, *dout = ws + 3 * stride;
+    rc = winattn_check_args(dq, dk, dv, theta, bias_feats, B, H_img, W_img, M, shift, heads, d, rank, dtype, dout);
+    if (rc != WINATTN_OK)
+        return rc;
+    rc = check_device();
+    if (rc != WINATTN_OK)
+        return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(dq, q_host, n, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(dk, k_host, n, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(dv, v_host, n, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return WINATTN_ERR_CUDA;
+    const Geometry g = Geometry::make(B, H_img, W_img, M, shift, heads, d, rank);
+    rc = dispatch(dq, dk, dv, theta, bias_feats, dout, g, dtype, s);
+    if (rc != WINATTN_OK)
+        return rc;
+    if (cudaMemcpyAsync(out_host, dout, n, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return WINATTN_ERR_CUDA;
+    return WINATTN_OK;
+}
+
+const char *winattn_strerror(int code)
+{
+    switch (code) {
+    case WINATTN_OK: return "success";
+    case WINATTN_ERR_ARG: return "invalid argument (null pointer, size, window/map mismatch, shift or head dim)";
+    case WINATTN_ERR_RANK: return "bias rank and bias_feats pointer disagree, or unsupported rank";
+    case WINATTN_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case WINATTN_ERR_DTYPE: return "unsupported dtype";
+    case WINATTN_ERR_ARCH: return "device is not compute capability 10.0 (B200, sm_100a)";
+    case WINATTN_ERR_CUDA: return "CUDA runtime error or kernel launch failure";
+    case WINATTN_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel timed out";
+    case WINATTN_ERR_ALIAS: return "out overlaps q, k or v";
+    case WINATTN_ERR_SIZE: return "problem too large for the index range, or workspace too small";
+    }
+    return "unknown error code";
+}
+
+int winattn_last_device_status(void *stream)
+{
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return WINATTN_ERR_CUDA;
+    unsigned int word = 0;
+    if (cudaMemcpyFromSymbol(&word, g_status_word, sizeof word) != cudaSuccess)
+        return WINATTN_ERR_CUDA;
+    if (word) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(g_status_word, &zero, sizeof zero) != cudaSuccess)
+            return WINATTN_ERR_CUDA;
+        return WINATTN_ERR_DEVICE_TIMEOUT;
+    }
+    return WINATTN_OK;
+}
+
+int winattn_launch_info(int B, int H_img, int W_img, int M, int shift, int heads, int d, int rank, int dtype,
+                        int64_t *work_items, int *grid, int *threads, int *smem_bytes, int *windows_per_tile)
+{
+    const int rc = check_sizes(B, H_img, W_img, M, shift, heads, d, rank, dtype);
+    if (rc != WINATTN_OK)
+        return rc;
+    const Geometry g = Geometry::make(B, H_img, W_img, M, shift, heads, d, rank);
+    if (work_items) *work_items = g.items;
+    if (grid) *grid = (int)g.items;
+    if (threads) *threads = kThreads;
+    if (smem_bytes) *smem_bytes = smem_bytes_for(g, dtype);
+    if (windows_per_tile) *windows_per_tile = g.U;
+    return WINATTN_OK;
+}
+
+}  // extern "C"
