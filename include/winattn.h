@@ -140,14 +140,17 @@ int winattn_last_device_status(void *stream);
 
 /*
  * winattn_launch_info — the launch plan winattn_fwd would use, for tests and
- * benchmarks: work items (query tiles of 128 rows), grid size, threads per
- * CTA, dynamic shared memory bytes and windows packed per tile.  Any output
- * pointer may be NULL.  Makes no CUDA call.  Returns the winattn_check_args
- * code for the sizes (pointers are not checked).
+ * benchmarks: work items (128-row query tiles), grid size (persistent kernels:
+ * one CTA per SM of a 148-SM B200, capped by the work items), threads per CTA,
+ * dynamic shared memory bytes, windows packed per tile and the kernel chosen
+ * (0 = generic tensor-core kernel, 1 = persistent small-window kernel,
+ * 3 = fp32 SIMT kernel).  Any output pointer may be NULL.  Makes no CUDA
+ * call.  Returns the winattn_check_args code for the sizes (pointers are not
+ * checked).
  */
 int winattn_launch_info(int B, int H_img, int W_img, int M, int shift, int heads, int d,
                         int rank, int dtype, int64_t *work_items, int *grid, int *threads,
-                        int *smem_bytes, int *windows_per_tile);
+                        int *smem_bytes, int *windows_per_tile, int *kernel);
 
 #ifdef __cplusplus
 }

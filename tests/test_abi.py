@@ -89,20 +89,33 @@ def test_host_workspace_bytes(lib):
     assert _lib.host_workspace_bytes(0, 16, 16, 2, 32, _lib.BF16) == 0
 
 
-@pytest.mark.parametrize("B,H,W,M,heads,d,rank,U,tiles", [
-    (64, 56, 56, 8, 3, 32, 0, 2, 1),      # Swin stage 1: two 64-token windows per tile
-    (16, 128, 128, 32, 3, 32, 0, 1, 8),   # 1024-token windows: 8 query tiles each
-    (4, 192, 192, 96, 6, 32, 16, 1, 72),  # 9216-token windows
-    (1, 24, 24, 12, 1, 32, 0, 1, 2),      # 144 tokens: a ragged second tile
-    (1, 9, 9, 3, 2, 64, 0, 14, 1),        # 9-token windows: 14 per tile
-    (2, 5, 5, 1, 1, 32, 0, 128, 1),       # one-token windows
-    (1, 10, 10, 10, 1, 32, 0, 1, 1),      # 100 tokens: one ragged tile
+GENERIC, SMALL, SIMT = 0, 1, 3
+
+
+@pytest.mark.parametrize("B,H,W,M,heads,d,rank,U,tiles,kernel", [
+    (64, 56, 56, 8, 3, 32, 0, 2, 1, SMALL),      # Swin stage 1: two 64-token windows per tile
+    (16, 128, 128, 32, 3, 32, 0, 1, 8, GENERIC),  # 1024-token windows: 8 query tiles each
+    (4, 192, 192, 96, 6, 32, 16, 1, 72, GENERIC),  # 9216-token windows
+    (1, 24, 24, 12, 1, 32, 0, 1, 2, GENERIC),     # 144 tokens: a ragged second tile
+    (1, 9, 9, 3, 2, 64, 0, 14, 1, SMALL),         # 9-token windows: 14 per tile
+    (2, 5, 5, 1, 1, 32, 0, 128, 1, SMALL),        # one-token windows
+    (1, 10, 10, 10, 1, 32, 0, 1, 1, SMALL),       # 100 tokens: one ragged tile
+    (1, 8, 8, 8, 80, 32, 0, 2, 1, GENERIC),       # too many heads for the small kernel's RoPE table
 ])
-def test_launch_plan(lib, B, H, W, M, heads, d, rank, U, tiles):
+def test_launch_plan(lib, B, H, W, M, heads, d, rank, U, tiles, kernel):
     rc, info = _lib.launch_info(B, H, W, M, 0, heads, d, rank, _lib.BF16)
     assert rc == _lib.OK
     windows = B * (H // M) * (W // M)
     assert info["windows_per_tile"] == U
     assert info["work_items"] == heads * math.ceil(windows / U) * tiles
-    assert info["threads"] == 128
+    assert info["kernel"] == kernel
+    if kernel == SMALL:
+        assert info["threads"] == 416 and info["grid"] == min(148, info["work_items"])
+    else:
+        assert info["threads"] == 128 and info["grid"] == info["work_items"]
     assert 0 < info["smem_bytes"] <= 227 * 1024
+
+
+def test_launch_plan_fp32(lib):
+    rc, info = _lib.launch_info(1, 16, 16, 8, 0, 2, 32, 0, _lib.FP32)
+    assert rc == _lib.OK and info["kernel"] == SIMT

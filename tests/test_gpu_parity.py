@@ -30,6 +30,9 @@ SMALL = [
     ("m12_s6", 1, 24, 24, 12, 6, 2, 32, "bf16", "learned", 0),      # 144 tokens: ragged second tile
     ("m16_s8_d64", 1, 32, 32, 16, 8, 2, 64, "bf16", "learned", 0),
     ("m32_s16", 1, 64, 64, 32, 16, 2, 32, "bf16", "standard", 0),
+    ("m8_s4_many_heads", 1, 16, 16, 8, 4, 80, 32, "bf16", "learned", 0),  # generic kernel at N = 64
+    ("m11_s5_d64_r16", 1, 22, 22, 11, 5, 2, 64, "bf16", "learned", 16),   # 121 tokens, small kernel
+    ("m9_s4_r32", 2, 18, 9, 9, 4, 3, 32, "bf16", None, 32),
     ("m24_s0_r16", 1, 48, 48, 24, 0, 2, 32, "bf16", None, 16),      # bias factors, no RoPE
     ("m8_s4_r32_rope", 2, 16, 16, 8, 4, 2, 32, "bf16", "learned", 32),
     ("m16_s8_d64_r16", 1, 32, 32, 16, 8, 1, 64, "bf16", "learned", 16),

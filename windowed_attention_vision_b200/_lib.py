@@ -52,7 +52,7 @@ def load(path: str = LIB_PATH):
     lib.winattn_strerror.restype = ctypes.c_char_p
     lib.winattn_last_device_status.argtypes = [vp]
     lib.winattn_last_device_status.restype = i32
-    lib.winattn_launch_info.argtypes = [i32] * 9 + [ctypes.POINTER(i64)] + [ctypes.POINTER(i32)] * 4
+    lib.winattn_launch_info.argtypes = [i32] * 9 + [ctypes.POINTER(i64)] + [ctypes.POINTER(i32)] * 5
     lib.winattn_launch_info.restype = i32
     _lib = lib
     return lib
@@ -89,11 +89,11 @@ def last_device_status(stream) -> int:
 
 
 def launch_info(B, H, W, M, shift, heads, d, rank, dtype):
-    """(rc, dict) with work_items, grid, threads, smem_bytes, windows_per_tile."""
+    """(rc, dict) with work_items, grid, threads, smem_bytes, windows_per_tile, kernel."""
     i64, i32 = ctypes.c_int64, ctypes.c_int
-    items, grid, threads, smem, wpt = i64(), i32(), i32(), i32(), i32()
+    items, grid, threads, smem, wpt, kern = i64(), i32(), i32(), i32(), i32(), i32()
     rc = load().winattn_launch_info(B, H, W, M, shift, heads, d, rank, dtype, ctypes.byref(items),
                                     ctypes.byref(grid), ctypes.byref(threads), ctypes.byref(smem),
-                                    ctypes.byref(wpt))
+                                    ctypes.byref(wpt), ctypes.byref(kern))
     return rc, dict(work_items=items.value, grid=grid.value, threads=threads.value, smem_bytes=smem.value,
-                    windows_per_tile=wpt.value)
+                    windows_per_tile=wpt.value, kernel=kern.value)

@@ -32,12 +32,6 @@
 
 namespace winattn {
 
-// Set (bit 0) by a kernel that gave up a bounded wait; read and cleared by
-// winattn_last_device_status.  One word per device (module-scope variable).
-__device__ unsigned int g_status_word = 0;
-
-constexpr float kLog2e = 1.4426950408889634f;
-
 template <int D, int R>
 struct TcLayout {
     static constexpr uint32_t QC = 0;                       // query content  [128][D]  bf16

@@ -10,6 +10,7 @@
 
 #include "../../include/winattn.h"
 #include "fwd_simt.cuh"
+#include "fwd_small.cuh"
 #include "fwd_tc.cuh"
 #include "geometry.cuh"
 
@@ -81,6 +82,54 @@ int smem_bytes_for(const Geometry &g, int dtype)
     return -1;
 }
 
+constexpr int kAssumedSMs = 148;          // B200; used only by winattn_launch_info
+constexpr uint32_t kMaxSmem = 227 * 1024;
+constexpr uint32_t kMaxSmallTable = 32 * 1024;
+
+enum KernelKind { kGeneric = 0, kSmall = 1, kSimt = 3 };
+
+uint32_t small_smem(const Geometry &g)
+{
+    switch (g.d * 100 + g.rank) {
+    case 3200: return SmallLayout<32, 0>::bytes(g.heads, g.M);
+    case 3216: return SmallLayout<32, 16>::bytes(g.heads, g.M);
+    case 3232: return SmallLayout<32, 32>::bytes(g.heads, g.M);
+    case 6400: return SmallLayout<64, 0>::bytes(g.heads, g.M);
+    case 6416: return SmallLayout<64, 16>::bytes(g.heads, g.M);
+    case 6432: return SmallLayout<64, 32>::bytes(g.heads, g.M);
+    }
+    return ~0u;
+}
+
+// Which kernel serves a problem: windows of <= 128 tokens go to the
+// persistent small-window kernel when its RoPE table and ring fit in shared
+// memory; fp32 goes to the SIMT kernel; everything else to the generic one.
+KernelKind choose_kernel(const Geometry &g, int dtype)
+{
+    if (dtype == WINATTN_FP32)
+        return kSimt;
+    if (g.N <= kTileRows && (uint64_t)g.heads * g.M * (g.d / 4) * 8 <= kMaxSmallTable && small_smem(g) <= kMaxSmem)
+        return kSmall;
+    return kGeneric;
+}
+
+int sm_count()
+{
+    static std::mutex mu;
+    static int cached[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return kAssumedSMs;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = kAssumedSMs;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
 // Compute capability check, cached per device.
 int check_device()
 {
@@ -122,6 +171,25 @@ int launch_tc(const void *q, const void *k, const void *v, const float *theta, c
 }
 
 template <int D, int R>
+int launch_small(const void *q, const void *k, const void *v, const float *theta, const void *bias, void *out,
+                 const Geometry &g, cudaStream_t stream)
+{
+    using T = __nv_bfloat16;
+    auto kernel = winattn_fwd_small_kernel<D, R>;
+    // The kernel takes all 512 TMEM columns: ask for enough shared memory that
+    // no second CTA can be resident on the same SM.
+    const int need = (int)SmallLayout<D, R>::bytes(g.heads, g.M);
+    const int smem = need > 116 * 1024 ? need : 116 * 1024;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return WINATTN_ERR_CUDA;
+    const int64_t grid = g.items < sm_count() ? g.items : sm_count();
+    kernel<<<(unsigned)grid, kSmallThreads, smem, stream>>>(
+        static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), theta,
+        static_cast<const T *>(bias), static_cast<T *>(out), g, 1.0f / std::sqrt((float)g.d));
+    return cudaGetLastError() == cudaSuccess ? WINATTN_OK : WINATTN_ERR_CUDA;
+}
+
+template <int D, int R>
 int launch_simt(const void *q, const void *k, const void *v, const float *theta, const void *bias, void *out,
                 const Geometry &g, cudaStream_t stream)
 {
@@ -133,7 +201,17 @@ int launch_simt(const void *q, const void *k, const void *v, const float *theta,
 int dispatch(const void *q, const void *k, const void *v, const float *theta, const void *bias, void *out,
              const Geometry &g, int dtype, cudaStream_t s)
 {
-    if (dtype == WINATTN_BF16) {
+    const KernelKind kind = choose_kernel(g, dtype);
+    if (kind == kSmall) {
+        switch (g.d * 100 + g.rank) {
+        case 3200: return launch_small<32, 0>(q, k, v, theta, bias, out, g, s);
+        case 3216: return launch_small<32, 16>(q, k, v, theta, bias, out, g, s);
+        case 3232: return launch_small<32, 32>(q, k, v, theta, bias, out, g, s);
+        case 6400: return launch_small<64, 0>(q, k, v, theta, bias, out, g, s);
+        case 6416: return launch_small<64, 16>(q, k, v, theta, bias, out, g, s);
+        case 6432: return launch_small<64, 32>(q, k, v, theta, bias, out, g, s);
+        }
+    } else if (kind == kGeneric) {
         switch (g.d * 100 + g.rank) {
         case 3200: return launch_tc<32, 0>(q, k, v, theta, bias, out, g, s);
         case 3216: return launch_tc<32, 16>(q, k, v, theta, bias, out, g, s);
@@ -279,17 +357,26 @@ int winattn_last_device_status(void *stream)
 }
 
 int winattn_launch_info(int B, int H_img, int W_img, int M, int shift, int heads, int d, int rank, int dtype,
-                        int64_t *work_items, int *grid, int *threads, int *smem_bytes, int *windows_per_tile)
+                        int64_t *work_items, int *grid, int *threads, int *smem_bytes, int *windows_per_tile,
+                        int *kernel)
 {
     const int rc = check_sizes(B, H_img, W_img, M, shift, heads, d, rank, dtype);
     if (rc != WINATTN_OK)
         return rc;
     const Geometry g = Geometry::make(B, H_img, W_img, M, shift, heads, d, rank);
+    const KernelKind kind = choose_kernel(g, dtype);
     if (work_items) *work_items = g.items;
-    if (grid) *grid = (int)g.items;
-    if (threads) *threads = kThreads;
-    if (smem_bytes) *smem_bytes = smem_bytes_for(g, dtype);
     if (windows_per_tile) *windows_per_tile = g.U;
+    if (kernel) *kernel = (int)kind;
+    if (kind == kSmall) {
+        if (grid) *grid = (int)(g.items < kAssumedSMs ? g.items : kAssumedSMs);
+        if (threads) *threads = kSmallThreads;
+        if (smem_bytes) *smem_bytes = (int)small_smem(g);
+    } else {
+        if (grid) *grid = (int)g.items;
+        if (threads) *threads = kThreads;
+        if (smem_bytes) *smem_bytes = smem_bytes_for(g, dtype);
+    }
     return WINATTN_OK;
 }
 
