@@ -120,16 +120,6 @@ __device__ __forceinline__ void rotate_row_inplace(uint8_t *tile, int row, const
     }
 }
 
-__device__ __forceinline__ bool window_wrapped(const Geometry &g, int64_t w)
-{
-    if (g.shift == 0)
-        return false;
-    const int64_t per_img = (int64_t)g.nWy * g.nWx;
-    const int rem = (int)(w % per_img);
-    const int wy = rem / g.nWx, wx = rem - wy * g.nWx;
-    return wy == g.nWy - 1 || wx == g.nWx - 1;
-}
-
 template <int D, int R>
 __global__ void __launch_bounds__(kSmallThreads, 1)
     winattn_fwd_small_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
@@ -150,9 +140,9 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
     volatile uint32_t *abort_flag = tslot + 1;
 
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-    const int64_t n_items = (int64_t)g.heads * g.packs;
-    const int64_t first = blockIdx.x, stride = gridDim.x;
-    const int count = first < n_items ? (int)((n_items - 1 - first) / stride + 1) : 0;
+    const int n_items = (int)g.items;
+    const int first = blockIdx.x, stride = gridDim.x;
+    const int count = first < n_items ? (n_items - 1 - first) / stride + 1 : 0;
     const int table_per_head = g.M * (D / 4);
 
     if (warp == 12) {
@@ -196,9 +186,8 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
             const int s = kk % NS;
             if (kk >= NS && !wait_or_abort(&empty[s], ((kk / NS) - 1) & 1, abort_flag))
                 return false;
-            const int64_t item = first + (int64_t)kk * stride;
-            const int64_t pack = item / g.heads;
-            const int h = (int)(item - pack * g.heads);
+            const Item it = decode_item_head_minor(g, first + kk * stride);
+            const int pack = it.pack, h = it.h;
             uint8_t *st = base + s * L::STAGE;
             const uint32_t sst = sbase + s * L::STAGE;
 #pragma unroll
@@ -258,9 +247,8 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
             if (named_bar_any(1, 128, failed))
                 break;
             const int s = kc % NS;
-            const int64_t item = first + (int64_t)kc * stride;
-            const int64_t pack = item / g.heads;
-            const int h = (int)(item - pack * g.heads);
+            const Item it = decode_item_head_minor(g, first + kc * stride);
+            const int pack = it.pack, h = it.h;
             const RowRef rr = tile_row(g, pack, 0, lt);
             if (rr.valid) {
                 const TokenRef tk = token_ref(g, rr.w, rr.p, h);
@@ -346,9 +334,8 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
             if (!warp_wait(&s_full[w], j & 1, abort_flag))
                 break;
             tc_fence_after_sync();
-            const int64_t item = first + (int64_t)kc * stride;
-            const int64_t pack = item / g.heads;
-            const int h = (int)(item - pack * g.heads);
+            const Item it = decode_item_head_minor(g, first + kc * stride);
+            const int pack = it.pack, h = it.h;
             const RowRef rr = tile_row(g, pack, 0, row);
             int qcode = 0xFFFF;
             TokenRef tk{};

@@ -45,7 +45,7 @@ int check_sizes(int B, int H, int W, int M, int shift, int heads, int d, int ran
         return WINATTN_ERR_RANK;
     const Geometry g = Geometry::make(B, H, W, M, shift, heads, d, rank);
     const double elems = (double)B * H * W * heads * d;
-    if (elems > 9.0e18 || g.items > 0x7FFFFFFFLL)
+    if (elems > 9.0e18 || g.items > 0x7FFFFFFFLL || g.wph > 0x7FFFFFFFLL)
         return WINATTN_ERR_SIZE;
     return WINATTN_OK;
 }
