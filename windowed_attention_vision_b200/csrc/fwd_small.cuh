@@ -229,10 +229,12 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
             return true;
         };
 
+        // Exactly PF - 1 groups go out before the loop (empty ones when the CTA
+        // has fewer items), and one more per iteration, so that waiting until
+        // at most PF - 1 groups are pending always covers item kc.
         bool failed = false;
-        const int pre = PF - 1 < count ? PF - 1 : count;
-        for (int kk = 0; kk < pre; ++kk) {
-            if (!failed)
+        for (int kk = 0; kk < PF - 1; ++kk) {
+            if (kk < count && !failed)
                 failed = !issue(kk);
             cp_async_commit();
         }
