@@ -9,21 +9,28 @@
 // are ordered pack-major, head-minor so that the heads of a token - which
 // share its DRAM lines - are read by neighbouring CTAs at the same time.
 //
-// Roles (416 threads):
-//   warps 8-11  loader: cp.async gathers of Q, K, V (and the rank-r factors)
-//               straight into the swizzled operand tiles of a ring of stages,
-//               several items ahead; then, per item, window-local RoPE on Q and
-//               K in place (fp32 registers), Q scaled by d^-1/2;
-//   warp 12     MMA issuer (one thread): S = Q~ K~^T into TMEM, then
-//               O = P V with P read from TMEM (the tensor core never waits for
-//               P in shared memory);
-//   warps 0-7   two softmax warpgroups, alternating items: each thread owns one
-//               row (TMEM lane), computes max / exp / sum over its window's
-//               keys only, writes P (bf16 pairs) over the consumed S columns,
-//               and after O lands normalises and stores it to the token's
-//               original (un-shifted) position.
-// Every wait is a bounded mbarrier wait; a timeout sets a CTA-wide abort flag
-// and the device status word, and every role drains and returns.
+// Roles (576 threads):
+//   warp 16     loader.  TMA mode (windows that split into whole swizzle
+//               atoms): tensor-map box loads of each window's Q, K, V head
+//               slices straight into the swizzled operand tiles - one box
+//               for an interior window, two for a window on the wrap seam's
+//               row or column, four for the corner window.  Otherwise:
+//               cp.async gathers of 16-byte chunks (rank-r factors too).
+//   warp 17     MMA issuer (one thread): polls the ring and issues, as soon
+//               as each is ready, S = Q~ K~^T into TMEM and O = P V with P
+//               read from TMEM;
+//   warps 0-15  four compute warpgroups, item k going to group k % 4: each
+//               thread owns one tile row (TMEM lane): it resolves its row's
+//               token (window-local coordinates, original position, wrap
+//               label), applies window-local RoPE to its Q and K rows in
+//               place (fp32, Q scaled by d^-1/2), runs max / exp / sum over
+//               its window's keys, writes P (bf16 pairs) over the consumed S
+//               columns, and once O lands normalises it and stores it to the
+//               token's original (un-shifted) position.
+// TMEM: 128 columns per group - S (fp32, 128 cols), then P over S[0, 64) and
+// O over S[64, 64 + d).
+// Every wait is bounded; a timeout sets a CTA-wide abort flag and the device
+// status word, and every role drains and returns.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -33,7 +40,15 @@
 
 namespace winattn {
 
-constexpr int kSmallThreads = 416;
+// Compute warpgroups per CTA: four for d = 32; three for d = 64, whose rows
+// need more registers (the CTA's register file is shared by all roles).
+template <int D>
+struct SmallRoles {
+    static constexpr int kGroups = D <= 32 ? 4 : 3;
+    static constexpr int kThreads = (kGroups * 4 + 2) * 32;
+    static constexpr int kLoaderWarp = kGroups * 4;
+    static constexpr int kMmaWarp = kGroups * 4 + 1;
+};
 
 template <int D, int R>
 struct SmallLayout {
@@ -42,18 +57,26 @@ struct SmallLayout {
     static constexpr uint32_t KC = QB + 256 * R;            // key content    [128][D]
     static constexpr uint32_t KB = KC + 256 * D;            // key factors    [128][R]
     static constexpr uint32_t VO = KB + 256 * R;            // values         [128][D]
-    static constexpr uint32_t CODES = VO + 256 * D;         // key mask codes u16[128]
-    static constexpr uint32_t STAGE = (CODES + 256 + 1023) & ~1023u;
-    static constexpr int NS = (200 * 1024 / STAGE) < 5 ? (200 * 1024 / STAGE) : 5;  // ring depth
-    static constexpr int PF = NS - 1;                       // items in flight ahead of conversion
+    static constexpr uint32_t CODES = VO + 256 * D;         // mask code per tile row, u16[128]
+    static constexpr uint32_t OFFS = CODES + 256;           // loader's row offsets (cp.async mode), i64[128]
+    static constexpr uint32_t STAGE = (OFFS + 128 * 8 + 1023) & ~1023u;
+    static constexpr int NS_FIT = (200 * 1024) / STAGE;
+    static constexpr int NS = NS_FIT < 6 ? NS_FIT : 6;      // ring depth
+    static constexpr int PF = NS - 2 > 2 ? NS - 2 : 2;      // cp.async mode: items issued ahead
     static constexpr uint32_t TABLE = NS * STAGE;           // RoPE (cos, sin) [heads][M][D/4]
-    static constexpr int kBars = 2 * NS + 9;
+    static constexpr int kBars = 3 * NS + 4 * SmallRoles<D>::kGroups + 1;
     static __host__ __device__ uint32_t table_bytes(int heads, int M)
     {
         return (uint32_t)(heads * M * (D / 4) * 8 + 15) & ~15u;
     }
     static __host__ __device__ uint32_t bars(int heads, int M) { return TABLE + table_bytes(heads, M); }
     static __host__ __device__ uint32_t bytes(int heads, int M) { return bars(heads, M) + kBars * 8 + 16 + 1024; }
+};
+
+// Tensor maps of one operand for the TMA mode: box shapes (width x height in
+// tokens) M x M, M/2 x M, M x M/2 and M/2 x M/2.
+struct WindowMaps {
+    CUtensorMap full, xhalf, yhalf, quarter;
 };
 
 // Bounded wait that also gives up as soon as another role has aborted.
@@ -120,22 +143,84 @@ __device__ __forceinline__ void rotate_row_inplace(uint8_t *tile, int row, const
     }
 }
 
-template <int D, int R>
-__global__ void __launch_bounds__(kSmallThreads, 1)
+// Window kind in the TMA mode: bit 0 = the window straddles the column wrap
+// seam (last window column of a shifted map), bit 1 = the row seam.
+__device__ __forceinline__ int window_kind(const Geometry &g, int wy, int wx)
+{
+    if (g.shift == 0)
+        return 0;
+    return (wx == g.nWx - 1 ? 1 : 0) | (wy == g.nWy - 1 ? 2 : 0);
+}
+
+// Window-local (i, j) of row rp of a window of the given kind, in the order
+// the TMA boxes land: kind 0 and 2 row-major (two M x M/2 boxes stacked keep
+// row-major order); kind 1 two M/2-wide boxes, each row-major; kind 3 four
+// M/2 x M/2 quadrants, each row-major.
+__device__ __forceinline__ void tma_row_coords(const Geometry &g, int kind, int rp, int &i, int &j)
+{
+    const int M = g.M, hm = M >> 1;
+    if (kind == 1) {
+        const int half = M * hm;
+        const int bx = rp >= half ? 1 : 0;
+        const int r = rp - bx * half;
+        i = r / hm;
+        j = bx * hm + (r - i * hm);
+    } else if (kind == 3) {
+        const int q2 = hm * hm;
+        const int qd = rp / q2, r = rp - qd * q2;
+        const int iy = r / hm;
+        i = (qd >> 1) * hm + iy;
+        j = (qd & 1) * hm + (r - iy * hm);
+    } else {
+        i = (int)g.div_M.div((uint32_t)rp);
+        j = rp - i * M;
+    }
+}
+
+// TMA loads apply when every box is a whole number of 8-row swizzle atoms:
+// unshifted windows with M*M % 8 == 0, or shift M/2 with (M/2)^2 % 8 == 0;
+// packed tiles only (at most 64 tokens per window), no rank-r factors.
+__host__ __device__ inline bool small_tma_ok(const Geometry &g)
+{
+    if (g.rank != 0 || g.U < 2)
+        return false;
+    if (g.shift == 0)
+        return (g.N % 8) == 0;
+    return 2 * g.shift == g.M && ((g.shift * g.shift) % 8) == 0;
+}
+
+// Tensor map of one operand for a window kind (see window_kind).
+__device__ __forceinline__ const CUtensorMap *pick_map(const WindowMaps &m, int kind)
+{
+    switch (kind) {
+    case 1: return &m.xhalf;
+    case 2: return &m.yhalf;
+    case 3: return &m.quarter;
+    default: return &m.full;
+    }
+}
+
+template <int D, int R, bool TMA>
+__global__ void __launch_bounds__(SmallRoles<D>::kThreads, 1)
     winattn_fwd_small_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                              const __nv_bfloat16 *__restrict__ v, const float *__restrict__ theta,
                              const __nv_bfloat16 *__restrict__ bias, __nv_bfloat16 *__restrict__ out,
-                             const Geometry g, const float scale)
+                             const Geometry g, const float scale, const __grid_constant__ WindowMaps tm_q,
+                             const __grid_constant__ WindowMaps tm_k, const __grid_constant__ WindowMaps tm_v)
 {
     using L = SmallLayout<D, R>;
-    constexpr int NS = L::NS, PF = L::PF;
+    constexpr int NS = L::NS, PF = L::PF, NW = SmallRoles<D>::kGroups;
+    constexpr int kLoaderWarp = SmallRoles<D>::kLoaderWarp, kMmaWarp = SmallRoles<D>::kMmaWarp;
+    static_assert(NS >= 3, "ring too shallow");
+    static_assert(!TMA || R == 0, "TMA loads carry no rank-r factors");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(base);
     float2 *table = reinterpret_cast<float2 *>(base + L::TABLE);
     uint64_t *bars = reinterpret_cast<uint64_t *>(base + L::bars(g.heads, g.M));
-    uint64_t *full = bars, *empty = bars + NS, *s_full = bars + 2 * NS, *p_full = s_full + 2, *o_full = p_full + 2,
-             *t_free = o_full + 2, *fin = t_free + 2;
+    uint64_t *full = bars, *conv = bars + NS, *empty = bars + 2 * NS;
+    uint64_t *s_full = bars + 3 * NS, *p_full = s_full + NW, *o_full = p_full + NW, *t_free = o_full + NW;
+    uint64_t *fin = t_free + NW;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + L::kBars);
     volatile uint32_t *abort_flag = tslot + 1;
 
@@ -145,16 +230,17 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
     const int count = first < n_items ? (n_items - 1 - first) / stride + 1 : 0;
     const int table_per_head = g.M * (D / 4);
 
-    if (warp == 12) {
+    if (warp == kMmaWarp) {
         tmem_alloc(tslot, 512);
         tmem_relinquish();
     }
     if (t == 0) {
         for (int s = 0; s < NS; ++s) {
-            mbar_init(&full[s], 128);
+            mbar_init(&full[s], TMA ? 1 : 32);
+            mbar_init(&conv[s], 128);
             mbar_init(&empty[s], 1);
         }
-        for (int w = 0; w < 2; ++w) {
+        for (int w = 0; w < NW; ++w) {
             mbar_init(&s_full[w], 1);
             mbar_init(&p_full[w], 128);
             mbar_init(&o_full[w], 1);
@@ -178,25 +264,75 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
     tc_fence_after_sync();
     const uint32_t tmem = *tslot;
 
-    if (warp >= 8 && warp < 12) {
-        // ------------------------------------------------------------ loader
-        const int lt = t - 256;
+    if (warp == kLoaderWarp && TMA) {
+        // ------------------------------------------------------------ loader (TMA)
+        if (lane == 0) {
+            for (int kind = 0; kind < 4; ++kind) {
+                tma_prefetch_map(pick_map(tm_q, kind));
+                tma_prefetch_map(pick_map(tm_k, kind));
+                tma_prefetch_map(pick_map(tm_v, kind));
+            }
+            const int M = g.M, hm = M >> 1;
+            for (int kk = 0; kk < count; ++kk) {
+                const int s = kk % NS;
+                if (kk >= NS && !wait_or_abort(&empty[s], ((kk / NS) - 1) & 1, abort_flag))
+                    break;
+                const Item it = decode_item_head_minor(g, first + kk * stride);
+                const uint32_t sst = sbase + s * L::STAGE;
+                const int64_t left = g.wph - (int64_t)it.pack * g.U;
+                const int nvalid = left < g.U ? (int)left : g.U;
+                mbar_arrive_expect_tx(&full[s], (uint32_t)(3 * nvalid * g.N * 2 * D));
+                const int c0 = it.h * D;
+                for (int slot = 0; slot < nvalid; ++slot) {
+                    const int w = it.pack * g.U + slot;
+                    const int b = (int)g.div_img.div((uint32_t)w);
+                    const int rem = w - b * g.nWy * g.nWx;
+                    const int wy = (int)g.div_nWx.div((uint32_t)rem);
+                    const int wx = rem - wy * g.nWx;
+                    const int kind = window_kind(g, wy, wx);
+                    const int nbox = kind == 3 ? 4 : (kind ? 2 : 1);
+                    const int box_rows = g.N / nbox;
+                    for (int bi = 0; bi < nbox; ++bi) {
+                        // rolled-local origin of the box, then its original position
+                        const int iy0 = (kind & 2) ? ((kind == 3 ? bi >> 1 : bi) * hm) : 0;
+                        const int jx0 = (kind & 1) ? ((kind == 3 ? bi & 1 : bi) * hm) : 0;
+                        int y0 = wy * M + iy0 + g.shift;
+                        if (y0 >= g.H) y0 -= g.H;
+                        int x0 = wx * M + jx0 + g.shift;
+                        if (x0 >= g.W) x0 -= g.W;
+                        const uint32_t roff = (uint32_t)((slot * g.N + bi * box_rows) * 2 * D);
+                        tma_load_4d(sst + L::QC + roff, pick_map(tm_q, kind), c0, x0, y0, b, &full[s]);
+                        tma_load_4d(sst + L::KC + roff, pick_map(tm_k, kind), c0, x0, y0, b, &full[s]);
+                        tma_load_4d(sst + L::VO + roff, pick_map(tm_v, kind), c0, x0, y0, b, &full[s]);
+                    }
+                }
+            }
+        }
+    } else if (warp == kLoaderWarp) {
+        // ------------------------------------------------------------ loader (cp.async)
         constexpr int CD = D / 8, CR = R / 8;
         auto issue = [&](int kk) -> bool {
             const int s = kk % NS;
-            if (kk >= NS && !wait_or_abort(&empty[s], ((kk / NS) - 1) & 1, abort_flag))
+            if (kk >= NS && !warp_wait(&empty[s], ((kk / NS) - 1) & 1, abort_flag))
                 return false;
             const Item it = decode_item_head_minor(g, first + kk * stride);
-            const int pack = it.pack, h = it.h;
             uint8_t *st = base + s * L::STAGE;
             const uint32_t sst = sbase + s * L::STAGE;
+            int64_t *offs = reinterpret_cast<int64_t *>(st + L::OFFS);
 #pragma unroll
-            for (int i = 0; i < CD; ++i) {
-                const int idx = i * 128 + lt, row = idx / CD, ch = idx % CD;
-                const RowRef rr = tile_row(g, pack, 0, row);
+            for (int r4 = 0; r4 < 4; ++r4) {
+                const int row = r4 * 32 + lane;
+                const RowRef rr = tile_row(g, it.pack, 0, row);
+                offs[row] = rr.valid ? token_ref(g, rr.w, rr.p, it.h).offset : int64_t(-1);
+            }
+            __syncwarp();
+#pragma unroll 4
+            for (int idx = lane; idx < 128 * CD; idx += 32) {
+                const int row = idx / CD, ch = idx % CD;
+                const int64_t ro = offs[row];
                 const uint32_t off = swz_offset(row, ch, 2 * D);
-                if (rr.valid) {
-                    const int64_t src = token_ref(g, rr.w, rr.p, h).offset + ch * 8;
+                if (ro >= 0) {
+                    const int64_t src = ro + ch * 8;
                     cp_async16(sst + L::QC + off, q + src);
                     cp_async16(sst + L::KC + off, k + src);
                     cp_async16(sst + L::VO + off, v + src);
@@ -207,118 +343,114 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
                 }
             }
             if constexpr (R > 0) {
-#pragma unroll
-                for (int i = 0; i < CR; ++i) {
-                    const int idx = i * 128 + lt, row = idx / CR, ch = idx % CR;
-                    const RowRef rr = tile_row(g, pack, 0, row);
+                const __nv_bfloat16 *u_h = bias + (int64_t)it.h * 2 * g.N * R;
+                const __nv_bfloat16 *w_h = u_h + (int64_t)g.N * R;
+#pragma unroll 4
+                for (int idx = lane; idx < 128 * CR; idx += 32) {
+                    const int row = idx / CR, ch = idx % CR;
+                    const RowRef rr = tile_row(g, it.pack, 0, row);
                     const uint32_t off = swz_offset(row, ch, 2 * R);
                     if (rr.valid) {
-                        cp_async16(sst + L::QB + off, bias + (((int64_t)h * 2 + 0) * g.N + rr.p) * R + ch * 8);
-                        cp_async16(sst + L::KB + off, bias + (((int64_t)h * 2 + 1) * g.N + rr.p) * R + ch * 8);
+                        cp_async16(sst + L::QB + off, u_h + rr.p * R + ch * 8);
+                        cp_async16(sst + L::KB + off, w_h + rr.p * R + ch * 8);
                     } else {
                         *reinterpret_cast<uint4 *>(st + L::QB + off) = make_uint4(0, 0, 0, 0);
                         *reinterpret_cast<uint4 *>(st + L::KB + off) = make_uint4(0, 0, 0, 0);
                     }
                 }
             }
-            const RowRef rr = tile_row(g, pack, 0, lt);
-            uint16_t code = 0xFFFE;
-            if (rr.valid)
-                code = (uint16_t)((rr.slot << 2) | token_ref(g, rr.w, rr.p, h).label);
-            reinterpret_cast<uint16_t *>(st + L::CODES)[lt] = code;
             return true;
         };
 
-        // Exactly PF - 1 groups go out before the loop (empty ones when the CTA
-        // has fewer items), and one more per iteration, so that waiting until
-        // at most PF - 1 groups are pending always covers item kc.
+        // Groups go out one per item, PF - 1 ahead (empty groups past the
+        // end keep the count uniform), so waiting until at most PF - 2 are
+        // pending covers the oldest item.
         bool failed = false;
         for (int kk = 0; kk < PF - 1; ++kk) {
             if (kk < count && !failed)
                 failed = !issue(kk);
             cp_async_commit();
         }
-        for (int kc = 0; kc < count; ++kc) {
+        for (int kc = 0; kc < count && !failed; ++kc) {
+            cp_async_wait<PF - 2>();
+            fence_proxy_async_smem();
+            mbar_arrive(&full[kc % NS]);
             const int kk = kc + PF - 1;
-            if (kk < count && !failed)
+            if (kk < count)
                 failed = !issue(kk);
             cp_async_commit();
-            cp_async_wait<PF - 1>();
-            // Every loader thread's copies of item kc have landed (and all
-            // loader threads agree on whether to stop).
-            if (named_bar_any(1, 128, failed))
-                break;
-            const int s = kc % NS;
-            const Item it = decode_item_head_minor(g, first + kc * stride);
-            const int pack = it.pack, h = it.h;
-            const RowRef rr = tile_row(g, pack, 0, lt);
-            if (rr.valid) {
-                const TokenRef tk = token_ref(g, rr.w, rr.p, h);
-                const float2 *tb = theta ? table + h * table_per_head : nullptr;
-                uint8_t *st = base + s * L::STAGE;
-                rotate_row_inplace<D>(st + L::QC, lt, tb, tk.i, tk.j, scale);
-                if (theta)
-                    rotate_row_inplace<D>(st + L::KC, lt, tb, tk.i, tk.j, 1.f);
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(&full[s]);
         }
         cp_async_wait_all();
-    } else if (warp == 12) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false);
             constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
-            auto issue_s = [&](int kc) -> bool {
-                const int s = kc % NS, w = kc & 1;
-                if (!wait_or_abort(&full[s], (kc / NS) & 1, abort_flag))
-                    return false;
-                if (kc >= 2 && !wait_or_abort(&t_free[w], ((kc - 2) >> 1) & 1, abort_flag))
-                    return false;
-                tc_fence_after_sync();
-                const uint32_t sst = sbase + s * L::STAGE;
-                const uint32_t d = tmem + w * 256;
+            int ns = 0, npv = 0;  // next item whose S / PV is to be issued
+            uint64_t t_last = globaltimer_ns();
+            while (npv < count) {
+                bool progress = false;
+                if (ns < count && ns - npv < NW) {
+                    const int s = ns % NS, w = ns % NW;
+                    if (mbar_test_wait(&conv[s], (ns / NS) & 1) &&
+                        (ns < NW || mbar_test_wait(&t_free[w], ((ns - NW) / NW) & 1))) {
+                        tc_fence_after_sync();
+                        const uint32_t sst = sbase + s * L::STAGE;
+                        const uint32_t d = tmem + w * 128;
 #pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks)
-                    umma_bf16_ss(d, smem_desc(sst + L::QC + ks * 32, 16, 16 * D, swizzle_code(2 * D)),
-                                 smem_desc(sst + L::KC + ks * 32, 16, 16 * D, swizzle_code(2 * D)), kIdescS, ks > 0);
+                        for (int ks = 0; ks < D / 16; ++ks)
+                            umma_bf16_ss(d, smem_desc(sst + L::QC + ks * 32, 16, 16 * D, swizzle_code(2 * D)),
+                                         smem_desc(sst + L::KC + ks * 32, 16, 16 * D, swizzle_code(2 * D)), kIdescS,
+                                         ks > 0);
 #pragma unroll
-                for (int ks = 0; ks < R / 16; ++ks)
-                    umma_bf16_ss(d, smem_desc(sst + L::QB + ks * 32, 16, 16 * R, swizzle_code(2 * R)),
-                                 smem_desc(sst + L::KB + ks * 32, 16, 16 * R, swizzle_code(2 * R)), kIdescS, 1);
-                umma_commit(&s_full[w]);
-                return true;
-            };
-            bool ok = count > 0 ? issue_s(0) : true;
-            for (int kc = 0; kc < count && ok; ++kc) {
-                if (kc + 1 < count && !(ok = issue_s(kc + 1)))
+                        for (int ks = 0; ks < R / 16; ++ks)
+                            umma_bf16_ss(d, smem_desc(sst + L::QB + ks * 32, 16, 16 * R, swizzle_code(2 * R)),
+                                         smem_desc(sst + L::KB + ks * 32, 16, 16 * R, swizzle_code(2 * R)), kIdescS,
+                                         1);
+                        umma_commit(&s_full[w]);
+                        ++ns;
+                        progress = true;
+                    }
+                }
+                if (npv < ns) {
+                    const int s = npv % NS, w = npv % NW;
+                    if (mbar_test_wait(&p_full[w], (npv / NW) & 1)) {
+                        tc_fence_after_sync();
+                        const uint32_t sst = sbase + s * L::STAGE;
+                        const uint32_t pa = tmem + w * 128;        // P: 64 columns of bf16 pairs over S
+                        const uint32_t od = tmem + w * 128 + 64;   // O: d columns over S[64, 64 + d)
+#pragma unroll
+                        for (int ks = 0; ks < 8; ++ks)
+                            umma_bf16_ts(od, pa + ks * 8,
+                                         smem_desc(sst + L::VO + ks * 32 * D, 8192, 16 * D, swizzle_code(2 * D)),
+                                         kIdescPV, ks > 0);
+                        umma_commit(&o_full[w]);
+                        umma_commit(&empty[s]);
+                        ++npv;
+                        progress = true;
+                    }
+                }
+                if (progress) {
+                    t_last = globaltimer_ns();
+                } else if (*abort_flag) {
                     break;
-                const int s = kc % NS, w = kc & 1;
-                if (!(ok = wait_or_abort(&p_full[w], (kc >> 1) & 1, abort_flag)))
+                } else if (globaltimer_ns() - t_last > kWaitLimitNs) {
+                    *abort_flag = 1u;
+                    atomicOr(&g_status_word, 1u);
                     break;
-                tc_fence_after_sync();
-                const uint32_t sst = sbase + s * L::STAGE;
-                const uint32_t pa = tmem + w * 256;        // P: 64 columns of bf16 pairs (over S)
-                const uint32_t od = tmem + w * 256 + 128;  // O: D columns
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    umma_bf16_ts(od, pa + ks * 8,
-                                 smem_desc(sst + L::VO + ks * 32 * D, 8192, 16 * D, swizzle_code(2 * D)), kIdescPV,
-                                 ks > 0);
-                umma_commit(&o_full[w]);
-                umma_commit(&empty[s]);
+                } else {
+                    __nanosleep(32);
+                }
             }
             // every UMMA issued above has completed before TMEM is released
             umma_commit(fin);
             mbar_wait(fin, 0);
         }
-    } else if (warp < 8) {
-        // ------------------------------------------------------------ softmax + epilogue
+    } else {
+        // ------------------------------------------------------------ compute groups
         const int w = warp >> 2;
         const int row = t - 128 * w;
-        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t s_addr = tmem + w * 256 + lane_base;
-        const uint32_t o_addr = s_addr + 128;
+        const uint32_t region = tmem + w * 128 + ((uint32_t)((warp & 3) * 32) << 16);
         const int r0 = (warp & 3) * 32;
         int c_lo = 0, c_hi = g.N < 128 ? g.N : 128;
         if (g.U > 1) {
@@ -328,68 +460,134 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
         }
         const int ch_lo = c_lo >> 5, ch_hi = (c_hi + 31) >> 5;
         const bool aligned = (g.N & 31) == 0;
+        // the fast path reads exactly two 32-column chunks: one 64-token window
+        const bool two_chunk = aligned && ch_hi - ch_lo == 2;
 
-        for (int kc = w; kc < count; kc += 2) {
-            const int s = kc % NS, j = kc >> 1;
+        for (int kc = w; kc < count; kc += NW) {
+            const int s = kc % NS, j = kc / NW;
             if (!warp_wait(&full[s], (kc / NS) & 1, abort_flag))
                 break;
+            uint8_t *st = base + s * L::STAGE;
+            const Item it = decode_item_head_minor(g, first + kc * stride);
+
+            // ---- resolve this row's token
+            const RowRef rr = tile_row(g, it.pack, 0, row);
+            bool wrapped = false;
+            TokenRef tk{};
+            int code = 0xFFFE;
+            if (rr.valid) {
+                int pi = 0, pj = 0, p = rr.p;
+                if (TMA) {
+                    const int b = (int)g.div_img.div((uint32_t)rr.w);
+                    const int rem = rr.w - b * g.nWy * g.nWx;
+                    const int wy = (int)g.div_nWx.div((uint32_t)rem);
+                    const int kind = window_kind(g, wy, rem - wy * g.nWx);
+                    tma_row_coords(g, kind, rr.p, pi, pj);
+                    p = pi * g.M + pj;
+                    wrapped = kind != 0;
+                } else {
+                    wrapped = window_wrapped(g, rr.w);
+                }
+                tk = token_ref(g, rr.w, p, it.h);
+                code = (rr.slot << 2) | tk.label;
+            }
+            uint16_t *codes = reinterpret_cast<uint16_t *>(st + L::CODES);
+            codes[row] = (uint16_t)code;
+
+            // ---- window-local RoPE on this row's query and key, in place; a
+            // row without a token (empty pack slot) is zeroed, so that its
+            // value row contributes exact zeros to P V
+            if (rr.valid) {
+                const float2 *tb = theta ? table + it.h * table_per_head : nullptr;
+                rotate_row_inplace<D>(st + L::QC, row, tb, tk.i, tk.j, scale);
+                if (theta)
+                    rotate_row_inplace<D>(st + L::KC, row, tb, tk.i, tk.j, 1.f);
+            } else {
+#pragma unroll
+                for (int c = 0; c < D / 8; ++c) {
+                    const uint32_t off = swz_offset(row, c, 2 * D);
+                    *reinterpret_cast<uint4 *>(st + L::QC + off) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4 *>(st + L::KC + off) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4 *>(st + L::VO + off) = make_uint4(0, 0, 0, 0);
+                }
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(2 + w, 128);  // this group's codes are all written
+            mbar_arrive(&conv[s]);
+
             if (!warp_wait(&s_full[w], j & 1, abort_flag))
                 break;
             tc_fence_after_sync();
-            const Item it = decode_item_head_minor(g, first + kc * stride);
-            const int pack = it.pack, h = it.h;
-            const RowRef rr = tile_row(g, pack, 0, row);
-            int qcode = 0xFFFF;
-            TokenRef tk{};
-            if (rr.valid) {
-                tk = token_ref(g, rr.w, rr.p, h);
-                qcode = (rr.slot << 2) | tk.label;
-            }
-            const uint16_t *codes = reinterpret_cast<const uint16_t *>(base + s * L::STAGE + L::CODES);
+            const int qcode = rr.valid ? code : 0xFFFF;
             // Keys need no per-element test when the row's window fills whole
             // 32-column chunks and is not wrapped.
-            const bool fast = __all_sync(0xffffffffu, aligned && rr.valid && !window_wrapped(g, rr.w));
-
-            float mx = -INFINITY;
-            for (int ch = ch_lo; ch < ch_hi; ++ch) {
-                float x[32];
-                tmem_ld32(s_addr + ch * 32, x);
-                if (fast) {
+            const bool fast = __all_sync(0xffffffffu, two_chunk && rr.valid && !wrapped);
+            float l = 0.f;
+            if (fast) {
+                float x[64];
+                tmem_ld32(region + ch_lo * 32, x);
+                tmem_ld32(region + ch_lo * 32 + 32, x + 32);
+                float mx = x[0];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        mx = fmaxf(mx, x[e]);
+                for (int e = 1; e < 64; ++e)
+                    mx = fmaxf(mx, x[e]);
+                const float m = mx * kLog2e;
+                uint32_t pk[32];
+#pragma unroll
+                for (int e = 0; e < 64; e += 2) {
+                    const float p0 = fast_exp2(fmaf(x[e], kLog2e, -m));
+                    const float p1 = fast_exp2(fmaf(x[e + 1], kLog2e, -m));
+                    l += p0 + p1;
+                    pk[e >> 1] = pack_bf16x2(p0, p1);
+                }
+                uint32_t zero[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    zero[e] = 0u;
+                if (ch_lo == 0) {
+                    tmem_st16(region + 0, pk);
+                    tmem_st16(region + 16, pk + 16);
+                    tmem_st16(region + 32, zero);
+                    tmem_st16(region + 48, zero);
                 } else {
+                    tmem_st16(region + 0, zero);
+                    tmem_st16(region + 16, zero);
+                    tmem_st16(region + 32, pk);
+                    tmem_st16(region + 48, pk + 16);
+                }
+            } else {
+                float mx = -INFINITY;
+                for (int ch = ch_lo; ch < ch_hi; ++ch) {
+                    float x[32];
+                    tmem_ld32(region + ch * 32, x);
 #pragma unroll
                     for (int e = 0; e < 32; ++e)
                         if (codes[ch * 32 + e] == qcode)
                             mx = fmaxf(mx, x[e]);
                 }
-            }
-            const float m = (mx == -INFINITY) ? 0.f : mx * kLog2e;
-            float l = 0.f;
+                const float m = (mx == -INFINITY) ? 0.f : mx * kLog2e;
 #pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-                uint32_t pk[16];
-                if (ch >= ch_lo && ch < ch_hi) {
-                    float x[32];
-                    tmem_ld32(s_addr + ch * 32, x);
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t pk[16];
+                    if (ch >= ch_lo && ch < ch_hi) {
+                        float x[32];
+                        tmem_ld32(region + ch * 32, x);
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        float p0 = fast_exp2(fmaf(x[e], kLog2e, -m));
-                        float p1 = fast_exp2(fmaf(x[e + 1], kLog2e, -m));
-                        if (!fast) {
+                        for (int e = 0; e < 32; e += 2) {
+                            float p0 = fast_exp2(fmaf(x[e], kLog2e, -m));
+                            float p1 = fast_exp2(fmaf(x[e + 1], kLog2e, -m));
                             p0 = codes[ch * 32 + e] == qcode ? p0 : 0.f;
                             p1 = codes[ch * 32 + e + 1] == qcode ? p1 : 0.f;
+                            l += p0 + p1;
+                            pk[e >> 1] = pack_bf16x2(p0, p1);
                         }
-                        l += p0 + p1;
-                        pk[e >> 1] = pack_bf16x2(p0, p1);
-                    }
-                } else {
+                    } else {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        pk[e] = 0u;
+                        for (int e = 0; e < 16; ++e)
+                            pk[e] = 0u;
+                    }
+                    tmem_st16(region + ch * 16, pk);
                 }
-                tmem_st16(s_addr + ch * 16, pk);
             }
             tmem_wait_st();
             tc_fence_before_sync();
@@ -401,7 +599,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
             float o[D];
 #pragma unroll
             for (int c = 0; c < D / 32; ++c)
-                tmem_ld32(o_addr + c * 32, o + c * 32);
+                tmem_ld32(region + 64 + c * 32, o + c * 32);
             if (rr.valid) {
                 const float inv = 1.f / l;
                 uint4 *dst = reinterpret_cast<uint4 *>(out + tk.offset);
@@ -422,7 +620,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1)
 
     tc_fence_before_sync();
     __syncthreads();
-    if (warp == 12) {
+    if (warp == kMmaWarp) {
         tc_fence_after_sync();
         tmem_dealloc(tmem, 512);
     }

@@ -1,6 +1,8 @@
 // C ABI of the fused window-attention forward (declared in include/winattn.h):
 // argument checks, launch planning, kernel dispatch, the host-buffer variant
 // and the per-device status word of the bounded waits.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -170,12 +172,62 @@ int launch_tc(const void *q, const void *k, const void *v, const float *theta, c
                   static_cast<const T *>(bias), static_cast<T *>(out));
 }
 
-template <int D, int R>
-int launch_small(const void *q, const void *k, const void *v, const float *theta, const void *bias, void *out,
-                 const Geometry &g, cudaStream_t stream)
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no
+// link-time dependency on libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult qr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
+            qr == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 4-D view (channels, x, y, image) of a bf16 [B][H][W][heads*d] map with a
+// (d, bw, bh, 1) box: one head's d-vector for a bw x bh rectangle of tokens,
+// swizzled to match the d*2-byte rows of the UMMA operand tiles.
+bool encode_window_map(CUtensorMap *m, const void *base, const Geometry &g, int bw, int bh)
+{
+    auto fn = tensor_map_encoder();
+    if (!fn)
+        return false;
+    const cuuint64_t C = (cuuint64_t)g.heads * g.d;
+    const cuuint64_t dims[4] = {C, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.B};
+    const cuuint64_t strides[3] = {C * 2, C * 2 * g.W, C * 2 * g.W * g.H};
+    const cuuint32_t box[4] = {(cuuint32_t)g.d, (cuuint32_t)bw, (cuuint32_t)bh, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          g.d == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// The four box shapes of one operand (see WindowMaps).
+bool encode_window_maps(WindowMaps *m, const void *base, const Geometry &g)
+{
+    if (!encode_window_map(&m->full, base, g, g.M, g.M))
+        return false;
+    if (g.shift == 0) {
+        m->xhalf = m->yhalf = m->quarter = m->full;
+        return true;
+    }
+    const int hm = g.M / 2;
+    return encode_window_map(&m->xhalf, base, g, hm, g.M) && encode_window_map(&m->yhalf, base, g, g.M, hm) &&
+           encode_window_map(&m->quarter, base, g, hm, hm);
+}
+
+template <int D, int R, bool TMA>
+int launch_small_variant(const void *q, const void *k, const void *v, const float *theta, const void *bias,
+                         void *out, const Geometry &g, cudaStream_t stream, const WindowMaps *maps)
 {
     using T = __nv_bfloat16;
-    auto kernel = winattn_fwd_small_kernel<D, R>;
+    auto kernel = winattn_fwd_small_kernel<D, R, TMA>;
     // The kernel takes all 512 TMEM columns: ask for enough shared memory that
     // no second CTA can be resident on the same SM.
     const int need = (int)SmallLayout<D, R>::bytes(g.heads, g.M);
@@ -183,10 +235,28 @@ int launch_small(const void *q, const void *k, const void *v, const float *theta
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return WINATTN_ERR_CUDA;
     const int64_t grid = g.items < sm_count() ? g.items : sm_count();
-    kernel<<<(unsigned)grid, kSmallThreads, smem, stream>>>(
+    kernel<<<(unsigned)grid, SmallRoles<D>::kThreads, smem, stream>>>(
         static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), theta,
-        static_cast<const T *>(bias), static_cast<T *>(out), g, 1.0f / std::sqrt((float)g.d));
+        static_cast<const T *>(bias), static_cast<T *>(out), g, 1.0f / std::sqrt((float)g.d), maps[0], maps[1],
+        maps[2]);
     return cudaGetLastError() == cudaSuccess ? WINATTN_OK : WINATTN_ERR_CUDA;
+}
+
+template <int D, int R>
+int launch_small(const void *q, const void *k, const void *v, const float *theta, const void *bias, void *out,
+                 const Geometry &g, cudaStream_t stream)
+{
+    WindowMaps maps[3];
+    std::memset(maps, 0, sizeof maps);
+    if constexpr (R == 0) {
+        if (small_tma_ok(g)) {
+            if (encode_window_maps(&maps[0], q, g) && encode_window_maps(&maps[1], k, g) &&
+                encode_window_maps(&maps[2], v, g))
+                return launch_small_variant<D, R, true>(q, k, v, theta, bias, out, g, stream, maps);
+            std::memset(maps, 0, sizeof maps);
+        }
+    }
+    return launch_small_variant<D, R, false>(q, k, v, theta, bias, out, g, stream, maps);
 }
 
 template <int D, int R>
@@ -370,7 +440,7 @@ int winattn_launch_info(int B, int H_img, int W_img, int M, int shift, int heads
     if (kernel) *kernel = (int)kind;
     if (kind == kSmall) {
         if (grid) *grid = (int)(g.items < kAssumedSMs ? g.items : kAssumedSMs);
-        if (threads) *threads = kSmallThreads;
+        if (threads) *threads = g.d <= 32 ? SmallRoles<32>::kThreads : SmallRoles<64>::kThreads;
         if (smem_bytes) *smem_bytes = (int)small_smem(g);
     } else {
         if (grid) *grid = (int)g.items;
