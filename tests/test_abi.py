@@ -110,8 +110,8 @@ def test_launch_plan(lib, B, H, W, M, heads, d, rank, U, tiles, kernel):
     assert info["work_items"] == heads * math.ceil(windows / U) * tiles
     assert info["kernel"] == kernel
     if kernel == SMALL:
-        groups = 4 if d == 32 else 3  # compute warpgroups, plus a loader and an MMA warp
-        assert info["threads"] == (4 * groups + 2) * 32 and info["grid"] == min(148, info["work_items"])
+        groups = 4 if d == 32 else 3  # compute warpgroups, plus a loader warp
+        assert info["threads"] == (4 * groups + 1) * 32 and info["grid"] == min(148, info["work_items"])
     else:
         assert info["threads"] == 128 and info["grid"] == info["work_items"]
     assert 0 < info["smem_bytes"] <= 227 * 1024

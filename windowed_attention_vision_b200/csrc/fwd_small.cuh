@@ -9,28 +9,29 @@
 // are ordered pack-major, head-minor so that the heads of a token - which
 // share its DRAM lines - are read by neighbouring CTAs at the same time.
 //
-// Roles (576 threads):
-//   warp 16     loader.  TMA mode (windows that split into whole swizzle
-//               atoms): tensor-map box loads of each window's Q, K, V head
-//               slices straight into the swizzled operand tiles - one box
-//               for an interior window, two for a window on the wrap seam's
-//               row or column, four for the corner window.  Otherwise:
-//               cp.async gathers of 16-byte chunks (rank-r factors too).
-//   warp 17     MMA issuer (one thread): polls the ring and issues, as soon
-//               as each is ready, S = Q~ K~^T into TMEM and O = P V with P
-//               read from TMEM;
-//   warps 0-15  four compute warpgroups, item k going to group k % 4: each
-//               thread owns one tile row (TMEM lane): it resolves its row's
-//               token (window-local coordinates, original position, wrap
-//               label), applies window-local RoPE to its Q and K rows in
-//               place (fp32, Q scaled by d^-1/2), runs max / exp / sum over
-//               its window's keys, writes P (bf16 pairs) over the consumed S
-//               columns, and once O lands normalises it and stores it to the
-//               token's original (un-shifted) position.
+// Roles (4 compute warpgroups + 1 loader warp at d = 32; 3 + 1 at d = 64):
+//   loader warp  TMA mode (windows that split into whole swizzle atoms):
+//                tensor-map box loads of each window's Q, K, V head slices
+//                straight into the swizzled operand tiles - one box for an
+//                interior window, two on the wrap seam's row or column, four
+//                for the corner window - issued by several lanes at once.
+//                Otherwise: cp.async gathers of 16-byte chunks (rank-r
+//                factors too).
+//   compute warpgroups, item k going to group k % groups: each thread owns
+//                one tile row (TMEM lane): it resolves its row's token
+//                (window-local coordinates, original position, wrap label),
+//                applies window-local RoPE to its Q and K rows in place (fp32,
+//                Q scaled by d^-1/2); after a group barrier one elected thread
+//                issues S = Q~ K~^T into the group's TMEM columns; every
+//                thread then runs max / exp / sum over its window's keys and
+//                writes P (bf16 pairs) over the consumed S columns; after a
+//                second barrier the elected thread issues O = P V (P read from
+//                TMEM); once O lands each thread normalises its row and
+//                stores it to the token's original (un-shifted) position.
 // TMEM: 128 columns per group - S (fp32, 128 cols), then P over S[0, 64) and
 // O over S[64, 64 + d).
 // Every wait is bounded; a timeout sets a CTA-wide abort flag and the device
-// status word, and every role drains and returns.
+// status word; a group leaves its loop only at a group barrier, all together.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -45,9 +46,8 @@ namespace winattn {
 template <int D>
 struct SmallRoles {
     static constexpr int kGroups = D <= 32 ? 4 : 3;
-    static constexpr int kThreads = (kGroups * 4 + 2) * 32;
+    static constexpr int kThreads = (kGroups * 4 + 1) * 32;
     static constexpr int kLoaderWarp = kGroups * 4;
-    static constexpr int kMmaWarp = kGroups * 4 + 1;
 };
 
 template <int D, int R>
@@ -63,8 +63,9 @@ struct SmallLayout {
     static constexpr int NS_FIT = (200 * 1024) / STAGE;
     static constexpr int NS = NS_FIT < 6 ? NS_FIT : 6;      // ring depth
     static constexpr int PF = NS - 2 > 2 ? NS - 2 : 2;      // cp.async mode: items issued ahead
-    static constexpr uint32_t TABLE = NS * STAGE;           // RoPE (cos, sin) [heads][M][D/4]
-    static constexpr int kBars = 3 * NS + 4 * SmallRoles<D>::kGroups + 1;
+    static constexpr uint32_t IJTAB = NS * STAGE;           // TMA row order: (i << 8 | j) u16[4 kinds][64]
+    static constexpr uint32_t TABLE = IJTAB + 512;          // RoPE (cos, sin) [heads][M][D/4]
+    static constexpr int kBars = 2 * NS + 3 * SmallRoles<D>::kGroups;
     static __host__ __device__ uint32_t table_bytes(int heads, int M)
     {
         return (uint32_t)(heads * M * (D / 4) * 8 + 15) & ~15u;
@@ -143,6 +144,54 @@ __device__ __forceinline__ void rotate_row_inplace(uint8_t *tile, int row, const
     }
 }
 
+// Rows `row` of the swizzled Q and K tiles: both rotated by R(i, j) (when
+// table != null; one table read serves both), Q multiplied by `qmul`,
+// written back in place, one 16-byte chunk (4 pairs) at a time.
+template <int D>
+__device__ __forceinline__ void rotate_qk_rows(uint8_t *qtile, uint8_t *ktile, int row, const float2 *table, int i,
+                                               int j, float qmul)
+{
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+        const uint32_t off = swz_offset(row, c, 2 * D);
+        const uint4 uq = *reinterpret_cast<const uint4 *>(qtile + off);
+        float xq[8] = {bf16lo(uq.x), bf16hi(uq.x), bf16lo(uq.y), bf16hi(uq.y),
+                       bf16lo(uq.z), bf16hi(uq.z), bf16lo(uq.w), bf16hi(uq.w)};
+        if (table) {
+            const uint4 uk = *reinterpret_cast<const uint4 *>(ktile + off);
+            float xk[8] = {bf16lo(uk.x), bf16hi(uk.x), bf16lo(uk.y), bf16hi(uk.y),
+                           bf16lo(uk.z), bf16hi(uk.z), bf16lo(uk.w), bf16hi(uk.w)};
+            // chunk c holds pairs 4c .. 4c+3 of the head dim: the first half
+            // (row coordinate i) or the second half (column coordinate j)
+            const bool second = 8 * c >= D / 2;
+            const int pos = second ? j : i;
+            const int k0 = second ? 4 * c - D / 4 : 4 * c;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 r = table[pos * (D / 4) + k0 + e];  // (cos, sin) of pos * theta_k
+                const float a0 = xq[2 * e], a1 = xq[2 * e + 1];
+                xq[2 * e] = a0 * r.x - a1 * r.y;
+                xq[2 * e + 1] = a0 * r.y + a1 * r.x;
+                const float b0 = xk[2 * e], b1 = xk[2 * e + 1];
+                xk[2 * e] = b0 * r.x - b1 * r.y;
+                xk[2 * e + 1] = b0 * r.y + b1 * r.x;
+            }
+            uint4 ok;
+            ok.x = pack_bf16x2(xk[0], xk[1]);
+            ok.y = pack_bf16x2(xk[2], xk[3]);
+            ok.z = pack_bf16x2(xk[4], xk[5]);
+            ok.w = pack_bf16x2(xk[6], xk[7]);
+            *reinterpret_cast<uint4 *>(ktile + off) = ok;
+        }
+        uint4 oq;
+        oq.x = pack_bf16x2(xq[0] * qmul, xq[1] * qmul);
+        oq.y = pack_bf16x2(xq[2] * qmul, xq[3] * qmul);
+        oq.z = pack_bf16x2(xq[4] * qmul, xq[5] * qmul);
+        oq.w = pack_bf16x2(xq[6] * qmul, xq[7] * qmul);
+        *reinterpret_cast<uint4 *>(qtile + off) = oq;
+    }
+}
+
 // Window kind in the TMA mode: bit 0 = the window straddles the column wrap
 // seam (last window column of a shifted map), bit 1 = the row seam.
 __device__ __forceinline__ int window_kind(const Geometry &g, int wy, int wx)
@@ -210,17 +259,17 @@ __global__ void __launch_bounds__(SmallRoles<D>::kThreads, 1)
 {
     using L = SmallLayout<D, R>;
     constexpr int NS = L::NS, PF = L::PF, NW = SmallRoles<D>::kGroups;
-    constexpr int kLoaderWarp = SmallRoles<D>::kLoaderWarp, kMmaWarp = SmallRoles<D>::kMmaWarp;
+    constexpr int kLoaderWarp = SmallRoles<D>::kLoaderWarp;
     static_assert(NS >= 3, "ring too shallow");
     static_assert(!TMA || R == 0, "TMA loads carry no rank-r factors");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(base);
+    uint16_t *ijtab = reinterpret_cast<uint16_t *>(base + L::IJTAB);
     float2 *table = reinterpret_cast<float2 *>(base + L::TABLE);
     uint64_t *bars = reinterpret_cast<uint64_t *>(base + L::bars(g.heads, g.M));
-    uint64_t *full = bars, *conv = bars + NS, *empty = bars + 2 * NS;
-    uint64_t *s_full = bars + 3 * NS, *p_full = s_full + NW, *o_full = p_full + NW, *t_free = o_full + NW;
-    uint64_t *fin = t_free + NW;
+    uint64_t *full = bars, *empty = bars + NS;
+    uint64_t *s_full = bars + 2 * NS, *o_full = s_full + NW, *fin = o_full + NW;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + L::kBars);
     volatile uint32_t *abort_flag = tslot + 1;
 
@@ -230,23 +279,20 @@ __global__ void __launch_bounds__(SmallRoles<D>::kThreads, 1)
     const int count = first < n_items ? (n_items - 1 - first) / stride + 1 : 0;
     const int table_per_head = g.M * (D / 4);
 
-    if (warp == kMmaWarp) {
+    if (warp == 0) {
         tmem_alloc(tslot, 512);
         tmem_relinquish();
     }
-    if (t == 0) {
+    if (t == 32) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], TMA ? 1 : 32);
-            mbar_init(&conv[s], 128);
             mbar_init(&empty[s], 1);
         }
         for (int w = 0; w < NW; ++w) {
             mbar_init(&s_full[w], 1);
-            mbar_init(&p_full[w], 128);
             mbar_init(&o_full[w], 1);
-            mbar_init(&t_free[w], 128);
+            mbar_init(&fin[w], 1);
         }
-        mbar_init(fin, 1);
         *abort_flag = 0u;
         fence_mbar_init();
     }
@@ -257,6 +303,14 @@ __global__ void __launch_bounds__(SmallRoles<D>::kThreads, 1)
             float sn, cs;
             sincosf((float)c * __ldg(theta + h * (D / 4) + kk), &sn, &cs);
             table[idx] = make_float2(cs, sn);
+        }
+    }
+    if (TMA) {
+        for (int idx = t; idx < 4 * g.N; idx += blockDim.x) {
+            const int kind = idx / g.N, rp = idx - kind * g.N;
+            int i, j;
+            tma_row_coords(g, kind, rp, i, j);
+            ijtab[kind * 64 + rp] = (uint16_t)((i << 8) | j);
         }
     }
     tc_fence_before_sync();
@@ -272,39 +326,42 @@ __global__ void __launch_bounds__(SmallRoles<D>::kThreads, 1)
                 tma_prefetch_map(pick_map(tm_k, kind));
                 tma_prefetch_map(pick_map(tm_v, kind));
             }
-            const int M = g.M, hm = M >> 1;
-            for (int kk = 0; kk < count; ++kk) {
-                const int s = kk % NS;
-                if (kk >= NS && !wait_or_abort(&empty[s], ((kk / NS) - 1) & 1, abort_flag))
-                    break;
-                const Item it = decode_item_head_minor(g, first + kk * stride);
-                const uint32_t sst = sbase + s * L::STAGE;
-                const int64_t left = g.wph - (int64_t)it.pack * g.U;
-                const int nvalid = left < g.U ? (int)left : g.U;
+        }
+        const int M = g.M, hm = M >> 1;
+        const int my_slot = lane >> 2, my_box = lane & 3;
+        for (int kk = 0; kk < count; ++kk) {
+            const int s = kk % NS;
+            if (kk >= NS && !warp_wait(&empty[s], ((kk / NS) - 1) & 1, abort_flag))
+                break;
+            const Item it = decode_item_head_minor(g, first + kk * stride);
+            const uint32_t sst = sbase + s * L::STAGE;
+            const int64_t left = g.wph - (int64_t)it.pack * g.U;
+            const int nvalid = left < g.U ? (int)left : g.U;
+            if (lane == 0)
                 mbar_arrive_expect_tx(&full[s], (uint32_t)(3 * nvalid * g.N * 2 * D));
-                const int c0 = it.h * D;
-                for (int slot = 0; slot < nvalid; ++slot) {
-                    const int w = it.pack * g.U + slot;
-                    const int b = (int)g.div_img.div((uint32_t)w);
-                    const int rem = w - b * g.nWy * g.nWx;
-                    const int wy = (int)g.div_nWx.div((uint32_t)rem);
-                    const int wx = rem - wy * g.nWx;
-                    const int kind = window_kind(g, wy, wx);
-                    const int nbox = kind == 3 ? 4 : (kind ? 2 : 1);
-                    const int box_rows = g.N / nbox;
-                    for (int bi = 0; bi < nbox; ++bi) {
-                        // rolled-local origin of the box, then its original position
-                        const int iy0 = (kind & 2) ? ((kind == 3 ? bi >> 1 : bi) * hm) : 0;
-                        const int jx0 = (kind & 1) ? ((kind == 3 ? bi & 1 : bi) * hm) : 0;
-                        int y0 = wy * M + iy0 + g.shift;
-                        if (y0 >= g.H) y0 -= g.H;
-                        int x0 = wx * M + jx0 + g.shift;
-                        if (x0 >= g.W) x0 -= g.W;
-                        const uint32_t roff = (uint32_t)((slot * g.N + bi * box_rows) * 2 * D);
-                        tma_load_4d(sst + L::QC + roff, pick_map(tm_q, kind), c0, x0, y0, b, &full[s]);
-                        tma_load_4d(sst + L::KC + roff, pick_map(tm_k, kind), c0, x0, y0, b, &full[s]);
-                        tma_load_4d(sst + L::VO + roff, pick_map(tm_v, kind), c0, x0, y0, b, &full[s]);
-                    }
+            __syncwarp();
+            if (my_slot < nvalid) {
+                const int w = it.pack * g.U + my_slot;
+                const int b = (int)g.div_img.div((uint32_t)w);
+                const int rem = w - b * g.nWy * g.nWx;
+                const int wy = (int)g.div_nWx.div((uint32_t)rem);
+                const int wx = rem - wy * g.nWx;
+                const int kind = window_kind(g, wy, wx);
+                const int nbox = kind == 3 ? 4 : (kind ? 2 : 1);
+                if (my_box < nbox) {
+                    const int bi = my_box;
+                    // rolled-local origin of the box, then its original position
+                    const int iy0 = (kind & 2) ? ((kind == 3 ? bi >> 1 : bi) * hm) : 0;
+                    const int jx0 = (kind & 1) ? ((kind == 3 ? bi & 1 : bi) * hm) : 0;
+                    int y0 = wy * M + iy0 + g.shift;
+                    if (y0 >= g.H) y0 -= g.H;
+                    int x0 = wx * M + jx0 + g.shift;
+                    if (x0 >= g.W) x0 -= g.W;
+                    const uint32_t roff = (uint32_t)((my_slot * g.N + bi * (g.N / nbox)) * 2 * D);
+                    const int c0 = it.h * D;
+                    tma_load_4d(sst + L::QC + roff, pick_map(tm_q, kind), c0, x0, y0, b, &full[s]);
+                    tma_load_4d(sst + L::KC + roff, pick_map(tm_k, kind), c0, x0, y0, b, &full[s]);
+                    tma_load_4d(sst + L::VO + roff, pick_map(tm_v, kind), c0, x0, y0, b, &full[s]);
                 }
             }
         }
@@ -336,10 +393,6 @@ __global__ void __launch_bounds__(SmallRoles<D>::kThreads, 1)
                     cp_async16(sst + L::QC + off, q + src);
                     cp_async16(sst + L::KC + off, k + src);
                     cp_async16(sst + L::VO + off, v + src);
-                } else {
-                    *reinterpret_cast<uint4 *>(st + L::QC + off) = make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4 *>(st + L::KC + off) = make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4 *>(st + L::VO + off) = make_uint4(0, 0, 0, 0);
                 }
             }
             if constexpr (R > 0) {
@@ -381,76 +434,13 @@ __global__ void __launch_bounds__(SmallRoles<D>::kThreads, 1)
             cp_async_commit();
         }
         cp_async_wait_all();
-    } else if (warp == kMmaWarp) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false);
-            constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
-            int ns = 0, npv = 0;  // next item whose S / PV is to be issued
-            uint64_t t_last = globaltimer_ns();
-            while (npv < count) {
-                bool progress = false;
-                if (ns < count && ns - npv < NW) {
-                    const int s = ns % NS, w = ns % NW;
-                    if (mbar_test_wait(&conv[s], (ns / NS) & 1) &&
-                        (ns < NW || mbar_test_wait(&t_free[w], ((ns - NW) / NW) & 1))) {
-                        tc_fence_after_sync();
-                        const uint32_t sst = sbase + s * L::STAGE;
-                        const uint32_t d = tmem + w * 128;
-#pragma unroll
-                        for (int ks = 0; ks < D / 16; ++ks)
-                            umma_bf16_ss(d, smem_desc(sst + L::QC + ks * 32, 16, 16 * D, swizzle_code(2 * D)),
-                                         smem_desc(sst + L::KC + ks * 32, 16, 16 * D, swizzle_code(2 * D)), kIdescS,
-                                         ks > 0);
-#pragma unroll
-                        for (int ks = 0; ks < R / 16; ++ks)
-                            umma_bf16_ss(d, smem_desc(sst + L::QB + ks * 32, 16, 16 * R, swizzle_code(2 * R)),
-                                         smem_desc(sst + L::KB + ks * 32, 16, 16 * R, swizzle_code(2 * R)), kIdescS,
-                                         1);
-                        umma_commit(&s_full[w]);
-                        ++ns;
-                        progress = true;
-                    }
-                }
-                if (npv < ns) {
-                    const int s = npv % NS, w = npv % NW;
-                    if (mbar_test_wait(&p_full[w], (npv / NW) & 1)) {
-                        tc_fence_after_sync();
-                        const uint32_t sst = sbase + s * L::STAGE;
-                        const uint32_t pa = tmem + w * 128;        // P: 64 columns of bf16 pairs over S
-                        const uint32_t od = tmem + w * 128 + 64;   // O: d columns over S[64, 64 + d)
-#pragma unroll
-                        for (int ks = 0; ks < 8; ++ks)
-                            umma_bf16_ts(od, pa + ks * 8,
-                                         smem_desc(sst + L::VO + ks * 32 * D, 8192, 16 * D, swizzle_code(2 * D)),
-                                         kIdescPV, ks > 0);
-                        umma_commit(&o_full[w]);
-                        umma_commit(&empty[s]);
-                        ++npv;
-                        progress = true;
-                    }
-                }
-                if (progress) {
-                    t_last = globaltimer_ns();
-                } else if (*abort_flag) {
-                    break;
-                } else if (globaltimer_ns() - t_last > kWaitLimitNs) {
-                    *abort_flag = 1u;
-                    atomicOr(&g_status_word, 1u);
-                    break;
-                } else {
-                    __nanosleep(32);
-                }
-            }
-            // every UMMA issued above has completed before TMEM is released
-            umma_commit(fin);
-            mbar_wait(fin, 0);
-        }
-    } else {
+    } else if (warp < 4 * NW) {
         // ------------------------------------------------------------ compute groups
         const int w = warp >> 2;
         const int row = t - 128 * w;
-        const uint32_t region = tmem + w * 128 + ((uint32_t)((warp & 3) * 32) << 16);
+        const bool elected = row == 0;
+        const uint32_t gbase = tmem + w * 128;  // this group's TMEM columns
+        const uint32_t region = gbase + ((uint32_t)((warp & 3) * 32) << 16);
         const int r0 = (warp & 3) * 32;
         int c_lo = 0, c_hi = g.N < 128 ? g.N : 128;
         if (g.U > 1) {
@@ -462,165 +452,199 @@ __global__ void __launch_bounds__(SmallRoles<D>::kThreads, 1)
         const bool aligned = (g.N & 31) == 0;
         // the fast path reads exactly two 32-column chunks: one 64-token window
         const bool two_chunk = aligned && ch_hi - ch_lo == 2;
+        constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false);
+        constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
+        bool failed = false;
+        int issued = 0;  // UMMA batches this thread issued (elected thread only)
 
         for (int kc = w; kc < count; kc += NW) {
             const int s = kc % NS, j = kc / NW;
-            if (!warp_wait(&full[s], (kc / NS) & 1, abort_flag))
-                break;
             uint8_t *st = base + s * L::STAGE;
+            const uint32_t sst = sbase + s * L::STAGE;
             const Item it = decode_item_head_minor(g, first + kc * stride);
-
-            // ---- resolve this row's token
             const RowRef rr = tile_row(g, it.pack, 0, row);
             bool wrapped = false;
             TokenRef tk{};
             int code = 0xFFFE;
-            if (rr.valid) {
-                int pi = 0, pj = 0, p = rr.p;
-                if (TMA) {
-                    const int b = (int)g.div_img.div((uint32_t)rr.w);
-                    const int rem = rr.w - b * g.nWy * g.nWx;
-                    const int wy = (int)g.div_nWx.div((uint32_t)rem);
-                    const int kind = window_kind(g, wy, rem - wy * g.nWx);
-                    tma_row_coords(g, kind, rr.p, pi, pj);
-                    p = pi * g.M + pj;
-                    wrapped = kind != 0;
+            float row_sum = 1.f;
+            failed = failed || !warp_wait(&full[s], (kc / NS) & 1, abort_flag);
+            if (!failed) {
+                // ---- resolve this row's token
+                if (rr.valid) {
+                    int p = rr.p;
+                    if (TMA) {
+                        const int b = (int)g.div_img.div((uint32_t)rr.w);
+                        const int rem = rr.w - b * g.nWy * g.nWx;
+                        const int wy = (int)g.div_nWx.div((uint32_t)rem);
+                        const int kind = window_kind(g, wy, rem - wy * g.nWx);
+                        const uint32_t ij = ijtab[kind * 64 + rr.p];
+                        p = (int)(ij >> 8) * g.M + (int)(ij & 0xFF);
+                        wrapped = kind != 0;
+                    } else {
+                        wrapped = window_wrapped(g, rr.w);
+                    }
+                    tk = token_ref(g, rr.w, p, it.h);
+                    code = (rr.slot << 2) | tk.label;
+                }
+                reinterpret_cast<uint16_t *>(st + L::CODES)[row] = (uint16_t)code;
+                // ---- window-local RoPE on this row's query and key, in place;
+                // a row without a token (empty pack slot) is zeroed, so that its
+                // value row contributes exact zeros to P V
+                if (rr.valid) {
+                    rotate_qk_rows<D>(st + L::QC, st + L::KC, row,
+                                      theta ? table + it.h * table_per_head : nullptr, tk.i, tk.j, scale);
                 } else {
-                    wrapped = window_wrapped(g, rr.w);
-                }
-                tk = token_ref(g, rr.w, p, it.h);
-                code = (rr.slot << 2) | tk.label;
-            }
-            uint16_t *codes = reinterpret_cast<uint16_t *>(st + L::CODES);
-            codes[row] = (uint16_t)code;
-
-            // ---- window-local RoPE on this row's query and key, in place; a
-            // row without a token (empty pack slot) is zeroed, so that its
-            // value row contributes exact zeros to P V
-            if (rr.valid) {
-                const float2 *tb = theta ? table + it.h * table_per_head : nullptr;
-                rotate_row_inplace<D>(st + L::QC, row, tb, tk.i, tk.j, scale);
-                if (theta)
-                    rotate_row_inplace<D>(st + L::KC, row, tb, tk.i, tk.j, 1.f);
-            } else {
 #pragma unroll
-                for (int c = 0; c < D / 8; ++c) {
-                    const uint32_t off = swz_offset(row, c, 2 * D);
-                    *reinterpret_cast<uint4 *>(st + L::QC + off) = make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4 *>(st + L::KC + off) = make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4 *>(st + L::VO + off) = make_uint4(0, 0, 0, 0);
+                    for (int c = 0; c < D / 8; ++c) {
+                        const uint32_t off = swz_offset(row, c, 2 * D);
+                        *reinterpret_cast<uint4 *>(st + L::QC + off) = make_uint4(0, 0, 0, 0);
+                        *reinterpret_cast<uint4 *>(st + L::KC + off) = make_uint4(0, 0, 0, 0);
+                        *reinterpret_cast<uint4 *>(st + L::VO + off) = make_uint4(0, 0, 0, 0);
+                    }
                 }
+                fence_proxy_async_smem();
             }
-            fence_proxy_async_smem();
-            named_bar_sync(2 + w, 128);  // this group's codes are all written
-            mbar_arrive(&conv[s]);
-
-            if (!warp_wait(&s_full[w], j & 1, abort_flag))
+            tc_fence_before_sync();
+            // operands and codes of the tile are complete (or someone failed)
+            if (named_bar_any(1 + w, 128, failed))
                 break;
-            tc_fence_after_sync();
-            const int qcode = rr.valid ? code : 0xFFFF;
-            // Keys need no per-element test when the row's window fills whole
-            // 32-column chunks and is not wrapped.
-            const bool fast = __all_sync(0xffffffffu, two_chunk && rr.valid && !wrapped);
-            float l = 0.f;
-            if (fast) {
-                float x[64];
-                tmem_ld32(region + ch_lo * 32, x);
-                tmem_ld32(region + ch_lo * 32 + 32, x + 32);
-                float mx = x[0];
+            if (elected) {
+                tc_fence_after_sync();
 #pragma unroll
-                for (int e = 1; e < 64; ++e)
-                    mx = fmaxf(mx, x[e]);
-                const float m = mx * kLog2e;
-                uint32_t pk[32];
+                for (int ks = 0; ks < D / 16; ++ks)
+                    umma_bf16_ss(gbase, smem_desc(sst + L::QC + ks * 32, 16, 16 * D, swizzle_code(2 * D)),
+                                 smem_desc(sst + L::KC + ks * 32, 16, 16 * D, swizzle_code(2 * D)), kIdescS, ks > 0);
 #pragma unroll
-                for (int e = 0; e < 64; e += 2) {
-                    const float p0 = fast_exp2(fmaf(x[e], kLog2e, -m));
-                    const float p1 = fast_exp2(fmaf(x[e + 1], kLog2e, -m));
-                    l += p0 + p1;
-                    pk[e >> 1] = pack_bf16x2(p0, p1);
-                }
-                uint32_t zero[16];
+                for (int ks = 0; ks < R / 16; ++ks)
+                    umma_bf16_ss(gbase, smem_desc(sst + L::QB + ks * 32, 16, 16 * R, swizzle_code(2 * R)),
+                                 smem_desc(sst + L::KB + ks * 32, 16, 16 * R, swizzle_code(2 * R)), kIdescS, 1);
+                umma_commit(&s_full[w]);
+                ++issued;
+            }
+            const uint16_t *codes = reinterpret_cast<const uint16_t *>(st + L::CODES);
+            failed = !warp_wait(&s_full[w], j & 1, abort_flag);
+            if (!failed) {
+                tc_fence_after_sync();
+                const int qcode = rr.valid ? code : 0xFFFF;
+                // Keys need no per-element test when the row's window fills
+                // whole 32-column chunks and is not wrapped.
+                const bool fast = __all_sync(0xffffffffu, two_chunk && rr.valid && !wrapped);
+                float l = 0.f;
+                if (fast) {
+                    float x[64];
+                    tmem_ld32(region + ch_lo * 32, x);
+                    tmem_ld32(region + ch_lo * 32 + 32, x + 32);
+                    float mx = x[0];
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    zero[e] = 0u;
-                if (ch_lo == 0) {
-                    tmem_st16(region + 0, pk);
-                    tmem_st16(region + 16, pk + 16);
-                    tmem_st16(region + 32, zero);
-                    tmem_st16(region + 48, zero);
+                    for (int e = 1; e < 64; ++e)
+                        mx = fmaxf(mx, x[e]);
+                    const float m = mx * kLog2e;
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int e = 0; e < 64; e += 2) {
+                        const float p0 = fast_exp2(fmaf(x[e], kLog2e, -m));
+                        const float p1 = fast_exp2(fmaf(x[e + 1], kLog2e, -m));
+                        l += p0 + p1;
+                        pk[e >> 1] = pack_bf16x2(p0, p1);
+                    }
+                    uint32_t zero[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        zero[e] = 0u;
+                    if (ch_lo == 0) {
+                        tmem_st16(region + 0, pk);
+                        tmem_st16(region + 16, pk + 16);
+                        tmem_st16(region + 32, zero);
+                        tmem_st16(region + 48, zero);
+                    } else {
+                        tmem_st16(region + 0, zero);
+                        tmem_st16(region + 16, zero);
+                        tmem_st16(region + 32, pk);
+                        tmem_st16(region + 48, pk + 16);
+                    }
                 } else {
-                    tmem_st16(region + 0, zero);
-                    tmem_st16(region + 16, zero);
-                    tmem_st16(region + 32, pk);
-                    tmem_st16(region + 48, pk + 16);
-                }
-            } else {
-                float mx = -INFINITY;
-                for (int ch = ch_lo; ch < ch_hi; ++ch) {
-                    float x[32];
-                    tmem_ld32(region + ch * 32, x);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (codes[ch * 32 + e] == qcode)
-                            mx = fmaxf(mx, x[e]);
-                }
-                const float m = (mx == -INFINITY) ? 0.f : mx * kLog2e;
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    uint32_t pk[16];
-                    if (ch >= ch_lo && ch < ch_hi) {
+                    float mx = -INFINITY;
+                    for (int ch = ch_lo; ch < ch_hi; ++ch) {
                         float x[32];
                         tmem_ld32(region + ch * 32, x);
 #pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            float p0 = fast_exp2(fmaf(x[e], kLog2e, -m));
-                            float p1 = fast_exp2(fmaf(x[e + 1], kLog2e, -m));
-                            p0 = codes[ch * 32 + e] == qcode ? p0 : 0.f;
-                            p1 = codes[ch * 32 + e + 1] == qcode ? p1 : 0.f;
-                            l += p0 + p1;
-                            pk[e >> 1] = pack_bf16x2(p0, p1);
-                        }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            pk[e] = 0u;
+                        for (int e = 0; e < 32; ++e)
+                            if (codes[ch * 32 + e] == qcode)
+                                mx = fmaxf(mx, x[e]);
                     }
-                    tmem_st16(region + ch * 16, pk);
+                    const float m = (mx == -INFINITY) ? 0.f : mx * kLog2e;
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t pk[16];
+                        if (ch >= ch_lo && ch < ch_hi) {
+                            float x[32];
+                            tmem_ld32(region + ch * 32, x);
+#pragma unroll
+                            for (int e = 0; e < 32; e += 2) {
+                                float p0 = fast_exp2(fmaf(x[e], kLog2e, -m));
+                                float p1 = fast_exp2(fmaf(x[e + 1], kLog2e, -m));
+                                p0 = codes[ch * 32 + e] == qcode ? p0 : 0.f;
+                                p1 = codes[ch * 32 + e + 1] == qcode ? p1 : 0.f;
+                                l += p0 + p1;
+                                pk[e >> 1] = pack_bf16x2(p0, p1);
+                            }
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e)
+                                pk[e] = 0u;
+                        }
+                        tmem_st16(region + ch * 16, pk);
+                    }
                 }
+                tmem_wait_st();
+                row_sum = l;
             }
-            tmem_wait_st();
             tc_fence_before_sync();
-            mbar_arrive(&p_full[w]);
-
-            if (!warp_wait(&o_full[w], j & 1, abort_flag))
+            // every row's P is in TMEM (or someone failed)
+            if (named_bar_any(1 + w, 128, failed))
                 break;
-            tc_fence_after_sync();
-            float o[D];
+            if (elected) {
+                tc_fence_after_sync();
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c)
-                tmem_ld32(region + 64 + c * 32, o + c * 32);
-            if (rr.valid) {
-                const float inv = 1.f / l;
-                uint4 *dst = reinterpret_cast<uint4 *>(out + tk.offset);
+                for (int ks = 0; ks < 8; ++ks)
+                    umma_bf16_ts(gbase + 64, gbase + ks * 8,
+                                 smem_desc(sst + L::VO + ks * 32 * D, 8192, 16 * D, swizzle_code(2 * D)), kIdescPV,
+                                 ks > 0);
+                umma_commit(&o_full[w]);
+                umma_commit(&empty[s]);
+            }
+            failed = !warp_wait(&o_full[w], j & 1, abort_flag);
+            if (!failed) {
+                tc_fence_after_sync();
+                float o[D];
 #pragma unroll
-                for (int c = 0; c < D / 8; ++c) {
-                    uint4 u;
-                    u.x = pack_bf16x2(o[8 * c + 0] * inv, o[8 * c + 1] * inv);
-                    u.y = pack_bf16x2(o[8 * c + 2] * inv, o[8 * c + 3] * inv);
-                    u.z = pack_bf16x2(o[8 * c + 4] * inv, o[8 * c + 5] * inv);
-                    u.w = pack_bf16x2(o[8 * c + 6] * inv, o[8 * c + 7] * inv);
-                    dst[c] = u;
+                for (int c = 0; c < D / 32; ++c)
+                    tmem_ld32(region + 64 + c * 32, o + c * 32);
+                if (rr.valid) {
+                    const float inv = 1.f / row_sum;
+                    uint4 *dst = reinterpret_cast<uint4 *>(out + tk.offset);
+#pragma unroll
+                    for (int c = 0; c < D / 8; ++c) {
+                        uint4 u;
+                        u.x = pack_bf16x2(o[8 * c + 0] * inv, o[8 * c + 1] * inv);
+                        u.y = pack_bf16x2(o[8 * c + 2] * inv, o[8 * c + 3] * inv);
+                        u.z = pack_bf16x2(o[8 * c + 4] * inv, o[8 * c + 5] * inv);
+                        u.w = pack_bf16x2(o[8 * c + 6] * inv, o[8 * c + 7] * inv);
+                        dst[c] = u;
+                    }
                 }
             }
-            tc_fence_before_sync();
-            mbar_arrive(&t_free[w]);
+        }
+        // every UMMA this thread issued has completed before TMEM is released
+        if (elected && issued) {
+            umma_commit(&fin[w]);
+            mbar_wait(&fin[w], 0);
         }
     }
 
     tc_fence_before_sync();
     __syncthreads();
-    if (warp == kMmaWarp) {
+    if (warp == 0) {
         tc_fence_after_sync();
         tmem_dealloc(tmem, 512);
     }
