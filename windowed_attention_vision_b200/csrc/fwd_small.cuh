@@ -105,89 +105,67 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     return __all_sync(0xffffffffu, wait_or_abort(bar, parity, abort_flag));
 }
 
-// Row `row` of a swizzled bf16 tile: rotate by R(i, j) (when table != null),
-// multiply by `mul`, write back in place.
-template <int D>
-__device__ __forceinline__ void rotate_row_inplace(uint8_t *tile, int row, const float2 *table, int i, int j,
-                                                   float mul)
-{
-    float x[D];
-#pragma unroll
-    for (int c = 0; c < D / 8; ++c) {
-        const uint4 u = *reinterpret_cast<const uint4 *>(tile + swz_offset(row, c, 2 * D));
-        x[8 * c + 0] = bf16lo(u.x); x[8 * c + 1] = bf16hi(u.x);
-        x[8 * c + 2] = bf16lo(u.y); x[8 * c + 3] = bf16hi(u.y);
-        x[8 * c + 4] = bf16lo(u.z); x[8 * c + 5] = bf16hi(u.z);
-        x[8 * c + 6] = bf16lo(u.w); x[8 * c + 7] = bf16hi(u.w);
-    }
-    if (table) {
-#pragma unroll
-        for (int k = 0; k < D / 4; ++k) {
-            const float2 ry = table[i * (D / 4) + k];
-            const float a0 = x[2 * k], a1 = x[2 * k + 1];
-            x[2 * k] = a0 * ry.x - a1 * ry.y;
-            x[2 * k + 1] = a0 * ry.y + a1 * ry.x;
-            const float2 rx = table[j * (D / 4) + k];
-            const float b0 = x[D / 2 + 2 * k], b1 = x[D / 2 + 2 * k + 1];
-            x[D / 2 + 2 * k] = b0 * rx.x - b1 * rx.y;
-            x[D / 2 + 2 * k + 1] = b0 * rx.y + b1 * rx.x;
-        }
-    }
-#pragma unroll
-    for (int c = 0; c < D / 8; ++c) {
-        uint4 o;
-        o.x = pack_bf16x2(x[8 * c + 0] * mul, x[8 * c + 1] * mul);
-        o.y = pack_bf16x2(x[8 * c + 2] * mul, x[8 * c + 3] * mul);
-        o.z = pack_bf16x2(x[8 * c + 4] * mul, x[8 * c + 5] * mul);
-        o.w = pack_bf16x2(x[8 * c + 6] * mul, x[8 * c + 7] * mul);
-        *reinterpret_cast<uint4 *>(tile + swz_offset(row, c, 2 * D)) = o;
-    }
-}
-
 // Rows `row` of the swizzled Q and K tiles: both rotated by R(i, j) (when
-// table != null; one table read serves both), Q multiplied by `qmul`,
-// written back in place, one 16-byte chunk (4 pairs) at a time.
+// table != null; one table read serves both), Q multiplied by `qmul` (when
+// scale_q), written back in place, one 16-byte chunk (4 pairs) at a time,
+// with packed two-lane fp32 arithmetic.  table4[pos][k/2] holds
+// (cos k, cos k+1, sin k, sin k+1) of pos * theta for even k.
 template <int D>
-__device__ __forceinline__ void rotate_qk_rows(uint8_t *qtile, uint8_t *ktile, int row, const float2 *table, int i,
-                                               int j, float qmul)
+__device__ __forceinline__ void rotate_qk_rows(uint8_t *qtile, uint8_t *ktile, int row, const float4 *table4, int i,
+                                               int j, bool scale_q, float qmul)
 {
 #pragma unroll
     for (int c = 0; c < D / 8; ++c) {
         const uint32_t off = swz_offset(row, c, 2 * D);
         const uint4 uq = *reinterpret_cast<const uint4 *>(qtile + off);
-        float xq[8] = {bf16lo(uq.x), bf16hi(uq.x), bf16lo(uq.y), bf16hi(uq.y),
-                       bf16lo(uq.z), bf16hi(uq.z), bf16lo(uq.w), bf16hi(uq.w)};
-        if (table) {
+        // pairs (a_e, b_e), e = 0..3, regrouped as (a0, a1), (b0, b1), (a2, a3), (b2, b3)
+        float2 qa01 = make_float2(bf16lo(uq.x), bf16lo(uq.y)), qb01 = make_float2(bf16hi(uq.x), bf16hi(uq.y));
+        float2 qa23 = make_float2(bf16lo(uq.z), bf16lo(uq.w)), qb23 = make_float2(bf16hi(uq.z), bf16hi(uq.w));
+        if (table4) {
             const uint4 uk = *reinterpret_cast<const uint4 *>(ktile + off);
-            float xk[8] = {bf16lo(uk.x), bf16hi(uk.x), bf16lo(uk.y), bf16hi(uk.y),
-                           bf16lo(uk.z), bf16hi(uk.z), bf16lo(uk.w), bf16hi(uk.w)};
+            float2 ka01 = make_float2(bf16lo(uk.x), bf16lo(uk.y)), kb01 = make_float2(bf16hi(uk.x), bf16hi(uk.y));
+            float2 ka23 = make_float2(bf16lo(uk.z), bf16lo(uk.w)), kb23 = make_float2(bf16hi(uk.z), bf16hi(uk.w));
             // chunk c holds pairs 4c .. 4c+3 of the head dim: the first half
             // (row coordinate i) or the second half (column coordinate j)
             const bool second = 8 * c >= D / 2;
-            const int pos = second ? j : i;
-            const int k0 = second ? 4 * c - D / 4 : 4 * c;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 r = table[pos * (D / 4) + k0 + e];  // (cos, sin) of pos * theta_k
-                const float a0 = xq[2 * e], a1 = xq[2 * e + 1];
-                xq[2 * e] = a0 * r.x - a1 * r.y;
-                xq[2 * e + 1] = a0 * r.y + a1 * r.x;
-                const float b0 = xk[2 * e], b1 = xk[2 * e + 1];
-                xk[2 * e] = b0 * r.x - b1 * r.y;
-                xk[2 * e + 1] = b0 * r.y + b1 * r.x;
-            }
+            const float4 *tp = table4 + (second ? j : i) * (D / 8) + (second ? 2 * c - D / 8 : 2 * c);
+            const float4 r01 = tp[0], r23 = tp[1];
+            const float2 c01 = make_float2(r01.x, r01.y), s01 = make_float2(r01.z, r01.w);
+            const float2 c23 = make_float2(r23.x, r23.y), s23 = make_float2(r23.z, r23.w);
+            const float2 n01 = make_float2(-r01.z, -r01.w), n23 = make_float2(-r23.z, -r23.w);
+            // (a, b) -> (a cos - b sin, a sin + b cos)
+            float2 t;
+            t = __ffma2_rn(qb01, n01, __fmul2_rn(qa01, c01));
+            qb01 = __ffma2_rn(qb01, c01, __fmul2_rn(qa01, s01));
+            qa01 = t;
+            t = __ffma2_rn(qb23, n23, __fmul2_rn(qa23, c23));
+            qb23 = __ffma2_rn(qb23, c23, __fmul2_rn(qa23, s23));
+            qa23 = t;
+            t = __ffma2_rn(kb01, n01, __fmul2_rn(ka01, c01));
+            kb01 = __ffma2_rn(kb01, c01, __fmul2_rn(ka01, s01));
+            ka01 = t;
+            t = __ffma2_rn(kb23, n23, __fmul2_rn(ka23, c23));
+            kb23 = __ffma2_rn(kb23, c23, __fmul2_rn(ka23, s23));
+            ka23 = t;
             uint4 ok;
-            ok.x = pack_bf16x2(xk[0], xk[1]);
-            ok.y = pack_bf16x2(xk[2], xk[3]);
-            ok.z = pack_bf16x2(xk[4], xk[5]);
-            ok.w = pack_bf16x2(xk[6], xk[7]);
+            ok.x = pack_bf16x2(ka01.x, kb01.x);
+            ok.y = pack_bf16x2(ka01.y, kb01.y);
+            ok.z = pack_bf16x2(ka23.x, kb23.x);
+            ok.w = pack_bf16x2(ka23.y, kb23.y);
             *reinterpret_cast<uint4 *>(ktile + off) = ok;
         }
+        if (scale_q) {
+            const float2 m2 = make_float2(qmul, qmul);
+            qa01 = __fmul2_rn(qa01, m2);
+            qb01 = __fmul2_rn(qb01, m2);
+            qa23 = __fmul2_rn(qa23, m2);
+            qb23 = __fmul2_rn(qb23, m2);
+        }
         uint4 oq;
-        oq.x = pack_bf16x2(xq[0] * qmul, xq[1] * qmul);
-        oq.y = pack_bf16x2(xq[2] * qmul, xq[3] * qmul);
-        oq.z = pack_bf16x2(xq[4] * qmul, xq[5] * qmul);
-        oq.w = pack_bf16x2(xq[6] * qmul, xq[7] * qmul);
+        oq.x = pack_bf16x2(qa01.x, qb01.x);
+        oq.y = pack_bf16x2(qa01.y, qb01.y);
+        oq.z = pack_bf16x2(qa23.x, qb23.x);
+        oq.w = pack_bf16x2(qa23.y, qb23.y);
         *reinterpret_cast<uint4 *>(qtile + off) = oq;
     }
 }
@@ -297,12 +275,16 @@ __global__ void __launch_bounds__(SmallRoles<D>::kThreads, 1)
         fence_mbar_init();
     }
     if (theta) {
+        // table4[h][pos][k/2] = (cos k, cos k+1, sin k, sin k+1) of pos * theta_h
+        float *tf = reinterpret_cast<float *>(table);
         for (int idx = t; idx < g.heads * table_per_head; idx += blockDim.x) {
             const int h = idx / table_per_head, r = idx - h * table_per_head;
             const int c = r / (D / 4), kk = r - c * (D / 4);
             float sn, cs;
             sincosf((float)c * __ldg(theta + h * (D / 4) + kk), &sn, &cs);
-            table[idx] = make_float2(cs, sn);
+            float *e = tf + 2 * ((h * g.M + c) * (D / 4) + (kk & ~1));
+            e[kk & 1] = cs;
+            e[2 + (kk & 1)] = sn;
         }
     }
     if (TMA) {
@@ -491,8 +473,11 @@ __global__ void __launch_bounds__(SmallRoles<D>::kThreads, 1)
                 // a row without a token (empty pack slot) is zeroed, so that its
                 // value row contributes exact zeros to P V
                 if (rr.valid) {
-                    rotate_qk_rows<D>(st + L::QC, st + L::KC, row,
-                                      theta ? table + it.h * table_per_head : nullptr, tk.i, tk.j, scale);
+                    if (theta || R > 0)
+                        rotate_qk_rows<D>(st + L::QC, st + L::KC, row,
+                                          theta ? reinterpret_cast<const float4 *>(table + it.h * table_per_head)
+                                                : nullptr,
+                                          tk.i, tk.j, R > 0, scale);
                 } else {
 #pragma unroll
                     for (int c = 0; c < D / 8; ++c) {
@@ -525,6 +510,9 @@ __global__ void __launch_bounds__(SmallRoles<D>::kThreads, 1)
             failed = !warp_wait(&s_full[w], j & 1, abort_flag);
             if (!failed) {
                 tc_fence_after_sync();
+                // scores in log2 units: without rank-r factors Q was not
+                // pre-scaled, so d^-1/2 joins log2(e) here
+                const float c2 = R > 0 ? kLog2e : scale * kLog2e;
                 const int qcode = rr.valid ? code : 0xFFFF;
                 // Keys need no per-element test when the row's window fills
                 // whole 32-column chunks and is not wrapped.
@@ -534,19 +522,23 @@ __global__ void __launch_bounds__(SmallRoles<D>::kThreads, 1)
                     float x[64];
                     tmem_ld32(region + ch_lo * 32, x);
                     tmem_ld32(region + ch_lo * 32 + 32, x + 32);
-                    float mx = x[0];
+                    float mx = fmax3(x[0], x[1], x[2]);
 #pragma unroll
-                    for (int e = 1; e < 64; ++e)
-                        mx = fmaxf(mx, x[e]);
-                    const float m = mx * kLog2e;
+                    for (int e = 3; e < 63; e += 2)
+                        mx = fmax3(mx, x[e], x[e + 1]);
+                    mx = fmaxf(mx, x[63]);
+                    const float2 cc = make_float2(c2, c2);
+                    const float2 mm = make_float2(-mx * c2, -mx * c2);
+                    float2 l2 = make_float2(0.f, 0.f);
                     uint32_t pk[32];
 #pragma unroll
                     for (int e = 0; e < 64; e += 2) {
-                        const float p0 = fast_exp2(fmaf(x[e], kLog2e, -m));
-                        const float p1 = fast_exp2(fmaf(x[e + 1], kLog2e, -m));
-                        l += p0 + p1;
-                        pk[e >> 1] = pack_bf16x2(p0, p1);
+                        const float2 z = __ffma2_rn(make_float2(x[e], x[e + 1]), cc, mm);
+                        const float2 p = make_float2(fast_exp2(z.x), fast_exp2(z.y));
+                        l2 = __fadd2_rn(l2, p);
+                        pk[e >> 1] = pack_bf16x2(p.x, p.y);
                     }
+                    l = l2.x + l2.y;
                     uint32_t zero[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e)
@@ -572,7 +564,7 @@ __global__ void __launch_bounds__(SmallRoles<D>::kThreads, 1)
                             if (codes[ch * 32 + e] == qcode)
                                 mx = fmaxf(mx, x[e]);
                     }
-                    const float m = (mx == -INFINITY) ? 0.f : mx * kLog2e;
+                    const float m = (mx == -INFINITY) ? 0.f : mx * c2;
 #pragma unroll
                     for (int ch = 0; ch < 4; ++ch) {
                         uint32_t pk[16];
@@ -581,8 +573,8 @@ __global__ void __launch_bounds__(SmallRoles<D>::kThreads, 1)
                             tmem_ld32(region + ch * 32, x);
 #pragma unroll
                             for (int e = 0; e < 32; e += 2) {
-                                float p0 = fast_exp2(fmaf(x[e], kLog2e, -m));
-                                float p1 = fast_exp2(fmaf(x[e + 1], kLog2e, -m));
+                                float p0 = fast_exp2(fmaf(x[e], c2, -m));
+                                float p1 = fast_exp2(fmaf(x[e + 1], c2, -m));
                                 p0 = codes[ch * 32 + e] == qcode ? p0 : 0.f;
                                 p1 = codes[ch * 32 + e + 1] == qcode ? p1 : 0.f;
                                 l += p0 + p1;
@@ -622,14 +614,19 @@ __global__ void __launch_bounds__(SmallRoles<D>::kThreads, 1)
                     tmem_ld32(region + 64 + c * 32, o + c * 32);
                 if (rr.valid) {
                     const float inv = 1.f / row_sum;
+                    const float2 i2 = make_float2(inv, inv);
                     uint4 *dst = reinterpret_cast<uint4 *>(out + tk.offset);
 #pragma unroll
                     for (int c = 0; c < D / 8; ++c) {
+                        float2 y[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            y[e] = __fmul2_rn(make_float2(o[8 * c + 2 * e], o[8 * c + 2 * e + 1]), i2);
                         uint4 u;
-                        u.x = pack_bf16x2(o[8 * c + 0] * inv, o[8 * c + 1] * inv);
-                        u.y = pack_bf16x2(o[8 * c + 2] * inv, o[8 * c + 3] * inv);
-                        u.z = pack_bf16x2(o[8 * c + 4] * inv, o[8 * c + 5] * inv);
-                        u.w = pack_bf16x2(o[8 * c + 6] * inv, o[8 * c + 7] * inv);
+                        u.x = pack_bf16x2(y[0].x, y[0].y);
+                        u.y = pack_bf16x2(y[1].x, y[1].y);
+                        u.z = pack_bf16x2(y[2].x, y[2].y);
+                        u.w = pack_bf16x2(y[3].x, y[3].y);
                         dst[c] = u;
                     }
                 }

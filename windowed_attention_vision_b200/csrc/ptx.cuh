@@ -52,6 +52,22 @@ __device__ __forceinline__ uint32_t mbar_try_wait(uint64_t *bar, uint32_t parity
     return ok;
 }
 
+// The same with a suspend-time hint: a thread whose phase is not complete
+// sleeps in hardware until it completes or about `hint_ns` pass, instead of
+// spinning through the issue slots other warps need.
+__device__ __forceinline__ uint32_t mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok;
+}
+
 // Non-blocking probe of a phase (for polling loops).
 __device__ __forceinline__ uint32_t mbar_test_wait(uint64_t *bar, uint32_t parity)
 {
@@ -80,7 +96,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
     if (mbar_try_wait(bar, parity))
         return true;
     const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_sleep(bar, parity, 100000u)) {
         if (globaltimer_ns() - t0 > kWaitLimitNs)
             return false;
     }
@@ -317,6 +333,14 @@ __device__ __forceinline__ float fast_exp2(float x)
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// max(a, b, c) in one instruction (three-input max of sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
