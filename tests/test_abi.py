@@ -89,13 +89,14 @@ def test_host_workspace_bytes(lib):
     assert _lib.host_workspace_bytes(0, 16, 16, 2, 32, _lib.BF16) == 0
 
 
-GENERIC, SMALL, SIMT = 0, 1, 3
+GENERIC, SMALL, LARGE, SIMT = 0, 1, 2, 3
 
 
 @pytest.mark.parametrize("B,H,W,M,heads,d,rank,U,tiles,kernel", [
     (64, 56, 56, 8, 3, 32, 0, 2, 1, SMALL),      # Swin stage 1: two 64-token windows per tile
-    (16, 128, 128, 32, 3, 32, 0, 1, 8, GENERIC),  # 1024-token windows: 8 query tiles each
-    (4, 192, 192, 96, 6, 32, 16, 1, 72, GENERIC),  # 9216-token windows
+    (16, 128, 128, 32, 3, 32, 0, 1, 8, LARGE),    # 1024-token windows: 8 query tiles each
+    (4, 192, 192, 96, 6, 32, 16, 1, 72, LARGE),   # 9216-token windows
+    (1, 48, 48, 24, 1, 32, 0, 1, 5, GENERIC),     # 576 tokens: no whole-row key tiles
     (1, 24, 24, 12, 1, 32, 0, 1, 2, GENERIC),     # 144 tokens: a ragged second tile
     (1, 9, 9, 3, 2, 64, 0, 14, 1, SMALL),         # 9-token windows: 14 per tile
     (2, 5, 5, 1, 1, 32, 0, 128, 1, SMALL),        # one-token windows
@@ -107,12 +108,16 @@ def test_launch_plan(lib, B, H, W, M, heads, d, rank, U, tiles, kernel):
     assert rc == _lib.OK
     windows = B * (H // M) * (W // M)
     assert info["windows_per_tile"] == U
-    assert info["work_items"] == heads * math.ceil(windows / U) * tiles
     assert info["kernel"] == kernel
+    if kernel == LARGE:  # items are pairs of query tiles
+        assert info["work_items"] == heads * windows * tiles // 2
+        assert info["threads"] == 448 and info["grid"] == min(148, info["work_items"])
+    else:
+        assert info["work_items"] == heads * math.ceil(windows / U) * tiles
     if kernel == SMALL:
         groups = 4 if d == 32 else 3  # compute warpgroups, plus a loader warp
         assert info["threads"] == (4 * groups + 1) * 32 and info["grid"] == min(148, info["work_items"])
-    else:
+    elif kernel == GENERIC:
         assert info["threads"] == 128 and info["grid"] == info["work_items"]
     assert 0 < info["smem_bytes"] <= 227 * 1024
 

@@ -37,6 +37,14 @@ SMALL = [
     ("m11_s5_d64_r16", 1, 22, 22, 11, 5, 2, 64, "bf16", "learned", 16),   # 121 tokens, small kernel
     ("m9_s4_r32", 2, 18, 9, 9, 4, 3, 32, "bf16", None, 32),
     ("m24_s0_r16", 1, 48, 48, 24, 0, 2, 32, "bf16", None, 16),      # bias factors, no RoPE
+    ("m16_s0_d32", 2, 32, 48, 16, 0, 2, 32, "bf16", "learned", 0),  # large-window kernel from here on
+    ("m16_s8_d32_nope", 1, 32, 32, 16, 8, 3, 32, "bf16", None, 0),
+    ("m32_s0_d64", 1, 64, 96, 32, 0, 2, 64, "bf16", "standard", 0),
+    ("m32_s0_r16", 1, 64, 64, 32, 0, 2, 32, "bf16", None, 16),
+    ("m32_s0_r32_rope", 1, 64, 64, 32, 0, 1, 64, "bf16", "learned", 32),
+    ("m64_s32", 1, 128, 128, 64, 32, 1, 32, "bf16", "learned", 0),
+    ("m96_s48_d64", 1, 192, 96, 96, 48, 1, 64, "bf16", "learned", 0),
+    ("m96_s0_r16", 1, 96, 96, 96, 0, 2, 32, "bf16", None, 16),
     ("m8_s4_r32_rope", 2, 16, 16, 8, 4, 2, 32, "bf16", "learned", 32),
     ("m16_s8_d64_r16", 1, 32, 32, 16, 8, 1, 64, "bf16", "learned", 16),
     ("fp32_m8_d16", 1, 16, 16, 8, 4, 2, 16, "fp32", "learned", 0),

@@ -1,0 +1,631 @@
+// Persistent, warp-specialised forward for large windows (M in {16, 32, 64,
+// 96}: 256 to 9216 tokens): the compute-bound regime ("FLASHSWIN" page,
+// section "어떻게 동작하나": an IO-aware fused kernel accumulates the softmax
+// online over key tiles, so the N x N score matrix is never stored; the
+// windows grow to 96 x 96 on the "Rank-Factorized Implicit Neural Bias"
+// page, section 3).
+//
+// Work item: one window-head (a "unit") and a pair of 128-row query tiles of
+// it; items are ordered unit-major, so the pairs of one window run side by
+// side on neighbouring SMs and its keys and values are read from L2.
+//
+// Key/value tiles are whole rows of the window (BN = 128 tokens, or 96 at
+// M = 96), loaded by TMA boxes straight into swizzled operand tiles of a
+// ring; when the window straddles the column wrap seam (shift M/2) a tile is
+// two boxes of M/2 columns, never a rolled copy.  Query tiles are gathered
+// with cp.async in the window's row-major order.
+//
+// Roles (14 warps):
+//   warps 0-3 / 4-7  softmax warpgroups A / B, one per query tile: each
+//                    thread owns one query row (TMEM lane), runs the online
+//                    softmax over the key tiles (running max m and sum l in
+//                    fp32, exp2 in log2 units), writes P (bf16 pairs) over the
+//                    consumed S columns, rescales its O row in TMEM only when
+//                    the max grows by more than 2^8, and at the end
+//                    normalises O and stores it to the token's original
+//                    (un-shifted) position;
+//   warps 8-11       converter: per item, the RoPE table of the head and the
+//                    query tiles (cp.async gather, window-local 2D RoPE in
+//                    fp32, d^-1/2 folded in when rank-r factors are present);
+//                    per key tile, RoPE on the K rows in place;
+//   warp 12          TMA loader of K, V (and the key-side factors w);
+//   warp 13          MMA issuer: S_A, S_B, then O_A += P_A V and O_B += P_B V
+//                    per key tile, the next S of a tile issued right behind its
+//                    PV so the softmax groups ping-pong with the tensor core.
+// TMEM: tile A at columns [0, BN + d), tile B at [256, 256 + BN + d): S (fp32,
+// BN columns) with P over its first BN/2 columns, then O (d columns).
+// Wrap masks are structural: a key tile lies on one side of the row seam,
+// and its two boxes on the two sides of the column seam, so each query row
+// keeps all, none, or one half of a tile.
+#pragma once
+#include <cuda_bf16.h>
+#include <cstdint>
+
+#include "geometry.cuh"
+#include "ptx.cuh"
+#include "waits.cuh"
+
+namespace winattn {
+
+constexpr int kLargeThreads = 14 * 32;
+constexpr uint32_t kLargeSmemBudget = 220 * 1024;
+
+// Key-tile rows of a window: 128 tokens per tile for M = 16, 32, 64, one
+// window row (96 tokens) for M = 96.
+__host__ __device__ inline int large_tile_keys(int M) { return M == 96 ? 96 : 128; }
+
+// Windows this kernel serves (the rest go to the generic kernel): M in
+// {16, 32, 64, 96}; shift 0 or M/2 (key tiles then never straddle the row
+// seam and split into two equal boxes at the column seam); rank-r factors
+// only without a shift.
+__host__ __device__ inline bool large_ok(const Geometry &g)
+{
+    if (g.M != 16 && g.M != 32 && g.M != 64 && g.M != 96)
+        return false;
+    if (g.shift != 0 && 2 * g.shift != g.M)
+        return false;
+    return g.rank == 0 || g.shift == 0;
+}
+
+// One tile row's token, resolved for the softmax groups.
+struct QRowInfo {
+    int64_t off;   // element offset of the (token, head) d-vector
+    int ly, lx;    // wrap label bits of the row (rolled row / column in the last `shift`)
+};
+static_assert(sizeof(QRowInfo) == 16, "QRowInfo is 16 bytes");
+
+template <int D, int R, int BN>
+struct LargeLayout {
+    static constexpr uint32_t QTILE = 256 * (D + R);             // 128 rows: content [128][D], factors [128][R]
+    static constexpr uint32_t QBUF = 2 * QTILE;                   // a pair of query tiles
+    static constexpr uint32_t KC = 0;                             // key content  [BN][D]   (in a stage)
+    static constexpr uint32_t KB = KC + BN * 2 * D;               // key factors  [BN][R]
+    static constexpr uint32_t VO = KB + BN * 2 * R;               // values       [BN][D]
+    static constexpr uint32_t STAGE = (VO + BN * 2 * D + 1023) & ~1023u;
+    static constexpr uint32_t STAGES = 2 * QBUF;                  // ring start
+    static constexpr uint32_t TABLE_BYTES = 96 * D * 2;           // RoPE (cos, sin) float4 [M][D/8], M <= 96
+    static constexpr uint32_t QINFO_BYTES = 2 * 256 * 16;         // QRowInfo [2 buffers][256]
+    static constexpr uint32_t FIXED = STAGES + TABLE_BYTES + QINFO_BYTES + 64 * 8 + 16 + 1024;
+    static constexpr int NS_FIT = (int)((kLargeSmemBudget - FIXED) / STAGE);
+    static constexpr int NS = NS_FIT < 8 ? NS_FIT : 8;
+    static constexpr uint32_t TABLE = STAGES + NS * STAGE;
+    static constexpr uint32_t QINFO = TABLE + TABLE_BYTES;
+    static constexpr uint32_t BARS = QINFO + QINFO_BYTES;
+    static constexpr uint32_t BYTES = BARS + 64 * 8 + 16 + 1024;
+};
+
+// Row `row` of a swizzled bf16 tile with D content columns: rotated by
+// R(i, j) with packed two-lane fp32 arithmetic (table4[pos][k/2] holds
+// (cos k, cos k+1, sin k, sin k+1) of pos * theta, even k), optionally
+// multiplied by `mul`, written back in place.
+template <int D>
+__device__ __forceinline__ void rotate_row_f2(uint8_t *tile, int row, const float4 *table4, int i, int j,
+                                              bool scale, float mul)
+{
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+        const uint32_t off = swz_offset(row, c, 2 * D);
+        const uint4 u = *reinterpret_cast<const uint4 *>(tile + off);
+        float2 a01 = make_float2(bf16lo(u.x), bf16lo(u.y)), b01 = make_float2(bf16hi(u.x), bf16hi(u.y));
+        float2 a23 = make_float2(bf16lo(u.z), bf16lo(u.w)), b23 = make_float2(bf16hi(u.z), bf16hi(u.w));
+        if (table4) {
+            const bool second = 8 * c >= D / 2;
+            const float4 *tp = table4 + (second ? j : i) * (D / 8) + (second ? 2 * c - D / 8 : 2 * c);
+            const float4 r01 = tp[0], r23 = tp[1];
+            const float2 c01 = make_float2(r01.x, r01.y), s01 = make_float2(r01.z, r01.w);
+            const float2 c23 = make_float2(r23.x, r23.y), s23 = make_float2(r23.z, r23.w);
+            const float2 n01 = make_float2(-r01.z, -r01.w), n23 = make_float2(-r23.z, -r23.w);
+            float2 t = __ffma2_rn(b01, n01, __fmul2_rn(a01, c01));
+            b01 = __ffma2_rn(b01, c01, __fmul2_rn(a01, s01));
+            a01 = t;
+            t = __ffma2_rn(b23, n23, __fmul2_rn(a23, c23));
+            b23 = __ffma2_rn(b23, c23, __fmul2_rn(a23, s23));
+            a23 = t;
+        }
+        if (scale) {
+            const float2 m2 = make_float2(mul, mul);
+            a01 = __fmul2_rn(a01, m2);
+            b01 = __fmul2_rn(b01, m2);
+            a23 = __fmul2_rn(a23, m2);
+            b23 = __fmul2_rn(b23, m2);
+        }
+        uint4 o;
+        o.x = pack_bf16x2(a01.x, b01.x);
+        o.y = pack_bf16x2(a01.y, b01.y);
+        o.z = pack_bf16x2(a23.x, b23.x);
+        o.w = pack_bf16x2(a23.y, b23.y);
+        *reinterpret_cast<uint4 *>(tile + off) = o;
+    }
+}
+
+// 8 consecutive 32-bit TMEM columns of this thread's lane, written from v[].
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t *v)
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+                 "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
+}
+
+// Tiled 2-D tensor load (no multicast), bytes counted on *bar.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst_smem, const CUtensorMap *map, int c0, int c1,
+                                            uint64_t *bar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+            "r"(dst_smem),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Tensor maps of the large-window kernel: K and V boxes of (d, M, kr) and
+// (d, M/2, kr) tokens, and the key-side factors w as (rank, BN) rows.
+struct LargeMaps {
+    CUtensorMap k_full, k_half, v_full, v_half, w;
+};
+
+template <int D, int R, int BN>
+__global__ void __launch_bounds__(kLargeThreads, 1)
+    winattn_fwd_large_kernel(const __nv_bfloat16 *__restrict__ q, const float *__restrict__ theta,
+                             const __nv_bfloat16 *__restrict__ bias, __nv_bfloat16 *__restrict__ out,
+                             const Geometry g, const float scale, const __grid_constant__ LargeMaps maps)
+{
+    using L = LargeLayout<D, R, BN>;
+    constexpr int NS = L::NS;
+    static_assert(NS >= 2, "ring too shallow");
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(base);
+    float4 *table4 = reinterpret_cast<float4 *>(base + L::TABLE);
+    QRowInfo *qinfo = reinterpret_cast<QRowInfo *>(base + L::QINFO);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(base + L::BARS);
+    uint64_t *kv_full = bars, *kv_ready = bars + NS, *kv_empty = bars + 2 * NS;
+    uint64_t *q_ready = bars + 3 * NS, *q_free = q_ready + 2, *s_full = q_free + 2, *p_full = s_full + 2;
+    uint64_t *o_done = p_full + 2, *t_free = o_done + 2, *fin = t_free + 2;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(fin + 1);
+    volatile uint32_t *abort_flag = tslot + 1;
+
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    const int M = g.M, N = g.N, kr = BN / M;  // key tile = kr window rows
+    const int nkv = N / BN;                   // key tiles per window
+    const int npairs = N / 256;               // query-tile pairs per window
+    const int n_items = (int)(g.wph * g.heads) * npairs;
+    const int first = blockIdx.x, stride = gridDim.x;
+    const int count = first < n_items ? (n_items - 1 - first) / stride + 1 : 0;
+    const bool has_rope = theta != nullptr;
+    // scores in log2 units: without rank-r factors Q is not pre-scaled, so
+    // d^-1/2 joins log2(e) in the exponent
+    const float c2 = R > 0 ? kLog2e : scale * kLog2e;
+
+    if (warp == 0) {
+        tmem_alloc(tslot, 512);
+        tmem_relinquish();
+    }
+    if (t == 32) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_ready[s], 128);
+            mbar_init(&kv_empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&q_ready[a], 128);
+            mbar_init(&q_free[a], 1);
+            mbar_init(&s_full[a], 1);
+            mbar_init(&p_full[a], 128);
+            mbar_init(&o_done[a], 1);
+            mbar_init(&t_free[a], 128);
+        }
+        mbar_init(fin, 1);
+        *abort_flag = 0u;
+        fence_mbar_init();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tslot;
+
+    // item -> (window, head, pair); units are head-minor
+    auto decode = [&](int kk, int &w, int &h, int &pair) {
+        const int item = first + kk * stride;
+        const int unit = item / npairs;
+        pair = item - unit * npairs;
+        w = (int)g.div_heads.div((uint32_t)unit);
+        h = unit - w * g.heads;
+    };
+    auto window_pos = [&](int w, int &b, int &wy, int &wx) {
+        b = (int)g.div_img.div((uint32_t)w);
+        const int rem = w - b * g.nWy * g.nWx;
+        wy = (int)g.div_nWx.div((uint32_t)rem);
+        wx = rem - wy * g.nWx;
+    };
+
+    if (warp == 12) {
+        // ============================================================ TMA loader
+        if (lane == 0) {
+            int c = 0;
+            bool ok = true;
+            const uint32_t bytes = (uint32_t)(BN * 2 * (2 * D + R));
+            for (int kk = 0; kk < count && ok; ++kk) {
+                int w, h, pair, b, wy, wx;
+                decode(kk, w, h, pair);
+                window_pos(w, b, wy, wx);
+                const bool xwrap = g.shift && wx == g.nWx - 1;
+                for (int jt = 0; jt < nkv; ++jt, ++c) {
+                    const int s = c % NS;
+                    if (c >= NS && !wait_or_abort(&kv_empty[s], ((c / NS) - 1) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t sst = sbase + L::STAGES + s * L::STAGE;
+                    mbar_arrive_expect_tx(&kv_full[s], bytes);
+                    int y0 = wy * M + jt * kr + g.shift;
+                    if (y0 >= g.H) y0 -= g.H;
+                    const int x0 = wx * M + g.shift;  // < W unless the window straddles the seam
+                    const int c0 = h * D;
+                    if (xwrap) {
+                        const int x1 = 0;             // the seam's far side
+                        const uint32_t half = (uint32_t)(BN / 2) * 2 * D;
+                        tma_load_4d(sst + L::KC, &maps.k_half, c0, x0, y0, b, &kv_full[s]);
+                        tma_load_4d(sst + L::KC + half, &maps.k_half, c0, x1, y0, b, &kv_full[s]);
+                        tma_load_4d(sst + L::VO, &maps.v_half, c0, x0, y0, b, &kv_full[s]);
+                        tma_load_4d(sst + L::VO + half, &maps.v_half, c0, x1, y0, b, &kv_full[s]);
+                    } else {
+                        tma_load_4d(sst + L::KC, &maps.k_full, c0, x0, y0, b, &kv_full[s]);
+                        tma_load_4d(sst + L::VO, &maps.v_full, c0, x0, y0, b, &kv_full[s]);
+                    }
+                    if constexpr (R > 0)
+                        tma_load_2d(sst + L::KB, &maps.w, 0, (h * 2 + 1) * N + jt * BN, &kv_full[s]);
+                }
+            }
+        }
+    } else if (warp == 13) {
+        // ============================================================ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t kIdescS = idesc_bf16_f32(128, BN, false);
+            constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
+            int c = 0;
+            bool ok = true;
+            int issued = 0;
+            auto issue_s = [&](int tile, uint32_t qtile, int s) {
+                const uint32_t d = tmem + tile * 256;
+                const uint32_t kst = sbase + L::STAGES + s * L::STAGE;
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks)
+                    umma_bf16_ss(d, smem_desc(qtile + ks * 32, 16, 16 * D, swizzle_code(2 * D)),
+                                 smem_desc(kst + L::KC + ks * 32, 16, 16 * D, swizzle_code(2 * D)), kIdescS, ks > 0);
+#pragma unroll
+                for (int ks = 0; ks < R / 16; ++ks)
+                    umma_bf16_ss(d, smem_desc(qtile + 256 * D + ks * 32, 16, 16 * R, swizzle_code(2 * R)),
+                                 smem_desc(kst + L::KB + ks * 32, 16, 16 * R, swizzle_code(2 * R)), kIdescS, 1);
+                umma_commit(&s_full[tile]);
+            };
+            auto issue_pv = [&](int tile, int s, bool acc) {
+                const uint32_t st = tmem + tile * 256;
+                const uint32_t vst = sbase + L::STAGES + s * L::STAGE + L::VO;
+#pragma unroll
+                for (int ks = 0; ks < BN / 16; ++ks)
+                    umma_bf16_ts(st + BN, st + ks * 8, smem_desc(vst + ks * 32 * D, 8192, 16 * D, swizzle_code(2 * D)),
+                                 kIdescPV, acc || ks > 0);
+                umma_commit(&o_done[tile]);
+            };
+            for (int kk = 0; kk < count && ok; ++kk) {
+                const int qb = kk & 1;
+                if (!(ok = wait_or_abort(&q_ready[qb], (kk >> 1) & 1, abort_flag)))
+                    break;
+                const uint32_t qa = sbase + qb * L::QBUF, qbt = qa + L::QTILE;
+                if (!(ok = wait_or_abort(&kv_ready[c % NS], (c / NS) & 1, abort_flag)))
+                    break;
+                tc_fence_after_sync();
+                issue_s(0, qa, c % NS);
+                issue_s(1, qbt, c % NS);
+                ++issued;
+                for (int jt = 0; jt < nkv && ok; ++jt, ++c) {
+                    const int s = c % NS;
+                    // tile A: PV of this key tile, then its next S
+                    if (!(ok = wait_or_abort(&p_full[0], c & 1, abort_flag)))
+                        break;
+                    if (jt == 0 && kk > 0 && !(ok = wait_or_abort(&t_free[0], (kk - 1) & 1, abort_flag)))
+                        break;
+                    tc_fence_after_sync();
+                    issue_pv(0, s, jt > 0);
+                    const bool more = jt + 1 < nkv;
+                    if (more) {
+                        if (!(ok = wait_or_abort(&kv_ready[(c + 1) % NS], ((c + 1) / NS) & 1, abort_flag)))
+                            break;
+                        tc_fence_after_sync();
+                        issue_s(0, qa, (c + 1) % NS);
+                    }
+                    // tile B
+                    if (!(ok = wait_or_abort(&p_full[1], c & 1, abort_flag)))
+                        break;
+                    if (jt == 0 && kk > 0 && !(ok = wait_or_abort(&t_free[1], (kk - 1) & 1, abort_flag)))
+                        break;
+                    tc_fence_after_sync();
+                    issue_pv(1, s, jt > 0);
+                    umma_commit(&kv_empty[s]);
+                    if (more)
+                        issue_s(1, qbt, (c + 1) % NS);
+                }
+                umma_commit(&q_free[qb]);
+            }
+            if (issued) {
+                umma_commit(fin);
+                mbar_wait(fin, 0);
+            }
+        }
+    } else if (warp >= 8) {
+        // ============================================================ converter
+        const int ct = t - 256;
+        constexpr int CD = D / 8, CR = R / 8;
+        int c = 0;
+        bool failed = false;
+        // cp.async gather of this thread's two query rows (and factors) of item kk
+        auto load_q = [&](int kk) {
+            int w, h, pair;
+            decode(kk, w, h, pair);
+            const uint32_t qbase = sbase + (kk & 1) * L::QBUF;
+            for (int t2 = 0; t2 < 2; ++t2) {
+                const int p = (2 * pair + t2) * 128 + ct;
+                const TokenRef tk = token_ref(g, w, p, h);
+                const uint32_t tile = qbase + t2 * L::QTILE;
+#pragma unroll
+                for (int ch = 0; ch < CD; ++ch)
+                    cp_async16(tile + swz_offset(ct, ch, 2 * D), q + tk.offset + ch * 8);
+                if constexpr (R > 0) {
+                    const __nv_bfloat16 *u = bias + (((int64_t)h * 2 + 0) * N + p) * R;
+#pragma unroll
+                    for (int ch = 0; ch < CR; ++ch)
+                        cp_async16(tile + 256 * D + swz_offset(ct, ch, 2 * R), u + ch * 8);
+                }
+            }
+            cp_async_commit();
+        };
+        if (count > 0)
+            load_q(0);
+        for (int kk = 0; kk < count; ++kk) {
+            int w, h, pair, b, wy, wx;
+            decode(kk, w, h, pair);
+            window_pos(w, b, wy, wx);
+            const bool xwrap = g.shift && wx == g.nWx - 1;
+            const int qb = kk & 1;
+            // ---- RoPE table of head h: table4[pos][k/2] = (cos k, cos k+1, sin k, sin k+1)
+            if (has_rope) {
+                float *tf = reinterpret_cast<float *>(table4);
+                for (int idx = ct; idx < M * (D / 4); idx += 128) {
+                    const int pos = idx / (D / 4), kq = idx - pos * (D / 4);
+                    float sn, cs;
+                    sincosf((float)pos * __ldg(theta + h * (D / 4) + kq), &sn, &cs);
+                    float *e = tf + 2 * (pos * (D / 4) + (kq & ~1));
+                    e[kq & 1] = cs;
+                    e[2 + (kq & 1)] = sn;
+                }
+            }
+            cp_async_wait<0>();
+            // table built, every query row landed (or someone failed)
+            if (named_bar_any(1, 128, failed))
+                break;
+            // ---- query rows: resolve, rotate (and scale with factors present)
+            {
+                uint8_t *qbase = base + qb * L::QBUF;
+                for (int t2 = 0; t2 < 2; ++t2) {
+                    const int p = (2 * pair + t2) * 128 + ct;
+                    const TokenRef tk = token_ref(g, w, p, h);
+                    QRowInfo ri;
+                    ri.off = tk.offset;
+                    ri.ly = tk.label >> 1;
+                    ri.lx = tk.label & 1;
+                    qinfo[qb * 256 + t2 * 128 + ct] = ri;
+                    if (has_rope || R > 0)
+                        rotate_row_f2<D>(qbase + t2 * L::QTILE, ct, has_rope ? table4 : nullptr, tk.i, tk.j, R > 0,
+                                         scale);
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&q_ready[qb]);
+            }
+            // ---- key tiles: RoPE on K rows in place (TMA row order)
+            for (int jt = 0; jt < nkv && !failed; ++jt, ++c) {
+                const int s = c % NS;
+                if (!warp_wait(&kv_full[s], (c / NS) & 1, abort_flag)) {
+                    failed = true;
+                    break;
+                }
+                if (has_rope && ct < BN) {
+                    int i, j;
+                    if (xwrap) {
+                        const int hm = M >> 1, hf = ct >= BN / 2 ? 1 : 0, cc = ct - hf * (BN / 2);
+                        const int ri = cc / hm;
+                        i = jt * kr + ri;
+                        j = hf * hm + (cc - ri * hm);
+                    } else {
+                        const int ri = ct / M;
+                        i = jt * kr + ri;
+                        j = ct - ri * M;
+                    }
+                    rotate_row_f2<D>(base + L::STAGES + s * L::STAGE + L::KC, ct, table4, i, j, false, 1.f);
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&kv_ready[s]);
+            }
+            // ---- prefetch the next item's query rows into the other buffer,
+            // once the tensor core is done with the item that used it
+            if (kk + 1 < count && !failed) {
+                if (kk + 1 >= 2 && !warp_wait(&q_free[(kk + 1) & 1], (((kk + 1) >> 1) - 1) & 1, abort_flag))
+                    failed = true;
+                else
+                    load_q(kk + 1);
+            }
+            // the table may be rebuilt for the next item (or someone failed)
+            if (named_bar_any(1, 128, failed))
+                break;
+        }
+        cp_async_wait_all();
+    } else {
+        // ============================================================ softmax groups
+        const int tile = warp >> 2;  // 0 = A, 1 = B
+        const int row = t - 128 * tile;
+        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t sreg = tmem + tile * 256 + lane_base;  // S / P
+        const uint32_t oreg = sreg + BN;                      // O
+        constexpr int NCH = BN / 16;                          // 16-column chunks of S
+        int c = 0;
+        bool failed = false;
+        for (int kk = 0; kk < count && !failed; ++kk) {
+            int w, h, pair, b, wy, wx;
+            decode(kk, w, h, pair);
+            window_pos(w, b, wy, wx);
+            const bool xwrap = g.shift && wx == g.nWx - 1;
+            const bool ywrap = g.shift && wy == g.nWy - 1;
+            const int qb = kk & 1;
+            if (!warp_wait(&q_ready[qb], (kk >> 1) & 1, abort_flag)) {
+                failed = true;
+                break;
+            }
+            const QRowInfo me = qinfo[qb * 256 + tile * 128 + row];
+            // Online softmax in log2 units: m is the reference of the row's P
+            // (exp2(s * c2 - m)); it moves, rescaling l and O, only when a
+            // tile's max exceeds it by more than 2^8.
+            float m = -INFINITY, l = 0.f;
+            constexpr int NC = BN / 32;  // 32-column chunks of S
+            for (int jt = 0; jt < nkv; ++jt, ++c) {
+                if (!warp_wait(&s_full[tile], c & 1, abort_flag)) {
+                    failed = true;
+                    break;
+                }
+                tc_fence_after_sync();
+                // allowed 16-column halves of this row: the tile lies on one
+                // side of the row seam, its halves on the two sides of the
+                // column seam
+                const int ky = ywrap && jt * kr >= (M >> 1) ? 1 : 0;
+                int a0 = 0, a1 = NCH;
+                if (ky != me.ly) {
+                    a0 = a1 = 0;
+                } else if (xwrap) {
+                    a0 = me.lx ? NCH / 2 : 0;
+                    a1 = a0 + NCH / 2;
+                }
+                uint32_t buf[2][32];
+                // ---- pass 1: row max over the allowed columns (loads pipelined)
+                float mx = -INFINITY;
+                tmem_ld32_issue(sreg, buf[0]);
+#pragma unroll
+                for (int ch = 0; ch < NC; ++ch) {
+                    tmem_wait_ld32(buf[ch & 1]);
+                    if (ch + 1 < NC)
+                        tmem_ld32_issue(sreg + (ch + 1) * 32, buf[(ch + 1) & 1]);
+                    const uint32_t *xb = buf[ch & 1];
+                    if (2 * ch >= a0 && 2 * ch < a1) {
+#pragma unroll
+                        for (int e = 0; e < 16; e += 2)
+                            mx = fmax3(mx, __uint_as_float(xb[e]), __uint_as_float(xb[e + 1]));
+                    }
+                    if (2 * ch + 1 >= a0 && 2 * ch + 1 < a1) {
+#pragma unroll
+                        for (int e = 16; e < 32; e += 2)
+                            mx = fmax3(mx, __uint_as_float(xb[e]), __uint_as_float(xb[e + 1]));
+                    }
+                }
+                float alpha = 1.f;
+                bool rescale = false;
+                if (mx > -INFINITY) {
+                    const float mn = mx * c2;
+                    if (m == -INFINITY) {
+                        m = mn;
+                    } else if (mn > m + 8.f) {
+                        alpha = fast_exp2(m - mn);
+                        m = mn;
+                        rescale = true;
+                    }
+                }
+                // ---- pass 2: P = exp2(s * c2 - m) into TMEM over the consumed S
+                const float2 cc = make_float2(c2, c2), mm2 = make_float2(-m, -m);
+                float2 l2 = make_float2(0.f, 0.f);
+                tmem_ld32_issue(sreg, buf[0]);
+#pragma unroll
+                for (int ch = 0; ch < NC; ++ch) {
+                    tmem_wait_ld32(buf[ch & 1]);
+                    // P chunk ch covers S columns [16 ch, 16 ch + 16), already read
+                    if (ch + 1 < NC)
+                        tmem_ld32_issue(sreg + (ch + 1) * 32, buf[(ch + 1) & 1]);
+                    const uint32_t *xb = buf[ch & 1];
+                    const bool lo = 2 * ch >= a0 && 2 * ch < a1;
+                    const bool hi = 2 * ch + 1 >= a0 && 2 * ch + 1 < a1;
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        if (e < 16 ? lo : hi) {
+                            const float2 z = __ffma2_rn(
+                                make_float2(__uint_as_float(xb[e]), __uint_as_float(xb[e + 1])), cc, mm2);
+                            const float2 p = make_float2(fast_exp2(z.x), fast_exp2(z.y));
+                            l2 = __fadd2_rn(l2, p);
+                            pk[e >> 1] = pack_bf16x2(p.x, p.y);
+                        } else {
+                            pk[e >> 1] = 0u;
+                        }
+                    }
+                    tmem_st16(sreg + ch * 16, pk);
+                }
+                l = l * alpha + (l2.x + l2.y);
+                if (__any_sync(0xffffffffu, rescale)) {
+                    // O must hold every earlier key tile's P V before it is rescaled
+                    if (!warp_wait(&o_done[tile], (c - 1) & 1, abort_flag)) {
+                        failed = true;
+                        break;
+                    }
+                    tc_fence_after_sync();
+#pragma unroll
+                    for (int ch = 0; ch < D / 16; ++ch) {
+                        float o[16];
+                        tmem_ld16(oreg + ch * 16, o);
+                        uint32_t ob[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            ob[e] = __float_as_uint(o[e] * alpha);
+                        tmem_st16(oreg + ch * 16, ob);
+                    }
+                }
+                tmem_wait_st();
+                tc_fence_before_sync();
+                mbar_arrive(&p_full[tile]);
+            }
+            if (failed)
+                break;
+            // ---- epilogue: O / l to the token's original position
+            if (!warp_wait(&o_done[tile], (c - 1) & 1, abort_flag)) {
+                failed = true;
+                break;
+            }
+            tc_fence_after_sync();
+            const float inv = 1.f / l;
+            const float2 i2 = make_float2(inv, inv);
+            uint4 *dst = reinterpret_cast<uint4 *>(out + me.off);
+#pragma unroll
+            for (int ch = 0; ch < D / 16; ++ch) {
+                float o[16];
+                tmem_ld16(oreg + ch * 16, o);
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float2 y[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        y[e] = __fmul2_rn(make_float2(o[8 * hh + 2 * e], o[8 * hh + 2 * e + 1]), i2);
+                    uint4 u;
+                    u.x = pack_bf16x2(y[0].x, y[0].y);
+                    u.y = pack_bf16x2(y[1].x, y[1].y);
+                    u.z = pack_bf16x2(y[2].x, y[2].y);
+                    u.w = pack_bf16x2(y[3].x, y[3].y);
+                    dst[2 * ch + hh] = u;
+                }
+            }
+            tc_fence_before_sync();
+            mbar_arrive(&t_free[tile]);
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace winattn

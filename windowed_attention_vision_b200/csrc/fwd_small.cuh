@@ -38,6 +38,7 @@
 
 #include "geometry.cuh"
 #include "ptx.cuh"
+#include "waits.cuh"
 
 namespace winattn {
 
@@ -79,31 +80,6 @@ struct SmallLayout {
 struct WindowMaps {
     CUtensorMap full, xhalf, yhalf, quarter;
 };
-
-// Bounded wait that also gives up as soon as another role has aborted.
-__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile uint32_t *abort_flag)
-{
-    if (mbar_try_wait(bar, parity))
-        return true;
-    const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait(bar, parity)) {
-        if (*abort_flag)
-            return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
-            *abort_flag = 1u;
-            atomicOr(&g_status_word, 1u);
-            return false;
-        }
-    }
-    return true;
-}
-
-// The same, with one verdict for the whole warp (its tcgen05 loads and stores
-// are warp-collective, so the warp must leave a loop together).
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile uint32_t *abort_flag)
-{
-    return __all_sync(0xffffffffu, wait_or_abort(bar, parity, abort_flag));
-}
 
 // Rows `row` of the swizzled Q and K tiles: both rotated by R(i, j) (when
 // table != null; one table read serves both), Q multiplied by `qmul` (when

@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "../../include/winattn.h"
+#include "fwd_large.cuh"
 #include "fwd_simt.cuh"
 #include "fwd_small.cuh"
 #include "fwd_tc.cuh"
@@ -88,7 +89,7 @@ constexpr int kAssumedSMs = 148;          // B200; used only by winattn_launch_i
 constexpr uint32_t kMaxSmem = 227 * 1024;
 constexpr uint32_t kMaxSmallTable = 32 * 1024;
 
-enum KernelKind { kGeneric = 0, kSmall = 1, kSimt = 3 };
+enum KernelKind { kGeneric = 0, kSmall = 1, kLarge = 2, kSimt = 3 };
 
 uint32_t small_smem(const Geometry &g)
 {
@@ -112,6 +113,8 @@ KernelKind choose_kernel(const Geometry &g, int dtype)
         return kSimt;
     if (g.N <= kTileRows && (uint64_t)g.heads * g.M * (g.d / 4) * 8 <= kMaxSmallTable && small_smem(g) <= kMaxSmem)
         return kSmall;
+    if (large_ok(g))
+        return kLarge;
     return kGeneric;
 }
 
@@ -222,6 +225,87 @@ bool encode_window_maps(WindowMaps *m, const void *base, const Geometry &g)
            encode_window_map(&m->quarter, base, g, hm, hm);
 }
 
+uint32_t large_smem(const Geometry &g)
+{
+    const bool b96 = large_tile_keys(g.M) == 96;
+    switch (g.d * 100 + g.rank) {
+    case 3200: return b96 ? LargeLayout<32, 0, 96>::BYTES : LargeLayout<32, 0, 128>::BYTES;
+    case 3216: return b96 ? LargeLayout<32, 16, 96>::BYTES : LargeLayout<32, 16, 128>::BYTES;
+    case 3232: return b96 ? LargeLayout<32, 32, 96>::BYTES : LargeLayout<32, 32, 128>::BYTES;
+    case 6400: return b96 ? LargeLayout<64, 0, 96>::BYTES : LargeLayout<64, 0, 128>::BYTES;
+    case 6416: return b96 ? LargeLayout<64, 16, 96>::BYTES : LargeLayout<64, 16, 128>::BYTES;
+    case 6432: return b96 ? LargeLayout<64, 32, 96>::BYTES : LargeLayout<64, 32, 128>::BYTES;
+    }
+    return ~0u;
+}
+
+// 4-D K or V box map for the large-window kernel: (d, bw, rows, 1).
+bool encode_kv_map(CUtensorMap *m, const void *base, const Geometry &g, int bw, int rows)
+{
+    auto fn = tensor_map_encoder();
+    if (!fn)
+        return false;
+    const cuuint64_t C = (cuuint64_t)g.heads * g.d;
+    const cuuint64_t dims[4] = {C, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.B};
+    const cuuint64_t strides[3] = {C * 2, C * 2 * g.W, C * 2 * g.W * g.H};
+    const cuuint32_t box[4] = {(cuuint32_t)g.d, (cuuint32_t)bw, (cuuint32_t)rows, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, g.d == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D map of the factor table [heads][2][N][rank] as rows of rank values,
+// box (rank, rows).
+bool encode_factor_map(CUtensorMap *m, const void *base, const Geometry &g, int rows)
+{
+    auto fn = tensor_map_encoder();
+    if (!fn)
+        return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)g.rank, (cuuint64_t)g.heads * 2 * g.N};
+    const cuuint64_t strides[1] = {(cuuint64_t)g.rank * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)g.rank, (cuuint32_t)rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, g.rank == 16 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int R, int BN>
+int launch_large(const void *q, const void *k, const void *v, const float *theta, const void *bias, void *out,
+                 const Geometry &g, cudaStream_t stream)
+{
+    using T = __nv_bfloat16;
+    LargeMaps maps;
+    std::memset(&maps, 0, sizeof maps);
+    const int kr = BN / g.M;
+    if (!encode_kv_map(&maps.k_full, k, g, g.M, kr) || !encode_kv_map(&maps.v_full, v, g, g.M, kr))
+        return WINATTN_ERR_CUDA;
+    if (g.shift && (!encode_kv_map(&maps.k_half, k, g, g.M / 2, kr) || !encode_kv_map(&maps.v_half, v, g, g.M / 2, kr)))
+        return WINATTN_ERR_CUDA;
+    if (R > 0 && !encode_factor_map(&maps.w, bias, g, BN))
+        return WINATTN_ERR_CUDA;
+    auto kernel = winattn_fwd_large_kernel<D, R, BN>;
+    const int smem = (int)LargeLayout<D, R, BN>::BYTES;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return WINATTN_ERR_CUDA;
+    const int64_t items = g.wph * g.heads * (g.N / 256);
+    const int64_t grid = items < sm_count() ? items : sm_count();
+    kernel<<<(unsigned)grid, kLargeThreads, smem, stream>>>(static_cast<const T *>(q), theta,
+                                                           static_cast<const T *>(bias), static_cast<T *>(out), g,
+                                                           1.0f / std::sqrt((float)g.d), maps);
+    return cudaGetLastError() == cudaSuccess ? WINATTN_OK : WINATTN_ERR_CUDA;
+}
+
+template <int D, int R>
+int launch_large_bn(const void *q, const void *k, const void *v, const float *theta, const void *bias, void *out,
+                    const Geometry &g, cudaStream_t s)
+{
+    if (large_tile_keys(g.M) == 96)
+        return launch_large<D, R, 96>(q, k, v, theta, bias, out, g, s);
+    return launch_large<D, R, 128>(q, k, v, theta, bias, out, g, s);
+}
+
 template <int D, int R, bool TMA>
 int launch_small_variant(const void *q, const void *k, const void *v, const float *theta, const void *bias,
                          void *out, const Geometry &g, cudaStream_t stream, const WindowMaps *maps)
@@ -280,6 +364,15 @@ int dispatch(const void *q, const void *k, const void *v, const float *theta, co
         case 6400: return launch_small<64, 0>(q, k, v, theta, bias, out, g, s);
         case 6416: return launch_small<64, 16>(q, k, v, theta, bias, out, g, s);
         case 6432: return launch_small<64, 32>(q, k, v, theta, bias, out, g, s);
+        }
+    } else if (kind == kLarge) {
+        switch (g.d * 100 + g.rank) {
+        case 3200: return launch_large_bn<32, 0>(q, k, v, theta, bias, out, g, s);
+        case 3216: return launch_large_bn<32, 16>(q, k, v, theta, bias, out, g, s);
+        case 3232: return launch_large_bn<32, 32>(q, k, v, theta, bias, out, g, s);
+        case 6400: return launch_large_bn<64, 0>(q, k, v, theta, bias, out, g, s);
+        case 6416: return launch_large_bn<64, 16>(q, k, v, theta, bias, out, g, s);
+        case 6432: return launch_large_bn<64, 32>(q, k, v, theta, bias, out, g, s);
         }
     } else if (kind == kGeneric) {
         switch (g.d * 100 + g.rank) {
@@ -438,7 +531,13 @@ int winattn_launch_info(int B, int H_img, int W_img, int M, int shift, int heads
     if (work_items) *work_items = g.items;
     if (windows_per_tile) *windows_per_tile = g.U;
     if (kernel) *kernel = (int)kind;
-    if (kind == kSmall) {
+    if (kind == kLarge) {
+        const int64_t items = g.wph * g.heads * (g.N / 256);
+        if (work_items) *work_items = items;
+        if (grid) *grid = (int)(items < kAssumedSMs ? items : kAssumedSMs);
+        if (threads) *threads = kLargeThreads;
+        if (smem_bytes) *smem_bytes = (int)large_smem(g);
+    } else if (kind == kSmall) {
         if (grid) *grid = (int)(g.items < kAssumedSMs ? g.items : kAssumedSMs);
         if (threads) *threads = g.d <= 32 ? SmallRoles<32>::kThreads : SmallRoles<64>::kThreads;
         if (smem_bytes) *smem_bytes = (int)small_smem(g);
