@@ -29,11 +29,15 @@
 //                    fp32, d^-1/2 folded in when rank-r factors are present);
 //                    per key tile, RoPE on the K rows in place;
 //   warp 12          TMA loader of K, V (and the key-side factors w);
-//   warp 13          MMA issuer: S_A, S_B, then O_A += P_A V and O_B += P_B V
-//                    per key tile, the next S of a tile issued right behind its
-//                    PV so the softmax groups ping-pong with the tensor core.
-// TMEM: tile A at columns [0, BN + d), tile B at [256, 256 + BN + d): S (fp32,
-// BN columns) with P over its first BN/2 columns, then O (d columns).
+//   warp 13          MMA issuer: the steps (key tile, query tile A or B) of all
+//                    the CTA's items form one sequence; S of a step is issued
+//                    NB steps ahead into a rotating TMEM buffer, right behind
+//                    the P V that frees it, so a softmax group finds its next
+//                    S already computed; O_A += P_A V, O_B += P_B V as soon as
+//                    each P is ready.
+// TMEM: NB S buffers of BN fp32 columns (NB = 3 at BN = 128, 4 at BN = 96;
+// P as bf16 pairs over the first BN/2 columns of its buffer), then O of tile
+// A and of tile B (d columns each).
 // Wrap masks are structural: a key tile lies on one side of the row seam,
 // and its two boxes on the two sides of the column seam, so each query row
 // keeps all, none, or one half of a tile.
@@ -50,7 +54,7 @@ namespace winattn {
 constexpr int kLargeThreads = 14 * 32;
 constexpr uint32_t kLargeSmemBudget = 220 * 1024;
 
-// Key-tile rows of a window: 128 tokens per tile for M = 16, 32, 64, one
+// Keys per tile: 128 (8, 4 or 2 window rows for M = 16, 32, 64), or one
 // window row (96 tokens) for M = 96.
 __host__ __device__ inline int large_tile_keys(int M) { return M == 96 ? 96 : 128; }
 
@@ -67,13 +71,6 @@ __host__ __device__ inline bool large_ok(const Geometry &g)
     return g.rank == 0 || g.shift == 0;
 }
 
-// One tile row's token, resolved for the softmax groups.
-struct QRowInfo {
-    int64_t off;   // element offset of the (token, head) d-vector
-    int ly, lx;    // wrap label bits of the row (rolled row / column in the last `shift`)
-};
-static_assert(sizeof(QRowInfo) == 16, "QRowInfo is 16 bytes");
-
 template <int D, int R, int BN>
 struct LargeLayout {
     static constexpr uint32_t QTILE = 256 * (D + R);             // 128 rows: content [128][D], factors [128][R]
@@ -84,13 +81,11 @@ struct LargeLayout {
     static constexpr uint32_t STAGE = (VO + BN * 2 * D + 1023) & ~1023u;
     static constexpr uint32_t STAGES = 2 * QBUF;                  // ring start
     static constexpr uint32_t TABLE_BYTES = 96 * D * 2;           // RoPE (cos, sin) float4 [M][D/8], M <= 96
-    static constexpr uint32_t QINFO_BYTES = 2 * 256 * 16;         // QRowInfo [2 buffers][256]
-    static constexpr uint32_t FIXED = STAGES + TABLE_BYTES + QINFO_BYTES + 64 * 8 + 16 + 1024;
+    static constexpr uint32_t FIXED = STAGES + TABLE_BYTES + 64 * 8 + 16 + 1024;
     static constexpr int NS_FIT = (int)((kLargeSmemBudget - FIXED) / STAGE);
     static constexpr int NS = NS_FIT < 8 ? NS_FIT : 8;
     static constexpr uint32_t TABLE = STAGES + NS * STAGE;
-    static constexpr uint32_t QINFO = TABLE + TABLE_BYTES;
-    static constexpr uint32_t BARS = QINFO + QINFO_BYTES;
+    static constexpr uint32_t BARS = TABLE + TABLE_BYTES;
     static constexpr uint32_t BYTES = BARS + 64 * 8 + 16 + 1024;
 };
 
@@ -171,16 +166,21 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
 {
     using L = LargeLayout<D, R, BN>;
     constexpr int NS = L::NS;
-    static_assert(NS >= 2, "ring too shallow");
+    // S buffers in TMEM (BN fp32 columns each, rotated over both query tiles),
+    // then O of tile A and of tile B (D columns each)
+    constexpr int NB = BN == 96 ? 4 : 3;
+    constexpr uint32_t kOCol = NB * BN;
+    static_assert(kOCol + 2 * D <= 512, "TMEM columns");
+    // S of step n + NB may need key tile cg + NB / 2 while tile cg (step n = 2 cg) is held
+    static_assert(NS >= NB / 2 + 1, "ring too shallow for the S lookahead");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(base);
     float4 *table4 = reinterpret_cast<float4 *>(base + L::TABLE);
-    QRowInfo *qinfo = reinterpret_cast<QRowInfo *>(base + L::QINFO);
     uint64_t *bars = reinterpret_cast<uint64_t *>(base + L::BARS);
     uint64_t *kv_full = bars, *kv_ready = bars + NS, *kv_empty = bars + 2 * NS;
-    uint64_t *q_ready = bars + 3 * NS, *q_free = q_ready + 2, *s_full = q_free + 2, *p_full = s_full + 2;
-    uint64_t *o_done = p_full + 2, *t_free = o_done + 2, *fin = t_free + 2;
+    uint64_t *q_ready = bars + 3 * NS, *q_free = q_ready + 2, *s_full = q_free + 2, *p_full = s_full + NB;
+    uint64_t *o_done = p_full + NB, *o_last = o_done + 2, *t_free = o_last + 2, *fin = t_free + 2;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(fin + 1);
     volatile uint32_t *abort_flag = tslot + 1;
 
@@ -209,10 +209,13 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
         for (int a = 0; a < 2; ++a) {
             mbar_init(&q_ready[a], 128);
             mbar_init(&q_free[a], 1);
-            mbar_init(&s_full[a], 1);
-            mbar_init(&p_full[a], 128);
             mbar_init(&o_done[a], 1);
+            mbar_init(&o_last[a], 1);
             mbar_init(&t_free[a], 128);
+        }
+        for (int b = 0; b < NB; ++b) {
+            mbar_init(&s_full[b], 1);
+            mbar_init(&p_full[b], 128);
         }
         mbar_init(fin, 1);
         *abort_flag = 0u;
@@ -279,75 +282,76 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
         }
     } else if (warp == 13) {
         // ============================================================ MMA issuer
+        // One sequence over the CTA's items: step n = 2 cg + t is query tile t
+        // (0 = A, 1 = B) against the CTA's cg-th key tile.  S of step n goes to
+        // TMEM buffer n % NB and is issued NB steps ahead, right behind the P V
+        // that frees its buffer, across item boundaries too.
         if (lane == 0) {
             constexpr uint32_t kIdescS = idesc_bf16_f32(128, BN, false);
             constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
-            int c = 0;
+            const int total = 2 * count * nkv;
             bool ok = true;
-            int issued = 0;
-            auto issue_s = [&](int tile, uint32_t qtile, int s) {
-                const uint32_t d = tmem + tile * 256;
-                const uint32_t kst = sbase + L::STAGES + s * L::STAGE;
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks)
-                    umma_bf16_ss(d, smem_desc(qtile + ks * 32, 16, 16 * D, swizzle_code(2 * D)),
-                                 smem_desc(kst + L::KC + ks * 32, 16, 16 * D, swizzle_code(2 * D)), kIdescS, ks > 0);
-#pragma unroll
-                for (int ks = 0; ks < R / 16; ++ks)
-                    umma_bf16_ss(d, smem_desc(qtile + 256 * D + ks * 32, 16, 16 * R, swizzle_code(2 * R)),
-                                 smem_desc(kst + L::KB + ks * 32, 16, 16 * R, swizzle_code(2 * R)), kIdescS, 1);
-                umma_commit(&s_full[tile]);
-            };
-            auto issue_pv = [&](int tile, int s, bool acc) {
-                const uint32_t st = tmem + tile * 256;
-                const uint32_t vst = sbase + L::STAGES + s * L::STAGE + L::VO;
-#pragma unroll
-                for (int ks = 0; ks < BN / 16; ++ks)
-                    umma_bf16_ts(st + BN, st + ks * 8, smem_desc(vst + ks * 32 * D, 8192, 16 * D, swizzle_code(2 * D)),
-                                 kIdescPV, acc || ks > 0);
-                umma_commit(&o_done[tile]);
-            };
-            for (int kk = 0; kk < count && ok; ++kk) {
-                const int qb = kk & 1;
-                if (!(ok = wait_or_abort(&q_ready[qb], (kk >> 1) & 1, abort_flag)))
-                    break;
-                const uint32_t qa = sbase + qb * L::QBUF, qbt = qa + L::QTILE;
-                if (!(ok = wait_or_abort(&kv_ready[c % NS], (c / NS) & 1, abort_flag)))
-                    break;
-                tc_fence_after_sync();
-                issue_s(0, qa, c % NS);
-                issue_s(1, qbt, c % NS);
-                ++issued;
-                for (int jt = 0; jt < nkv && ok; ++jt, ++c) {
-                    const int s = c % NS;
-                    // tile A: PV of this key tile, then its next S
-                    if (!(ok = wait_or_abort(&p_full[0], c & 1, abort_flag)))
-                        break;
-                    if (jt == 0 && kk > 0 && !(ok = wait_or_abort(&t_free[0], (kk - 1) & 1, abort_flag)))
-                        break;
-                    tc_fence_after_sync();
-                    issue_pv(0, s, jt > 0);
-                    const bool more = jt + 1 < nkv;
-                    if (more) {
-                        if (!(ok = wait_or_abort(&kv_ready[(c + 1) % NS], ((c + 1) / NS) & 1, abort_flag)))
+            int ns = 0, s_kk = 0, s_jt = 0;  // next S step, its item and key tile
+            auto issue_s_upto = [&](int upto) {
+                for (; ns < upto && ns < total && ok; ++ns) {
+                    const int tl = ns & 1, cg = ns >> 1;
+                    if (tl == 0) {
+                        if (s_jt == 0 && !(ok = wait_or_abort(&q_ready[s_kk & 1], (s_kk >> 1) & 1, abort_flag)))
+                            break;
+                        if (!(ok = wait_or_abort(&kv_ready[cg % NS], (cg / NS) & 1, abort_flag)))
                             break;
                         tc_fence_after_sync();
-                        issue_s(0, qa, (c + 1) % NS);
                     }
-                    // tile B
-                    if (!(ok = wait_or_abort(&p_full[1], c & 1, abort_flag)))
-                        break;
-                    if (jt == 0 && kk > 0 && !(ok = wait_or_abort(&t_free[1], (kk - 1) & 1, abort_flag)))
-                        break;
-                    tc_fence_after_sync();
-                    issue_pv(1, s, jt > 0);
-                    umma_commit(&kv_empty[s]);
-                    if (more)
-                        issue_s(1, qbt, (c + 1) % NS);
+                    const uint32_t qtile = sbase + (s_kk & 1) * L::QBUF + tl * L::QTILE;
+                    const uint32_t d = tmem + (ns % NB) * BN;
+                    const uint32_t kst = sbase + L::STAGES + (cg % NS) * L::STAGE;
+#pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks)
+                        umma_bf16_ss(d, smem_desc(qtile + ks * 32, 16, 16 * D, swizzle_code(2 * D)),
+                                     smem_desc(kst + L::KC + ks * 32, 16, 16 * D, swizzle_code(2 * D)), kIdescS,
+                                     ks > 0);
+#pragma unroll
+                    for (int ks = 0; ks < R / 16; ++ks)
+                        umma_bf16_ss(d, smem_desc(qtile + 256 * D + ks * 32, 16, 16 * R, swizzle_code(2 * R)),
+                                     smem_desc(kst + L::KB + ks * 32, 16, 16 * R, swizzle_code(2 * R)), kIdescS, 1);
+                    umma_commit(&s_full[ns % NB]);
+                    if (tl == 1 && ++s_jt == nkv) {
+                        umma_commit(&q_free[s_kk & 1]);  // the last S that reads this item's Q
+                        s_jt = 0;
+                        ++s_kk;
+                    }
                 }
-                umma_commit(&q_free[qb]);
+            };
+            issue_s_upto(NB);
+            int p_kk = 0, p_jt = 0;
+            for (int n = 0; n < total && ok; ++n) {
+                const int tl = n & 1, cg = n >> 1;
+                if (!(ok = wait_or_abort(&p_full[n % NB], (n / NB) & 1, abort_flag)))
+                    break;
+                // O of this tile is free once the previous item's epilogue read it
+                if (p_jt == 0 && p_kk > 0 && !(ok = wait_or_abort(&t_free[tl], (p_kk - 1) & 1, abort_flag)))
+                    break;
+                tc_fence_after_sync();
+                const uint32_t pa = tmem + (n % NB) * BN;  // P over the first BN/2 columns of the buffer
+                const uint32_t vst = sbase + L::STAGES + (cg % NS) * L::STAGE + L::VO;
+                const uint32_t od = tmem + kOCol + tl * D;
+#pragma unroll
+                for (int ks = 0; ks < BN / 16; ++ks)
+                    umma_bf16_ts(od, pa + ks * 8, smem_desc(vst + ks * 32 * D, 8192, 16 * D, swizzle_code(2 * D)),
+                                 kIdescPV, p_jt > 0 || ks > 0);
+                umma_commit(&o_done[tl]);
+                if (p_jt == nkv - 1)
+                    umma_commit(&o_last[tl]);
+                if (tl == 1) {
+                    umma_commit(&kv_empty[cg % NS]);
+                    if (++p_jt == nkv) {
+                        p_jt = 0;
+                        ++p_kk;
+                    }
+                }
+                issue_s_upto(n + 1 + NB);
             }
-            if (issued) {
+            if (total > 0) {
                 umma_commit(fin);
                 mbar_wait(fin, 0);
             }
@@ -409,11 +413,6 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
                 for (int t2 = 0; t2 < 2; ++t2) {
                     const int p = (2 * pair + t2) * 128 + ct;
                     const TokenRef tk = token_ref(g, w, p, h);
-                    QRowInfo ri;
-                    ri.off = tk.offset;
-                    ri.ly = tk.label >> 1;
-                    ri.lx = tk.label & 1;
-                    qinfo[qb * 256 + t2 * 128 + ct] = ri;
                     if (has_rope || R > 0)
                         rotate_row_f2<D>(qbase + t2 * L::QTILE, ct, has_rope ? table4 : nullptr, tk.i, tk.j, R > 0,
                                          scale);
@@ -463,8 +462,7 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
         const int tile = warp >> 2;  // 0 = A, 1 = B
         const int row = t - 128 * tile;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t sreg = tmem + tile * 256 + lane_base;  // S / P
-        const uint32_t oreg = sreg + BN;                      // O
+        const uint32_t oreg = tmem + lane_base + kOCol + tile * D;  // O of this tile, this warp's lanes
         constexpr int NCH = BN / 16;                          // 16-column chunks of S
         int c = 0;
         bool failed = false;
@@ -474,32 +472,32 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
             window_pos(w, b, wy, wx);
             const bool xwrap = g.shift && wx == g.nWx - 1;
             const bool ywrap = g.shift && wy == g.nWy - 1;
-            const int qb = kk & 1;
-            if (!warp_wait(&q_ready[qb], (kk >> 1) & 1, abort_flag)) {
-                failed = true;
-                break;
-            }
-            const QRowInfo me = qinfo[qb * 256 + tile * 128 + row];
+            // this thread's query row: token, and its wrap label bits (S of
+            // the item implies its query tiles are ready)
+            const TokenRef me = token_ref(g, w, (2 * pair + tile) * 128 + row, h);
+            const int me_ly = me.label >> 1, me_lx = me.label & 1;
             // Online softmax in log2 units: m is the reference of the row's P
             // (exp2(s * c2 - m)); it moves, rescaling l and O, only when a
             // tile's max exceeds it by more than 2^8.
             float m = -INFINITY, l = 0.f;
             constexpr int NC = BN / 32;  // 32-column chunks of S
             for (int jt = 0; jt < nkv; ++jt, ++c) {
-                if (!warp_wait(&s_full[tile], c & 1, abort_flag)) {
+                const int n = 2 * c + tile;  // step of the CTA's S / P sequence
+                if (!warp_wait(&s_full[n % NB], (n / NB) & 1, abort_flag)) {
                     failed = true;
                     break;
                 }
                 tc_fence_after_sync();
+                const uint32_t sreg = tmem + lane_base + (n % NB) * BN;  // S (then P) of this step
                 // allowed 16-column halves of this row: the tile lies on one
                 // side of the row seam, its halves on the two sides of the
                 // column seam
                 const int ky = ywrap && jt * kr >= (M >> 1) ? 1 : 0;
                 int a0 = 0, a1 = NCH;
-                if (ky != me.ly) {
+                if (ky != me_ly) {
                     a0 = a1 = 0;
                 } else if (xwrap) {
-                    a0 = me.lx ? NCH / 2 : 0;
+                    a0 = me_lx ? NCH / 2 : 0;
                     a1 = a0 + NCH / 2;
                 }
                 uint32_t buf[2][32];
@@ -565,7 +563,10 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
                 }
                 l = l * alpha + (l2.x + l2.y);
                 if (__any_sync(0xffffffffu, rescale)) {
-                    // O must hold every earlier key tile's P V before it is rescaled
+                    // O must hold every earlier key tile's P V before it is
+                    // rescaled; S of this step was issued after P V of step
+                    // n - NB, so for this tile only P V of c - 1 can still be
+                    // in flight
                     if (!warp_wait(&o_done[tile], (c - 1) & 1, abort_flag)) {
                         failed = true;
                         break;
@@ -584,19 +585,19 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
                 }
                 tmem_wait_st();
                 tc_fence_before_sync();
-                mbar_arrive(&p_full[tile]);
+                mbar_arrive(&p_full[n % NB]);
             }
             if (failed)
                 break;
             // ---- epilogue: O / l to the token's original position
-            if (!warp_wait(&o_done[tile], (c - 1) & 1, abort_flag)) {
+            if (!warp_wait(&o_last[tile], kk & 1, abort_flag)) {
                 failed = true;
                 break;
             }
             tc_fence_after_sync();
             const float inv = 1.f / l;
             const float2 i2 = make_float2(inv, inv);
-            uint4 *dst = reinterpret_cast<uint4 *>(out + me.off);
+            uint4 *dst = reinterpret_cast<uint4 *>(out + me.offset);
 #pragma unroll
             for (int ch = 0; ch < D / 16; ++ch) {
                 float o[16];

@@ -225,7 +225,7 @@ bool encode_window_maps(WindowMaps *m, const void *base, const Geometry &g)
            encode_window_map(&m->quarter, base, g, hm, hm);
 }
 
-uint32_t large_smem(const Geometry &g)
+uint32_t large_layout_bytes(const Geometry &g)
 {
     const bool b96 = large_tile_keys(g.M) == 96;
     switch (g.d * 100 + g.rank) {
@@ -237,6 +237,14 @@ uint32_t large_smem(const Geometry &g)
     case 6432: return b96 ? LargeLayout<64, 32, 96>::BYTES : LargeLayout<64, 32, 128>::BYTES;
     }
     return ~0u;
+}
+
+// Dynamic shared memory of a large-kernel launch: its layout, at least 116 KB
+// so that one CTA (holding all of TMEM) is resident per SM.
+uint32_t large_smem(const Geometry &g)
+{
+    const uint32_t need = large_layout_bytes(g);
+    return need > 116u * 1024 ? need : 116u * 1024;
 }
 
 // 4-D K or V box map for the large-window kernel: (d, bw, rows, 1).
@@ -286,7 +294,10 @@ int launch_large(const void *q, const void *k, const void *v, const float *theta
     if (R > 0 && !encode_factor_map(&maps.w, bias, g, BN))
         return WINATTN_ERR_CUDA;
     auto kernel = winattn_fwd_large_kernel<D, R, BN>;
-    const int smem = (int)LargeLayout<D, R, BN>::BYTES;
+    // all 512 TMEM columns per CTA: enough shared memory that no second CTA
+    // is resident on the same SM
+    const int need = (int)LargeLayout<D, R, BN>::BYTES;
+    const int smem = need > 116 * 1024 ? need : 116 * 1024;
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return WINATTN_ERR_CUDA;
     const int64_t items = g.wph * g.heads * (g.N / 256);
