@@ -30,8 +30,11 @@ if ROOT not in sys.path:
 
 METRIC = "window-attn fwd TFLOP/s & tokens/s on 1 B200 vs M; % of roofline"
 L2_BYTES = 126 * 2**20
-KERNEL_SOURCES = ["windowed_attention_vision_b200/csrc/fwd_tc.cuh", "windowed_attention_vision_b200/csrc/ptx.cuh",
-                  "windowed_attention_vision_b200/csrc/geometry.cuh"]
+_CSRC = "windowed_attention_vision_b200/csrc/"
+_COMMON = [_CSRC + "ptx.cuh", _CSRC + "geometry.cuh", _CSRC + "waits.cuh"]
+# kernel id of winattn_launch_info -> (name used in profiles/, source files whose change voids a capture)
+KERNELS = {0: ("tc", [_CSRC + "fwd_tc.cuh"] + _COMMON), 1: ("small", [_CSRC + "fwd_small.cuh"] + _COMMON),
+           2: ("large", [_CSRC + "fwd_large.cuh"] + _COMMON), 3: ("simt", [_CSRC + "fwd_simt.cuh"] + _COMMON)}
 
 
 def parse():
@@ -54,12 +57,21 @@ def cpu_cores() -> int:
         return os.cpu_count() or 1
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(files) -> str:
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
+    for p in files:
         with open(os.path.join(ROOT, p), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
+
+
+def kernel_of(w):
+    """(profile name, source files) of the kernel the library picks for the
+    workload's last call."""
+    from windowed_attention_vision_b200 import _lib
+    dt = _lib.BF16 if w.dtype == "bf16" else _lib.FP32
+    rc, info = _lib.launch_info(w.B, w.H, w.W, w.M, w.shifts[-1], w.heads, w.d, w.rank, dt)
+    return KERNELS.get(info["kernel"], ("unknown", _COMMON)) if rc == 0 else ("unknown", _COMMON)
 
 
 def read_peaks():
@@ -74,16 +86,18 @@ def read_peaks():
         return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
 
 
-def recorded_traffic(workload: str):
-    """DRAM bytes per launch of the attention kernel from the committed ncu
-    summary for this workload, if it was taken on the current kernel source."""
-    path = os.path.join(ROOT, "profiles", f"winattn_fwd_tc_{workload}.md")
+def recorded_traffic(w):
+    """DRAM bytes (read + write) per launch of the workload's kernel from the
+    committed ncu summary ``profiles/winattn_fwd_<kernel>_<workload>.md``, or
+    None when there is none or it was taken on a different kernel source."""
+    name, files = kernel_of(w)
+    path = os.path.join(ROOT, "profiles", f"winattn_fwd_{name}_{w.name}.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
     m_bytes = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
     m_hash = re.search(r"kernel_source_hash:\s*([0-9a-f]+)", text)
-    if not m_bytes or not m_hash or m_hash.group(1) != kernel_source_hash():
+    if not m_bytes or not m_hash or m_hash.group(1) != kernel_source_hash(files):
         return None
     return float(m_bytes.group(1))
 
@@ -216,14 +230,37 @@ def oracle_sample_rate(w, target_s, base=0):
     per_batch = time.perf_counter() - t0
     n = int(min(total_units, max(probe, probe * max(1.0, target_s / max(per_batch, 1e-6)))))
     units = rng.choice(total_units, n, replace=False)
+    # when the whole call is faster than the target, repeat it (at most 100
+    # times) so that the timed CPU work still lasts about target_s
+    reps, dt = 0, 0.0
     t0 = time.perf_counter()
-    orc.fwd_units(*args, units, M=w.M, shift=shift, theta=th, bias=bs, nthreads=cores)
-    dt = time.perf_counter() - t0
+    while reps == 0 or (n == total_units and dt < target_s and reps < 100):
+        orc.fwd_units(*args, units, M=w.M, shift=shift, theta=th, bias=bs, nthreads=cores)
+        reps += 1
+        dt = time.perf_counter() - t0
     calls = len(workload_calls(w))
-    tokens_per_s = w.tokens * (n / total_units) / dt
-    sample = (f"{n} of {total_units} (window, head) units of one {w.name} call (shift {shift}), "
-              f"{dt:.1f} s on {cores} threads, extrapolated by unit count")
+    tokens_per_s = w.tokens * (n / total_units) * reps / dt
+    sample = (f"{n} of {total_units} (window, head) units of one {w.name} call (shift {shift})"
+              + (f", repeated {reps} times" if reps > 1 else "")
+              + f", {dt:.1f} s on {cores} threads, extrapolated by unit count")
     return tokens_per_s, sample, cores, calls
+
+
+def max_over_ranks(values, device):
+    """Element-wise maximum of per-rank timings over all ranks (every rank
+    calls it at the same point; the job is as slow as its slowest rank)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(list(values), device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_tokens_per_s(w, calls_per_step, steps, world, elapsed_ms):
+    """Whole-job throughput: every rank processes its own batch of the
+    workload (weak scaling), so the job handles world times one rank's tokens
+    in the slowest rank's time."""
+    return w.tokens * calls_per_step * steps * world / (elapsed_ms / 1e3)
 
 
 # ----------------------------------------------------------------- reference arm
@@ -326,12 +363,9 @@ def run_ours(args):
     elapsed_ms = start.elapsed_time(end)
     kernel_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
     if world > 1:
-        t = torch.tensor([elapsed_ms, kernel_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms, kernel_ms = t.tolist()
+        elapsed_ms, kernel_ms = max_over_ranks([elapsed_ms, kernel_ms], dev)
 
-    tokens_all = w.tokens * len(calls) * args.steps * world
-    value = tokens_all / (elapsed_ms / 1e3)
+    value = job_tokens_per_s(w, len(calls), args.steps, world, elapsed_ms)
     tflops = w.flops() * len(calls) * args.steps * world / (elapsed_ms / 1e3) / 1e12
 
     # end to end through the C ABI on host buffers (pinned), copies inside the region
@@ -357,9 +391,7 @@ def run_ours(args):
         torch.cuda.synchronize(dev)
         e2e_ms = e0.elapsed_time(e1)
         if world > 1:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = t.item()
+            (e2e_ms,) = max_over_ranks([e2e_ms], dev)
         e2e = {"value": w.tokens * len(calls) * args.e2e_steps * world / (e2e_ms / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": 3 * map_bytes * len(calls), "d2h_bytes_per_step": map_bytes * len(calls),
                "steps": args.e2e_steps, "api": "winattn_fwd_host (C ABI, pinned host buffers)"}
@@ -373,7 +405,7 @@ def run_ours(args):
                                l2=f"inputs larger than L2: {copies} rotating input sets of "
                                   f"{4 * map_bytes / 1e6:.0f} MB (q, k, v, out)"),
                 "tflops": tflops, "kernel_ms_per_launch": kernel_ms, "gpu_launches": args.steps * len(calls),
-                "roofline": roofline(w, kernel_ms / 1e3, peaks, recorded_traffic(w.name)),
+                "roofline": roofline(w, kernel_ms / 1e3, peaks, recorded_traffic(w)),
                 "clocks": clocks.summary(), "e2e": e2e, "device_status": status}
         if world == 1 and not args.no_cpu_baseline:
             rate, sample, cores, _ = oracle_sample_rate(w, args.cpu_seconds)
