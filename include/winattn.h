@@ -144,7 +144,8 @@ int winattn_last_device_status(void *stream);
  * one CTA per SM of a 148-SM B200, capped by the work items), threads per CTA,
  * dynamic shared memory bytes, windows packed per tile and the kernel chosen
  * (0 = generic tensor-core kernel, 1 = persistent small-window kernel,
- * 3 = fp32 SIMT kernel).  Any output pointer may be NULL.  Makes no CUDA
+ * 2 = persistent large-window kernel, 3 = fp32 SIMT kernel, 4 = pipelined
+ * kernel for 8 x 8 windows).  Any output pointer may be NULL.  Makes no CUDA
  * call.  Returns the winattn_check_args code for the sizes (pointers are not
  * checked).
  */

@@ -89,22 +89,26 @@ def test_host_workspace_bytes(lib):
     assert _lib.host_workspace_bytes(0, 16, 16, 2, 32, _lib.BF16) == 0
 
 
-GENERIC, SMALL, LARGE, SIMT = 0, 1, 2, 3
+GENERIC, SMALL, LARGE, SIMT, PIPE = 0, 1, 2, 3, 4
 
 
-@pytest.mark.parametrize("B,H,W,M,heads,d,rank,U,tiles,kernel", [
-    (64, 56, 56, 8, 3, 32, 0, 2, 1, SMALL),      # Swin stage 1: two 64-token windows per tile
-    (16, 128, 128, 32, 3, 32, 0, 1, 8, LARGE),    # 1024-token windows: 8 query tiles each
-    (4, 192, 192, 96, 6, 32, 16, 1, 72, LARGE),   # 9216-token windows
-    (1, 48, 48, 24, 1, 32, 0, 1, 5, GENERIC),     # 576 tokens: no whole-row key tiles
-    (1, 24, 24, 12, 1, 32, 0, 1, 2, GENERIC),     # 144 tokens: a ragged second tile
-    (1, 9, 9, 3, 2, 64, 0, 14, 1, SMALL),         # 9-token windows: 14 per tile
-    (2, 5, 5, 1, 1, 32, 0, 128, 1, SMALL),        # one-token windows
-    (1, 10, 10, 10, 1, 32, 0, 1, 1, SMALL),       # 100 tokens: one ragged tile
-    (1, 8, 8, 8, 80, 32, 0, 2, 1, GENERIC),       # too many heads for the small kernel's RoPE table
+@pytest.mark.parametrize("B,H,W,M,shift,heads,d,rank,U,tiles,kernel", [
+    (64, 56, 56, 8, 4, 3, 32, 0, 2, 1, PIPE),        # Swin stage 1: two 64-token windows per tile
+    (64, 56, 56, 8, 0, 3, 32, 0, 2, 1, PIPE),
+    (4, 32, 32, 8, 4, 4, 64, 0, 2, 1, PIPE),
+    (4, 32, 32, 8, 3, 4, 32, 0, 2, 1, SMALL),        # shift 3: boxes are not whole swizzle atoms
+    (4, 32, 32, 8, 4, 4, 32, 16, 2, 1, SMALL),       # rank-r factors
+    (16, 128, 128, 32, 0, 3, 32, 0, 1, 8, LARGE),    # 1024-token windows: 8 query tiles each
+    (4, 192, 192, 96, 0, 6, 32, 16, 1, 72, LARGE),   # 9216-token windows
+    (1, 48, 48, 24, 0, 1, 32, 0, 1, 5, GENERIC),     # 576 tokens: no whole-row key tiles
+    (1, 24, 24, 12, 0, 1, 32, 0, 1, 2, GENERIC),     # 144 tokens: a ragged second tile
+    (1, 9, 9, 3, 0, 2, 64, 0, 14, 1, SMALL),         # 9-token windows: 14 per tile
+    (2, 5, 5, 1, 0, 1, 32, 0, 128, 1, SMALL),        # one-token windows
+    (1, 10, 10, 10, 0, 1, 32, 0, 1, 1, SMALL),       # 100 tokens: one ragged tile
+    (1, 8, 8, 8, 0, 80, 32, 0, 2, 1, GENERIC),       # too many heads for a shared-memory RoPE table
 ])
-def test_launch_plan(lib, B, H, W, M, heads, d, rank, U, tiles, kernel):
-    rc, info = _lib.launch_info(B, H, W, M, 0, heads, d, rank, _lib.BF16)
+def test_launch_plan(lib, B, H, W, M, shift, heads, d, rank, U, tiles, kernel):
+    rc, info = _lib.launch_info(B, H, W, M, shift, heads, d, rank, _lib.BF16)
     assert rc == _lib.OK
     windows = B * (H // M) * (W // M)
     assert info["windows_per_tile"] == U
@@ -117,6 +121,8 @@ def test_launch_plan(lib, B, H, W, M, heads, d, rank, U, tiles, kernel):
     if kernel == SMALL:
         groups = 4 if d == 32 else 3  # compute warpgroups, plus a loader warp
         assert info["threads"] == (4 * groups + 1) * 32 and info["grid"] == min(148, info["work_items"])
+    elif kernel == PIPE:  # RoPE x3, softmax x2, epilogue warpgroups, loader and two MMA warps
+        assert info["threads"] == 27 * 32 and info["grid"] == min(148, info["work_items"])
     elif kernel == GENERIC:
         assert info["threads"] == 128 and info["grid"] == info["work_items"]
     assert 0 < info["smem_bytes"] <= 227 * 1024

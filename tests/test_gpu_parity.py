@@ -23,6 +23,9 @@ SMALL = [
     ("m8_odd_pack", 1, 24, 8, 8, 3, 1, 32, "bf16", "learned", 0),   # 3 windows: a half-empty pack
     ("m8_odd_pack_tma", 1, 24, 8, 8, 4, 2, 32, "bf16", "learned", 0),  # TMA quadrants + empty slot
     ("m8_s4_d64_tma", 3, 16, 16, 8, 4, 2, 64, "bf16", "learned", 0),
+    ("m8_s0_d64_nope", 1, 16, 16, 8, 0, 3, 64, "bf16", None, 0),
+    ("m8_s4_d32_nope_odd", 5, 24, 40, 8, 4, 3, 32, "bf16", None, 0),  # 75 windows per head: odd packs
+    ("m8_s4_d32_deep", 8, 64, 64, 8, 4, 4, 32, "bf16", "learned", 0),  # many tiles per CTA
     ("m4_s0_tma", 2, 8, 12, 4, 0, 2, 32, "bf16", "learned", 0),      # 8 windows per tile via TMA
     ("m7_s3", 2, 14, 21, 7, 3, 2, 32, "bf16", "learned", 0),        # 49-token windows, 2 per tile
     ("m4_s2", 1, 12, 8, 4, 2, 3, 32, "bf16", "learned", 0),         # 16-token windows, 8 per tile

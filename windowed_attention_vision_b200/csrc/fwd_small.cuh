@@ -51,6 +51,10 @@ struct SmallRoles {
     static constexpr int kLoaderWarp = kGroups * 4;
 };
 
+// Largest RoPE (cos, sin) table the small-window kernel keeps in shared
+// memory: heads * M * (d/4) * 8 bytes.
+constexpr uint32_t kSmallTableMax = 8 * 1024;
+
 template <int D, int R>
 struct SmallLayout {
     static constexpr uint32_t QC = 0;                       // query content  [128][D] bf16, swizzled
@@ -61,8 +65,10 @@ struct SmallLayout {
     static constexpr uint32_t CODES = VO + 256 * D;         // mask code per tile row, u16[128]
     static constexpr uint32_t OFFS = CODES + 256;           // loader's row offsets (cp.async mode), i64[128]
     static constexpr uint32_t STAGE = (OFFS + 128 * 8 + 1023) & ~1023u;
-    static constexpr int NS_FIT = (200 * 1024) / STAGE;
-    static constexpr int NS = NS_FIT < 6 ? NS_FIT : 6;      // ring depth
+    // ring depth: as many stages as fit beside a RoPE table of up to
+    // kSmallTableMax bytes, at most 8
+    static constexpr int NS_FIT = (int)((216u * 1024 - kSmallTableMax) / STAGE);
+    static constexpr int NS = NS_FIT < 8 ? NS_FIT : 8;
     static constexpr int PF = NS - 2 > 2 ? NS - 2 : 2;      // cp.async mode: items issued ahead
     static constexpr uint32_t IJTAB = NS * STAGE;           // TMA row order: (i << 8 | j) u16[4 kinds][64]
     static constexpr uint32_t TABLE = IJTAB + 512;          // RoPE (cos, sin) [heads][M][D/4]
@@ -410,6 +416,8 @@ __global__ void __launch_bounds__(SmallRoles<D>::kThreads, 1)
         const bool aligned = (g.N & 31) == 0;
         // the fast path reads exactly two 32-column chunks: one 64-token window
         const bool two_chunk = aligned && ch_hi - ch_lo == 2;
+        // TMA row order with 64-token windows (M = 8): granule-masked softmax
+        const bool gran = TMA && g.N == 64;
         constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false);
         constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
         bool failed = false;
@@ -422,6 +430,7 @@ __global__ void __launch_bounds__(SmallRoles<D>::kThreads, 1)
             const Item it = decode_item_head_minor(g, first + kc * stride);
             const RowRef rr = tile_row(g, it.pack, 0, row);
             bool wrapped = false;
+            int kind = 0;
             TokenRef tk{};
             int code = 0xFFFE;
             float row_sum = 1.f;
@@ -434,7 +443,7 @@ __global__ void __launch_bounds__(SmallRoles<D>::kThreads, 1)
                         const int b = (int)g.div_img.div((uint32_t)rr.w);
                         const int rem = rr.w - b * g.nWy * g.nWx;
                         const int wy = (int)g.div_nWx.div((uint32_t)rem);
-                        const int kind = window_kind(g, wy, rem - wy * g.nWx);
+                        kind = window_kind(g, wy, rem - wy * g.nWx);
                         const uint32_t ij = ijtab[kind * 64 + rr.p];
                         p = (int)(ij >> 8) * g.M + (int)(ij & 0xFF);
                         wrapped = kind != 0;
@@ -492,9 +501,68 @@ __global__ void __launch_bounds__(SmallRoles<D>::kThreads, 1)
                 const int qcode = rr.valid ? code : 0xFFFF;
                 // Keys need no per-element test when the row's window fills
                 // whole 32-column chunks and is not wrapped.
-                const bool fast = __all_sync(0xffffffffu, two_chunk && rr.valid && !wrapped);
+                const bool fast = !gran && __all_sync(0xffffffffu, two_chunk && rr.valid && !wrapped);
                 float l = 0.f;
-                if (fast) {
+                if (gran) {
+                    // 64-token windows in TMA row order: the boxes of a window
+                    // are its wrap-label regions, so the keys a row may see
+                    // are whole 16-key granules of its own window (all four
+                    // inside, the row's box of two on a seam, its quadrant in
+                    // the corner window).  Masked granules get -inf in the
+                    // exponent instead of a per-key test.
+                    uint32_t gmask = 0u;
+                    if (rr.valid)
+                        gmask = kind == 0 ? 0xFu : (kind == 3 ? 1u << (rr.p >> 4) : ((rr.p >> 5) ? 0xCu : 0x3u));
+                    float x[64];
+                    tmem_ld32(region + ch_lo * 32, x);
+                    tmem_ld32(region + ch_lo * 32 + 32, x + 32);
+                    float gm[4];
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const float *xg = x + 16 * q4;
+                        float a = fmax3(xg[0], xg[1], xg[2]);
+#pragma unroll
+                        for (int e = 3; e < 15; e += 2)
+                            a = fmax3(a, xg[e], xg[e + 1]);
+                        gm[q4] = fmaxf(a, xg[15]);
+                    }
+                    const float ninf = -INFINITY;
+                    const float mx = fmaxf(fmax3((gmask & 1u) ? gm[0] : ninf, (gmask & 2u) ? gm[1] : ninf,
+                                                 (gmask & 4u) ? gm[2] : ninf),
+                                           (gmask & 8u) ? gm[3] : ninf);
+                    const float mneg = mx == ninf ? 0.f : -mx * c2;
+                    const float2 cc = make_float2(c2, c2);
+                    float2 l2 = make_float2(0.f, 0.f);
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const float b = ((gmask >> q4) & 1u) ? mneg : ninf;
+                        const float2 bb = make_float2(b, b);
+#pragma unroll
+                        for (int e = 16 * q4; e < 16 * q4 + 16; e += 2) {
+                            const float2 z = __ffma2_rn(make_float2(x[e], x[e + 1]), cc, bb);
+                            const float2 p = make_float2(fast_exp2(z.x), fast_exp2(z.y));
+                            l2 = __fadd2_rn(l2, p);
+                            pk[e >> 1] = pack_bf16x2(p.x, p.y);
+                        }
+                    }
+                    l = l2.x + l2.y;
+                    uint32_t zero[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        zero[e] = 0u;
+                    if (ch_lo == 0) {
+                        tmem_st16(region + 0, pk);
+                        tmem_st16(region + 16, pk + 16);
+                        tmem_st16(region + 32, zero);
+                        tmem_st16(region + 48, zero);
+                    } else {
+                        tmem_st16(region + 0, zero);
+                        tmem_st16(region + 16, zero);
+                        tmem_st16(region + 32, pk);
+                        tmem_st16(region + 48, pk + 16);
+                    }
+                } else if (fast) {
                     float x[64];
                     tmem_ld32(region + ch_lo * 32, x);
                     tmem_ld32(region + ch_lo * 32 + 32, x + 32);

@@ -12,6 +12,7 @@
 
 #include "../../include/winattn.h"
 #include "fwd_large.cuh"
+#include "fwd_pipe.cuh"
 #include "fwd_simt.cuh"
 #include "fwd_small.cuh"
 #include "fwd_tc.cuh"
@@ -87,9 +88,13 @@ int smem_bytes_for(const Geometry &g, int dtype)
 
 constexpr int kAssumedSMs = 148;          // B200; used only by winattn_launch_info
 constexpr uint32_t kMaxSmem = 227 * 1024;
-constexpr uint32_t kMaxSmallTable = 32 * 1024;
 
-enum KernelKind { kGeneric = 0, kSmall = 1, kLarge = 2, kSimt = 3 };
+enum KernelKind { kGeneric = 0, kSmall = 1, kLarge = 2, kSimt = 3, kPipe = 4 };
+
+uint32_t pipe_smem(const Geometry &g)
+{
+    return g.d == 32 ? PipeLayout<32>::bytes(g.heads) : PipeLayout<64>::bytes(g.heads);
+}
 
 uint32_t small_smem(const Geometry &g)
 {
@@ -111,7 +116,9 @@ KernelKind choose_kernel(const Geometry &g, int dtype)
 {
     if (dtype == WINATTN_FP32)
         return kSimt;
-    if (g.N <= kTileRows && (uint64_t)g.heads * g.M * (g.d / 4) * 8 <= kMaxSmallTable && small_smem(g) <= kMaxSmem)
+    if (pipe_ok(g) && (uint64_t)g.heads * g.M * (g.d / 4) * 8 <= kSmallTableMax && pipe_smem(g) <= kMaxSmem)
+        return kPipe;
+    if (g.N <= kTileRows && (uint64_t)g.heads * g.M * (g.d / 4) * 8 <= kSmallTableMax && small_smem(g) <= kMaxSmem)
         return kSmall;
     if (large_ok(g))
         return kLarge;
@@ -354,6 +361,26 @@ int launch_small(const void *q, const void *k, const void *v, const float *theta
     return launch_small_variant<D, R, false>(q, k, v, theta, bias, out, g, stream, maps);
 }
 
+template <int D>
+int launch_pipe(const void *q, const void *k, const void *v, const float *theta, void *out, const Geometry &g,
+                cudaStream_t stream)
+{
+    WindowMaps maps[3];
+    std::memset(maps, 0, sizeof maps);
+    if (!encode_window_maps(&maps[0], q, g) || !encode_window_maps(&maps[1], k, g) ||
+        !encode_window_maps(&maps[2], v, g))
+        return WINATTN_ERR_CUDA;
+    auto kernel = winattn_fwd_pipe_kernel<D>;
+    const int smem = (int)PipeLayout<D>::bytes(g.heads);
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return WINATTN_ERR_CUDA;
+    const int64_t grid = g.items < sm_count() ? g.items : sm_count();
+    kernel<<<(unsigned)grid, kPipeThreads, smem, stream>>>(theta, static_cast<__nv_bfloat16 *>(out), g,
+                                                           1.0f / std::sqrt((float)g.d), maps[0], maps[1],
+                                                           maps[2]);
+    return cudaGetLastError() == cudaSuccess ? WINATTN_OK : WINATTN_ERR_CUDA;
+}
+
 template <int D, int R>
 int launch_simt(const void *q, const void *k, const void *v, const float *theta, const void *bias, void *out,
                 const Geometry &g, cudaStream_t stream)
@@ -367,6 +394,8 @@ int dispatch(const void *q, const void *k, const void *v, const float *theta, co
              const Geometry &g, int dtype, cudaStream_t s)
 {
     const KernelKind kind = choose_kernel(g, dtype);
+    if (kind == kPipe)
+        return g.d == 32 ? launch_pipe<32>(q, k, v, theta, out, g, s) : launch_pipe<64>(q, k, v, theta, out, g, s);
     if (kind == kSmall) {
         switch (g.d * 100 + g.rank) {
         case 3200: return launch_small<32, 0>(q, k, v, theta, bias, out, g, s);
@@ -548,6 +577,10 @@ int winattn_launch_info(int B, int H_img, int W_img, int M, int shift, int heads
         if (grid) *grid = (int)(items < kAssumedSMs ? items : kAssumedSMs);
         if (threads) *threads = kLargeThreads;
         if (smem_bytes) *smem_bytes = (int)large_smem(g);
+    } else if (kind == kPipe) {
+        if (grid) *grid = (int)(g.items < kAssumedSMs ? g.items : kAssumedSMs);
+        if (threads) *threads = kPipeThreads;
+        if (smem_bytes) *smem_bytes = (int)pipe_smem(g);
     } else if (kind == kSmall) {
         if (grid) *grid = (int)(g.items < kAssumedSMs ? g.items : kAssumedSMs);
         if (threads) *threads = g.d <= 32 ? SmallRoles<32>::kThreads : SmallRoles<64>::kThreads;
