@@ -7,23 +7,23 @@
 // so that the latencies of one (TMA arrivals, tcgen05 round trips, the long
 // per-row RoPE and softmax chains) hide behind the others:
 //
-//   warp 24       TMA loader: each window's Q, K, V head slice as one box
+//   warp 20       TMA loader: each window's Q, K, V head slice as one box
 //                 (interior), two (a seam's row or column) or four (corner)
 //                 boxes straight into the swizzled operand tiles of an
 //                 NS-stage ring;
-//   warps 0-11    three RoPE warpgroups, tiles in turn: a thread owns one
+//   warps 0-7     two RoPE warpgroups, alternate tiles: a thread owns one
 //                 tile row: it resolves the row's token (window-local (i, j)
 //                 in box order, original position, wrap-label granules) and
 //                 rotates its Q and K rows in place in fp32;
-//   warps 25, 26  MMA issuers: S = Q K^T of each tile into TMEM buffer
+//   warps 21, 22  MMA issuers: S = Q K^T of each tile into TMEM buffer
 //                 k % 4 as soon as its RoPE is done and the buffer is free
 //                 (up to four tiles ahead); O = P V as soon as its P is
 //                 written.  Each issuer sleeps in bounded mbarrier waits, so
 //                 neither spins on the issue slots the other roles need;
-//   warps 12-19   two softmax warpgroups, alternate tiles: max / exp2 / sum
+//   warps 8-15    two softmax warpgroups, alternate tiles: max / exp2 / sum
 //                 of a row over its own window's allowed keys, P (bf16 pairs)
 //                 written over the consumed S columns;
-//   warps 20-23   epilogue: O / l of each row stored (16-byte stores) to the
+//   warps 16-19   epilogue: O / l of each row stored (16-byte stores) to the
 //                 token's original, un-shifted position.
 //
 // TMEM: four buffers of 128 columns: S (fp32), P over its first 64 columns,
@@ -45,7 +45,7 @@
 
 namespace winattn {
 
-constexpr int kPipeRope = 3;                    // RoPE warpgroups (tile k goes to group k % 3)
+constexpr int kPipeRope = 2;                    // RoPE warpgroups (tile k goes to group k % 2)
 constexpr int kPipeSoftmaxWarp = 4 * kPipeRope; // first softmax warp
 constexpr int kPipeEpiWarp = kPipeSoftmaxWarp + 8;
 constexpr int kPipeLoadWarp = kPipeEpiWarp + 4;
@@ -86,6 +86,13 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     using L = PipeLayout<D>;
     constexpr int NS = L::NS, NB = kPipeBufs;
     static_assert(NS >= 3, "ring too shallow");
+    // mbarrier waits test a phase's parity only, so a waiter must never reach
+    // phase u + 2 of a barrier before phase u has completed: tiles k and
+    // k + NS share ring stage s, and the same RoPE group (which takes them in
+    // order) must wait for both; likewise tiles k and k + NB share a TMEM
+    // buffer and must fall to the same softmax group.
+    static_assert(NS % kPipeRope == 0, "a ring stage must always be consumed by the same RoPE group");
+    static_assert(NB % 2 == 0, "a TMEM buffer must always be consumed by the same softmax group");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(base);

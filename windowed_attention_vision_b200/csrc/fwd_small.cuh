@@ -68,7 +68,12 @@ struct SmallLayout {
     // ring depth: as many stages as fit beside a RoPE table of up to
     // kSmallTableMax bytes, at most 8
     static constexpr int NS_FIT = (int)((216u * 1024 - kSmallTableMax) / STAGE);
-    static constexpr int NS = NS_FIT < 8 ? NS_FIT : 8;
+    // a whole number of rounds of the compute groups, so that tiles k and
+    // k + NS (which share a stage) fall to the same group: mbarrier waits
+    // test a phase's parity only, and a group must not reach a stage's next
+    // phase while an earlier phase is still pending for another group
+    static constexpr int NS_CAP = NS_FIT < 8 ? NS_FIT : 8;
+    static constexpr int NS = NS_CAP - NS_CAP % SmallRoles<D>::kGroups;
     static constexpr int PF = NS - 2 > 2 ? NS - 2 : 2;      // cp.async mode: items issued ahead
     static constexpr uint32_t IJTAB = NS * STAGE;           // TMA row order: (i << 8 | j) u16[4 kinds][64]
     static constexpr uint32_t TABLE = IJTAB + 512;          // RoPE (cos, sin) [heads][M][D/4]
@@ -221,6 +226,7 @@ __global__ void __launch_bounds__(SmallRoles<D>::kThreads, 1)
     constexpr int NS = L::NS, PF = L::PF, NW = SmallRoles<D>::kGroups;
     constexpr int kLoaderWarp = SmallRoles<D>::kLoaderWarp;
     static_assert(NS >= 3, "ring too shallow");
+    static_assert(NS % NW == 0, "a ring stage must always be consumed by the same compute group");
     static_assert(!TMA || R == 0, "TMA loads carry no rank-r factors");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);

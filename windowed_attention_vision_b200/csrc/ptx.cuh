@@ -90,13 +90,16 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar)
 // Every wait in this library is bounded: it gives up after kWaitLimitNs of
 // wall time (read from %globaltimer) and reports false.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Longest a thread stays suspended in one try_wait before it re-checks the
+// time limit and the abort flag (it wakes as soon as the phase completes).
+constexpr uint32_t kSuspendHintNs = 1000000u;
 
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
 {
-    if (mbar_try_wait(bar, parity))
+    if (mbar_try_wait_sleep(bar, parity, kSuspendHintNs))
         return true;
     const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait_sleep(bar, parity, 100000u)) {
+    while (!mbar_try_wait_sleep(bar, parity, kSuspendHintNs)) {
         if (globaltimer_ns() - t0 > kWaitLimitNs)
             return false;
     }

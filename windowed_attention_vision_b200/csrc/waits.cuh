@@ -8,13 +8,16 @@
 
 namespace winattn {
 
-// Bounded wait that also gives up as soon as another role has aborted.
+// Bounded wait that also gives up as soon as another role has aborted.  The
+// try_wait carries a suspend-time hint, so a waiting thread sleeps in
+// hardware until the phase completes (or the hint runs out) instead of
+// polling: a polling warp takes issue slots from the warps doing the work.
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile uint32_t *abort_flag)
 {
-    if (mbar_try_wait(bar, parity))
+    if (mbar_try_wait_sleep(bar, parity, kSuspendHintNs))
         return true;
     const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait_sleep(bar, parity, 100000u)) {
+    while (!mbar_try_wait_sleep(bar, parity, kSuspendHintNs)) {
         if (*abort_flag)
             return false;
         if (globaltimer_ns() - t0 > kWaitLimitNs) {
