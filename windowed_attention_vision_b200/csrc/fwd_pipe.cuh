@@ -3,37 +3,40 @@
 // Swin's stage-1 shape at patch 4 ("FLASHSWIN" page, section "무엇과
 // 다른가"), where the fused kernel has to run at memory speed.
 //
-// Every tile passes five roles, each working on a different tile at a time,
+// Every tile passes six roles, each working on a different tile at a time,
 // so that the latencies of one (TMA arrivals, tcgen05 round trips, the long
 // per-row RoPE and softmax chains) hide behind the others:
 //
-//   warp 20       TMA loader: each window's Q, K, V head slice as one box
+//   warp 20       Q/K loader: each window's Q and K head slices as one box
 //                 (interior), two (a seam's row or column) or four (corner)
 //                 boxes straight into the swizzled operand tiles of an
-//                 NS-stage ring;
+//                 NSQ-stage ring;
+//   warp 23       V loader: the same boxes of V into an NSV-stage ring, issued
+//                 once the tile's RoPE is done, so that V arrives about when
+//                 P V needs it instead of occupying shared memory through the
+//                 whole pipeline;
 //   warps 0-7     two RoPE warpgroups, alternate tiles: a thread owns one
 //                 tile row: it resolves the row's token (window-local (i, j)
 //                 in box order, original position, wrap-label granules) and
 //                 rotates its Q and K rows in place in fp32;
 //   warps 21, 22  MMA issuers: S = Q K^T of each tile into TMEM buffer
 //                 k % 4 as soon as its RoPE is done and the buffer is free
-//                 (up to four tiles ahead); O = P V as soon as its P is
-//                 written.  Each issuer sleeps in bounded mbarrier waits, so
-//                 neither spins on the issue slots the other roles need;
+//                 (the commit also frees the tile's Q/K stage); O = P V as
+//                 soon as its P is written and its V has landed (the commit
+//                 frees the V stage).  Each issuer sleeps in bounded mbarrier
+//                 waits, so neither spins on the issue slots others need;
 //   warps 8-15    two softmax warpgroups, alternate tiles: max / exp2 / sum
 //                 of a row over its own window's allowed keys, P (bf16 pairs)
 //                 written over the consumed S columns;
-//   warps 16-19   epilogue: O / l of each row stored (16-byte stores) to the
-//                 token's original, un-shifted position.
+//   warps 16-19   epilogue: O / l of each row, as bf16, into a staging tile
+//                 written back with TMA stores of the same boxes the loaders
+//                 read: the token's original, un-shifted position.
 //
-// TMEM: four buffers of 128 columns: S (fp32), P over its first 64 columns,
-// O over columns [64, 64 + d).  Wrap masks need no per-key test: the boxes
-// of a window are exactly its wrap-label regions, so a row may see whole
-// 16-key granules of its own window (all four inside, the row's box of two
-// on a seam, its quadrant in the corner window); masked granules get -inf
-// in the exponent.
-// Every wait is bounded; a timeout sets the CTA's abort flag and the device
-// status word, and every role leaves its loop at its next wait.
+// The rate is bounded by how long a tile holds shared memory: the rings must
+// cover the DRAM latency plus the processing latency of the tiles in flight,
+// so Q/K (needed until S) and V (needed from P V only) have rings of their
+// own.  Per-row metadata (wrap-label granules) lives in a ring of its own
+// that outlasts the Q/K stage.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -48,24 +51,30 @@ namespace winattn {
 constexpr int kPipeRope = 2;                    // RoPE warpgroups (tile k goes to group k % 2)
 constexpr int kPipeSoftmaxWarp = 4 * kPipeRope; // first softmax warp
 constexpr int kPipeEpiWarp = kPipeSoftmaxWarp + 8;
-constexpr int kPipeLoadWarp = kPipeEpiWarp + 4;
-constexpr int kPipeThreads = (kPipeLoadWarp + 3) * 32;
+constexpr int kPipeLoadWarp = kPipeEpiWarp + 4; // Q/K loader; S issuer, P V issuer and V loader follow
+constexpr int kPipeThreads = (kPipeLoadWarp + 4) * 32;
 constexpr int kPipeBufs = 4;  // TMEM buffers (tiles between S and the epilogue)
 
 template <int D>
 struct PipeLayout {
-    static constexpr uint32_t QC = 0;                 // query content [128][D] bf16, swizzled
-    static constexpr uint32_t KC = QC + 256 * D;      // key content
-    static constexpr uint32_t VO = KC + 256 * D;      // values
-    static constexpr uint32_t META = VO + 256 * D;    // per row: original offset | granule mask, i64[128]
-    static constexpr uint32_t STAGE = (META + 128 * 8 + 1023) & ~1023u;
-    static constexpr int NS_FIT = (int)((208u * 1024 - kSmallTableMax) / STAGE);
-    static constexpr int NS = NS_FIT < 8 ? NS_FIT : 8;
-    static constexpr uint32_t OMETA = NS * STAGE;                   // per TMEM buffer: row meta, i64[4][128]
-    static constexpr uint32_t OSUM = OMETA + kPipeBufs * 128 * 8;   // per TMEM buffer: row sum l, f32[4][128]
+    // Q/K ring: query and key content [128][D] bf16 each, swizzled
+    static constexpr uint32_t QC = 0, KC = 256 * D;
+    static constexpr uint32_t QK_STAGE = 512 * D;
+    static constexpr int NSQ = D == 32 ? 8 : 4;
+    // V ring: values [128][D]
+    static constexpr uint32_t V_STAGE = 256 * D;
+    static constexpr int NSV = D == 32 ? 6 : 3;
+    // row metadata ring: original element offset | granule mask, i64[128]
+    static constexpr int NM = NSQ + kPipeBufs;
+    static constexpr uint32_t VRING = NSQ * QK_STAGE;
+    static constexpr uint32_t MRING = VRING + NSV * V_STAGE;
+    // output staging for the TMA stores: [128][D] bf16, swizzled like the operands
+    static constexpr int NO = D == 32 ? 2 : 1;
+    static constexpr uint32_t OSTAGE = MRING + NM * 1024;
+    static constexpr uint32_t OSUM = OSTAGE + NO * 256 * D;         // per TMEM buffer: row sum l, f32[4][128]
     static constexpr uint32_t IJTAB = OSUM + kPipeBufs * 128 * 4;   // box row order: (i << 8 | j) u16[4][64]
     static constexpr uint32_t TABLE = IJTAB + 512;                  // RoPE (cos, sin) float4 [heads][8][D/8]
-    static constexpr int kBars = 3 * NS + 4 * kPipeBufs + 2;
+    static constexpr int kBars = 3 * NSQ + 2 * NSV + NM + 4 * kPipeBufs + 2;
     static __host__ __device__ uint32_t bars(int heads) { return TABLE + ((heads * 8 * (D / 4) * 8 + 15) & ~15u); }
     static __host__ __device__ uint32_t bytes(int heads) { return bars(heads) + kBars * 8 + 16 + 1024; }
 };
@@ -81,28 +90,31 @@ template <int D>
 __global__ void __launch_bounds__(kPipeThreads, 1)
     winattn_fwd_pipe_kernel(const float *__restrict__ theta, __nv_bfloat16 *__restrict__ out, const Geometry g,
                             const float scale, const __grid_constant__ WindowMaps tm_q,
-                            const __grid_constant__ WindowMaps tm_k, const __grid_constant__ WindowMaps tm_v)
+                            const __grid_constant__ WindowMaps tm_k, const __grid_constant__ WindowMaps tm_v,
+                            const __grid_constant__ WindowMaps tm_o)
 {
     using L = PipeLayout<D>;
-    constexpr int NS = L::NS, NB = kPipeBufs;
-    static_assert(NS >= 3, "ring too shallow");
+    constexpr int NSQ = L::NSQ, NSV = L::NSV, NM = L::NM, NB = kPipeBufs;
+    static_assert(NSQ >= 3 && NSV >= 2, "rings too shallow");
     // mbarrier waits test a phase's parity only, so a waiter must never reach
-    // phase u + 2 of a barrier before phase u has completed: tiles k and
-    // k + NS share ring stage s, and the same RoPE group (which takes them in
-    // order) must wait for both; likewise tiles k and k + NB share a TMEM
-    // buffer and must fall to the same softmax group.
-    static_assert(NS % kPipeRope == 0, "a ring stage must always be consumed by the same RoPE group");
-    static_assert(NB % 2 == 0, "a TMEM buffer must always be consumed by the same softmax group");
+    // phase u + 2 of a barrier while phase u is still pending.  Tiles k and
+    // k + NSQ share a Q/K stage and must fall to the same RoPE group (which
+    // takes them in order); tiles k and k + NM share a metadata slot and must
+    // fall to the same softmax group.  NM = NSQ + NB also orders the metadata
+    // writer of tile k + NM after the last reader of tile k (S of tile
+    // k + NB needs tile k's TMEM buffer back from the epilogue).
+    static_assert(NSQ % kPipeRope == 0, "a Q/K stage must always be consumed by the same RoPE group");
+    static_assert(NM % 2 == 0 && NM == NSQ + NB, "metadata ring must order its writers after its readers");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(base);
     uint16_t *ijtab = reinterpret_cast<uint16_t *>(base + L::IJTAB);
     float2 *table = reinterpret_cast<float2 *>(base + L::TABLE);
-    int64_t *ometa = reinterpret_cast<int64_t *>(base + L::OMETA);
     float *osum = reinterpret_cast<float *>(base + L::OSUM);
     uint64_t *bars = reinterpret_cast<uint64_t *>(base + L::bars(g.heads));
-    uint64_t *full = bars, *ready = bars + NS, *empty = bars + 2 * NS;
-    uint64_t *s_full = bars + 3 * NS, *p_full = s_full + NB, *o_full = p_full + NB, *t_free = o_full + NB;
+    uint64_t *qk_full = bars, *ready = qk_full + NSQ, *qk_empty = ready + NSQ;
+    uint64_t *v_full = qk_empty + NSQ, *v_empty = v_full + NSV, *meta_full = v_empty + NSV;
+    uint64_t *s_full = meta_full + NM, *p_full = s_full + NB, *o_full = p_full + NB, *t_free = o_full + NB;
     uint64_t *fin = t_free + NB;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + L::kBars);
     volatile uint32_t *abort_flag = tslot + 1;
@@ -111,18 +123,24 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     const int n_items = (int)g.items;
     const int first = blockIdx.x, stride = gridDim.x;
     const int count = first < n_items ? (n_items - 1 - first) / stride + 1 : 0;
-    constexpr int kTab = 8 * (D / 4);  // table floats-pairs per head: 8 positions x D/4 frequencies
+    constexpr int kTab = 8 * (D / 4);  // table float pairs per head: 8 positions x D/4 frequencies
 
     if (warp == 0) {
         tmem_alloc(tslot, 512);
         tmem_relinquish();
     }
     if (t == 32) {
-        for (int s = 0; s < NS; ++s) {
-            mbar_init(&full[s], 1);
+        for (int s = 0; s < NSQ; ++s) {
+            mbar_init(&qk_full[s], 1);
             mbar_init(&ready[s], 128);
-            mbar_init(&empty[s], 1);
+            mbar_init(&qk_empty[s], 1);
         }
+        for (int s = 0; s < NSV; ++s) {
+            mbar_init(&v_full[s], 1);
+            mbar_init(&v_empty[s], 1);
+        }
+        for (int m = 0; m < NM; ++m)
+            mbar_init(&meta_full[m], 128);
         for (int b = 0; b < NB; ++b) {
             mbar_init(&s_full[b], 1);
             mbar_init(&p_full[b], 128);
@@ -158,71 +176,126 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     tc_fence_after_sync();
     const uint32_t tmem = *tslot;
 
+    // The boxes of tile k, one per loader lane (window slot, box): the
+    // rolled-window origin of the box, its original coordinates and its row
+    // offset in the operand tile.
+    struct Box {
+        bool go;
+        int kind, c0, x0, y0, b;
+        uint32_t roff;
+    };
+    auto box_of = [&](const Item &it, int nvalid) -> Box {
+        Box r{};
+        r.go = false;
+        const int my_slot = lane >> 2, my_box = lane & 3;
+        if (my_slot >= nvalid)
+            return r;
+        const int w = it.pack * 2 + my_slot;
+        r.b = (int)g.div_img.div((uint32_t)w);
+        const int rem = w - r.b * g.nWy * g.nWx;
+        const int wy = (int)g.div_nWx.div((uint32_t)rem);
+        const int wx = rem - wy * g.nWx;
+        r.kind = window_kind(g, wy, wx);
+        const int nbox = r.kind == 3 ? 4 : (r.kind ? 2 : 1);
+        if (my_box >= nbox)
+            return r;
+        const int bi = my_box;
+        const int iy0 = (r.kind & 2) ? ((r.kind == 3 ? bi >> 1 : bi) * 4) : 0;
+        const int jx0 = (r.kind & 1) ? ((r.kind == 3 ? bi & 1 : bi) * 4) : 0;
+        r.y0 = wy * 8 + iy0 + g.shift;
+        if (r.y0 >= g.H) r.y0 -= g.H;
+        r.x0 = wx * 8 + jx0 + g.shift;
+        if (r.x0 >= g.W) r.x0 -= g.W;
+        r.roff = (uint32_t)((my_slot * 64 + bi * (64 / nbox)) * 2 * D);
+        r.c0 = it.h * D;
+        r.go = true;
+        return r;
+    };
+    auto valid_windows = [&](const Item &it) -> int {
+        const int64_t left = g.wph - (int64_t)it.pack * 2;
+        return left < 2 ? (int)left : 2;
+    };
+
     if (warp == kPipeLoadWarp) {
-        // ================================================================ TMA loader
+        // ================================================================ Q/K loader
         if (lane == 0) {
             for (int kind = 0; kind < 4; ++kind) {
                 tma_prefetch_map(pick_map(tm_q, kind));
                 tma_prefetch_map(pick_map(tm_k, kind));
-                tma_prefetch_map(pick_map(tm_v, kind));
+                tma_prefetch_map(pick_map(tm_o, kind));
             }
         }
-        const int my_slot = lane >> 2, my_box = lane & 3;
         for (int kk = 0; kk < count; ++kk) {
-            const int s = kk % NS;
-            if (kk >= NS && !warp_wait(&empty[s], ((kk / NS) - 1) & 1, abort_flag))
+            const int s = kk % NSQ;
+            if (kk >= NSQ && !warp_wait(&qk_empty[s], ((kk / NSQ) - 1) & 1, abort_flag))
                 break;
             const Item it = decode_item_head_minor(g, first + kk * stride);
-            const uint32_t sst = sbase + s * L::STAGE;
-            const int64_t left = g.wph - (int64_t)it.pack * 2;
-            const int nvalid = left < 2 ? (int)left : 2;
+            const int nvalid = valid_windows(it);
+            const uint32_t sst = sbase + s * L::QK_STAGE;
             if (lane == 0)
-                mbar_arrive_expect_tx(&full[s], (uint32_t)(3 * nvalid * 64 * 2 * D));
+                mbar_arrive_expect_tx(&qk_full[s], (uint32_t)(2 * nvalid * 64 * 2 * D));
             __syncwarp();
-            if (my_slot < nvalid) {
-                const int w = it.pack * 2 + my_slot;
-                const int b = (int)g.div_img.div((uint32_t)w);
-                const int rem = w - b * g.nWy * g.nWx;
-                const int wy = (int)g.div_nWx.div((uint32_t)rem);
-                const int wx = rem - wy * g.nWx;
-                const int kind = window_kind(g, wy, wx);
-                const int nbox = kind == 3 ? 4 : (kind ? 2 : 1);
-                if (my_box < nbox) {
-                    const int bi = my_box;
-                    const int iy0 = (kind & 2) ? ((kind == 3 ? bi >> 1 : bi) * 4) : 0;
-                    const int jx0 = (kind & 1) ? ((kind == 3 ? bi & 1 : bi) * 4) : 0;
-                    int y0 = wy * 8 + iy0 + g.shift;
-                    if (y0 >= g.H) y0 -= g.H;
-                    int x0 = wx * 8 + jx0 + g.shift;
-                    if (x0 >= g.W) x0 -= g.W;
-                    const uint32_t roff = (uint32_t)((my_slot * 64 + bi * (64 / nbox)) * 2 * D);
-                    const int c0 = it.h * D;
-                    tma_load_4d(sst + L::QC + roff, pick_map(tm_q, kind), c0, x0, y0, b, &full[s]);
-                    tma_load_4d(sst + L::KC + roff, pick_map(tm_k, kind), c0, x0, y0, b, &full[s]);
-                    tma_load_4d(sst + L::VO + roff, pick_map(tm_v, kind), c0, x0, y0, b, &full[s]);
-                }
+            const Box r = box_of(it, nvalid);
+            if (r.go) {
+                tma_load_4d(sst + L::QC + r.roff, pick_map(tm_q, r.kind), r.c0, r.x0, r.y0, r.b, &qk_full[s]);
+                tma_load_4d(sst + L::KC + r.roff, pick_map(tm_k, r.kind), r.c0, r.x0, r.y0, r.b, &qk_full[s]);
             }
+        }
+    } else if (warp == kPipeLoadWarp + 3) {
+        // ================================================================ V loader
+        if (lane == 0) {
+            for (int kind = 0; kind < 4; ++kind)
+                tma_prefetch_map(pick_map(tm_v, kind));
+        }
+        for (int kk = 0; kk < count; ++kk) {
+            const int s = kk % NSV;
+            // once the tile's RoPE is done, V has about the S and softmax
+            // time to arrive before P V needs it
+            if (!warp_wait(&meta_full[kk % NM], (kk / NM) & 1, abort_flag))
+                break;
+            if (kk >= NSV && !warp_wait(&v_empty[s], ((kk / NSV) - 1) & 1, abort_flag))
+                break;
+            const Item it = decode_item_head_minor(g, first + kk * stride);
+            const int nvalid = valid_windows(it);
+            const uint32_t sst = sbase + L::VRING + s * L::V_STAGE;
+            if (nvalid < 2) {
+                // the empty second slot of the last pack: zero value rows (its
+                // P is zero, so they only have to be finite)
+                uint4 *z = reinterpret_cast<uint4 *>(base + L::VRING + s * L::V_STAGE + 64 * 2 * D);
+                for (int c = lane; c < 64 * 2 * D / 16; c += 32)
+                    z[c] = make_uint4(0, 0, 0, 0);
+                fence_proxy_async_smem();
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive_expect_tx(&v_full[s], (uint32_t)(nvalid * 64 * 2 * D));
+            __syncwarp();
+            const Box r = box_of(it, nvalid);
+            if (r.go)
+                tma_load_4d(sst + r.roff, pick_map(tm_v, r.kind), r.c0, r.x0, r.y0, r.b, &v_full[s]);
         }
     } else if (warp == kPipeLoadWarp + 1) {
         // ================================================================ S issuer
         // S = Q K^T of each tile into TMEM buffer k % 4 as soon as its RoPE is
-        // done and the buffer's previous tile has left the epilogue.
+        // done and the buffer's previous tile has left the epilogue; the
+        // commit also hands the Q/K stage back to its loader.
         if (lane == 0) {
             constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false);
             int kk = 0;
             for (; kk < count; ++kk) {
-                const int s = kk % NS, b = kk % NB;
-                if (!wait_or_abort(&ready[s], (kk / NS) & 1, abort_flag))
+                const int s = kk % NSQ, b = kk % NB;
+                if (!wait_or_abort(&ready[s], (kk / NSQ) & 1, abort_flag))
                     break;
                 if (kk >= NB && !wait_or_abort(&t_free[b], ((kk / NB) - 1) & 1, abort_flag))
                     break;
                 tc_fence_after_sync();
-                const uint32_t sst = sbase + s * L::STAGE;
+                const uint32_t sst = sbase + s * L::QK_STAGE;
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks)
                     umma_bf16_ss(tmem + b * 128, smem_desc(sst + L::QC + ks * 32, 16, 16 * D, swizzle_code(2 * D)),
                                  smem_desc(sst + L::KC + ks * 32, 16, 16 * D, swizzle_code(2 * D)), kIdescS, ks > 0);
                 umma_commit(&s_full[b]);
+                umma_commit(&qk_empty[s]);
             }
             if (kk > 0) {
                 umma_commit(&fin[0]);
@@ -231,23 +304,25 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         }
     } else if (warp == kPipeLoadWarp + 2) {
         // ================================================================ P V issuer
-        // O = P V of each tile as soon as its P is written; the commit also
-        // hands the tile's ring stage back to the loader.
+        // O = P V of each tile once its P is written and its V has landed;
+        // the commit also hands the V stage back to its loader.
         if (lane == 0) {
             constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
             int kk = 0;
             for (; kk < count; ++kk) {
-                const int s = kk % NS, b = kk % NB;
+                const int s = kk % NSV, b = kk % NB;
                 if (!wait_or_abort(&p_full[b], (kk / NB) & 1, abort_flag))
                     break;
+                if (!wait_or_abort(&v_full[s], (kk / NSV) & 1, abort_flag))
+                    break;
                 tc_fence_after_sync();
-                const uint32_t vst = sbase + s * L::STAGE + L::VO;
+                const uint32_t vst = sbase + L::VRING + s * L::V_STAGE;
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
                     umma_bf16_ts(tmem + b * 128 + 64, tmem + b * 128 + ks * 8,
                                  smem_desc(vst + ks * 32 * D, 8192, 16 * D, swizzle_code(2 * D)), kIdescPV, ks > 0);
                 umma_commit(&o_full[b]);
-                umma_commit(&empty[s]);
+                umma_commit(&v_empty[s]);
             }
             if (kk > 0) {
                 umma_commit(&fin[1]);
@@ -260,13 +335,13 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         const int row = t - 128 * grp;
         const int slot = row >> 6, rp = row & 63;
         for (int kk = grp; kk < count; kk += kPipeRope) {
-            const int s = kk % NS;
-            if (!warp_wait(&full[s], (kk / NS) & 1, abort_flag))
+            const int s = kk % NSQ, m = kk % NM;
+            if (!warp_wait(&qk_full[s], (kk / NSQ) & 1, abort_flag))
                 break;
-            uint8_t *st = base + s * L::STAGE;
+            uint8_t *st = base + s * L::QK_STAGE;
             const Item it = decode_item_head_minor(g, first + kk * stride);
             const int w = it.pack * 2 + slot;
-            int64_t meta = -1;
+            int64_t meta = -1;  // allowed 16-key granules of the row's window, -1 for no token
             if (w < g.wph) {
                 const int b = (int)g.div_img.div((uint32_t)w);
                 const int rem = w - b * g.nWy * g.nWx;
@@ -275,30 +350,24 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
                 const int kind = window_kind(g, wy, wx);
                 const uint32_t ij = ijtab[kind * 64 + rp];
                 const int i = (int)(ij >> 8), j = (int)(ij & 0xFF);
-                int y = wy * 8 + i + g.shift;
-                if (y >= g.H) y -= g.H;
-                int x = wx * 8 + j + g.shift;
-                if (x >= g.W) x -= g.W;
-                const int64_t off = ((((int64_t)b * g.H + y) * g.W + x) * g.heads + it.h) * D;
-                const uint32_t gmask = kind == 0 ? 0xFu : (kind == 3 ? 1u << (rp >> 4) : ((rp >> 5) ? 0xCu : 0x3u));
-                meta = off | (int64_t)gmask;
+                meta = kind == 0 ? 0xF : (kind == 3 ? 1 << (rp >> 4) : ((rp >> 5) ? 0xC : 0x3));
                 if (theta)
                     rotate_qk_rows<D>(st + L::QC, st + L::KC, row,
                                       reinterpret_cast<const float4 *>(table + it.h * kTab), i, j, false, 1.f);
             } else {
-                // an empty slot of the last pack: zero rows keep its keys and
-                // values finite (their P is zero)
+                // an empty slot of the last pack: zero rows keep its keys finite
+                // (their P is zero)
 #pragma unroll
                 for (int c = 0; c < D / 8; ++c) {
                     const uint32_t off = swz_offset(row, c, 2 * D);
                     *reinterpret_cast<uint4 *>(st + L::QC + off) = make_uint4(0, 0, 0, 0);
                     *reinterpret_cast<uint4 *>(st + L::KC + off) = make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4 *>(st + L::VO + off) = make_uint4(0, 0, 0, 0);
                 }
             }
-            reinterpret_cast<int64_t *>(st + L::META)[row] = meta;
+            reinterpret_cast<int64_t *>(base + L::MRING + m * 1024)[row] = meta;
             fence_proxy_async_smem();
             mbar_arrive(&ready[s]);
+            mbar_arrive(&meta_full[m]);
         }
     } else if (warp < kPipeEpiWarp) {
         // ================================================================ softmax groups
@@ -311,14 +380,14 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         const float2 cc = make_float2(c2, c2);
         const float ninf = -INFINITY;
         for (int kk = grp; kk < count; kk += 2) {
-            const int s = kk % NS, b = kk % NB;
+            const int b = kk % NB, m = kk % NM;
             if (!warp_wait(&s_full[b], (kk / NB) & 1, abort_flag))
                 break;
-            // the row's meta was written before ready[s] (complete: S was issued)
-            if (!warp_wait(&ready[s], (kk / NS) & 1, abort_flag))
+            // the row's metadata (written with the tile's RoPE)
+            if (!warp_wait(&meta_full[m], (kk / NM) & 1, abort_flag))
                 break;
             tc_fence_after_sync();
-            const int64_t meta = reinterpret_cast<const int64_t *>(base + s * L::STAGE + L::META)[row];
+            const int64_t meta = reinterpret_cast<const int64_t *>(base + L::MRING + m * 1024)[row];
             const uint32_t gmask = meta < 0 ? 0u : (uint32_t)(meta & 15);
             const uint32_t sreg = tmem + lane_base + b * 128 + slot * 64;  // this row's window: 64 S columns
             // pass 1: granule maxima
@@ -370,7 +439,6 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
             // the other window's keys contribute nothing to this row
             tmem_st16(tmem + lane_base + b * 128 + (1 - slot) * 32, zero);
             tmem_st16(tmem + lane_base + b * 128 + (1 - slot) * 32 + 16, zero);
-            ometa[b * 128 + row] = meta;
             osum[b * 128 + row] = l2.x + l2.y;
             tmem_wait_st();
             tc_fence_before_sync();
@@ -378,54 +446,95 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         }
     } else if (warp < kPipeLoadWarp) {
         // ================================================================ epilogue
-        const int row = t - 32 * kPipeEpiWarp;
-        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        for (int kk = 0; kk < count; ++kk) {
-            const int b = kk % NB;
-            if (!warp_wait(&o_full[b], (kk / NB) & 1, abort_flag))
-                break;
-            // row meta and sum were written before p_full[b] (complete: P V ran)
-            if (!warp_wait(&p_full[b], (kk / NB) & 1, abort_flag))
+        // O / l of each row, as bf16, into a staging tile laid out like the
+        // operand tiles; each warp then writes its own 32 rows back with TMA
+        // stores: half a window (an M x M/2 or M/2 x M box) or, in the corner
+        // window, two quadrants, at the rows' original (un-shifted) position.
+        const int quarter = warp & 3;
+        const int row = quarter * 32 + lane;
+        const int slot = quarter >> 1, half = quarter & 1;
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+        int kk = 0;
+        for (; kk < count; ++kk) {
+            const int b = kk % NB, e = kk % L::NO;
+            // the row sum was written before p_full[b] (complete: P V ran)
+            if (!warp_wait(&o_full[b], (kk / NB) & 1, abort_flag) ||
+                !warp_wait(&p_full[b], (kk / NB) & 1, abort_flag))
                 break;
             tc_fence_after_sync();
-            const int64_t meta = ometa[b * 128 + row];
             const float inv = 1.f / osum[b * 128 + row];
             const float2 i2 = make_float2(inv, inv);
-            // normalise 32 columns of O and store them (16-byte stores)
-            auto store32 = [&](const float *o, int h2) {
-                if (meta < 0)
-                    return;
-                uint4 *dst = reinterpret_cast<uint4 *>(out + (meta & ~(int64_t)15)) + h2 * 4;
+            uint4 y[D / 8];
+            // the buffer goes back to the S issuer as soon as O is in registers
+#pragma unroll
+            for (int h2 = 0; h2 < D / 32; ++h2) {
+                float o[32];
+                tmem_ld32(tmem + lane_base + b * 128 + 64 + h2 * 32, o);
+                if (h2 == D / 32 - 1) {
+                    tc_fence_before_sync();
+                    mbar_arrive(&t_free[b]);
+                }
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    float2 y[4];
+                    float2 f[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        y[e] = __fmul2_rn(make_float2(o[8 * c + 2 * e], o[8 * c + 2 * e + 1]), i2);
-                    uint4 u;
-                    u.x = pack_bf16x2(y[0].x, y[0].y);
-                    u.y = pack_bf16x2(y[1].x, y[1].y);
-                    u.z = pack_bf16x2(y[2].x, y[2].y);
-                    u.w = pack_bf16x2(y[3].x, y[3].y);
-                    dst[c] = u;
+                    for (int q = 0; q < 4; ++q)
+                        f[q] = __fmul2_rn(make_float2(o[8 * c + 2 * q], o[8 * c + 2 * q + 1]), i2);
+                    y[h2 * 4 + c] = make_uint4(pack_bf16x2(f[0].x, f[0].y), pack_bf16x2(f[1].x, f[1].y),
+                                               pack_bf16x2(f[2].x, f[2].y), pack_bf16x2(f[3].x, f[3].y));
                 }
-            };
-            // the buffer goes back to the S issuer as soon as the last O
-            // columns are in registers, before the stores
-            float o[32];
-            tmem_ld32(tmem + lane_base + b * 128 + 64, o);
-            if constexpr (D == 32) {
-                tc_fence_before_sync();
-                mbar_arrive(&t_free[b]);
-                store32(o, 0);
-            } else {
-                store32(o, 0);
-                tmem_ld32(tmem + lane_base + b * 128 + 96, o);
-                tc_fence_before_sync();
-                mbar_arrive(&t_free[b]);
-                store32(o, 1);
             }
+            // this warp's staging rows have been read by its stores of tile kk - NO
+            if (kk >= L::NO)
+                bulk_wait_group_read<L::NO - 1>();
+            __syncwarp();
+            uint8_t *ost = base + L::OSTAGE + e * 256 * D;
+#pragma unroll
+            for (int c = 0; c < D / 8; ++c)
+                *reinterpret_cast<uint4 *>(ost + swz_offset(row, c, 2 * D)) = y[c];
+            fence_proxy_async_smem();
+            __syncwarp();
+            const Item it = decode_item_head_minor(g, first + kk * stride);
+            const int w = it.pack * 2 + slot;
+            if (lane < 2 && w < g.wph) {
+                const int bimg = (int)g.div_img.div((uint32_t)w);
+                const int rem = w - bimg * g.nWy * g.nWx;
+                const int wy = (int)g.div_nWx.div((uint32_t)rem);
+                const int wx = rem - wy * g.nWx;
+                const int kind = window_kind(g, wy, wx);
+                if (lane == 0 || kind == 3) {
+                    // box origin in the rolled window: rows of TMA order
+                    // [32 half, 32 half + 32) are the window's top / bottom half
+                    // (kinds 0, 2), left / right half (kind 1) or quadrants
+                    // 2 half and 2 half + 1 (kind 3)
+                    int iy0, jx0;
+                    const CUtensorMap *map;
+                    if (kind == 3) {
+                        const int qd = 2 * half + lane;
+                        iy0 = (qd >> 1) * 4;
+                        jx0 = (qd & 1) * 4;
+                        map = &tm_o.quarter;
+                    } else if (kind == 1) {
+                        iy0 = 0;
+                        jx0 = 4 * half;
+                        map = &tm_o.xhalf;
+                    } else {
+                        iy0 = 4 * half;
+                        jx0 = 0;
+                        map = &tm_o.yhalf;
+                    }
+                    int y0 = wy * 8 + iy0 + g.shift;
+                    if (y0 >= g.H) y0 -= g.H;
+                    int x0 = wx * 8 + jx0 + g.shift;
+                    if (x0 >= g.W) x0 -= g.W;
+                    tma_store_4d(map, sbase + L::OSTAGE + e * 256 * D + (uint32_t)((quarter * 32 + lane * 16) * 2 * D),
+                                 it.h * D, x0, y0, bimg);
+                }
+            }
+            bulk_commit_group();
         }
+        // every store has landed before the CTA exits
+        bulk_wait_group<0>();
     }
 
     tc_fence_before_sync();

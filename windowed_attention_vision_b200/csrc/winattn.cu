@@ -218,15 +218,13 @@ bool encode_window_map(CUtensorMap *m, const void *base, const Geometry &g, int 
     return r == CUDA_SUCCESS;
 }
 
-// The four box shapes of one operand (see WindowMaps).
+// The four box shapes of one operand (see WindowMaps).  All four are encoded
+// whatever the shift: the pipelined kernel's epilogue stores half windows and
+// quadrants of unshifted windows too.
 bool encode_window_maps(WindowMaps *m, const void *base, const Geometry &g)
 {
     if (!encode_window_map(&m->full, base, g, g.M, g.M))
         return false;
-    if (g.shift == 0) {
-        m->xhalf = m->yhalf = m->quarter = m->full;
-        return true;
-    }
     const int hm = g.M / 2;
     return encode_window_map(&m->xhalf, base, g, hm, g.M) && encode_window_map(&m->yhalf, base, g, g.M, hm) &&
            encode_window_map(&m->quarter, base, g, hm, hm);
@@ -365,10 +363,10 @@ template <int D>
 int launch_pipe(const void *q, const void *k, const void *v, const float *theta, void *out, const Geometry &g,
                 cudaStream_t stream)
 {
-    WindowMaps maps[3];
+    WindowMaps maps[4];
     std::memset(maps, 0, sizeof maps);
     if (!encode_window_maps(&maps[0], q, g) || !encode_window_maps(&maps[1], k, g) ||
-        !encode_window_maps(&maps[2], v, g))
+        !encode_window_maps(&maps[2], v, g) || !encode_window_maps(&maps[3], out, g))
         return WINATTN_ERR_CUDA;
     auto kernel = winattn_fwd_pipe_kernel<D>;
     const int smem = (int)PipeLayout<D>::bytes(g.heads);
@@ -377,7 +375,7 @@ int launch_pipe(const void *q, const void *k, const void *v, const float *theta,
     const int64_t grid = g.items < sm_count() ? g.items : sm_count();
     kernel<<<(unsigned)grid, kPipeThreads, smem, stream>>>(theta, static_cast<__nv_bfloat16 *>(out), g,
                                                            1.0f / std::sqrt((float)g.d), maps[0], maps[1],
-                                                           maps[2]);
+                                                           maps[2], maps[3]);
     return cudaGetLastError() == cudaSuccess ? WINATTN_OK : WINATTN_ERR_CUDA;
 }
 
