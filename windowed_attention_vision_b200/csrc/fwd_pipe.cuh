@@ -64,13 +64,16 @@ struct PipeLayout {
     // V ring: values [128][D]
     static constexpr uint32_t V_STAGE = 256 * D;
     static constexpr int NSV = D == 32 ? 6 : 3;
-    // row metadata ring: original element offset | granule mask, i64[128]
+    // metadata ring, per tile: allowed granules of each row, i64[128], then
+    // the output TMA stores of each warp: int4[4 warps][2] = {x0, y0, image,
+    // box shape | head column << 4} (box shape -1: no store)
     static constexpr int NM = NSQ + kPipeBufs;
+    static constexpr uint32_t MSLOT = 128 * 8 + 8 * 16;
     static constexpr uint32_t VRING = NSQ * QK_STAGE;
     static constexpr uint32_t MRING = VRING + NSV * V_STAGE;
     // output staging for the TMA stores: [128][D] bf16, swizzled like the operands
     static constexpr int NO = D == 32 ? 2 : 1;
-    static constexpr uint32_t OSTAGE = MRING + NM * 1024;
+    static constexpr uint32_t OSTAGE = (MRING + NM * MSLOT + 1023) & ~1023u;
     static constexpr uint32_t OSUM = OSTAGE + NO * 256 * D;         // per TMEM buffer: row sum l, f32[4][128]
     static constexpr uint32_t IJTAB = OSUM + kPipeBufs * 128 * 4;   // box row order: (i << 8 | j) u16[4][64]
     static constexpr uint32_t TABLE = IJTAB + 512;                  // RoPE (cos, sin) float4 [heads][8][D/8]
@@ -342,6 +345,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
             const Item it = decode_item_head_minor(g, first + kk * stride);
             const int w = it.pack * 2 + slot;
             int64_t meta = -1;  // allowed 16-key granules of the row's window, -1 for no token
+            uint8_t *ms = base + L::MRING + m * L::MSLOT;
             if (w < g.wph) {
                 const int b = (int)g.div_img.div((uint32_t)w);
                 const int rem = w - b * g.nWy * g.nWx;
@@ -351,20 +355,53 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
                 const uint32_t ij = ijtab[kind * 64 + rp];
                 const int i = (int)(ij >> 8), j = (int)(ij & 0xFF);
                 meta = kind == 0 ? 0xF : (kind == 3 ? 1 << (rp >> 4) : ((rp >> 5) ? 0xC : 0x3));
+                if (lane < 2) {
+                    // the output store(s) of the epilogue warp on this lane
+                    // quarter: rows [32 h, 32 h + 32) of the window in box order
+                    // are its top / bottom half (kinds 0, 2), left / right half
+                    // (kind 1), or quadrants 2 h and 2 h + 1 (kind 3)
+                    const int hh = (row >> 5) & 1;
+                    int4 rec = make_int4(0, 0, 0, -1);
+                    if (lane == 0 || kind == 3) {
+                        int iy0, jx0, shape;
+                        if (kind == 3) {
+                            const int qd = 2 * hh + lane;
+                            iy0 = (qd >> 1) * 4;
+                            jx0 = (qd & 1) * 4;
+                            shape = 3;
+                        } else if (kind == 1) {
+                            iy0 = 0;
+                            jx0 = 4 * hh;
+                            shape = 1;
+                        } else {
+                            iy0 = 4 * hh;
+                            jx0 = 0;
+                            shape = 2;
+                        }
+                        int y0 = wy * 8 + iy0 + g.shift;
+                        if (y0 >= g.H) y0 -= g.H;
+                        int x0 = wx * 8 + jx0 + g.shift;
+                        if (x0 >= g.W) x0 -= g.W;
+                        rec = make_int4(x0, y0, b, shape | (it.h * D) << 4);
+                    }
+                    reinterpret_cast<int4 *>(ms + 1024)[(row >> 5) * 2 + lane] = rec;
+                }
                 if (theta)
                     rotate_qk_rows<D>(st + L::QC, st + L::KC, row,
                                       reinterpret_cast<const float4 *>(table + it.h * kTab), i, j, false, 1.f);
             } else {
                 // an empty slot of the last pack: zero rows keep its keys finite
-                // (their P is zero)
+                // (their P is zero); nothing of it is stored
 #pragma unroll
                 for (int c = 0; c < D / 8; ++c) {
                     const uint32_t off = swz_offset(row, c, 2 * D);
                     *reinterpret_cast<uint4 *>(st + L::QC + off) = make_uint4(0, 0, 0, 0);
                     *reinterpret_cast<uint4 *>(st + L::KC + off) = make_uint4(0, 0, 0, 0);
                 }
+                if (lane < 2)
+                    reinterpret_cast<int4 *>(ms + 1024)[(row >> 5) * 2 + lane] = make_int4(0, 0, 0, -1);
             }
-            reinterpret_cast<int64_t *>(base + L::MRING + m * 1024)[row] = meta;
+            reinterpret_cast<int64_t *>(ms)[row] = meta;
             fence_proxy_async_smem();
             mbar_arrive(&ready[s]);
             mbar_arrive(&meta_full[m]);
@@ -387,7 +424,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
             if (!warp_wait(&meta_full[m], (kk / NM) & 1, abort_flag))
                 break;
             tc_fence_after_sync();
-            const int64_t meta = reinterpret_cast<const int64_t *>(base + L::MRING + m * 1024)[row];
+            const int64_t meta = reinterpret_cast<const int64_t *>(base + L::MRING + m * L::MSLOT)[row];
             const uint32_t gmask = meta < 0 ? 0u : (uint32_t)(meta & 15);
             const uint32_t sreg = tmem + lane_base + b * 128 + slot * 64;  // this row's window: 64 S columns
             // pass 1: granule maxima
@@ -452,16 +489,21 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         // window, two quadrants, at the rows' original (un-shifted) position.
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
-        const int slot = quarter >> 1, half = quarter & 1;
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         int kk = 0;
         for (; kk < count; ++kk) {
-            const int b = kk % NB, e = kk % L::NO;
-            // the row sum was written before p_full[b] (complete: P V ran)
+            const int b = kk % NB, e = kk % L::NO, m = kk % NM;
+            // the row sum was written before p_full[b] (complete: P V ran), the
+            // store record with the tile's RoPE (meta_full[m])
             if (!warp_wait(&o_full[b], (kk / NB) & 1, abort_flag) ||
-                !warp_wait(&p_full[b], (kk / NB) & 1, abort_flag))
+                !warp_wait(&p_full[b], (kk / NB) & 1, abort_flag) ||
+                !warp_wait(&meta_full[m], (kk / NM) & 1, abort_flag))
                 break;
             tc_fence_after_sync();
+            // read before the buffer is released: the slot is rewritten only
+            // after S of tile kk + 4, which needs this buffer back
+            const int4 rec = lane < 2 ? reinterpret_cast<const int4 *>(base + L::MRING + m * L::MSLOT + 1024)[quarter * 2 + lane]
+                                      : make_int4(0, 0, 0, -1);
             const float inv = 1.f / osum[b * 128 + row];
             const float2 i2 = make_float2(inv, inv);
             uint4 y[D / 8];
@@ -494,42 +536,11 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
                 *reinterpret_cast<uint4 *>(ost + swz_offset(row, c, 2 * D)) = y[c];
             fence_proxy_async_smem();
             __syncwarp();
-            const Item it = decode_item_head_minor(g, first + kk * stride);
-            const int w = it.pack * 2 + slot;
-            if (lane < 2 && w < g.wph) {
-                const int bimg = (int)g.div_img.div((uint32_t)w);
-                const int rem = w - bimg * g.nWy * g.nWx;
-                const int wy = (int)g.div_nWx.div((uint32_t)rem);
-                const int wx = rem - wy * g.nWx;
-                const int kind = window_kind(g, wy, wx);
-                if (lane == 0 || kind == 3) {
-                    // box origin in the rolled window: rows of TMA order
-                    // [32 half, 32 half + 32) are the window's top / bottom half
-                    // (kinds 0, 2), left / right half (kind 1) or quadrants
-                    // 2 half and 2 half + 1 (kind 3)
-                    int iy0, jx0;
-                    const CUtensorMap *map;
-                    if (kind == 3) {
-                        const int qd = 2 * half + lane;
-                        iy0 = (qd >> 1) * 4;
-                        jx0 = (qd & 1) * 4;
-                        map = &tm_o.quarter;
-                    } else if (kind == 1) {
-                        iy0 = 0;
-                        jx0 = 4 * half;
-                        map = &tm_o.xhalf;
-                    } else {
-                        iy0 = 4 * half;
-                        jx0 = 0;
-                        map = &tm_o.yhalf;
-                    }
-                    int y0 = wy * 8 + iy0 + g.shift;
-                    if (y0 >= g.H) y0 -= g.H;
-                    int x0 = wx * 8 + jx0 + g.shift;
-                    if (x0 >= g.W) x0 -= g.W;
-                    tma_store_4d(map, sbase + L::OSTAGE + e * 256 * D + (uint32_t)((quarter * 32 + lane * 16) * 2 * D),
-                                 it.h * D, x0, y0, bimg);
-                }
+            if (rec.w >= 0) {
+                const int shape = rec.w & 3;
+                const CUtensorMap *map = shape == 3 ? &tm_o.quarter : (shape == 1 ? &tm_o.xhalf : &tm_o.yhalf);
+                tma_store_4d(map, sbase + L::OSTAGE + e * 256 * D + (uint32_t)((quarter * 32 + lane * 16) * 2 * D),
+                             rec.w >> 4, rec.x, rec.y, rec.z);
             }
             bulk_commit_group();
         }
