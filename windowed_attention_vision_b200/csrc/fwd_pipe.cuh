@@ -155,6 +155,10 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         *abort_flag = 0u;
         fence_mbar_init();
     }
+    // TMEM and the barriers are set up; nothing of global memory is touched
+    // before the previous kernel of the stream has completed
+    grid_launch_dependents();
+    grid_dependency_wait();
     if (theta) {
         // table4[h][pos][k/2] = (cos k, cos k+1, sin k, sin k+1) of pos * theta_h[k], even k
         float *tf = reinterpret_cast<float *>(table);

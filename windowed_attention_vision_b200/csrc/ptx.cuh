@@ -166,6 +166,22 @@ __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap *map)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// ------------------------------------------------------------------ launch overlap
+
+// Programmatic dependent launch: let the next kernel of the stream (when it
+// was launched as a programmatic dependent) start its prologue on SMs this
+// grid frees, and wait until every earlier grid of the stream has completed
+// and its memory is visible.  Both are no-ops without the launch attribute.
+__device__ __forceinline__ void grid_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void grid_dependency_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ fences
 
 __device__ __forceinline__ void fence_proxy_async_smem()

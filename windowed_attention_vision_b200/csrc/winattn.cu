@@ -373,9 +373,23 @@ int launch_pipe(const void *q, const void *k, const void *v, const float *theta,
     if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return WINATTN_ERR_CUDA;
     const int64_t grid = g.items < sm_count() ? g.items : sm_count();
-    kernel<<<(unsigned)grid, kPipeThreads, smem, stream>>>(theta, static_cast<__nv_bfloat16 *>(out), g,
-                                                           1.0f / std::sqrt((float)g.d), maps[0], maps[1],
-                                                           maps[2], maps[3]);
+    // a programmatic dependent of the previous kernel in the stream: its
+    // launch and prologue overlap that kernel's tail (the kernel waits for it
+    // before touching global memory)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kPipeThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const float scale = 1.0f / std::sqrt((float)g.d);
+    if (cudaLaunchKernelEx(&cfg, kernel, theta, static_cast<__nv_bfloat16 *>(out), g, scale, maps[0], maps[1],
+                           maps[2], maps[3]) != cudaSuccess)
+        return WINATTN_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? WINATTN_OK : WINATTN_ERR_CUDA;
 }
 
