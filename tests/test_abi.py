@@ -115,7 +115,7 @@ def test_launch_plan(lib, B, H, W, M, shift, heads, d, rank, U, tiles, kernel):
     assert info["kernel"] == kernel
     if kernel == LARGE:  # items are pairs of query tiles
         assert info["work_items"] == heads * windows * tiles // 2
-        assert info["threads"] == 448 and info["grid"] == min(148, info["work_items"])
+        assert info["threads"] == 512 and info["grid"] == min(148, info["work_items"])
     else:
         assert info["work_items"] == heads * math.ceil(windows / U) * tiles
     if kernel == SMALL:

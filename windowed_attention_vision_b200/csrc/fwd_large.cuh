@@ -51,7 +51,7 @@
 
 namespace winattn {
 
-constexpr int kLargeThreads = 14 * 32;
+constexpr int kLargeThreads = 16 * 32;
 constexpr uint32_t kLargeSmemBudget = 220 * 1024;
 
 // Keys per tile: 128 (8, 4 or 2 window rows for M = 16, 32, 64), or one
@@ -179,9 +179,11 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
     float4 *table4 = reinterpret_cast<float4 *>(base + L::TABLE);
     uint64_t *bars = reinterpret_cast<uint64_t *>(base + L::BARS);
     uint64_t *kv_full = bars, *kv_ready = bars + NS, *kv_empty = bars + 2 * NS;
-    uint64_t *q_ready = bars + 3 * NS, *q_free = q_ready + 2, *s_full = q_free + 2, *p_full = s_full + NB;
-    uint64_t *o_done = p_full + NB, *o_last = o_done + 2, *t_free = o_last + 2, *fin = t_free + 2;
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(fin + 1);
+    // p_part[b * 4 + ch]: chunk ch (32 keys) of the P in S buffer b is written
+    uint64_t *q_ready = bars + 3 * NS, *q_free = q_ready + 2, *s_full = q_free + 2, *p_part = s_full + NB;
+    uint64_t *pv_done = p_part + 4 * NB, *o_done = pv_done + NB, *o_last = o_done + 2, *t_free = o_last + 2;
+    uint64_t *fin = t_free + 2;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(fin + 3);
     volatile uint32_t *abort_flag = tslot + 1;
 
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
@@ -204,7 +206,7 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
         for (int s = 0; s < NS; ++s) {
             mbar_init(&kv_full[s], 1);
             mbar_init(&kv_ready[s], 128);
-            mbar_init(&kv_empty[s], 1);
+            mbar_init(&kv_empty[s], 2);  // P V of both query tiles
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(&q_ready[a], 128);
@@ -215,9 +217,12 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
         }
         for (int b = 0; b < NB; ++b) {
             mbar_init(&s_full[b], 1);
-            mbar_init(&p_full[b], 128);
+            mbar_init(&pv_done[b], 1);
+            for (int ch = 0; ch < 4; ++ch)
+                mbar_init(&p_part[b * 4 + ch], 128);
         }
-        mbar_init(fin, 1);
+        for (int f = 0; f < 3; ++f)
+            mbar_init(&fin[f], 1);
         *abort_flag = 0u;
         fence_mbar_init();
     }
@@ -281,79 +286,113 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
             }
         }
     } else if (warp == 13) {
-        // ============================================================ MMA issuer
+        // ============================================================ S issuer
         // One sequence over the CTA's items: step n = 2 cg + t is query tile t
         // (0 = A, 1 = B) against the CTA's cg-th key tile.  S of step n goes to
-        // TMEM buffer n % NB and is issued NB steps ahead, right behind the P V
-        // that frees its buffer, across item boundaries too.
+        // TMEM buffer n % NB once P V of step n - NB (the buffer's previous
+        // tenant) has completed.
         if (lane == 0) {
             constexpr uint32_t kIdescS = idesc_bf16_f32(128, BN, false);
-            constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
             const int total = 2 * count * nkv;
-            bool ok = true;
-            int ns = 0, s_kk = 0, s_jt = 0;  // next S step, its item and key tile
-            auto issue_s_upto = [&](int upto) {
-                for (; ns < upto && ns < total && ok; ++ns) {
-                    const int tl = ns & 1, cg = ns >> 1;
-                    if (tl == 0) {
-                        if (s_jt == 0 && !(ok = wait_or_abort(&q_ready[s_kk & 1], (s_kk >> 1) & 1, abort_flag)))
-                            break;
-                        if (!(ok = wait_or_abort(&kv_ready[cg % NS], (cg / NS) & 1, abort_flag)))
-                            break;
-                        tc_fence_after_sync();
-                    }
-                    const uint32_t qtile = sbase + (s_kk & 1) * L::QBUF + tl * L::QTILE;
-                    const uint32_t d = tmem + (ns % NB) * BN;
-                    const uint32_t kst = sbase + L::STAGES + (cg % NS) * L::STAGE;
+            int s_kk = 0, s_jt = 0;  // item and key tile of the next S
+            int ns = 0;
+            for (; ns < total; ++ns) {
+                const int tl = ns & 1, cg = ns >> 1;
+                if (ns >= NB && !wait_or_abort(&pv_done[ns % NB], ((ns / NB) - 1) & 1, abort_flag))
+                    break;
+                if (tl == 0) {
+                    if (s_jt == 0 && !wait_or_abort(&q_ready[s_kk & 1], (s_kk >> 1) & 1, abort_flag))
+                        break;
+                    if (!wait_or_abort(&kv_ready[cg % NS], (cg / NS) & 1, abort_flag))
+                        break;
+                }
+                tc_fence_after_sync();
+                const uint32_t qtile = sbase + (s_kk & 1) * L::QBUF + tl * L::QTILE;
+                const uint32_t d = tmem + (ns % NB) * BN;
+                const uint32_t kst = sbase + L::STAGES + (cg % NS) * L::STAGE;
+                // descriptors built once per step; a 16-element K step is
+                // +32 bytes, i.e. +2 in the 16-byte start-address field
+                const uint64_t qd = smem_desc(qtile, 16, 16 * D, swizzle_code(2 * D));
+                const uint64_t kd = smem_desc(kst + L::KC, 16, 16 * D, swizzle_code(2 * D));
 #pragma unroll
-                    for (int ks = 0; ks < D / 16; ++ks)
-                        umma_bf16_ss(d, smem_desc(qtile + ks * 32, 16, 16 * D, swizzle_code(2 * D)),
-                                     smem_desc(kst + L::KC + ks * 32, 16, 16 * D, swizzle_code(2 * D)), kIdescS,
-                                     ks > 0);
+                for (int ks = 0; ks < D / 16; ++ks)
+                    umma_bf16_ss(d, qd + 2 * ks, kd + 2 * ks, kIdescS, ks > 0);
+                if constexpr (R > 0) {
+                    const uint64_t qbd = smem_desc(qtile + 256 * D, 16, 16 * R, swizzle_code(2 * R));
+                    const uint64_t kbd = smem_desc(kst + L::KB, 16, 16 * R, swizzle_code(2 * R));
 #pragma unroll
                     for (int ks = 0; ks < R / 16; ++ks)
-                        umma_bf16_ss(d, smem_desc(qtile + 256 * D + ks * 32, 16, 16 * R, swizzle_code(2 * R)),
-                                     smem_desc(kst + L::KB + ks * 32, 16, 16 * R, swizzle_code(2 * R)), kIdescS, 1);
-                    umma_commit(&s_full[ns % NB]);
-                    if (tl == 1 && ++s_jt == nkv) {
-                        umma_commit(&q_free[s_kk & 1]);  // the last S that reads this item's Q
-                        s_jt = 0;
-                        ++s_kk;
-                    }
+                        umma_bf16_ss(d, qbd + 2 * ks, kbd + 2 * ks, kIdescS, 1);
                 }
-            };
-            issue_s_upto(NB);
-            int p_kk = 0, p_jt = 0;
-            for (int n = 0; n < total && ok; ++n) {
-                const int tl = n & 1, cg = n >> 1;
-                if (!(ok = wait_or_abort(&p_full[n % NB], (n / NB) & 1, abort_flag)))
-                    break;
+                umma_commit(&s_full[ns % NB]);
+                if (tl == 1 && ++s_jt == nkv) {
+                    umma_commit(&q_free[s_kk & 1]);  // the last S that reads this item's Q
+                    s_jt = 0;
+                    ++s_kk;
+                }
+            }
+            if (ns > 0) {
+                umma_commit(&fin[0]);
+                mbar_wait(&fin[0], 0);
+            }
+        }
+    } else if (warp == 14 || warp == 15) {
+        // ============================================================ P V issuers
+        // One per query tile: O_t += P V chunk by chunk (32 keys, two MMAs)
+        // as the softmax writes each chunk of P, so that P V overlaps the
+        // exponentials and the S buffer returns right after the last chunk.
+        const int tl = warp - 14;
+        if (lane == 0) {
+            constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
+            constexpr int NC = BN / 32;
+            const int steps = count * nkv;
+            int p_kk = 0, p_jt = 0;  // item and key tile of this tile's next P V
+            int c = 0;
+            bool ok = true;
+            for (; c < steps && ok; ++c) {
+                const int n = 2 * c + tl, b = n % NB;
                 // O of this tile is free once the previous item's epilogue read it
                 if (p_jt == 0 && p_kk > 0 && !(ok = wait_or_abort(&t_free[tl], (p_kk - 1) & 1, abort_flag)))
                     break;
-                tc_fence_after_sync();
-                const uint32_t pa = tmem + (n % NB) * BN;  // P over the first BN/2 columns of the buffer
-                const uint32_t vst = sbase + L::STAGES + (cg % NS) * L::STAGE + L::VO;
-                const uint32_t od = tmem + kOCol + tl * D;
+                // S of this step exists, hence P V of the buffer's previous
+                // tenant (step n - NB, the other tile's) has completed and the
+                // chunk barriers of buffer b are on this step's phase: a
+                // parity wait must never run a phase ahead of its barrier
+                if (!(ok = wait_or_abort(&s_full[b], (n / NB) & 1, abort_flag)))
+                    break;
+                const uint32_t pa = tmem + b * BN;  // P over the first BN/2 columns of the buffer
+                const uint32_t vst = sbase + L::STAGES + (c % NS) * L::STAGE + L::VO;
+                const uint32_t od = tmem + NB * BN + tl * D;
+                // 16 keys of V are 32 D bytes: +2 D in the start-address field
+                const uint64_t vd = smem_desc(vst, 8192, 16 * D, swizzle_code(2 * D));
+                // parts end at chunks 1, 3 (and at the last chunk for BN = 96)
 #pragma unroll
-                for (int ks = 0; ks < BN / 16; ++ks)
-                    umma_bf16_ts(od, pa + ks * 8, smem_desc(vst + ks * 32 * D, 8192, 16 * D, swizzle_code(2 * D)),
-                                 kIdescPV, p_jt > 0 || ks > 0);
+                for (int ch = 0; ch < NC; ++ch) {
+                    if ((ch & 1) || ch == NC - 1) {
+                        if (!(ok = wait_or_abort(&p_part[b * 4 + ch], (n / NB) & 1, abort_flag)))
+                            break;
+                        tc_fence_after_sync();
+                        const int c0 = ch & ~1;
+#pragma unroll
+                        for (int ks = 2 * c0; ks < 2 * ch + 2; ++ks)
+                            umma_bf16_ts(od, pa + ks * 8, vd + (uint64_t)(2 * D * ks), kIdescPV, p_jt > 0 || ks > 0);
+                    }
+                }
+                if (!ok)
+                    break;
                 umma_commit(&o_done[tl]);
                 if (p_jt == nkv - 1)
                     umma_commit(&o_last[tl]);
-                if (tl == 1) {
-                    umma_commit(&kv_empty[cg % NS]);
-                    if (++p_jt == nkv) {
-                        p_jt = 0;
-                        ++p_kk;
-                    }
+                umma_commit(&pv_done[b]);
+                umma_commit(&kv_empty[c % NS]);
+                if (++p_jt == nkv) {
+                    p_jt = 0;
+                    ++p_kk;
                 }
-                issue_s_upto(n + 1 + NB);
             }
-            if (total > 0) {
-                umma_commit(fin);
-                mbar_wait(fin, 0);
+            if (c > 0) {
+                umma_commit(&fin[1 + tl]);
+                mbar_wait(&fin[1 + tl], 0);
             }
         }
     } else if (warp >= 8) {
@@ -533,9 +572,32 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
                         rescale = true;
                     }
                 }
-                // ---- pass 2: P = exp2(s * c2 - m) into TMEM over the consumed S
+                if (__any_sync(0xffffffffu, rescale)) {
+                    // O must hold every earlier key tile's P V before it is
+                    // rescaled: only P V of this tile's previous step (c - 1)
+                    // can still be in flight.  The rescale lands before the
+                    // first chunk of this step's P is handed to P V.
+                    if (!warp_wait(&o_done[tile], (c - 1) & 1, abort_flag)) {
+                        failed = true;
+                        break;
+                    }
+                    tc_fence_after_sync();
+#pragma unroll
+                    for (int ch = 0; ch < D / 16; ++ch) {
+                        float o[16];
+                        tmem_ld16(oreg + ch * 16, o);
+                        uint32_t ob[16];
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            ob[e] = __float_as_uint(o[e] * alpha);
+                        tmem_st16(oreg + ch * 16, ob);
+                    }
+                }
+                // ---- pass 2: P = exp2(s * c2 - m) into TMEM over the consumed
+                // S; each 32-key chunk goes to P V as soon as it is written
                 const float2 cc = make_float2(c2, c2), mm2 = make_float2(-m, -m);
                 float2 l2 = make_float2(0.f, 0.f);
+                uint64_t *parts = p_part + (n % NB) * 4;
                 tmem_ld32_issue(sreg, buf[0]);
 #pragma unroll
                 for (int ch = 0; ch < NC; ++ch) {
@@ -560,32 +622,15 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
                         }
                     }
                     tmem_st16(sreg + ch * 16, pk);
+                    // P goes to P V in parts of two chunks (64 keys): fewer
+                    // store waits on the softmax side
+                    if ((ch & 1) || ch == NC - 1) {
+                        tmem_wait_st();
+                        tc_fence_before_sync();
+                        mbar_arrive(&parts[ch]);
+                    }
                 }
                 l = l * alpha + (l2.x + l2.y);
-                if (__any_sync(0xffffffffu, rescale)) {
-                    // O must hold every earlier key tile's P V before it is
-                    // rescaled; S of this step was issued after P V of step
-                    // n - NB, so for this tile only P V of c - 1 can still be
-                    // in flight
-                    if (!warp_wait(&o_done[tile], (c - 1) & 1, abort_flag)) {
-                        failed = true;
-                        break;
-                    }
-                    tc_fence_after_sync();
-#pragma unroll
-                    for (int ch = 0; ch < D / 16; ++ch) {
-                        float o[16];
-                        tmem_ld16(oreg + ch * 16, o);
-                        uint32_t ob[16];
-#pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            ob[e] = __float_as_uint(o[e] * alpha);
-                        tmem_st16(oreg + ch * 16, ob);
-                    }
-                }
-                tmem_wait_st();
-                tc_fence_before_sync();
-                mbar_arrive(&p_full[n % NB]);
             }
             if (failed)
                 break;

@@ -297,10 +297,13 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
                     break;
                 tc_fence_after_sync();
                 const uint32_t sst = sbase + s * L::QK_STAGE;
+                // descriptors built once per tile; a 16-element K step is +32
+                // bytes, i.e. +2 in the 16-byte start-address field
+                const uint64_t qd = smem_desc(sst + L::QC, 16, 16 * D, swizzle_code(2 * D));
+                const uint64_t kd = smem_desc(sst + L::KC, 16, 16 * D, swizzle_code(2 * D));
 #pragma unroll
                 for (int ks = 0; ks < D / 16; ++ks)
-                    umma_bf16_ss(tmem + b * 128, smem_desc(sst + L::QC + ks * 32, 16, 16 * D, swizzle_code(2 * D)),
-                                 smem_desc(sst + L::KC + ks * 32, 16, 16 * D, swizzle_code(2 * D)), kIdescS, ks > 0);
+                    umma_bf16_ss(tmem + b * 128, qd + 2 * ks, kd + 2 * ks, kIdescS, ks > 0);
                 umma_commit(&s_full[b]);
                 umma_commit(&qk_empty[s]);
             }
@@ -324,10 +327,12 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
                     break;
                 tc_fence_after_sync();
                 const uint32_t vst = sbase + L::VRING + s * L::V_STAGE;
+                // 16 keys of V are 32 D bytes: +2 D in the start-address field
+                const uint64_t vd = smem_desc(vst, 8192, 16 * D, swizzle_code(2 * D));
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    umma_bf16_ts(tmem + b * 128 + 64, tmem + b * 128 + ks * 8,
-                                 smem_desc(vst + ks * 32 * D, 8192, 16 * D, swizzle_code(2 * D)), kIdescPV, ks > 0);
+                    umma_bf16_ts(tmem + b * 128 + 64, tmem + b * 128 + ks * 8, vd + (uint64_t)(2 * D * ks), kIdescPV,
+                                 ks > 0);
                 umma_commit(&o_full[b]);
                 umma_commit(&v_empty[s]);
             }

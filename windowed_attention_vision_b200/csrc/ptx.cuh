@@ -320,7 +320,9 @@ __host__ __device__ constexpr uint32_t swizzle_code(int row_bytes)
     return row_bytes == 128 ? 2u : (row_bytes == 64 ? 4u : 6u);
 }
 
-// Shared-memory matrix descriptor (sm_100 version 1).  Offsets in bytes.
+// Shared-memory matrix descriptor (sm_100 version 1).  Offsets in bytes.  The
+// start address sits in bits 0-13 in 16-byte units, so a descriptor of a
+// tile at saddr + k * 16 is this one plus k (addresses stay below 256 KiB).
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t swz)
 {
     uint64_t d = (uint64_t)((saddr & 0x3FFFFu) >> 4);
