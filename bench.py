@@ -272,7 +272,8 @@ def run_reference(args):
         return 0
     from windowed_attention_vision_b200 import inputs as I
     w = I.WORKLOADS[args.workload]
-    per_step = max(2.0, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
+    # the whole run stays within about 150 s of CPU time whatever K and W are
+    per_step = max(0.2, min(20.0, 150.0 / max(1, args.steps + args.warmup)))
     rates = []
     for s in range(args.warmup + args.steps):
         rate, sample, cores, _ = oracle_sample_rate(w, per_step, base=s)
