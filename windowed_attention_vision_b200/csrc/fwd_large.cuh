@@ -540,8 +540,9 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
                     a1 = a0 + NCH / 2;
                 }
                 uint32_t buf[2][32];
-                // ---- pass 1: row max over the allowed columns (loads pipelined)
-                float mx = -INFINITY;
+                // ---- pass 1: row max over the allowed columns (loads
+                // pipelined; four independent max chains)
+                float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
                 tmem_ld32_issue(sreg, buf[0]);
 #pragma unroll
                 for (int ch = 0; ch < NC; ++ch) {
@@ -552,14 +553,15 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
                     if (2 * ch >= a0 && 2 * ch < a1) {
 #pragma unroll
                         for (int e = 0; e < 16; e += 2)
-                            mx = fmax3(mx, __uint_as_float(xb[e]), __uint_as_float(xb[e + 1]));
+                            mq[(e >> 1) & 3] = fmax3(mq[(e >> 1) & 3], __uint_as_float(xb[e]), __uint_as_float(xb[e + 1]));
                     }
                     if (2 * ch + 1 >= a0 && 2 * ch + 1 < a1) {
 #pragma unroll
                         for (int e = 16; e < 32; e += 2)
-                            mx = fmax3(mx, __uint_as_float(xb[e]), __uint_as_float(xb[e + 1]));
+                            mq[(e >> 1) & 3] = fmax3(mq[(e >> 1) & 3], __uint_as_float(xb[e]), __uint_as_float(xb[e + 1]));
                     }
                 }
+                const float mx = fmaxf(fmax3(mq[0], mq[1], mq[2]), mq[3]);
                 float alpha = 1.f;
                 bool rescale = false;
                 if (mx > -INFINITY) {
@@ -596,7 +598,7 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
                 // ---- pass 2: P = exp2(s * c2 - m) into TMEM over the consumed
                 // S; each 32-key chunk goes to P V as soon as it is written
                 const float2 cc = make_float2(c2, c2), mm2 = make_float2(-m, -m);
-                float2 l2 = make_float2(0.f, 0.f);
+                float2 lq[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // two sum chains
                 uint64_t *parts = p_part + (n % NB) * 4;
                 tmem_ld32_issue(sreg, buf[0]);
 #pragma unroll
@@ -615,7 +617,7 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
                             const float2 z = __ffma2_rn(
                                 make_float2(__uint_as_float(xb[e]), __uint_as_float(xb[e + 1])), cc, mm2);
                             const float2 p = make_float2(fast_exp2(z.x), fast_exp2(z.y));
-                            l2 = __fadd2_rn(l2, p);
+                            lq[(e >> 1) & 1] = __fadd2_rn(lq[(e >> 1) & 1], p);
                             pk[e >> 1] = pack_bf16x2(p.x, p.y);
                         } else {
                             pk[e >> 1] = 0u;
@@ -630,6 +632,7 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
                         mbar_arrive(&parts[ch]);
                     }
                 }
+                const float2 l2 = __fadd2_rn(lq[0], lq[1]);
                 l = l * alpha + (l2.x + l2.y);
             }
             if (failed)

@@ -457,7 +457,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
                                    (gmask & 8u) ? gm[3] : ninf);
             const float mneg = mx == ninf ? 0.f : -mx * c2;
             // pass 2: P = exp2(s c2 - m), masked granules -> 0, over the S columns just read
-            float2 l2 = make_float2(0.f, 0.f);
+            float2 lq[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // two sum chains
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
                 float x[32];
@@ -471,7 +471,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
                     for (int e = 16 * q2; e < 16 * q2 + 16; e += 2) {
                         const float2 z = __ffma2_rn(make_float2(x[e], x[e + 1]), cc, bb);
                         const float2 p = make_float2(fast_exp2(z.x), fast_exp2(z.y));
-                        l2 = __fadd2_rn(l2, p);
+                        lq[(e >> 1) & 1] = __fadd2_rn(lq[(e >> 1) & 1], p);
                         pk[e >> 1] = pack_bf16x2(p.x, p.y);
                     }
                 }
@@ -485,6 +485,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
             // the other window's keys contribute nothing to this row
             tmem_st16(tmem + lane_base + b * 128 + (1 - slot) * 32, zero);
             tmem_st16(tmem + lane_base + b * 128 + (1 - slot) * 32 + 16, zero);
+            const float2 l2 = __fadd2_rn(lq[0], lq[1]);
             osum[b * 128 + row] = l2.x + l2.y;
             tmem_wait_st();
             tc_fence_before_sync();
