@@ -127,6 +127,36 @@ int winattn_fwd_host(const void *q_host, const void *k_host, const void *v_host,
  * 256 bytes), or 0 for invalid sizes. */
 size_t winattn_host_workspace_bytes(int B, int H_img, int W_img, int heads, int d, int dtype);
 
+/*
+ * winattn_fwd_host_static — winattn_fwd_host for callers that cannot allocate
+ * device memory: code that links this library into a process whose device
+ * memory is owned by someone else (a host application that must not grow the
+ * GPU's allocations, a plug-in without access to the owner's allocator), so
+ * it can pass neither a workspace nor device buffers.  (There is no
+ * counterpart on the pages: this is an interface convenience, not part of the
+ * method.)
+ *
+ * Same arguments and result as winattn_fwd_host, without the workspace: the
+ * device copies of q, k, v and out live in one library-owned static device
+ * buffer of WINATTN_STATIC_WORKSPACE_BYTES (every GPU that loads the library
+ * holds it until the process exits).  Problems whose four maps do not fit
+ * (winattn_host_workspace_bytes(...) > WINATTN_STATIC_WORKSPACE_BYTES) return
+ * WINATTN_ERR_SIZE before anything is enqueued.  Allocates nothing: no
+ * cudaMalloc, cudaFree or allocating library call.
+ *
+ * The first call on a device looks up the buffer's device address with that
+ * device current; make that first call before any stream capture.  Every call
+ * on a device shares the one buffer and leaves its contents behind (each call
+ * overwrites all of what it reads), so calls whose work overlaps on the GPU
+ * (other streams, or host threads) race on it: order them on one stream.
+ */
+#define WINATTN_STATIC_WORKSPACE_BYTES ((size_t)32 << 20)
+int winattn_fwd_host_static(const void *q_host, const void *k_host, const void *v_host,
+                            const float *theta, const void *bias_feats,
+                            int B, int H_img, int W_img, int M, int shift,
+                            int heads, int d, int rank, int dtype,
+                            void *out_host, void *stream);
+
 /* A static, human-readable description of a return code. */
 const char *winattn_strerror(int code);
 

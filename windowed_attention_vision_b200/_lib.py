@@ -18,7 +18,8 @@ ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_ALIAS, ERR_SIZE = -6, -7, -8, -9
 BF16, FP32 = 0, 1
 
 EXPORTS = ("winattn_fwd", "winattn_check_args", "winattn_fwd_host", "winattn_host_workspace_bytes",
-           "winattn_strerror", "winattn_last_device_status", "winattn_launch_info")
+           "winattn_strerror", "winattn_last_device_status", "winattn_launch_info", "winattn_fwd_host_static")
+STATIC_WORKSPACE_BYTES = 32 << 20
 
 
 class WinattnError(RuntimeError):
@@ -46,6 +47,8 @@ def load(path: str = LIB_PATH):
     lib.winattn_check_args.restype = i32
     lib.winattn_fwd_host.argtypes = [vp, vp, vp, vp, vp] + [i32] * 9 + [vp, vp, sz, vp]
     lib.winattn_fwd_host.restype = i32
+    lib.winattn_fwd_host_static.argtypes = [vp, vp, vp, vp, vp] + [i32] * 9 + [vp, vp]
+    lib.winattn_fwd_host_static.restype = i32
     lib.winattn_host_workspace_bytes.argtypes = [i32] * 6
     lib.winattn_host_workspace_bytes.restype = sz
     lib.winattn_strerror.argtypes = [i32]
@@ -78,6 +81,12 @@ def fwd_host(q_ptr, k_ptr, v_ptr, theta_ptr, bias_ptr, B, H, W, M, shift, heads,
              ws_ptr, ws_bytes, stream) -> int:
     return load().winattn_fwd_host(q_ptr, k_ptr, v_ptr, theta_ptr, bias_ptr, B, H, W, M, shift, heads, d,
                                    rank, dtype, out_ptr, ws_ptr, ws_bytes, stream)
+
+
+def fwd_host_static(q_ptr, k_ptr, v_ptr, theta_ptr, bias_ptr, B, H, W, M, shift, heads, d, rank, dtype, out_ptr,
+                    stream) -> int:
+    return load().winattn_fwd_host_static(q_ptr, k_ptr, v_ptr, theta_ptr, bias_ptr, B, H, W, M, shift, heads, d,
+                                          rank, dtype, out_ptr, stream)
 
 
 def host_workspace_bytes(B, H, W, heads, d, dtype) -> int:

@@ -538,6 +538,58 @@ int winattn_fwd_host(const void *q_host, const void *k_host, const void *v_host,
     return WINATTN_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
+// Library-owned device workspace of winattn_fwd_host_static (the device copies
+// of q, k, v and out).  In host code the name stands for a host-side shadow,
+// not a device address: the device address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) uint8_t g_static_workspace[WINATTN_STATIC_WORKSPACE_BYTES];
+
+// Device address of g_static_workspace on the current device, looked up once
+// per device with that device current; nullptr if the lookup failed.
+void *static_workspace_ptr()
+{
+    static std::mutex mu;
+    static void *cached[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!cached[dev]) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_static_workspace) != cudaSuccess)
+            return nullptr;
+        cached[dev] = ptr;
+    }
+    return cached[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+int winattn_fwd_host_static(const void *q_host, const void *k_host, const void *v_host, const float *theta,
+                            const void *bias_feats, int B, int H_img, int W_img, int M, int shift, int heads, int d,
+                            int rank, int dtype, void *out_host, void *stream)
+{
+    const int rc = check_sizes(B, H_img, W_img, M, shift, heads, d, rank, dtype);
+    if (rc != WINATTN_OK)
+        return rc;
+    const size_t need = winattn_host_workspace_bytes(B, H_img, W_img, heads, d, dtype);
+    if (need == 0 || need > WINATTN_STATIC_WORKSPACE_BYTES)
+        return WINATTN_ERR_SIZE;
+    const int dev_rc = check_device();
+    if (dev_rc != WINATTN_OK)
+        return dev_rc;
+    void *ws = static_workspace_ptr();
+    if (!ws)
+        return WINATTN_ERR_CUDA;
+    return winattn_fwd_host(q_host, k_host, v_host, theta, bias_feats, B, H_img, W_img, M, shift, heads, d, rank,
+                            dtype, out_host, ws, WINATTN_STATIC_WORKSPACE_BYTES, stream);
+}
+
 const char *winattn_strerror(int code)
 {
     switch (code) {
