@@ -155,29 +155,15 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         *abort_flag = 0u;
         fence_mbar_init();
     }
+    // the tensor maps (kernel parameters, not data) are fetched one per lane
+    if (warp == kPipeLoadWarp && lane < 12)
+        tma_prefetch_map(pick_map(lane < 4 ? tm_q : (lane < 8 ? tm_k : tm_o), lane & 3));
+    if (warp == kPipeLoadWarp + 3 && lane < 4)
+        tma_prefetch_map(pick_map(tm_v, lane));
     // TMEM and the barriers are set up; nothing of global memory is touched
     // before the previous kernel of the stream has completed
     grid_launch_dependents();
     grid_dependency_wait();
-    if (theta) {
-        // table4[h][pos][k/2] = (cos k, cos k+1, sin k, sin k+1) of pos * theta_h[k], even k
-        float *tf = reinterpret_cast<float *>(table);
-        for (int idx = t; idx < g.heads * kTab; idx += blockDim.x) {
-            const int h = idx / kTab, r = idx - h * kTab;
-            const int c = r / (D / 4), kk = r - c * (D / 4);
-            float sn, cs;
-            sincosf((float)c * __ldg(theta + h * (D / 4) + kk), &sn, &cs);
-            float *e = tf + 2 * ((h * 8 + c) * (D / 4) + (kk & ~1));
-            e[kk & 1] = cs;
-            e[2 + (kk & 1)] = sn;
-        }
-    }
-    for (int idx = t; idx < 4 * 64; idx += blockDim.x) {
-        const int kind = idx >> 6, rp = idx & 63;
-        int i, j;
-        tma_row_coords(g, kind, rp, i, j);
-        ijtab[idx] = (uint16_t)((i << 8) | j);
-    }
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
@@ -225,13 +211,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
 
     if (warp == kPipeLoadWarp) {
         // ================================================================ Q/K loader
-        if (lane == 0) {
-            for (int kind = 0; kind < 4; ++kind) {
-                tma_prefetch_map(pick_map(tm_q, kind));
-                tma_prefetch_map(pick_map(tm_k, kind));
-                tma_prefetch_map(pick_map(tm_o, kind));
-            }
-        }
+        // (starts right after the CTA barrier: the first tiles' DRAM latency
+        // overlaps the RoPE warps' table setup)
         for (int kk = 0; kk < count; ++kk) {
             const int s = kk % NSQ;
             if (kk >= NSQ && !warp_wait(&qk_empty[s], ((kk / NSQ) - 1) & 1, abort_flag))
@@ -250,10 +231,6 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         }
     } else if (warp == kPipeLoadWarp + 3) {
         // ================================================================ V loader
-        if (lane == 0) {
-            for (int kind = 0; kind < 4; ++kind)
-                tma_prefetch_map(pick_map(tm_v, kind));
-        }
         for (int kk = 0; kk < count; ++kk) {
             const int s = kk % NSV;
             // once the tile's RoPE is done, V has about the S and softmax
@@ -343,6 +320,29 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         }
     } else if (warp < kPipeSoftmaxWarp) {
         // ================================================================ RoPE groups
+        // the tables only these warps read: RoPE (cos, sin) of each head,
+        // table4[h][pos][k/2] = (cos k, cos k+1, sin k, sin k+1) of
+        // pos * theta_h[k], even k; and the window-local (i, j) of each row
+        // of a box of each kind
+        if (theta) {
+            float *tf = reinterpret_cast<float *>(table);
+            for (int idx = t; idx < g.heads * kTab; idx += 32 * kPipeSoftmaxWarp) {
+                const int h = idx / kTab, r = idx - h * kTab;
+                const int c = r / (D / 4), kk = r - c * (D / 4);
+                float sn, cs;
+                sincosf((float)c * __ldg(theta + h * (D / 4) + kk), &sn, &cs);
+                float *e = tf + 2 * ((h * 8 + c) * (D / 4) + (kk & ~1));
+                e[kk & 1] = cs;
+                e[2 + (kk & 1)] = sn;
+            }
+        }
+        for (int idx = t; idx < 4 * 64; idx += 32 * kPipeSoftmaxWarp) {
+            const int kind = idx >> 6, rp = idx & 63;
+            int i, j;
+            tma_row_coords(g, kind, rp, i, j);
+            ijtab[idx] = (uint16_t)((i << 8) | j);
+        }
+        named_bar_sync(1, 32 * kPipeSoftmaxWarp);
         const int grp = warp >> 2;
         const int row = t - 128 * grp;
         const int slot = row >> 6, rp = row & 63;

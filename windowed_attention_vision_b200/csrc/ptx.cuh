@@ -52,22 +52,6 @@ __device__ __forceinline__ uint32_t mbar_try_wait(uint64_t *bar, uint32_t parity
     return ok;
 }
 
-// The same with a suspend-time hint: a thread whose phase is not complete
-// sleeps in hardware until it completes or about `hint_ns` pass, instead of
-// spinning through the issue slots other warps need.
-__device__ __forceinline__ uint32_t mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns)
-{
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
-        : "memory");
-    return ok;
-}
-
 // Non-blocking probe of a phase (for polling loops).
 __device__ __forceinline__ uint32_t mbar_test_wait(uint64_t *bar, uint32_t parity)
 {
@@ -90,16 +74,13 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar)
 // Every wait in this library is bounded: it gives up after kWaitLimitNs of
 // wall time (read from %globaltimer) and reports false.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-// Longest a thread stays suspended in one try_wait before it re-checks the
-// time limit and the abort flag (it wakes as soon as the phase completes).
-constexpr uint32_t kSuspendHintNs = 1000000u;
 
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
 {
-    if (mbar_try_wait_sleep(bar, parity, kSuspendHintNs))
+    if (mbar_try_wait(bar, parity))
         return true;
     const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait_sleep(bar, parity, kSuspendHintNs)) {
+    while (!mbar_try_wait(bar, parity)) {
         if (globaltimer_ns() - t0 > kWaitLimitNs)
             return false;
     }

@@ -8,16 +8,17 @@
 
 namespace winattn {
 
-// Bounded wait that also gives up as soon as another role has aborted.  The
-// try_wait carries a suspend-time hint, so a waiting thread sleeps in
-// hardware until the phase completes (or the hint runs out) instead of
-// polling: a polling warp takes issue slots from the warps doing the work.
+// Bounded wait that also gives up as soon as another role has aborted.  A
+// try_wait blocks in hardware until the phase completes or a system-dependent
+// time passes (thousands of cycles), so a waiting warp takes almost no issue
+// slots from the warps doing the work.  Without a suspend-time hint it wakes
+// sooner after the phase completes (measured per tile on the pipelined kernel).
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile uint32_t *abort_flag)
 {
-    if (mbar_try_wait_sleep(bar, parity, kSuspendHintNs))
+    if (mbar_try_wait(bar, parity))
         return true;
     const uint64_t t0 = globaltimer_ns();
-    while (!mbar_try_wait_sleep(bar, parity, kSuspendHintNs)) {
+    while (!mbar_try_wait(bar, parity)) {
         if (*abort_flag)
             return false;
         if (globaltimer_ns() - t0 > kWaitLimitNs) {
