@@ -37,7 +37,9 @@
 //                    each P is ready.
 // TMEM: NB S buffers of BN fp32 columns (NB = 3 at BN = 128, 4 at BN = 96;
 // P as bf16 pairs over the first BN/2 columns of its buffer), then O of tile
-// A and of tile B (d columns each).
+// A and of tile B (d columns each), twice at d = 32: items alternate between
+// the two O buffers, so an item's epilogue can trail the next item's first
+// step.
 // Wrap masks are structural: a key tile lies on one side of the row seam,
 // and its two boxes on the two sides of the column seam, so each query row
 // keeps all, none, or one half of a tile.
@@ -158,6 +160,52 @@ struct LargeMaps {
     CUtensorMap k_full, k_half, v_full, v_half, w;
 };
 
+// Epilogue of one query row of item ke: waits for the item's last P V, writes
+// O / l (bf16) to `dst` (the token's original position) and hands the O
+// buffer (ke % NOB) back to the P V issuer.
+template <int D, int NOB>
+__device__ __forceinline__ bool large_epilogue_body(__nv_bfloat16 *dst_row, uint32_t obase, int ke, float le, uint64_t *o_last,
+                                            uint64_t *t_free, volatile uint32_t *abort_flag)
+{
+    if (!warp_wait(o_last, ke & 1, abort_flag))
+        return false;
+    tc_fence_after_sync();
+    const uint32_t oe = obase + (ke % NOB) * 2 * D;
+    const float inv = 1.f / le;
+    const float2 i2 = make_float2(inv, inv);
+    uint4 *dst = reinterpret_cast<uint4 *>(dst_row);
+#pragma unroll
+    for (int ch = 0; ch < D / 16; ++ch) {
+        float o[16];
+        tmem_ld16(oe + ch * 16, o);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            float2 y[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                y[e] = __fmul2_rn(make_float2(o[8 * hh + 2 * e], o[8 * hh + 2 * e + 1]), i2);
+            uint4 u;
+            u.x = pack_bf16x2(y[0].x, y[0].y);
+            u.y = pack_bf16x2(y[1].x, y[1].y);
+            u.z = pack_bf16x2(y[2].x, y[2].y);
+            u.w = pack_bf16x2(y[3].x, y[3].y);
+            dst[2 * ch + hh] = u;
+        }
+    }
+    tc_fence_before_sync();
+    mbar_arrive(t_free);
+    return true;
+}
+
+// The same kept out of line, for the deferred epilogue inside the step loop,
+// where inlined it would cost the softmax registers.
+template <int D, int NOB>
+__device__ __noinline__ bool large_epilogue_call(__nv_bfloat16 *dst_row, uint32_t obase, int ke, float le,
+                                                 uint64_t *o_last, uint64_t *t_free, volatile uint32_t *abort_flag)
+{
+    return large_epilogue_body<D, NOB>(dst_row, obase, ke, le, o_last, t_free, abort_flag);
+}
+
 template <int D, int R, int BN>
 __global__ void __launch_bounds__(kLargeThreads, 1)
     winattn_fwd_large_kernel(const __nv_bfloat16 *__restrict__ q, const float *__restrict__ theta,
@@ -170,7 +218,11 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
     // then O of tile A and of tile B (D columns each)
     constexpr int NB = BN == 96 ? 4 : 3;
     constexpr uint32_t kOCol = NB * BN;
-    static_assert(kOCol + 2 * D <= 512, "TMEM columns");
+    // O buffers per query tile: two where TMEM has room (d = 32), so that an
+    // item's epilogue can wait behind the next item's first step; one at
+    // M = 96, where an item has 96 key tiles and the boundary is rare
+    constexpr int NOB = BN == 128 && kOCol + 4 * D <= 512 ? 2 : 1;
+    static_assert(kOCol + 2 * NOB * D <= 512, "TMEM columns");
     // S of step n + NB may need key tile cg + NB / 2 while tile cg (step n = 2 cg) is held
     static_assert(NS >= NB / 2 + 1, "ring too shallow for the S lookahead");
     extern __shared__ uint8_t smem_raw[];
@@ -351,8 +403,13 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
             bool ok = true;
             for (; c < steps && ok; ++c) {
                 const int n = 2 * c + tl, b = n % NB;
-                // O of this tile is free once the previous item's epilogue read it
-                if (p_jt == 0 && p_kk > 0 && !(ok = wait_or_abort(&t_free[tl], (p_kk - 1) & 1, abort_flag)))
+                // O buffer p_kk % NOB of this tile is free once the epilogue of
+                // item p_kk - NOB read it (with two buffers the softmax group
+                // has done that epilogue before it wrote any P of item
+                // p_kk - 1, all of which this issuer has consumed: no phase of
+                // t_free is pending behind the one waited for)
+                if (p_jt == 0 && p_kk >= NOB &&
+                    !(ok = wait_or_abort(&t_free[tl], (p_kk - NOB) & 1, abort_flag)))
                     break;
                 // S of this step exists, hence P V of the buffer's previous
                 // tenant (step n - NB, the other tile's) has completed and the
@@ -362,7 +419,7 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
                     break;
                 const uint32_t pa = tmem + b * BN;  // P over the first BN/2 columns of the buffer
                 const uint32_t vst = sbase + L::STAGES + (c % NS) * L::STAGE + L::VO;
-                const uint32_t od = tmem + NB * BN + tl * D;
+                const uint32_t od = tmem + kOCol + ((p_kk % NOB) * 2 + tl) * D;
                 // 16 keys of V are 32 D bytes: +2 D in the start-address field
                 const uint64_t vd = smem_desc(vst, 8192, 16 * D, swizzle_code(2 * D));
                 // parts end at chunks 1, 3 (and at the last chunk for BN = 96)
@@ -501,10 +558,24 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
         const int tile = warp >> 2;  // 0 = A, 1 = B
         const int row = t - 128 * tile;
         const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t oreg = tmem + lane_base + kOCol + tile * D;  // O of this tile, this warp's lanes
-        constexpr int NCH = BN / 16;                          // 16-column chunks of S
+        const uint32_t obase = tmem + lane_base + kOCol + tile * D;  // O buffer 0 of this tile, this warp's lanes
+        constexpr int NCH = BN / 16;                           // 16-column chunks of S
         int c = 0;
         bool failed = false;
+        auto epilogue = [&](int ke, int64_t off, float le) -> bool {
+            if constexpr (NOB == 2)
+                return large_epilogue_call<D, NOB>(out + off, obase, ke, le, &o_last[tile], &t_free[tile], abort_flag);
+            else
+                return large_epilogue_body<D, NOB>(out + off, obase, ke, le, &o_last[tile], &t_free[tile], abort_flag);
+        };
+        // With two O buffers an item's epilogue runs after the first step of
+        // the next item, when its last P V has long completed, instead of
+        // stalling the group at the item boundary.  Its wait on o_last cannot
+        // alias the next item's phase: a window has at least two key tiles,
+        // so that phase needs P this group has not yet written.
+        int pend_kk = -1;
+        int64_t pend_off = 0;
+        float pend_l = 1.f;
         for (int kk = 0; kk < count && !failed; ++kk) {
             int w, h, pair, b, wy, wx;
             decode(kk, w, h, pair);
@@ -515,6 +586,7 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
             // the item implies its query tiles are ready)
             const TokenRef me = token_ref(g, w, (2 * pair + tile) * 128 + row, h);
             const int me_ly = me.label >> 1, me_lx = me.label & 1;
+            const uint32_t oreg = obase + (kk % NOB) * 2 * D;  // O of this item
             // Online softmax in log2 units: m is the reference of the row's P
             // (exp2(s * c2 - m)); it moves, rescaling l and O, only when a
             // tile's max exceeds it by more than 2^8.
@@ -634,39 +706,27 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
                 }
                 const float2 l2 = __fadd2_rn(lq[0], lq[1]);
                 l = l * alpha + (l2.x + l2.y);
+                if (pend_kk >= 0) {
+                    if (!epilogue(pend_kk, pend_off, pend_l)) {
+                        failed = true;
+                        break;
+                    }
+                    pend_kk = -1;
+                }
             }
             if (failed)
                 break;
-            // ---- epilogue: O / l to the token's original position
-            if (!warp_wait(&o_last[tile], kk & 1, abort_flag)) {
+            if constexpr (NOB == 2) {
+                pend_kk = kk;
+                pend_off = me.offset;
+                pend_l = l;
+            } else if (!epilogue(kk, me.offset, l)) {
                 failed = true;
                 break;
             }
-            tc_fence_after_sync();
-            const float inv = 1.f / l;
-            const float2 i2 = make_float2(inv, inv);
-            uint4 *dst = reinterpret_cast<uint4 *>(out + me.offset);
-#pragma unroll
-            for (int ch = 0; ch < D / 16; ++ch) {
-                float o[16];
-                tmem_ld16(oreg + ch * 16, o);
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    float2 y[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        y[e] = __fmul2_rn(make_float2(o[8 * hh + 2 * e], o[8 * hh + 2 * e + 1]), i2);
-                    uint4 u;
-                    u.x = pack_bf16x2(y[0].x, y[0].y);
-                    u.y = pack_bf16x2(y[1].x, y[1].y);
-                    u.z = pack_bf16x2(y[2].x, y[2].y);
-                    u.w = pack_bf16x2(y[3].x, y[3].y);
-                    dst[2 * ch + hh] = u;
-                }
-            }
-            tc_fence_before_sync();
-            mbar_arrive(&t_free[tile]);
         }
+        if (!failed && pend_kk >= 0)
+            epilogue(pend_kk, pend_off, pend_l);
     }
 
     tc_fence_before_sync();
