@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     if (t == 32) {
         for (int s = 0; s < NSQ; ++s) {
             mbar_init(&qk_full[s], 1);
-            mbar_init(&ready[s], 128);
+            mbar_init(&ready[s], 4);       // one arrival per RoPE warp
             mbar_init(&qk_empty[s], 1);
         }
         for (int s = 0; s < NSV; ++s) {
@@ -143,12 +143,12 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
             mbar_init(&v_empty[s], 1);
         }
         for (int m = 0; m < NM; ++m)
-            mbar_init(&meta_full[m], 128);
+            mbar_init(&meta_full[m], 4);    // one arrival per RoPE warp
         for (int b = 0; b < NB; ++b) {
             mbar_init(&s_full[b], 1);
-            mbar_init(&p_full[b], 128);
+            mbar_init(&p_full[b], 4);       // one arrival per softmax warp
             mbar_init(&o_full[b], 1);
-            mbar_init(&t_free[b], 128);
+            mbar_init(&t_free[b], 4);       // one arrival per epilogue warp
         }
         mbar_init(&fin[0], 1);
         mbar_init(&fin[1], 1);
@@ -412,8 +412,11 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
             }
             reinterpret_cast<int64_t *>(ms)[row] = meta;
             fence_proxy_async_smem();
-            mbar_arrive(&ready[s]);
-            mbar_arrive(&meta_full[m]);
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&ready[s]);
+                mbar_arrive(&meta_full[m]);
+            }
         }
     } else if (warp < kPipeEpiWarp) {
         // ================================================================ softmax groups
@@ -489,7 +492,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
             osum[b * 128 + row] = l2.x + l2.y;
             tmem_wait_st();
             tc_fence_before_sync();
-            mbar_arrive(&p_full[b]);
+            warp_arrive(&p_full[b]);
         }
     } else if (warp < kPipeLoadWarp) {
         // ================================================================ epilogue
@@ -524,7 +527,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
                 tmem_ld32(tmem + lane_base + b * 128 + 64 + h2 * 32, o);
                 if (h2 == D / 32 - 1) {
                     tc_fence_before_sync();
-                    mbar_arrive(&t_free[b]);
+                    warp_arrive(&t_free[b]);
                 }
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
