@@ -48,6 +48,18 @@
 
 namespace winattn {
 
+// One arrival per warp on a barrier that counts warps rather than threads:
+// the warp barrier orders every lane's earlier writes (shared memory, and
+// tcgen05 operations the caller has fenced with tcgen05.fence::before_thread_sync)
+// before lane 0's release-arrive.  One arrive instead of 32 same-address
+// shared-memory atomics per warp.
+__device__ __forceinline__ void warp_arrive(uint64_t *bar)
+{
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0)
+        mbar_arrive(bar);
+}
+
 constexpr int kPipeRope = 2;                    // RoPE warpgroups (tile k goes to group k % 2)
 constexpr int kPipeSoftmaxWarp = 4 * kPipeRope; // first softmax warp
 constexpr int kPipeEpiWarp = kPipeSoftmaxWarp + 8;

@@ -37,16 +37,4 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     return __all_sync(0xffffffffu, wait_or_abort(bar, parity, abort_flag));
 }
 
-// One arrival per warp on a barrier that counts warps rather than threads:
-// the warp barrier orders every lane's earlier writes (shared memory, and
-// tcgen05 operations the caller has fenced with tcgen05.fence::before_thread_sync)
-// before lane 0's release-arrive.  One arrive instead of 32 same-address
-// shared-memory atomics per warp.
-__device__ __forceinline__ void warp_arrive(uint64_t *bar)
-{
-    __syncwarp();
-    if ((threadIdx.x & 31) == 0)
-        mbar_arrive(bar);
-}
-
 }  // namespace winattn
