@@ -41,6 +41,12 @@ SMALL = [
     ("m9_s4_r32", 2, 18, 9, 9, 4, 3, 32, "bf16", None, 32),
     ("m24_s0_r16", 1, 48, 48, 24, 0, 2, 32, "bf16", None, 16),      # bias factors, no RoPE
     ("m16_s0_d32", 2, 32, 48, 16, 0, 2, 32, "bf16", "learned", 0),  # large-window kernel from here on
+    # several items per CTA: both O buffers of a query tile in turn, and the
+    # epilogue of each item trailing the next item's first step
+    ("m16_s8_d32_items", 8, 64, 64, 16, 8, 4, 32, "bf16", "learned", 0),
+    ("m32_s16_d32_items", 8, 64, 64, 32, 16, 3, 32, "bf16", "learned", 0),
+    ("m32_s0_d32_items", 8, 64, 64, 32, 0, 3, 32, "bf16", "standard", 0),
+    ("m16_s8_d64_items", 8, 64, 64, 16, 8, 2, 64, "bf16", "learned", 0),  # one O buffer
     ("m16_s8_d32_nope", 1, 32, 32, 16, 8, 3, 32, "bf16", None, 0),
     ("m32_s0_d64", 1, 64, 96, 32, 0, 2, 64, "bf16", "standard", 0),
     ("m32_s0_r16", 1, 64, 64, 32, 0, 2, 32, "bf16", None, 16),
