@@ -54,6 +54,14 @@
 namespace winattn {
 
 constexpr int kLargeThreads = 16 * 32;
+// Register split of a CTA launched with 128 registers per thread: the two
+// softmax warpgroups hold a whole row of S (BN fp32 values) in registers
+// between the max and the exp pass; the converter and the single-thread roles
+// need far fewer.  The shares add up to the launch's total, so no .inc waits.
+constexpr uint32_t kLargeRegsLaunch = 128, kLargeRegsSoftmax = 184, kLargeRegsConv = 80, kLargeRegsIssue = 64;
+static_assert(2 * 128 * kLargeRegsSoftmax + 128 * kLargeRegsConv + 128 * kLargeRegsIssue ==
+                  kLargeThreads * kLargeRegsLaunch,
+              "register split must add up to the launch's registers");
 constexpr uint32_t kLargeSmemBudget = 220 * 1024;
 
 // Keys per tile: 128 (8, 4 or 2 window rows for M = 16, 32, 64), or one
@@ -298,161 +306,169 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
         wx = rem - wy * g.nWx;
     };
 
-    if (warp == 12) {
-        // ============================================================ TMA loader
-        if (lane == 0) {
-            int c = 0;
-            bool ok = true;
-            const uint32_t bytes = (uint32_t)(BN * 2 * (2 * D + R));
-            for (int kk = 0; kk < count && ok; ++kk) {
-                int w, h, pair, b, wy, wx;
-                decode(kk, w, h, pair);
-                window_pos(w, b, wy, wx);
-                const bool xwrap = g.shift && wx == g.nWx - 1;
-                for (int jt = 0; jt < nkv; ++jt, ++c) {
-                    const int s = c % NS;
-                    if (c >= NS && !wait_or_abort(&kv_empty[s], ((c / NS) - 1) & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    const uint32_t sst = sbase + L::STAGES + s * L::STAGE;
-                    mbar_arrive_expect_tx(&kv_full[s], bytes);
-                    int y0 = wy * M + jt * kr + g.shift;
-                    if (y0 >= g.H) y0 -= g.H;
-                    const int x0 = wx * M + g.shift;  // < W unless the window straddles the seam
-                    const int c0 = h * D;
-                    if (xwrap) {
-                        const int x1 = 0;             // the seam's far side
-                        const uint32_t half = (uint32_t)(BN / 2) * 2 * D;
-                        tma_load_4d(sst + L::KC, &maps.k_half, c0, x0, y0, b, &kv_full[s]);
-                        tma_load_4d(sst + L::KC + half, &maps.k_half, c0, x1, y0, b, &kv_full[s]);
-                        tma_load_4d(sst + L::VO, &maps.v_half, c0, x0, y0, b, &kv_full[s]);
-                        tma_load_4d(sst + L::VO + half, &maps.v_half, c0, x1, y0, b, &kv_full[s]);
-                    } else {
-                        tma_load_4d(sst + L::KC, &maps.k_full, c0, x0, y0, b, &kv_full[s]);
-                        tma_load_4d(sst + L::VO, &maps.v_full, c0, x0, y0, b, &kv_full[s]);
-                    }
-                    if constexpr (R > 0)
-                        tma_load_2d(sst + L::KB, &maps.w, 0, (h * 2 + 1) * N + jt * BN, &kv_full[s]);
-                }
-            }
-        }
-    } else if (warp == 13) {
-        // ============================================================ S issuer
-        // One sequence over the CTA's items: step n = 2 cg + t is query tile t
-        // (0 = A, 1 = B) against the CTA's cg-th key tile.  S of step n goes to
-        // TMEM buffer n % NB once P V of step n - NB (the buffer's previous
-        // tenant) has completed.
-        if (lane == 0) {
-            constexpr uint32_t kIdescS = idesc_bf16_f32(128, BN, false);
-            const int total = 2 * count * nkv;
-            int s_kk = 0, s_jt = 0;  // item and key tile of the next S
-            int ns = 0;
-            for (; ns < total; ++ns) {
-                const int tl = ns & 1, cg = ns >> 1;
-                if (ns >= NB && !wait_or_abort(&pv_done[ns % NB], ((ns / NB) - 1) & 1, abort_flag))
-                    break;
-                if (tl == 0) {
-                    if (s_jt == 0 && !wait_or_abort(&q_ready[s_kk & 1], (s_kk >> 1) & 1, abort_flag))
-                        break;
-                    if (!wait_or_abort(&kv_ready[cg % NS], (cg / NS) & 1, abort_flag))
-                        break;
-                }
-                tc_fence_after_sync();
-                const uint32_t qtile = sbase + (s_kk & 1) * L::QBUF + tl * L::QTILE;
-                const uint32_t d = tmem + (ns % NB) * BN;
-                const uint32_t kst = sbase + L::STAGES + (cg % NS) * L::STAGE;
-                // descriptors built once per step; a 16-element K step is
-                // +32 bytes, i.e. +2 in the 16-byte start-address field
-                const uint64_t qd = smem_desc(qtile, 16, 16 * D, swizzle_code(2 * D));
-                const uint64_t kd = smem_desc(kst + L::KC, 16, 16 * D, swizzle_code(2 * D));
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks)
-                    umma_bf16_ss(d, qd + 2 * ks, kd + 2 * ks, kIdescS, ks > 0);
-                if constexpr (R > 0) {
-                    const uint64_t qbd = smem_desc(qtile + 256 * D, 16, 16 * R, swizzle_code(2 * R));
-                    const uint64_t kbd = smem_desc(kst + L::KB, 16, 16 * R, swizzle_code(2 * R));
-#pragma unroll
-                    for (int ks = 0; ks < R / 16; ++ks)
-                        umma_bf16_ss(d, qbd + 2 * ks, kbd + 2 * ks, kIdescS, 1);
-                }
-                umma_commit(&s_full[ns % NB]);
-                if (tl == 1 && ++s_jt == nkv) {
-                    umma_commit(&q_free[s_kk & 1]);  // the last S that reads this item's Q
-                    s_jt = 0;
-                    ++s_kk;
-                }
-            }
-            if (ns > 0) {
-                umma_commit(&fin[0]);
-                mbar_wait(&fin[0], 0);
-            }
-        }
-    } else if (warp == 14 || warp == 15) {
-        // ============================================================ P V issuers
-        // One per query tile: O_t += P V chunk by chunk (32 keys, two MMAs)
-        // as the softmax writes each chunk of P, so that P V overlaps the
-        // exponentials and the S buffer returns right after the last chunk.
-        const int tl = warp - 14;
-        if (lane == 0) {
-            constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
-            constexpr int NC = BN / 32;
-            const int steps = count * nkv;
-            int p_kk = 0, p_jt = 0;  // item and key tile of this tile's next P V
-            int c = 0;
-            bool ok = true;
-            for (; c < steps && ok; ++c) {
-                const int n = 2 * c + tl, b = n % NB;
-                // O buffer p_kk % NOB of this tile is free once the epilogue of
-                // item p_kk - NOB read it (with two buffers the softmax group
-                // has done that epilogue before it wrote any P of item
-                // p_kk - 1, all of which this issuer has consumed: no phase of
-                // t_free is pending behind the one waited for)
-                if (p_jt == 0 && p_kk >= NOB &&
-                    !(ok = wait_or_abort(&t_free[tl], (p_kk - NOB) & 1, abort_flag)))
-                    break;
-                // S of this step exists, hence P V of the buffer's previous
-                // tenant (step n - NB, the other tile's) has completed and the
-                // chunk barriers of buffer b are on this step's phase: a
-                // parity wait must never run a phase ahead of its barrier
-                if (!(ok = wait_or_abort(&s_full[b], (n / NB) & 1, abort_flag)))
-                    break;
-                const uint32_t pa = tmem + b * BN;  // P over the first BN/2 columns of the buffer
-                const uint32_t vst = sbase + L::STAGES + (c % NS) * L::STAGE + L::VO;
-                const uint32_t od = tmem + kOCol + ((p_kk % NOB) * 2 + tl) * D;
-                // 16 keys of V are 32 D bytes: +2 D in the start-address field
-                const uint64_t vd = smem_desc(vst, 8192, 16 * D, swizzle_code(2 * D));
-                // parts end at chunks 1, 3 (and at the last chunk for BN = 96)
-#pragma unroll
-                for (int ch = 0; ch < NC; ++ch) {
-                    if ((ch & 1) || ch == NC - 1) {
-                        if (!(ok = wait_or_abort(&p_part[b * 4 + ch], (n / NB) & 1, abort_flag)))
+    // Each warpgroup takes its register share first (one setmaxnreg per
+    // warpgroup, at the head of its branch; the host launches this kernel
+    // only when it was built with exactly kLargeRegsLaunch registers per
+    // thread, so the shares add up).
+    if (warp >= 12) {
+        warpgroup_regs_dec<kLargeRegsIssue>();
+        if (warp == 12) {
+            // ============================================================ TMA loader
+            if (lane == 0) {
+                int c = 0;
+                bool ok = true;
+                const uint32_t bytes = (uint32_t)(BN * 2 * (2 * D + R));
+                for (int kk = 0; kk < count && ok; ++kk) {
+                    int w, h, pair, b, wy, wx;
+                    decode(kk, w, h, pair);
+                    window_pos(w, b, wy, wx);
+                    const bool xwrap = g.shift && wx == g.nWx - 1;
+                    for (int jt = 0; jt < nkv; ++jt, ++c) {
+                        const int s = c % NS;
+                        if (c >= NS && !wait_or_abort(&kv_empty[s], ((c / NS) - 1) & 1, abort_flag)) {
+                            ok = false;
                             break;
-                        tc_fence_after_sync();
-                        const int c0 = ch & ~1;
-#pragma unroll
-                        for (int ks = 2 * c0; ks < 2 * ch + 2; ++ks)
-                            umma_bf16_ts(od, pa + ks * 8, vd + (uint64_t)(2 * D * ks), kIdescPV, p_jt > 0 || ks > 0);
+                        }
+                        const uint32_t sst = sbase + L::STAGES + s * L::STAGE;
+                        mbar_arrive_expect_tx(&kv_full[s], bytes);
+                        int y0 = wy * M + jt * kr + g.shift;
+                        if (y0 >= g.H) y0 -= g.H;
+                        const int x0 = wx * M + g.shift;  // < W unless the window straddles the seam
+                        const int c0 = h * D;
+                        if (xwrap) {
+                            const int x1 = 0;             // the seam's far side
+                            const uint32_t half = (uint32_t)(BN / 2) * 2 * D;
+                            tma_load_4d(sst + L::KC, &maps.k_half, c0, x0, y0, b, &kv_full[s]);
+                            tma_load_4d(sst + L::KC + half, &maps.k_half, c0, x1, y0, b, &kv_full[s]);
+                            tma_load_4d(sst + L::VO, &maps.v_half, c0, x0, y0, b, &kv_full[s]);
+                            tma_load_4d(sst + L::VO + half, &maps.v_half, c0, x1, y0, b, &kv_full[s]);
+                        } else {
+                            tma_load_4d(sst + L::KC, &maps.k_full, c0, x0, y0, b, &kv_full[s]);
+                            tma_load_4d(sst + L::VO, &maps.v_full, c0, x0, y0, b, &kv_full[s]);
+                        }
+                        if constexpr (R > 0)
+                            tma_load_2d(sst + L::KB, &maps.w, 0, (h * 2 + 1) * N + jt * BN, &kv_full[s]);
                     }
                 }
-                if (!ok)
-                    break;
-                umma_commit(&o_done[tl]);
-                if (p_jt == nkv - 1)
-                    umma_commit(&o_last[tl]);
-                umma_commit(&pv_done[b]);
-                umma_commit(&kv_empty[c % NS]);
-                if (++p_jt == nkv) {
-                    p_jt = 0;
-                    ++p_kk;
+            }
+        } else if (warp == 13) {
+            // ============================================================ S issuer
+            // One sequence over the CTA's items: step n = 2 cg + t is query tile t
+            // (0 = A, 1 = B) against the CTA's cg-th key tile.  S of step n goes to
+            // TMEM buffer n % NB once P V of step n - NB (the buffer's previous
+            // tenant) has completed.
+            if (lane == 0) {
+                constexpr uint32_t kIdescS = idesc_bf16_f32(128, BN, false);
+                const int total = 2 * count * nkv;
+                int s_kk = 0, s_jt = 0;  // item and key tile of the next S
+                int ns = 0;
+                for (; ns < total; ++ns) {
+                    const int tl = ns & 1, cg = ns >> 1;
+                    if (ns >= NB && !wait_or_abort(&pv_done[ns % NB], ((ns / NB) - 1) & 1, abort_flag))
+                        break;
+                    if (tl == 0) {
+                        if (s_jt == 0 && !wait_or_abort(&q_ready[s_kk & 1], (s_kk >> 1) & 1, abort_flag))
+                            break;
+                        if (!wait_or_abort(&kv_ready[cg % NS], (cg / NS) & 1, abort_flag))
+                            break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t qtile = sbase + (s_kk & 1) * L::QBUF + tl * L::QTILE;
+                    const uint32_t d = tmem + (ns % NB) * BN;
+                    const uint32_t kst = sbase + L::STAGES + (cg % NS) * L::STAGE;
+                    // descriptors built once per step; a 16-element K step is
+                    // +32 bytes, i.e. +2 in the 16-byte start-address field
+                    const uint64_t qd = smem_desc(qtile, 16, 16 * D, swizzle_code(2 * D));
+                    const uint64_t kd = smem_desc(kst + L::KC, 16, 16 * D, swizzle_code(2 * D));
+    #pragma unroll
+                    for (int ks = 0; ks < D / 16; ++ks)
+                        umma_bf16_ss(d, qd + 2 * ks, kd + 2 * ks, kIdescS, ks > 0);
+                    if constexpr (R > 0) {
+                        const uint64_t qbd = smem_desc(qtile + 256 * D, 16, 16 * R, swizzle_code(2 * R));
+                        const uint64_t kbd = smem_desc(kst + L::KB, 16, 16 * R, swizzle_code(2 * R));
+    #pragma unroll
+                        for (int ks = 0; ks < R / 16; ++ks)
+                            umma_bf16_ss(d, qbd + 2 * ks, kbd + 2 * ks, kIdescS, 1);
+                    }
+                    umma_commit(&s_full[ns % NB]);
+                    if (tl == 1 && ++s_jt == nkv) {
+                        umma_commit(&q_free[s_kk & 1]);  // the last S that reads this item's Q
+                        s_jt = 0;
+                        ++s_kk;
+                    }
+                }
+                if (ns > 0) {
+                    umma_commit(&fin[0]);
+                    mbar_wait(&fin[0], 0);
                 }
             }
-            if (c > 0) {
-                umma_commit(&fin[1 + tl]);
-                mbar_wait(&fin[1 + tl], 0);
+        } else if (warp == 14 || warp == 15) {
+            // ============================================================ P V issuers
+            // One per query tile: O_t += P V chunk by chunk (32 keys, two MMAs)
+            // as the softmax writes each chunk of P, so that P V overlaps the
+            // exponentials and the S buffer returns right after the last chunk.
+            const int tl = warp - 14;
+            if (lane == 0) {
+                constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
+                constexpr int NC = BN / 32;
+                const int steps = count * nkv;
+                int p_kk = 0, p_jt = 0;  // item and key tile of this tile's next P V
+                int c = 0;
+                bool ok = true;
+                for (; c < steps && ok; ++c) {
+                    const int n = 2 * c + tl, b = n % NB;
+                    // O buffer p_kk % NOB of this tile is free once the epilogue of
+                    // item p_kk - NOB read it (with two buffers the softmax group
+                    // has done that epilogue before it wrote any P of item
+                    // p_kk - 1, all of which this issuer has consumed: no phase of
+                    // t_free is pending behind the one waited for)
+                    if (p_jt == 0 && p_kk >= NOB &&
+                        !(ok = wait_or_abort(&t_free[tl], (p_kk - NOB) & 1, abort_flag)))
+                        break;
+                    // S of this step exists, hence P V of the buffer's previous
+                    // tenant (step n - NB, the other tile's) has completed and the
+                    // chunk barriers of buffer b are on this step's phase: a
+                    // parity wait must never run a phase ahead of its barrier
+                    if (!(ok = wait_or_abort(&s_full[b], (n / NB) & 1, abort_flag)))
+                        break;
+                    const uint32_t pa = tmem + b * BN;  // P over the first BN/2 columns of the buffer
+                    const uint32_t vst = sbase + L::STAGES + (c % NS) * L::STAGE + L::VO;
+                    const uint32_t od = tmem + kOCol + ((p_kk % NOB) * 2 + tl) * D;
+                    // 16 keys of V are 32 D bytes: +2 D in the start-address field
+                    const uint64_t vd = smem_desc(vst, 8192, 16 * D, swizzle_code(2 * D));
+                    // parts end at chunks 1, 3 (and at the last chunk for BN = 96)
+    #pragma unroll
+                    for (int ch = 0; ch < NC; ++ch) {
+                        if ((ch & 1) || ch == NC - 1) {
+                            if (!(ok = wait_or_abort(&p_part[b * 4 + ch], (n / NB) & 1, abort_flag)))
+                                break;
+                            tc_fence_after_sync();
+                            const int c0 = ch & ~1;
+    #pragma unroll
+                            for (int ks = 2 * c0; ks < 2 * ch + 2; ++ks)
+                                umma_bf16_ts(od, pa + ks * 8, vd + (uint64_t)(2 * D * ks), kIdescPV, p_jt > 0 || ks > 0);
+                        }
+                    }
+                    if (!ok)
+                        break;
+                    umma_commit(&o_done[tl]);
+                    if (p_jt == nkv - 1)
+                        umma_commit(&o_last[tl]);
+                    umma_commit(&pv_done[b]);
+                    umma_commit(&kv_empty[c % NS]);
+                    if (++p_jt == nkv) {
+                        p_jt = 0;
+                        ++p_kk;
+                    }
+                }
+                if (c > 0) {
+                    umma_commit(&fin[1 + tl]);
+                    mbar_wait(&fin[1 + tl], 0);
+                }
             }
         }
     } else if (warp >= 8) {
+        warpgroup_regs_dec<kLargeRegsConv>();
         // ============================================================ converter
         const int ct = t - 256;
         constexpr int CD = D / 8, CR = R / 8;
@@ -554,6 +570,7 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
         }
         cp_async_wait_all();
     } else {
+        warpgroup_regs_inc<kLargeRegsSoftmax>();
         // ============================================================ softmax groups
         const int tile = warp >> 2;  // 0 = A, 1 = B
         const int row = t - 128 * tile;
@@ -611,17 +628,21 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
                     a0 = me_lx ? NCH / 2 : 0;
                     a1 = a0 + NCH / 2;
                 }
-                uint32_t buf[2][32];
-                // ---- pass 1: row max over the allowed columns (loads
-                // pipelined; four independent max chains)
+                // ---- pass 1: the row of S into registers (all loads in
+                // flight at once, one wait), then its max over the allowed
+                // columns (four independent max chains)
+                uint32_t sv[NC][32];
+#pragma unroll
+                for (int ch = 0; ch < NC; ++ch)
+                    tmem_ld32_issue(sreg + ch * 32, sv[ch]);
+                tmem_wait_ld32(sv[0]);
+#pragma unroll
+                for (int ch = 1; ch < NC; ++ch)
+                    reg_fence32(sv[ch]);
                 float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-                tmem_ld32_issue(sreg, buf[0]);
 #pragma unroll
                 for (int ch = 0; ch < NC; ++ch) {
-                    tmem_wait_ld32(buf[ch & 1]);
-                    if (ch + 1 < NC)
-                        tmem_ld32_issue(sreg + (ch + 1) * 32, buf[(ch + 1) & 1]);
-                    const uint32_t *xb = buf[ch & 1];
+                    const uint32_t *xb = sv[ch];
                     if (2 * ch >= a0 && 2 * ch < a1) {
 #pragma unroll
                         for (int e = 0; e < 16; e += 2)
@@ -667,19 +688,15 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
                         tmem_st16(oreg + ch * 16, ob);
                     }
                 }
-                // ---- pass 2: P = exp2(s * c2 - m) into TMEM over the consumed
-                // S; each 32-key chunk goes to P V as soon as it is written
+                // ---- pass 2: P = exp2(s * c2 - m) from the registers into
+                // TMEM over the consumed S; P goes to P V part by part
                 const float2 cc = make_float2(c2, c2), mm2 = make_float2(-m, -m);
                 float2 lq[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // two sum chains
                 uint64_t *parts = p_part + (n % NB) * 4;
-                tmem_ld32_issue(sreg, buf[0]);
 #pragma unroll
                 for (int ch = 0; ch < NC; ++ch) {
-                    tmem_wait_ld32(buf[ch & 1]);
                     // P chunk ch covers S columns [16 ch, 16 ch + 16), already read
-                    if (ch + 1 < NC)
-                        tmem_ld32_issue(sreg + (ch + 1) * 32, buf[(ch + 1) & 1]);
-                    const uint32_t *xb = buf[ch & 1];
+                    const uint32_t *xb = sv[ch];
                     const bool lo = 2 * ch >= a0 && 2 * ch < a1;
                     const bool hi = 2 * ch + 1 >= a0 && 2 * ch + 1 < a1;
                     uint32_t pk[16];

@@ -261,6 +261,32 @@ __device__ __forceinline__ void tmem_wait_ld32(uint32_t (&r)[32])
                  : "memory");
 }
 
+// Marks r[] as (re)defined here without emitting an instruction: placed after
+// a tcgen05.wait::ld that covered the load into r[] (issued with
+// tmem_ld32_issue), so that no use of r[] is scheduled before that wait.
+__device__ __forceinline__ void reg_fence32(uint32_t (&r)[32])
+{
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
+}
+
+// Per-thread register budget of the executing warpgroup (all four warps run
+// the same instruction): .inc waits until the CTA has released enough
+// registers, .dec releases them.  The launch's registers (threads x
+// registers per thread) bound the sum over the warpgroups.
+template <uint32_t N>
+__device__ __forceinline__ void warpgroup_regs_inc()
+{
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void warpgroup_regs_dec()
+{
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ------------------------------------------------------------------ UMMA
 
 // D[tmem] (+)= A[smem desc] * B[smem desc]^T, bf16 inputs, fp32 accumulator.

@@ -299,6 +299,14 @@ int launch_large(const void *q, const void *k, const void *v, const float *theta
     if (R > 0 && !encode_factor_map(&maps.w, bias, g, BN))
         return WINATTN_ERR_CUDA;
     auto kernel = winattn_fwd_large_kernel<D, R, BN>;
+    // the warpgroups' register shares add up to the launch's registers only
+    // at exactly kLargeRegsLaunch registers per thread: refuse any other build
+    static const bool regs_ok = [&] {
+        cudaFuncAttributes fa;
+        return cudaFuncGetAttributes(&fa, kernel) == cudaSuccess && fa.numRegs == (int)kLargeRegsLaunch;
+    }();
+    if (!regs_ok)
+        return WINATTN_ERR_CUDA;
     // all 512 TMEM columns per CTA: enough shared memory that no second CTA
     // is resident on the same SM
     const int need = (int)LargeLayout<D, R, BN>::BYTES;
