@@ -183,6 +183,19 @@ int winattn_launch_info(int B, int H_img, int W_img, int M, int shift, int heads
                         int rank, int dtype, int64_t *work_items, int *grid, int *threads,
                         int *smem_bytes, int *windows_per_tile, int *kernel);
 
+/*
+ * winattn_selftest_wait_timeout — failure-detection self-test (the pages
+ * have no counterpart): enqueues on `stream` a one-warp kernel that waits on
+ * an mbarrier nothing arrives at, through the bounded wait the attention
+ * kernels use.  The wait gives up after its limit (2 s of %globaltimer), the
+ * kernel records WINATTN_ERR_DEVICE_TIMEOUT in the status word and returns;
+ * a following winattn_last_device_status(stream) returns that code and the
+ * device stays usable.  Returns WINATTN_OK once enqueued, WINATTN_ERR_ARCH
+ * off sm_100, WINATTN_ERR_CUDA if the launch failed.  Touches no caller
+ * memory.
+ */
+int winattn_selftest_wait_timeout(void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -18,7 +18,8 @@ ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_ALIAS, ERR_SIZE = -6, -7, -8, -9
 BF16, FP32 = 0, 1
 
 EXPORTS = ("winattn_fwd", "winattn_check_args", "winattn_fwd_host", "winattn_host_workspace_bytes",
-           "winattn_strerror", "winattn_last_device_status", "winattn_launch_info", "winattn_fwd_host_static")
+           "winattn_strerror", "winattn_last_device_status", "winattn_launch_info", "winattn_fwd_host_static",
+           "winattn_selftest_wait_timeout")
 STATIC_WORKSPACE_BYTES = 32 << 20
 
 
@@ -57,6 +58,8 @@ def load(path: str = LIB_PATH):
     lib.winattn_last_device_status.restype = i32
     lib.winattn_launch_info.argtypes = [i32] * 9 + [ctypes.POINTER(i64)] + [ctypes.POINTER(i32)] * 5
     lib.winattn_launch_info.restype = i32
+    lib.winattn_selftest_wait_timeout.argtypes = [vp]
+    lib.winattn_selftest_wait_timeout.restype = i32
     _lib = lib
     return lib
 
@@ -95,6 +98,10 @@ def host_workspace_bytes(B, H, W, heads, d, dtype) -> int:
 
 def last_device_status(stream) -> int:
     return load().winattn_last_device_status(stream)
+
+
+def selftest_wait_timeout(stream) -> int:
+    return load().winattn_selftest_wait_timeout(stream)
 
 
 def launch_info(B, H, W, M, shift, heads, d, rank, dtype):

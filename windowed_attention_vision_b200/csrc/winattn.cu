@@ -576,6 +576,27 @@ void *static_workspace_ptr()
 
 }  // namespace
 
+namespace winattn {
+
+// One warp waits on an mbarrier that nothing arrives at, through the same
+// bounded wait every persistent kernel uses: the wait must give up after its
+// time limit, set the CTA's abort flag and the device status word, and
+// return, so the context stays usable.
+__global__ void selftest_wait_kernel()
+{
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ uint32_t abort_word;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_word = 0u;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    warp_wait(&bar, 0, &abort_word);
+}
+
+}  // namespace winattn
+
 extern "C" {
 
 int winattn_fwd_host_static(const void *q_host, const void *k_host, const void *v_host, const float *theta,
@@ -663,6 +684,15 @@ int winattn_launch_info(int B, int H_img, int W_img, int M, int shift, int heads
         if (smem_bytes) *smem_bytes = smem_bytes_for(g, dtype);
     }
     return WINATTN_OK;
+}
+
+int winattn_selftest_wait_timeout(void *stream)
+{
+    const int rc = check_device();
+    if (rc != WINATTN_OK)
+        return rc;
+    selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+    return cudaGetLastError() == cudaSuccess ? WINATTN_OK : WINATTN_ERR_CUDA;
 }
 
 }  // extern "C"
