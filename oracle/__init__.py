@@ -60,6 +60,8 @@ def _bind(lib):
     lib.oracle_rope.restype = i32
     lib.oracle_token_origin.argtypes = [i32] * 7 + [vp, vp]
     lib.oracle_token_origin.restype = i32
+    lib.oracle_bwd.argtypes = [vp, vp, vp, i32, vp, vp] + [i32] * 8 + [vp] * 6 + [i32]
+    lib.oracle_bwd.restype = i32
     return lib
 
 
@@ -128,6 +130,24 @@ class Oracle:
         if rc < 0:
             raise ValueError(f"oracle rejected the problem (code {rc})")
         return out
+
+    def bwd(self, q, k, v, dout, *, M, shift=0, theta=None, bias=None, nthreads=0):
+        """Gradients of a scalar loss given dout = dL/dO [B, H, W, heads, d]:
+        (dq, dk, dv, dtheta, dbias) in fp64; dtheta [heads, d/4] (None without
+        theta), dbias [heads, 2, M*M, rank] (None without bias)."""
+        q, k, v, theta, bias, code, (B, H, W, heads, d, rank) = self._prep(q, k, v, theta, bias, M)
+        dout = np.ascontiguousarray(dout, dtype=np.float64)
+        if dout.shape != q.shape:
+            raise ValueError("dout must have the shape of q")
+        dq, dk, dv = (np.zeros(q.shape, dtype=np.float64) for _ in range(3))
+        dtheta = None if theta is None else np.zeros((heads, d // 4), dtype=np.float64)
+        dbias = None if bias is None else np.zeros(bias.shape, dtype=np.float64)
+        rc = self.lib.oracle_bwd(_ptr(q), _ptr(k), _ptr(v), code, _ptr(theta), _ptr(bias),
+                                 B, H, W, M, shift, heads, d, rank, _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                                 _ptr(dtheta), _ptr(dbias), nthreads)
+        if rc < 0:
+            raise ValueError(f"oracle rejected the problem (code {rc})")
+        return dq, dk, dv, dtheta, dbias
 
     def rope(self, vec, i, j, theta_h) -> np.ndarray:
         """R(i, j) vec for one d-vector (window-local row i, column j)."""

@@ -38,6 +38,14 @@
  * Parity of every function here is pinned by the not-gpu tests (closed
  * forms, the displacement identity of the rotation, brute-force masked
  * global attention, Swin's slice-based region labels, planted mistakes).
+ *
+ * The backward (oracle_bwd) is the chain rule through the same steps: the
+ * gradients of a scalar loss with respect to q, k, v, the RoPE frequencies
+ * theta and the bias table, given the loss gradient dO at the output map.
+ * The FLASHSWIN page trains the model (section "무엇과 다른가": memory was
+ * what blocked training at large windows) with theta = exp(omega) learned
+ * (section "어떻게 동작하나"); dL/domega = theta * dL/dtheta.  It is pinned
+ * by central finite differences of the forward above.
  */
 #include <math.h>
 #include <pthread.h>
@@ -364,4 +372,235 @@ int oracle_token_origin(int H, int W, int M, int shift, int wy, int wx, int p, i
     *y = (wy * M + p / M + shift) % H;
     *x = (wx * M + p % M + shift) % W;
     return 0;
+}
+
+/* ---- backward ---------------------------------------------------------------
+ * For one unit, after unit_forward has left the rotated q~, k~, v and the
+ * probabilities P in the scratch, with dO the loss gradient at the unit's
+ * output rows (gathered from the same original positions):
+ *   dV[c]    = sum_a P[a][c] dO[a]
+ *   dP[a][c] = dO[a] . v[c]
+ *   dS[a][c] = P[a][c] (dP[a][c] - sum_c' P[a][c'] dP[a][c'])
+ *   dq~[a] = scale sum_c dS[a][c] k~[c],   dk~[c] = scale sum_a dS[a][c] q~[a]
+ *   du[a]  = sum_c dS[a][c] w[c],          dw[c]  = sum_a dS[a][c] u[a]
+ *   dq = R(i, j)^T dq~ = R(-i, -j) dq~,    dk likewise
+ *   dtheta_k += i (dx~_{2k+1} x~_{2k} - dx~_{2k} x~_{2k+1})
+ *             + j (dx~_{h+2k+1} x~_{h+2k} - dx~_{h+2k} x~_{h+2k+1})  for x = q and k, h = d/2
+ * (d/dtheta of the pair rotation by angle i*theta maps (x~0, x~1) to
+ * i (-x~1, x~0)).  Every token lies in exactly one window of a call, so dq,
+ * dk, dv are written, not accumulated; dtheta and the bias-table gradient sum
+ * over all windows and images of a head. */
+
+typedef struct {
+    const problem_t *p;
+    const double *dout;
+    double *dq, *dk, *dv;   /* maps like dout */
+    double *dtheta;         /* [heads][d/4] or NULL */
+    double *dbias;          /* [heads][2][N][rank] or NULL */
+    int64_t n_units;
+    int64_t next;
+    int failed;
+    pthread_mutex_t mu;
+} bwd_job_t;
+
+static void unit_backward(const problem_t *p, int b, int wy, int wx, int h, const scratch_t *w,
+                          const double *dout, double *dq, double *dk, double *dv,
+                          double *dtheta_h, double *dbias_h, double *g_o, double *g_s, double *g_q, double *g_k)
+{
+    const int M = p->M, N = M * M, d = p->d, r = p->rank;
+    const double scale = 1.0 / sqrt((double)p->d);  /* the forward's d^-1/2 */
+
+    /* dO of the unit's rows, from the tokens' original positions */
+    for (int t = 0; t < N; ++t) {
+        size_t off = rolled_token_offset(p, b, wy * M + t / M, wx * M + t % M, h);
+        memcpy(g_o + (size_t)t * d, dout + off, (size_t)d * sizeof(double));
+    }
+    /* dV, scattered straight to the map */
+    for (int c = 0; c < N; ++c) {
+        size_t off = rolled_token_offset(p, b, wy * M + c / M, wx * M + c % M, h);
+        for (int e = 0; e < d; ++e) {
+            double acc = 0.0;
+            for (int a = 0; a < N; ++a)
+                acc += w->s[(size_t)a * N + c] * g_o[(size_t)a * d + e];
+            dv[off + e] = acc;
+        }
+    }
+    /* dP, then dS in place */
+    for (int a = 0; a < N; ++a) {
+        double rowdot = 0.0;
+        for (int c = 0; c < N; ++c) {
+            double dp = 0.0;
+            for (int e = 0; e < d; ++e)
+                dp += g_o[(size_t)a * d + e] * w->v[(size_t)c * d + e];
+            g_s[(size_t)a * N + c] = dp;
+            rowdot += w->s[(size_t)a * N + c] * dp;
+        }
+        for (int c = 0; c < N; ++c)
+            g_s[(size_t)a * N + c] = w->s[(size_t)a * N + c] * (g_s[(size_t)a * N + c] - rowdot);
+    }
+    /* dq~, dk~ */
+    for (int a = 0; a < N; ++a)
+        for (int e = 0; e < d; ++e) {
+            double acc = 0.0;
+            for (int c = 0; c < N; ++c)
+                acc += g_s[(size_t)a * N + c] * w->k[(size_t)c * d + e];
+            g_q[(size_t)a * d + e] = scale * acc;
+        }
+    for (int c = 0; c < N; ++c)
+        for (int e = 0; e < d; ++e) {
+            double acc = 0.0;
+            for (int a = 0; a < N; ++a)
+                acc += g_s[(size_t)a * N + c] * w->q[(size_t)a * d + e];
+            g_k[(size_t)c * d + e] = scale * acc;
+        }
+    /* bias-table gradient: du (side 0, query rows) and dw (side 1, key rows) */
+    if (p->bias && dbias_h) {
+        for (int a = 0; a < N; ++a)
+            for (int e = 0; e < r; ++e) {
+                double acc = 0.0;
+                for (int c = 0; c < N; ++c)
+                    acc += g_s[(size_t)a * N + c] * read_elem(p->bias, p->dtype, (((size_t)h * 2 + 1) * N + c) * r + e);
+                dbias_h[(size_t)a * r + e] += acc;
+            }
+        for (int c = 0; c < N; ++c)
+            for (int e = 0; e < r; ++e) {
+                double acc = 0.0;
+                for (int a = 0; a < N; ++a)
+                    acc += g_s[(size_t)a * N + c] * read_elem(p->bias, p->dtype, (((size_t)h * 2 + 0) * N + a) * r + e);
+                dbias_h[((size_t)N + c) * r + e] += acc;
+            }
+    }
+    /* theta gradient, then back through the rotation */
+    const int half = d / 2;
+    for (int t = 0; t < N; ++t) {
+        const double i = (double)(t / M), j = (double)(t % M);
+        double *gq = g_q + (size_t)t * d, *gk = g_k + (size_t)t * d;
+        const double *xq = w->q + (size_t)t * d, *xk = w->k + (size_t)t * d;
+        if (p->theta) {
+            if (dtheta_h)
+                for (int k = 0; k < d / 4; ++k) {
+                    const int a0 = 2 * k, a1 = 2 * k + 1, b0 = half + 2 * k, b1 = half + 2 * k + 1;
+                    dtheta_h[k] += i * (gq[a1] * xq[a0] - gq[a0] * xq[a1]) + j * (gq[b1] * xq[b0] - gq[b0] * xq[b1]) +
+                                   i * (gk[a1] * xk[a0] - gk[a0] * xk[a1]) + j * (gk[b1] * xk[b0] - gk[b0] * xk[b1]);
+                }
+            const float *th = p->theta + (size_t)h * (d / 4);
+            rope_rotate(gq, d, -i, -j, th);
+            rope_rotate(gk, d, -i, -j, th);
+        }
+        size_t off = rolled_token_offset(p, b, wy * M + t / M, wx * M + t % M, h);
+        memcpy(dq + off, gq, (size_t)d * sizeof(double));
+        memcpy(dk + off, gk, (size_t)d * sizeof(double));
+    }
+}
+
+static void *bwd_worker(void *arg)
+{
+    bwd_job_t *job = (bwd_job_t *)arg;
+    const problem_t *p = job->p;
+    const size_t N = (size_t)p->M * p->M, d = (size_t)p->d, r = (size_t)p->rank;
+    const size_t nth = (size_t)p->heads * (d / 4), nbias = (size_t)p->heads * 2 * N * r;
+    scratch_t w;
+    w.q = malloc(N * d * sizeof(double));
+    w.k = malloc(N * d * sizeof(double));
+    w.v = malloc(N * d * sizeof(double));
+    w.s = malloc(N * N * sizeof(double));
+    double *o = malloc(N * d * sizeof(double));
+    double *g_o = malloc(N * d * sizeof(double)), *g_s = malloc(N * N * sizeof(double));
+    double *g_q = malloc(N * d * sizeof(double)), *g_k = malloc(N * d * sizeof(double));
+    double *dth = job->dtheta ? calloc(nth, sizeof(double)) : NULL;
+    double *dbi = job->dbias ? calloc(nbias > 0 ? nbias : 1, sizeof(double)) : NULL;
+    if (!w.q || !w.k || !w.v || !w.s || !o || !g_o || !g_s || !g_q || !g_k || (job->dtheta && !dth) ||
+        (job->dbias && !dbi)) {
+        __atomic_store_n(&job->failed, 1, __ATOMIC_RELAXED);
+        goto done;
+    }
+    for (;;) {
+        int64_t n = __atomic_fetch_add(&job->next, 1, __ATOMIC_RELAXED);
+        if (n >= job->n_units)
+            break;
+        int b, wy, wx, h;
+        unit_coords(p, n, &b, &wy, &wx, &h);
+        unit_forward(p, b, wy, wx, h, &w, o);
+        unit_backward(p, b, wy, wx, h, &w, job->dout, job->dq, job->dk, job->dv,
+                      dth ? dth + (size_t)h * (d / 4) : NULL, dbi ? dbi + (size_t)h * 2 * N * r : NULL,
+                      g_o, g_s, g_q, g_k);
+    }
+    pthread_mutex_lock(&job->mu);
+    if (dth)
+        for (size_t e = 0; e < nth; ++e)
+            job->dtheta[e] += dth[e];
+    if (dbi)
+        for (size_t e = 0; e < nbias; ++e)
+            job->dbias[e] += dbi[e];
+    pthread_mutex_unlock(&job->mu);
+done:
+    free(w.q);
+    free(w.k);
+    free(w.v);
+    free(w.s);
+    free(o);
+    free(g_o);
+    free(g_s);
+    free(g_q);
+    free(g_k);
+    free(dth);
+    free(dbi);
+    return NULL;
+}
+
+/* Gradients of a scalar loss L given dout = dL/dO [B][H][W][heads][d] (fp64):
+ * dq, dk, dv in the same layout, dtheta [heads][d/4] (NULL without theta),
+ * dbias [heads][2][M*M][rank] (NULL without bias), all fp64 and overwritten.
+ * Returns the number of threads used (> 0), or < 0 on bad arguments. */
+int oracle_bwd(const void *q, const void *k, const void *v, int dtype,
+               const float *theta, const void *bias,
+               int B, int H, int W, int M, int shift, int heads, int d, int rank,
+               const double *dout, double *dq, double *dk, double *dv, double *dtheta, double *dbias,
+               int nthreads)
+{
+    problem_t p = {q, k, v, dtype, theta, bias, B, H, W, M, shift, heads, d, rank};
+    if (check_problem(&p) || !dout || !dq || !dk || !dv)
+        return -1;
+    if ((dtheta != NULL && theta == NULL) || (dbias != NULL && bias == NULL))
+        return -1;
+    const size_t N = (size_t)M * M;
+    if (dtheta)
+        memset(dtheta, 0, (size_t)heads * (d / 4) * sizeof(double));
+    if (dbias)
+        memset(dbias, 0, (size_t)heads * 2 * N * rank * sizeof(double));
+    int64_t n_units = (int64_t)B * (H / M) * (W / M) * heads;
+    long ncpu = sysconf(_SC_NPROCESSORS_ONLN);
+    if (nthreads <= 0)
+        nthreads = ncpu > 0 ? (int)ncpu : 1;
+    if (nthreads > n_units)
+        nthreads = (int)n_units;
+    bwd_job_t job;
+    memset(&job, 0, sizeof job);
+    job.p = &p;
+    job.dout = dout;
+    job.dq = dq;
+    job.dk = dk;
+    job.dv = dv;
+    job.dtheta = dtheta;
+    job.dbias = dbias;
+    job.n_units = n_units;
+    pthread_mutex_init(&job.mu, NULL);
+    pthread_t *th = malloc(sizeof(pthread_t) * (size_t)nthreads);
+    if (!th) {
+        pthread_mutex_destroy(&job.mu);
+        return -2;
+    }
+    int started = 0;
+    for (int t = 0; t < nthreads; ++t) {
+        if (pthread_create(&th[t], NULL, bwd_worker, &job) != 0)
+            break;
+        ++started;
+    }
+    if (started == 0)
+        bwd_worker(&job);
+    for (int t = 0; t < started; ++t)
+        pthread_join(th[t], NULL);
+    free(th);
+    pthread_mutex_destroy(&job.mu);
+    return job.failed ? -2 : (started == 0 ? 1 : started);
 }
