@@ -43,6 +43,9 @@
 // Wrap masks are structural: a key tile lies on one side of the row seam,
 // and its two boxes on the two sides of the column seam, so each query row
 // keeps all, none, or one half of a tile.
+// Registers: the CTA launches with 128 per thread; each warpgroup then takes
+// its share (softmax 184, converter 80, loader and issuers 64), so a softmax
+// thread holds its whole row of S between the max pass and the exp pass.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>

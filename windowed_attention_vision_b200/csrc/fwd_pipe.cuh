@@ -23,8 +23,9 @@
 //                 k % 4 as soon as its RoPE is done and the buffer is free
 //                 (the commit also frees the tile's Q/K stage); O = P V as
 //                 soon as its P is written and its V has landed (the commit
-//                 frees the V stage).  Each issuer sleeps in bounded mbarrier
-//                 waits, so neither spins on the issue slots others need;
+//                 frees the V stage).  Each issuer blocks in bounded mbarrier
+//                 waits (a try_wait holds the thread in hardware), so neither
+//                 spins on the issue slots others need;
 //   warps 8-15    two softmax warpgroups, alternate tiles: max / exp2 / sum
 //                 of a row over its own window's allowed keys, P (bf16 pairs)
 //                 written over the consumed S columns;
@@ -32,11 +33,12 @@
 //                 written back with TMA stores of the same boxes the loaders
 //                 read: the token's original, un-shifted position.
 //
-// The rate is bounded by how long a tile holds shared memory: the rings must
-// cover the DRAM latency plus the processing latency of the tiles in flight,
-// so Q/K (needed until S) and V (needed from P V only) have rings of their
-// own.  Per-row metadata (wrap-label granules) lives in a ring of its own
-// that outlasts the Q/K stage.
+// The rings must cover the DRAM latency plus the processing latency of the
+// tiles in flight, so Q/K (needed until S) and V (needed from P V only) have
+// rings of their own.  Per-row metadata (wrap-label granules) lives in a ring
+// of its own that outlasts the Q/K stage.  Measured per tile, the steady rate
+// is set by the TMA issue rate of the SM (four box loads and two to four box
+// stores per tile), not by the ring depths or any one role.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
