@@ -48,6 +48,7 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-m", action="store_true", help="skip the per-M table (sweep, dense and SR calls)")
     return ap.parse_args()
 
 
@@ -247,6 +248,58 @@ def oracle_sample_rate(w, target_s, base=0):
     return tokens_per_s, sample, cores, calls
 
 
+# The metric is throughput against the window size M: besides the headline
+# workload, one line per sweep point (shift M/2, both head dims) and the dense
+# and SR calls, each timed with CUDA events over back-to-back calls.
+PER_M = [f"sweep_M{M}_d{d}_s{M // 2}" for M in (8, 16, 32, 64, 96) for d in (32, 64)] + ["dense", "sr"]
+
+
+def per_m_table(dev, peaks, target_s=0.25):
+    import torch
+
+    import windowed_attention_vision_b200 as wa
+    from windowed_attention_vision_b200 import _lib
+    from windowed_attention_vision_b200 import inputs as I
+    stream = torch.cuda.current_stream(dev)
+    rows = []
+    for name in PER_M:
+        w = I.WORKLOADS[name]
+        (qkv,), theta, bias = I.make_inputs(w, dev)
+        out = torch.empty_like(qkv[0])
+        calls = workload_calls(w)
+
+        def one():
+            for s in calls:
+                wa.window_attention(*qkv, w.M, s, theta=theta, bias_feats=bias, out=out)
+
+        one()
+        torch.cuda.synchronize(dev)
+        t0 = time.perf_counter()
+        one()
+        torch.cuda.synchronize(dev)
+        est = max(time.perf_counter() - t0, 1e-5)
+        reps = int(max(3, min(200, target_s / est)))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            one()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        call_s = e0.elapsed_time(e1) / 1e3 / (reps * len(calls))
+        r = roofline(w, call_s, peaks, None)
+        rc, info = _lib.launch_info(w.B, w.H, w.W, w.M, calls[-1], w.heads, w.d, w.rank,
+                                    _lib.BF16 if w.dtype == "bf16" else _lib.FP32)
+        rows.append({"workload": name, "M": w.M, "d": w.d, "rank": w.rank, "shifts": list(calls),
+                     "tokens": w.tokens, "kernel": KERNELS.get(info["kernel"], ("unknown",))[0],
+                     "us_per_call": call_s * 1e6, "calls_timed": reps * len(calls),
+                     "tflops": w.flops() / call_s / 1e12, "tokens_per_s": w.tokens / call_s,
+                     "gbs": w.bytes() / call_s / 1e9, "bound": r["bound"], "achieved": r["achieved"],
+                     "peak": r["peak"], "unit": r["unit"], "frac": r["frac"]})
+        del qkv, out
+        torch.cuda.empty_cache()
+    return rows
+
+
 def max_over_ranks(values, device):
     """Element-wise maximum of per-rank timings over all ranks (every rank
     calls it at the same point; the job is as slow as its slowest rank)."""
@@ -334,24 +387,47 @@ def run_ours(args):
         step(i)
     torch.cuda.synchronize(dev)
 
+    def enqueue_steps():
+        n = 0
+        for i in range(args.steps):
+            q, k, v = sets[i % copies]
+            for s in calls:
+                wa.window_attention(q, k, v, w.M, s, theta=theta, bias_feats=bias, out=outs[i % copies])
+                n += 1
+        return n
+
+    # Eager launches first (reported, not the headline): the host time to
+    # enqueue a call next to the device time per call.
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    h0 = time.perf_counter()
+    n_eager = enqueue_steps()
+    host_us = (time.perf_counter() - h0) / n_eager * 1e6
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    eager_ms = e0.elapsed_time(e1) / n_eager
+
+    # The timed region: the K steps captured once as a CUDA graph (the same
+    # launches, each a programmatic dependent of the previous one) and
+    # replayed; the graph is replayed once untimed first.  The host then never
+    # sits between two launches, so the device time is the kernels' own.
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        n = enqueue_steps()
+    graph.replay()
+    torch.cuda.synchronize(dev)
+
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.01)
-    # the timed region holds only the attention launches, back to back (no
-    # event between them, so that each launch may overlap the previous one's
-    # tail): the kernel's average launch duration is the region over launches
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     clocks.mark("timed_start")
     start.record(stream)
-    n = 0
-    for i in range(args.steps):
-        q, k, v = sets[i % copies]
-        for s in calls:
-            wa.window_attention(q, k, v, w.M, s, theta=theta, bias_feats=bias, out=outs[i % copies])
-            n += 1
+    graph.replay()
     end.record(stream)
     torch.cuda.synchronize(dev)
     clocks.mark("timed_end")
@@ -359,6 +435,7 @@ def run_ours(args):
         dist.barrier()
     time.sleep(0.01)
     clocks.stop()
+    del graph
     status = wa.device_status(dev)
     elapsed_ms = start.elapsed_time(end)
     kernel_ms = elapsed_ms / n
@@ -404,9 +481,16 @@ def run_ours(args):
                 "config": dict(config_of(w, world),
                                l2=f"inputs larger than L2: {copies} rotating input sets of "
                                   f"{4 * map_bytes / 1e6:.0f} MB (q, k, v, out)"),
-                "tflops": tflops, "kernel_ms_per_launch": kernel_ms, "gpu_launches": args.steps * len(calls),
+                "tflops": tflops, "kernel_ms_per_launch": kernel_ms,
+                "timing": "CUDA events around one replay of a CUDA graph holding the K steps' launches",
+                "eager": {"ms_per_launch": eager_ms, "host_us_per_call": host_us,
+                          "note": "the same K steps launched one by one from Python (host time per call "
+                                  "= wall time to enqueue them / K)"},
+                "gpu_launches": args.steps * len(calls),
                 "roofline": roofline(w, kernel_ms / 1e3, peaks, recorded_traffic(w)),
                 "clocks": clocks.summary(), "e2e": e2e, "device_status": status}
+        if not args.no_per_m:
+            line["per_M"] = per_m_table(dev, peaks)
         if world == 1 and not args.no_cpu_baseline:
             rate, sample, cores, _ = oracle_sample_rate(w, args.cpu_seconds)
             line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",

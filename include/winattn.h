@@ -112,9 +112,16 @@ int winattn_check_args(const void *q, const void *k, const void *v,
  * then block).  theta and bias_feats stay device pointers (resident
  * parameters).  `workspace` is a caller-owned device buffer of at least
  * winattn_host_workspace_bytes(...) bytes, 16-byte aligned, that holds the
- * device copies of q, k, v and out.  Enqueues H2D copies, the kernel and the
- * D2H copy of out on `stream` and returns; synchronise the stream before
- * reading out.  Allocates nothing.
+ * device copies of q, k, v and out.  Enqueues the H2D copies, the kernels and
+ * the D2H copy of out and returns; synchronise `stream` before reading out.
+ * The work is stream-ordered on `stream` (it starts after the work already
+ * enqueued there, and work enqueued there later starts after it), but runs on
+ * library-owned streams ("lanes", created once per device by the first call,
+ * which should therefore come before any stream capture): the batch is cut
+ * into up to 8 chunks of whole images that take turns on 3 lanes, so that one
+ * chunk's kernel and read-back overlap the next chunk's upload.  Concurrent
+ * host-buffer calls on one device are serialised on those lanes.  Allocates
+ * no device memory.
  */
 int winattn_fwd_host(const void *q_host, const void *k_host, const void *v_host,
                      const float *theta, const void *bias_feats,
@@ -143,6 +150,9 @@ size_t winattn_host_workspace_bytes(int B, int H_img, int W_img, int heads, int 
  * (winattn_host_workspace_bytes(...) > WINATTN_STATIC_WORKSPACE_BYTES) return
  * WINATTN_ERR_SIZE before anything is enqueued.  Allocates nothing: no
  * cudaMalloc, cudaFree or allocating library call.
+ *
+ * Unlike winattn_fwd_host it enqueues its copies and kernel on `stream`
+ * alone, one after the other (no lanes, no chunks).
  *
  * The first call on a device looks up the buffer's device address with that
  * device current; make that first call before any stream capture.  Every call
@@ -195,6 +205,21 @@ int winattn_launch_info(int B, int H_img, int W_img, int M, int shift, int heads
  * memory.
  */
 int winattn_selftest_wait_timeout(void *stream);
+
+/*
+ * winattn_set_kernel_enabled — process-wide switch of a specialised kernel
+ * (the kernel ids of winattn_launch_info: 1 = persistent small-window,
+ * 2 = persistent large-window, 4 = pipelined 8 x 8 kernel).  While a kernel is
+ * disabled, winattn_fwd and winattn_launch_info route its problems to the
+ * next kernel that serves them (in the end the generic tensor-core kernel,
+ * which serves every bf16 problem); the results agree within the bf16
+ * tolerance.  For testing the fallbacks and for isolating a kernel; the
+ * generic and fp32 kernels cannot be disabled.  Returns the previous state
+ * (1 enabled, 0 disabled) or WINATTN_ERR_ARG for another id.  Makes no CUDA
+ * call.  The large-window kernel is also bypassed, without this switch, when
+ * its build does not have the register count its warpgroup split assumes.
+ */
+int winattn_set_kernel_enabled(int kernel, int enabled);
 
 #ifdef __cplusplus
 }

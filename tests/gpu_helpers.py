@@ -95,10 +95,21 @@ def sampled_compare(w: I.Workload, shift: int, images, heads=None, extra_windows
                 units.append((wy * nWx + wx) * w.heads + h)
                 locs.append((wy, wx, h))
         if max_units is not None:
-            keep = rng.permutation(len(units))[:max_units]
-            keep = sorted(set(keep.tolist()) | {0, len(units) - 1})
-            units = [units[i] for i in keep]
-            locs = [locs[i] for i in keep]
+            # always the four corner windows (every wrap case of a shifted map,
+            # heads taken in turn) and an edge window of each seam; then random
+            # units up to max_units
+            must = {}
+            corners = [(0, 0), (0, nWx - 1), (nWy - 1, 0), (nWy - 1, nWx - 1)]
+            edges = [(nWy - 1, nWx // 2), (nWy // 2, nWx - 1)]
+            for n_, (wy, wx) in enumerate(corners + edges):
+                if (wy, wx) in [(a, b) for (a, b, _) in must.values()]:
+                    continue
+                h = heads[n_ % len(heads)]
+                must[(wy * nWx + wx) * w.heads + h] = (wy, wx, h)
+            rest = [i for i in rng.permutation(len(units)) if units[i] not in must]
+            extra = max(0, max_units - len(must))
+            units = list(must) + [units[i] for i in rest[:extra]]
+            locs = list(must.values()) + [locs[i] for i in rest[:extra]]
         ref = orc().fwd_units(*sub, units, M=w.M, shift=shift, theta=th, bias=bs)
         got_img = out[b].float().cpu().numpy().astype(np.float64)
         got = np.stack([got_img[window_positions(w.H, w.W, w.M, shift, wy, wx) + (h,)]

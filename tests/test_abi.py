@@ -131,3 +131,29 @@ def test_launch_plan(lib, B, H, W, M, shift, heads, d, rank, U, tiles, kernel):
 def test_launch_plan_fp32(lib):
     rc, info = _lib.launch_info(1, 16, 16, 8, 0, 2, 32, 0, _lib.FP32)
     assert rc == _lib.OK and info["kernel"] == SIMT
+
+
+def test_kernel_switch_routes_to_fallbacks(lib):
+    """Disabling a specialised kernel sends its problems to the next kernel
+    that serves them (in the end the generic tensor-core kernel); the switch
+    is process-wide and returns its previous state."""
+    dense = (16, 128, 128, 32, 16, 3, 32, 0, _lib.BF16)
+    swin = (64, 56, 56, 8, 4, 3, 32, 0, _lib.BF16)
+    assert _lib.launch_info(*dense)[1]["kernel"] == _lib.KERNEL_LARGE
+    assert _lib.launch_info(*swin)[1]["kernel"] == _lib.KERNEL_PIPE
+    try:
+        assert _lib.set_kernel_enabled(_lib.KERNEL_LARGE, False) == 1
+        assert _lib.launch_info(*dense)[1]["kernel"] == _lib.KERNEL_GENERIC
+        assert _lib.set_kernel_enabled(_lib.KERNEL_PIPE, False) == 1
+        assert _lib.launch_info(*swin)[1]["kernel"] == _lib.KERNEL_SMALL
+        assert _lib.set_kernel_enabled(_lib.KERNEL_SMALL, False) == 1
+        assert _lib.launch_info(*swin)[1]["kernel"] == _lib.KERNEL_GENERIC
+        assert _lib.set_kernel_enabled(_lib.KERNEL_SMALL, False) == 0
+    finally:
+        for k in (_lib.KERNEL_LARGE, _lib.KERNEL_PIPE, _lib.KERNEL_SMALL):
+            _lib.set_kernel_enabled(k, True)
+    assert _lib.launch_info(*dense)[1]["kernel"] == _lib.KERNEL_LARGE
+    assert _lib.launch_info(*swin)[1]["kernel"] == _lib.KERNEL_PIPE
+    # the generic and fp32 kernels have no switch
+    assert _lib.set_kernel_enabled(_lib.KERNEL_GENERIC, False) == _lib.ERR_ARG
+    assert _lib.set_kernel_enabled(_lib.KERNEL_SIMT, False) == _lib.ERR_ARG

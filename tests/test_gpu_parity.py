@@ -11,6 +11,7 @@ import pytest
 import torch
 
 import windowed_attention_vision_b200 as wa
+from windowed_attention_vision_b200 import _lib
 from windowed_attention_vision_b200 import inputs as I
 from tests import gpu_helpers as G
 
@@ -131,6 +132,18 @@ def test_host_path_matches_device_path():
     assert torch.equal(out, ref.cpu())
 
 
+def test_host_path_chunks_odd_windows_per_image():
+    """The host-buffer path cuts the batch into chunks of whole images; with
+    49 windows per image (Swin's map) the window pairs of a chunk differ from
+    those of the whole batch, and the result still matches the oracle."""
+    w = I.WORKLOADS["swin"]
+    (qkv,), theta, _ = I.make_inputs(w)
+    pinned = [t.pin_memory() for t in qkv]
+    out = wa.window_attention_host(*pinned, w.M, 4, theta=theta.cuda())
+    ref = G.orc().fwd(*(I.to_storage_numpy(t) for t in qkv), M=w.M, shift=4, theta=theta.numpy())
+    G.check(G.as_f64(out), ref, "bf16", "host path, swin")
+
+
 def test_deterministic():
     w = I.WORKLOADS["swin"]
     (qkv,), theta, _ = I.make_inputs(w, "cuda")
@@ -151,3 +164,31 @@ def test_errors_leave_out_untouched():
     torch.cuda.synchronize()
     assert bool((out == 7.0).all())
     assert wa.device_status() == 0
+
+
+FALLBACKS = [
+    # switched off, workload, shift, kernel that serves it then
+    ((_lib.KERNEL_LARGE,), "dense", 16, _lib.KERNEL_GENERIC),
+    ((_lib.KERNEL_PIPE,), "swin", 4, _lib.KERNEL_SMALL),
+    ((_lib.KERNEL_PIPE, _lib.KERNEL_SMALL), "swin", 4, _lib.KERNEL_GENERIC),
+]
+
+
+@pytest.mark.parametrize("off,name,shift,serves", FALLBACKS, ids=["large-off", "pipe-off", "pipe-small-off"])
+def test_fallback_kernels(off, name, shift, serves):
+    """With specialised kernels switched off, their problems run on the next
+    kernel that serves them (the path a build with an unexpected register
+    count takes for the large-window kernel) and still match the oracle."""
+    w = I.WORKLOADS[name]
+    try:
+        for k in off:
+            assert _lib.set_kernel_enabled(k, False) == 1
+        rc, info = _lib.launch_info(w.B, w.H, w.W, w.M, shift, w.heads, w.d, w.rank, _lib.BF16)
+        assert rc == 0 and info["kernel"] == serves
+        if w.name == "dense":
+            G.sampled_compare(w, shift, images=[0, w.B - 1], extra_windows=2)
+        else:
+            G.full_compare(w, shift)
+    finally:
+        for k in off:
+            _lib.set_kernel_enabled(k, True)

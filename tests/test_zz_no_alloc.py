@@ -4,10 +4,11 @@ Some callers cannot allocate device memory (the process's device memory
 belongs to someone else, or no allocator is reachable from the calling
 code), so they can pass neither device buffers nor a workspace.  For them
 the library keeps one static device buffer and does the host-buffer call
-with it.  Here it must give the same result as winattn_fwd_host with a
-caller-owned workspace, on two calls in a row with different inputs (the
-buffer keeps the previous call's contents), and refuse problems that do not
-fit its fixed size.  This file is collected last on purpose.
+with it.  Here it must give the result winattn_fwd gives on device copies of
+the same inputs, bit for bit, on two calls in a row with different inputs
+(the buffer keeps the previous call's contents), match the fp64 oracle, leave
+the device's free memory unchanged, and refuse problems that do not fit its
+fixed size.  This file is collected last on purpose.
 """
 import pytest
 import torch
@@ -31,15 +32,31 @@ def _static_call(q, k, v, theta, M, shift):
     return out
 
 
-def test_static_workspace_matches_host_entry_point_on_two_calls():
+def test_static_workspace_matches_device_entry_point_on_two_calls():
+    """Two calls in a row with different inputs (the buffer keeps the previous
+    call's contents): each equals winattn_fwd on device copies of the same
+    inputs bit for bit (the same kernel on the same problem), matches the fp64
+    oracle within the bf16 tolerance, and leaves the device's free memory
+    unchanged (the call allocates nothing)."""
+    w = I.Workload("no-alloc", 2, 16, 24, 8, (4,), 3, 32, "bf16", "learned")
+    cases = []
     for base in (0, 1):
-        w = I.Workload("no-alloc", 2, 16, 24, 8, (4,), 3, 32, "bf16", "learned")
         (qkv,), theta, _ = I.make_inputs(w, base=base)
-        q, k, v = (t.pin_memory() for t in qkv)
-        theta = theta.cuda()
-        got = _static_call(q, k, v, theta, w.M, 4)
-        ref = wa.window_attention_host(q, k, v, w.M, 4, theta=theta)
-        G.check(G.as_f64(got), G.as_f64(ref), "bf16", f"static workspace, call {base + 1}")
+        pinned = [t.pin_memory() for t in qkv]
+        dev = G.run_gpu(*(t.cuda() for t in qkv), w.M, 4, theta.cuda())
+        ref = G.orc().fwd(*(I.to_storage_numpy(t) for t in qkv), M=w.M, shift=4, theta=theta.numpy())
+        cases.append((pinned, theta.cuda(), dev.cpu(), ref))
+    # the first call on the device looks up the buffer's address (and may load
+    # the library's module, which holds the buffer): not part of the check
+    _static_call(*cases[0][0], cases[0][1], w.M, 4)
+    torch.cuda.synchronize()
+    free_before = torch.cuda.mem_get_info()[0]
+    for n, (pinned, theta, dev, ref) in enumerate(cases):
+        got = _static_call(*pinned, theta, w.M, 4)
+        assert torch.equal(got, dev), f"call {n + 1}: static-workspace result differs from winattn_fwd"
+        G.check(G.as_f64(got), ref, "bf16", f"static workspace, call {n + 1}")
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] >= free_before, "free device memory dropped during the calls"
     assert wa.device_status() == 0
 
 

@@ -60,10 +60,16 @@ def window_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, M: int, 
             raise WinattnError(_lib.ERR_ARG, "window_attention takes CUDA tensors")
     if out is None:
         out = torch.empty_like(q)
-    stream = torch.cuda.current_stream(q.device).cuda_stream
-    with torch.cuda.device(q.device):
-        rc = _lib.fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(theta), _ptr(bias_feats), B, H, W, M, shift, heads, d,
-                      rank, _dtype_code(q), _ptr(out), stream)
+    dev = q.device
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(theta), _ptr(bias_feats), B, H, W, M, shift, heads, d, rank,
+            _dtype_code(q), _ptr(out), stream)
+    # the library works on the current device: switch only when q lives elsewhere
+    if torch.cuda.current_device() == dev.index:
+        rc = _lib.fwd(*args)
+    else:
+        with torch.cuda.device(dev):
+            rc = _lib.fwd(*args)
     if rc != _lib.OK:
         raise WinattnError(rc, "winattn_fwd")
     return out

@@ -19,7 +19,7 @@ BF16, FP32 = 0, 1
 
 EXPORTS = ("winattn_fwd", "winattn_check_args", "winattn_fwd_host", "winattn_host_workspace_bytes",
            "winattn_strerror", "winattn_last_device_status", "winattn_launch_info", "winattn_fwd_host_static",
-           "winattn_selftest_wait_timeout")
+           "winattn_selftest_wait_timeout", "winattn_set_kernel_enabled")
 STATIC_WORKSPACE_BYTES = 32 << 20
 
 
@@ -60,6 +60,8 @@ def load(path: str = LIB_PATH):
     lib.winattn_launch_info.restype = i32
     lib.winattn_selftest_wait_timeout.argtypes = [vp]
     lib.winattn_selftest_wait_timeout.restype = i32
+    lib.winattn_set_kernel_enabled.argtypes = [i32, i32]
+    lib.winattn_set_kernel_enabled.restype = i32
     _lib = lib
     return lib
 
@@ -102,6 +104,15 @@ def last_device_status(stream) -> int:
 
 def selftest_wait_timeout(stream) -> int:
     return load().winattn_selftest_wait_timeout(stream)
+
+
+KERNEL_GENERIC, KERNEL_SMALL, KERNEL_LARGE, KERNEL_SIMT, KERNEL_PIPE = 0, 1, 2, 3, 4
+
+
+def set_kernel_enabled(kernel: int, enabled: bool) -> int:
+    """Switch a specialised kernel off (its problems go to the next kernel that
+    serves them) or back on; returns the previous state or ERR_ARG."""
+    return load().winattn_set_kernel_enabled(kernel, 1 if enabled else 0)
 
 
 def launch_info(B, H, W, M, shift, heads, d, rank, dtype):

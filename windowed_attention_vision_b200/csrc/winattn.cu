@@ -5,6 +5,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -89,7 +90,112 @@ int smem_bytes_for(const Geometry &g, int dtype)
 constexpr int kAssumedSMs = 148;          // B200; used only by winattn_launch_info
 constexpr uint32_t kMaxSmem = 227 * 1024;
 
-enum KernelKind { kGeneric = 0, kSmall = 1, kLarge = 2, kSimt = 3, kPipe = 4 };
+enum KernelKind { kGeneric = 0, kSmall = 1, kLarge = 2, kSimt = 3, kPipe = 4, kKinds = 5 };
+
+// Process-wide switches of the specialised kernels (winattn_set_kernel_enabled):
+// a disabled kind's problems go to the generic kernel.  The generic and SIMT
+// kernels cannot be disabled.
+std::atomic<int> g_kernel_enabled[kKinds] = {1, 1, 1, 1, 1};
+
+bool kernel_enabled(KernelKind k) { return g_kernel_enabled[k].load(std::memory_order_relaxed) != 0; }
+
+int current_device()
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return -1;
+    return dev;
+}
+
+// cudaFuncAttributeMaxDynamicSharedMemorySize is a per-function, per-device
+// setting: raised to the largest opt-in size once per (kernel, device) and
+// never again (the launch itself passes the bytes it needs).
+template <auto Kernel>
+bool smem_attr_once()
+{
+    static std::atomic<uint64_t> done{0};
+    const int dev = current_device();
+    if (dev < 0)
+        return false;
+    const uint64_t bit = 1ull << dev;
+    if (done.load(std::memory_order_acquire) & bit)
+        return true;
+    if (cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024) != cudaSuccess)
+        return false;
+    done.fetch_or(bit, std::memory_order_release);
+    return true;
+}
+
+// Tensor maps of a launch depend only on the device, the buffers' addresses
+// and the problem's sizes, so they are encoded once per such key and reused:
+// a repeated key always denotes the same encoding, even after the caller has
+// freed and reallocated a buffer at the same address.  A small table per
+// process, replaced round-robin, guarded by a mutex (the lookup is a few
+// hundred nanoseconds; encoding the 16 maps of an 8 x 8 window call costs
+// several microseconds).
+struct MapKey {
+    int kind, dev, B, H, W, M, shift, heads, d, rank;
+    const void *ptr[5];
+    bool operator==(const MapKey &o) const { return std::memcmp(this, &o, sizeof *this) == 0; }
+};
+
+struct MapSet {
+    alignas(64) CUtensorMap m[16];
+};
+
+constexpr int kMapCacheEntries = 64;
+
+struct MapCache {
+    std::mutex mu;
+    MapKey key[kMapCacheEntries];
+    MapSet val[kMapCacheEntries];
+    bool used[kMapCacheEntries] = {};
+    int next = 0;
+};
+
+MapCache &map_cache()
+{
+    static MapCache c;
+    return c;
+}
+
+MapKey make_key(KernelKind kind, const Geometry &g, const void *a, const void *b, const void *c, const void *d,
+                const void *e)
+{
+    MapKey k;
+    std::memset(&k, 0, sizeof k);  // padding bytes take part in the comparison
+    k.kind = kind;
+    k.dev = current_device();
+    k.B = g.B; k.H = g.H; k.W = g.W; k.M = g.M; k.shift = g.shift; k.heads = g.heads; k.d = g.d; k.rank = g.rank;
+    k.ptr[0] = a; k.ptr[1] = b; k.ptr[2] = c; k.ptr[3] = d; k.ptr[4] = e;
+    return k;
+}
+
+// The cached maps of `key`, or those `encode(MapSet *)` produces (then
+// cached); false if encoding failed (nothing is cached then).
+template <typename Encode>
+bool cached_maps(const MapKey &key, MapSet *out, Encode encode)
+{
+    MapCache &c = map_cache();
+    {
+        std::lock_guard<std::mutex> lock(c.mu);
+        for (int i = 0; i < kMapCacheEntries; ++i)
+            if (c.used[i] && c.key[i] == key) {
+                *out = c.val[i];
+                return true;
+            }
+    }
+    std::memset(out, 0, sizeof *out);
+    if (!encode(out))
+        return false;
+    std::lock_guard<std::mutex> lock(c.mu);
+    const int i = c.next;
+    c.next = (c.next + 1) % kMapCacheEntries;
+    c.key[i] = key;
+    c.val[i] = *out;
+    c.used[i] = true;
+    return true;
+}
 
 uint32_t pipe_smem(const Geometry &g)
 {
@@ -116,11 +222,13 @@ KernelKind choose_kernel(const Geometry &g, int dtype)
 {
     if (dtype == WINATTN_FP32)
         return kSimt;
-    if (pipe_ok(g) && (uint64_t)g.heads * g.M * (g.d / 4) * 8 <= kSmallTableMax && pipe_smem(g) <= kMaxSmem)
+    if (kernel_enabled(kPipe) && pipe_ok(g) && (uint64_t)g.heads * g.M * (g.d / 4) * 8 <= kSmallTableMax &&
+        pipe_smem(g) <= kMaxSmem)
         return kPipe;
-    if (g.N <= kTileRows && (uint64_t)g.heads * g.M * (g.d / 4) * 8 <= kSmallTableMax && small_smem(g) <= kMaxSmem)
+    if (kernel_enabled(kSmall) && g.N <= kTileRows && (uint64_t)g.heads * g.M * (g.d / 4) * 8 <= kSmallTableMax &&
+        small_smem(g) <= kMaxSmem)
         return kSmall;
-    if (large_ok(g))
+    if (kernel_enabled(kLarge) && large_ok(g))
         return kLarge;
     return kGeneric;
 }
@@ -163,12 +271,12 @@ int check_device()
     return cached[dev] == 1 ? WINATTN_OK : WINATTN_ERR_ARCH;
 }
 
-template <typename Kernel>
-int launch(Kernel kernel, int smem, const Geometry &g, cudaStream_t stream, auto... args)
+template <auto Kernel>
+int launch(int smem, const Geometry &g, cudaStream_t stream, auto... args)
 {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    if (!smem_attr_once<Kernel>())
         return WINATTN_ERR_CUDA;
-    kernel<<<(unsigned)g.items, kThreads, smem, stream>>>(args..., g, 1.0f / std::sqrt((float)g.d));
+    Kernel<<<(unsigned)g.items, kThreads, smem, stream>>>(args..., g, 1.0f / std::sqrt((float)g.d));
     return cudaGetLastError() == cudaSuccess ? WINATTN_OK : WINATTN_ERR_CUDA;
 }
 
@@ -177,7 +285,7 @@ int launch_tc(const void *q, const void *k, const void *v, const float *theta, c
               const Geometry &g, cudaStream_t stream)
 {
     using T = __nv_bfloat16;
-    return launch(winattn_fwd_tc_kernel<D, R>, (int)TcLayout<D, R>::bytes(g.M), g, stream,
+    return launch<winattn_fwd_tc_kernel<D, R>>((int)TcLayout<D, R>::bytes(g.M), g, stream,
                   static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), theta,
                   static_cast<const T *>(bias), static_cast<T *>(out));
 }
@@ -284,35 +392,51 @@ bool encode_factor_map(CUtensorMap *m, const void *base, const Geometry &g, int 
               CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Whether the built large-window kernel has exactly kLargeRegsLaunch
+// registers per thread: its warpgroups' setmaxnreg shares add up to the
+// launch's registers only then.  Looked up once per instantiation.
+template <int D, int R, int BN>
+bool large_regs_ok()
+{
+    static const bool ok = [] {
+        cudaFuncAttributes fa;
+        return cudaFuncGetAttributes(&fa, winattn_fwd_large_kernel<D, R, BN>) == cudaSuccess &&
+               fa.numRegs == (int)kLargeRegsLaunch;
+    }();
+    return ok;
+}
+
 template <int D, int R, int BN>
 int launch_large(const void *q, const void *k, const void *v, const float *theta, const void *bias, void *out,
                  const Geometry &g, cudaStream_t stream)
 {
     using T = __nv_bfloat16;
+    // a build whose register count differs would wait forever in setmaxnreg:
+    // its problems go to the generic tensor-core kernel instead
+    if (!large_regs_ok<D, R, BN>())
+        return launch_tc<D, R>(q, k, v, theta, bias, out, g, stream);
+    MapSet ms;
+    const MapKey key = make_key(kLarge, g, k, v, bias, nullptr, nullptr);
+    const bool ok = cached_maps(key, &ms, [&](MapSet *m) {
+        const int kr = BN / g.M;
+        if (!encode_kv_map(&m->m[0], k, g, g.M, kr) || !encode_kv_map(&m->m[2], v, g, g.M, kr))
+            return false;
+        if (g.shift && (!encode_kv_map(&m->m[1], k, g, g.M / 2, kr) || !encode_kv_map(&m->m[3], v, g, g.M / 2, kr)))
+            return false;
+        return R == 0 || encode_factor_map(&m->m[4], bias, g, BN);
+    });
+    if (!ok)
+        return WINATTN_ERR_CUDA;
+    static_assert(sizeof(LargeMaps) == 5 * sizeof(CUtensorMap), "LargeMaps is five maps");
     LargeMaps maps;
-    std::memset(&maps, 0, sizeof maps);
-    const int kr = BN / g.M;
-    if (!encode_kv_map(&maps.k_full, k, g, g.M, kr) || !encode_kv_map(&maps.v_full, v, g, g.M, kr))
-        return WINATTN_ERR_CUDA;
-    if (g.shift && (!encode_kv_map(&maps.k_half, k, g, g.M / 2, kr) || !encode_kv_map(&maps.v_half, v, g, g.M / 2, kr)))
-        return WINATTN_ERR_CUDA;
-    if (R > 0 && !encode_factor_map(&maps.w, bias, g, BN))
-        return WINATTN_ERR_CUDA;
+    std::memcpy(&maps, ms.m, sizeof maps);
     auto kernel = winattn_fwd_large_kernel<D, R, BN>;
-    // the warpgroups' register shares add up to the launch's registers only
-    // at exactly kLargeRegsLaunch registers per thread: refuse any other build
-    static const bool regs_ok = [&] {
-        cudaFuncAttributes fa;
-        return cudaFuncGetAttributes(&fa, kernel) == cudaSuccess && fa.numRegs == (int)kLargeRegsLaunch;
-    }();
-    if (!regs_ok)
+    if (!smem_attr_once<winattn_fwd_large_kernel<D, R, BN>>())
         return WINATTN_ERR_CUDA;
     // all 512 TMEM columns per CTA: enough shared memory that no second CTA
     // is resident on the same SM
     const int need = (int)LargeLayout<D, R, BN>::BYTES;
     const int smem = need > 116 * 1024 ? need : 116 * 1024;
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-        return WINATTN_ERR_CUDA;
     const int64_t items = g.wph * g.heads * (g.N / 256);
     const int64_t grid = items < sm_count() ? items : sm_count();
     kernel<<<(unsigned)grid, kLargeThreads, smem, stream>>>(static_cast<const T *>(q), theta,
@@ -340,7 +464,7 @@ int launch_small_variant(const void *q, const void *k, const void *v, const floa
     // no second CTA can be resident on the same SM.
     const int need = (int)SmallLayout<D, R>::bytes(g.heads, g.M);
     const int smem = need > 116 * 1024 ? need : 116 * 1024;
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    if (!smem_attr_once<winattn_fwd_small_kernel<D, R, TMA>>())
         return WINATTN_ERR_CUDA;
     const int64_t grid = g.items < sm_count() ? g.items : sm_count();
     kernel<<<(unsigned)grid, SmallRoles<D>::kThreads, smem, stream>>>(
@@ -358,9 +482,16 @@ int launch_small(const void *q, const void *k, const void *v, const float *theta
     std::memset(maps, 0, sizeof maps);
     if constexpr (R == 0) {
         if (small_tma_ok(g)) {
-            if (encode_window_maps(&maps[0], q, g) && encode_window_maps(&maps[1], k, g) &&
-                encode_window_maps(&maps[2], v, g))
+            MapSet ms;
+            const MapKey key = make_key(kSmall, g, q, k, v, nullptr, nullptr);
+            if (cached_maps(key, &ms, [&](MapSet *m) {
+                    WindowMaps *w = reinterpret_cast<WindowMaps *>(m->m);
+                    return encode_window_maps(&w[0], q, g) && encode_window_maps(&w[1], k, g) &&
+                           encode_window_maps(&w[2], v, g);
+                })) {
+                std::memcpy(maps, ms.m, sizeof maps);
                 return launch_small_variant<D, R, true>(q, k, v, theta, bias, out, g, stream, maps);
+            }
             std::memset(maps, 0, sizeof maps);
         }
     }
@@ -371,14 +502,20 @@ template <int D>
 int launch_pipe(const void *q, const void *k, const void *v, const float *theta, void *out, const Geometry &g,
                 cudaStream_t stream)
 {
-    WindowMaps maps[4];
-    std::memset(maps, 0, sizeof maps);
-    if (!encode_window_maps(&maps[0], q, g) || !encode_window_maps(&maps[1], k, g) ||
-        !encode_window_maps(&maps[2], v, g) || !encode_window_maps(&maps[3], out, g))
+    static_assert(sizeof(WindowMaps) == 4 * sizeof(CUtensorMap), "WindowMaps is four maps");
+    MapSet ms;
+    const MapKey key = make_key(kPipe, g, q, k, v, out, nullptr);
+    if (!cached_maps(key, &ms, [&](MapSet *m) {
+            WindowMaps *w = reinterpret_cast<WindowMaps *>(m->m);
+            return encode_window_maps(&w[0], q, g) && encode_window_maps(&w[1], k, g) &&
+                   encode_window_maps(&w[2], v, g) && encode_window_maps(&w[3], out, g);
+        }))
         return WINATTN_ERR_CUDA;
+    WindowMaps maps[4];
+    std::memcpy(maps, ms.m, sizeof maps);
     auto kernel = winattn_fwd_pipe_kernel<D>;
     const int smem = (int)PipeLayout<D>::bytes(g.heads);
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    if (!smem_attr_once<winattn_fwd_pipe_kernel<D>>())
         return WINATTN_ERR_CUDA;
     const int64_t grid = g.items < sm_count() ? g.items : sm_count();
     // a programmatic dependent of the previous kernel in the stream: its
@@ -405,7 +542,7 @@ template <int D, int R>
 int launch_simt(const void *q, const void *k, const void *v, const float *theta, const void *bias, void *out,
                 const Geometry &g, cudaStream_t stream)
 {
-    return launch(winattn_fwd_simt_kernel<D, R>, (int)SimtLayout<D, R>::bytes(g.M), g, stream,
+    return launch<winattn_fwd_simt_kernel<D, R>>((int)SimtLayout<D, R>::bytes(g.M), g, stream,
                   static_cast<const float *>(q), static_cast<const float *>(k), static_cast<const float *>(v),
                   theta, static_cast<const float *>(bias), static_cast<float *>(out));
 }
@@ -459,6 +596,40 @@ int dispatch(const void *q, const void *k, const void *v, const float *theta, co
     return WINATTN_ERR_ARG;
 }
 
+// Streams and events of the host-buffer entry points, created once per device
+// (with that device current) and kept until the process exits; a mutex per
+// device keeps concurrent host-buffer calls from interleaving their records.
+constexpr int kHostLanes = 3, kHostChunks = 8;
+
+struct HostLanes {
+    std::mutex mu;
+    cudaStream_t lane[kHostLanes];
+    cudaEvent_t entry, done[kHostLanes];
+};
+
+HostLanes *host_lanes()
+{
+    static std::mutex mu;
+    static HostLanes *per_dev[64];
+    const int dev = current_device();
+    if (dev < 0)
+        return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!per_dev[dev]) {
+        HostLanes *h = new HostLanes;
+        bool ok = cudaEventCreateWithFlags(&h->entry, cudaEventDisableTiming) == cudaSuccess;
+        for (int l = 0; ok && l < kHostLanes; ++l)
+            ok = cudaStreamCreateWithFlags(&h->lane[l], cudaStreamNonBlocking) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&h->done[l], cudaEventDisableTiming) == cudaSuccess;
+        if (!ok) {
+            delete h;  // the handles created so far stay with the context
+            return nullptr;
+        }
+        per_dev[dev] = h;
+    }
+    return per_dev[dev];
+}
+
 }  // namespace
 }  // namespace winattn
 
@@ -509,9 +680,19 @@ size_t winattn_host_workspace_bytes(int B, int H_img, int W_img, int heads, int 
     return 4 * n;
 }
 
-int winattn_fwd_host(const void *q_host, const void *k_host, const void *v_host, const float *theta,
-                     const void *bias_feats, int B, int H_img, int W_img, int M, int shift, int heads, int d,
-                     int rank, int dtype, void *out_host, void *workspace, size_t workspace_bytes, void *stream)
+}  // extern "C"
+
+namespace {
+
+// The host-buffer call.  With `overlap`, the batch is cut into chunks of
+// whole images (a window never spans two images, so each chunk is an exact
+// sub-problem) that take turns on the library's lanes, so that one chunk's
+// kernel and read-back overlap the next chunk's upload (host-to-device and
+// device-to-host copies run on separate copy engines); without it, copies and
+// kernel are enqueued on the caller's stream alone.
+int fwd_host_impl(const void *q_host, const void *k_host, const void *v_host, const float *theta,
+                  const void *bias_feats, int B, int H_img, int W_img, int M, int shift, int heads, int d, int rank,
+                  int dtype, void *out_host, void *workspace, size_t workspace_bytes, void *stream, bool overlap)
 {
     int rc = check_sizes(B, H_img, W_img, M, shift, heads, d, rank, dtype);
     if (rc != WINATTN_OK)
@@ -525,7 +706,7 @@ int winattn_fwd_host(const void *q_host, const void *k_host, const void *v_host,
     const size_t n = map_bytes(B, H_img, W_img, heads, d, dtype);
     const size_t stride = (n + 255) & ~size_t(255);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    void *dq = ws, *dk = ws + stride, *dv = ws + 2 * stride, *dout = ws + 3 * stride;
+    uint8_t *dq = ws, *dk = ws + stride, *dv = ws + 2 * stride, *dout = ws + 3 * stride;
     rc = winattn_check_args(dq, dk, dv, theta, bias_feats, B, H_img, W_img, M, shift, heads, d, rank, dtype, dout);
     if (rc != WINATTN_OK)
         return rc;
@@ -533,17 +714,68 @@ int winattn_fwd_host(const void *q_host, const void *k_host, const void *v_host,
     if (rc != WINATTN_OK)
         return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (cudaMemcpyAsync(dq, q_host, n, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(dk, k_host, n, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(dv, v_host, n, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    if (!overlap) {
+        if (cudaMemcpyAsync(dq, q_host, n, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+            cudaMemcpyAsync(dk, k_host, n, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+            cudaMemcpyAsync(dv, v_host, n, cudaMemcpyHostToDevice, s) != cudaSuccess)
+            return WINATTN_ERR_CUDA;
+        const Geometry g = Geometry::make(B, H_img, W_img, M, shift, heads, d, rank);
+        rc = dispatch(dq, dk, dv, theta, bias_feats, dout, g, dtype, s);
+        if (rc != WINATTN_OK)
+            return rc;
+        return cudaMemcpyAsync(out_host, dout, n, cudaMemcpyDeviceToHost, s) == cudaSuccess ? WINATTN_OK
+                                                                                           : WINATTN_ERR_CUDA;
+    }
+    HostLanes *lanes = host_lanes();
+    if (!lanes)
         return WINATTN_ERR_CUDA;
-    const Geometry g = Geometry::make(B, H_img, W_img, M, shift, heads, d, rank);
-    rc = dispatch(dq, dk, dv, theta, bias_feats, dout, g, dtype, s);
-    if (rc != WINATTN_OK)
-        return rc;
-    if (cudaMemcpyAsync(out_host, dout, n, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    std::lock_guard<std::mutex> lock(lanes->mu);
+    const int chunks = B < kHostChunks ? B : kHostChunks;
+    const size_t img = n / (size_t)B;
+    if (cudaEventRecord(lanes->entry, s) != cudaSuccess)
         return WINATTN_ERR_CUDA;
+    for (int l = 0; l < kHostLanes && l < chunks; ++l)
+        if (cudaStreamWaitEvent(lanes->lane[l], lanes->entry, 0) != cudaSuccess)
+            return WINATTN_ERR_CUDA;
+    int b0 = 0;
+    for (int c = 0; c < chunks; ++c) {
+        const int nb = B / chunks + (c < B % chunks ? 1 : 0);
+        const size_t off = (size_t)b0 * img, len = (size_t)nb * img;
+        cudaStream_t ls = lanes->lane[c % kHostLanes];
+        const uint8_t *hq = static_cast<const uint8_t *>(q_host) + off;
+        const uint8_t *hk = static_cast<const uint8_t *>(k_host) + off;
+        const uint8_t *hv = static_cast<const uint8_t *>(v_host) + off;
+        if (cudaMemcpyAsync(dq + off, hq, len, cudaMemcpyHostToDevice, ls) != cudaSuccess ||
+            cudaMemcpyAsync(dk + off, hk, len, cudaMemcpyHostToDevice, ls) != cudaSuccess ||
+            cudaMemcpyAsync(dv + off, hv, len, cudaMemcpyHostToDevice, ls) != cudaSuccess)
+            return WINATTN_ERR_CUDA;
+        const Geometry g = Geometry::make(nb, H_img, W_img, M, shift, heads, d, rank);
+        rc = dispatch(dq + off, dk + off, dv + off, theta, bias_feats, dout + off, g, dtype, ls);
+        if (rc != WINATTN_OK)
+            return rc;
+        if (cudaMemcpyAsync(static_cast<uint8_t *>(out_host) + off, dout + off, len, cudaMemcpyDeviceToHost, ls) !=
+            cudaSuccess)
+            return WINATTN_ERR_CUDA;
+        b0 += nb;
+    }
+    // the caller's stream resumes once every lane has finished its chunks
+    for (int l = 0; l < kHostLanes && l < chunks; ++l)
+        if (cudaEventRecord(lanes->done[l], lanes->lane[l]) != cudaSuccess ||
+            cudaStreamWaitEvent(s, lanes->done[l], 0) != cudaSuccess)
+            return WINATTN_ERR_CUDA;
     return WINATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int winattn_fwd_host(const void *q_host, const void *k_host, const void *v_host, const float *theta,
+                     const void *bias_feats, int B, int H_img, int W_img, int M, int shift, int heads, int d,
+                     int rank, int dtype, void *out_host, void *workspace, size_t workspace_bytes, void *stream)
+{
+    return fwd_host_impl(q_host, k_host, v_host, theta, bias_feats, B, H_img, W_img, M, shift, heads, d, rank,
+                         dtype, out_host, workspace, workspace_bytes, stream, true);
 }
 
 }  // extern "C"
@@ -615,8 +847,8 @@ int winattn_fwd_host_static(const void *q_host, const void *k_host, const void *
     void *ws = static_workspace_ptr();
     if (!ws)
         return WINATTN_ERR_CUDA;
-    return winattn_fwd_host(q_host, k_host, v_host, theta, bias_feats, B, H_img, W_img, M, shift, heads, d, rank,
-                            dtype, out_host, ws, WINATTN_STATIC_WORKSPACE_BYTES, stream);
+    return fwd_host_impl(q_host, k_host, v_host, theta, bias_feats, B, H_img, W_img, M, shift, heads, d, rank,
+                         dtype, out_host, ws, WINATTN_STATIC_WORKSPACE_BYTES, stream, false);
 }
 
 const char *winattn_strerror(int code)
@@ -693,6 +925,13 @@ int winattn_selftest_wait_timeout(void *stream)
         return rc;
     selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
     return cudaGetLastError() == cudaSuccess ? WINATTN_OK : WINATTN_ERR_CUDA;
+}
+
+int winattn_set_kernel_enabled(int kernel, int enabled)
+{
+    if (kernel != kSmall && kernel != kLarge && kernel != kPipe)
+        return WINATTN_ERR_ARG;
+    return g_kernel_enabled[kernel].exchange(enabled ? 1 : 0);
 }
 
 }  // extern "C"
