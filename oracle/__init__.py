@@ -120,7 +120,8 @@ class Oracle:
     def fwd_units(self, q, k, v, units, *, M, shift=0, theta=None, bias=None,
                   nthreads=0, mem_budget=8e9) -> np.ndarray:
         """Selected units u = ((b*nWy + wy)*nWx + wx)*heads + h -> [n, M*M, d] fp64,
-        each in window order p = i*M + j."""
+        each in window order p = i*M + j (nWy, nWx count the windows of the
+        grid padded to multiples of M; rows at pad positions are NaN)."""
         q, k, v, theta, bias, code, (B, H, W, heads, d, rank) = self._prep(q, k, v, theta, bias, M)
         units = np.ascontiguousarray(units, dtype=np.int64)
         out = np.zeros((len(units), M * M, d), dtype=np.float64)
@@ -159,9 +160,10 @@ class Oracle:
         return out
 
     def token_origin(self, H, W, M, shift, wy, wx, p):
-        """Original (row, col) of token p of rolled window (wy, wx)."""
+        """Original (row, col) of token p of rolled window (wy, wx) in the grid
+        padded to multiples of M (row >= H or col >= W: a pad position)."""
         y, x = ctypes.c_int(), ctypes.c_int()
-        if self.lib.oracle_token_origin(H, W, M, shift, wy, wx, p, ctypes.byref(y), ctypes.byref(x)):
+        if self.lib.oracle_token_origin(H, W, M, shift, wy, wx, p, ctypes.byref(y), ctypes.byref(x)) < 0:
             raise ValueError("bad token arguments")
         return y.value, x.value
 

@@ -32,6 +32,11 @@
  *    (i + s, j + s) mod (H, W)), inverse roll on write-back;
  *  - wrap label L = 2*[row in last s rows] + [col in last s cols] of the
  *    rolled map, mask value -inf where labels differ;
+ *  - maps whose sides are not multiples of M (FlashSwin-T's 56 x 56 map at
+ *    M = 16 or 32) are padded at the bottom and right to the next multiples
+ *    Hp x Wp, the padded map is rolled and cut into windows (Swin pads before
+ *    its roll), and the pad positions hold no token: they are masked as keys
+ *    (-inf) and never written; the labels above use Hp and Wp;
  *  - scale d^-1/2 applies to the content dot product only, the bias dot
  *    product u.w is added unscaled.
  *
@@ -63,7 +68,20 @@ typedef struct {
     const float *theta;      /* [heads][d/4] or NULL */
     const void *bias;        /* [heads][2][M*M][rank] storage dtype, or NULL */
     int B, H, W, M, shift, heads, d, rank;
+    int Hp, Wp;              /* H and W rounded up to multiples of M (the padded map) */
 } problem_t;
+
+static problem_t make_problem(const void *q, const void *k, const void *v, int dtype, const float *theta,
+                              const void *bias, int B, int H, int W, int M, int shift, int heads, int d,
+                              int rank)
+{
+    problem_t p = {q, k, v, dtype, theta, bias, B, H, W, M, shift, heads, d, rank, 0, 0};
+    if (M > 0) {
+        p.Hp = (H + M - 1) / M * M;
+        p.Wp = (W + M - 1) / M * M;
+    }
+    return p;
+}
 
 /* Step 1: read one stored element as fp64 (bf16 -> fp64 and fp32 -> fp64 are exact). */
 static double read_elem(const void *base, int dtype, size_t idx)
@@ -76,13 +94,17 @@ static double read_elem(const void *base, int dtype, size_t idx)
     return (double)f;
 }
 
-/* Step 2: the rolled map.  Rolled row yr, rolled column xr hold the original
- * token at row (yr + s) mod H, column (xr + s) mod W. */
-static size_t rolled_token_offset(const problem_t *p, int b, int yr, int xr, int h)
+/* Step 2: the rolled map.  Rolled row yr, rolled column xr hold the padded
+ * map's token at row (yr + s) mod Hp, column (xr + s) mod Wp (Hp = H and
+ * Wp = W when M divides them).  Returns its element offset in the original
+ * map, or -1 when that position is padding (row >= H or column >= W). */
+static int64_t rolled_token_offset(const problem_t *p, int b, int yr, int xr, int h)
 {
-    int y = (yr + p->shift) % p->H;
-    int x = (xr + p->shift) % p->W;
-    return ((((size_t)b * p->H + y) * p->W + x) * p->heads + h) * p->d;
+    int y = (yr + p->shift) % p->Hp;
+    int x = (xr + p->shift) % p->Wp;
+    if (y >= p->H || x >= p->W)
+        return -1;
+    return (int64_t)(((((size_t)b * p->H + y) * p->W + x) * p->heads + h) * p->d);
 }
 
 /* Step 4: window-local 2D RoPE on one d-vector at window-local (row i, col j).
@@ -108,11 +130,12 @@ static int wrap_label(const problem_t *p, int yr, int xr)
 {
     if (p->shift == 0)
         return 0;
-    return 2 * (yr >= p->H - p->shift) + (xr >= p->W - p->shift);
+    return 2 * (yr >= p->Hp - p->shift) + (xr >= p->Wp - p->shift);
 }
 
 typedef struct {
     double *q, *k, *v, *s; /* N x d, N x d, N x d, N x N */
+    int64_t *off;          /* N: element offset of each window token, -1 for padding */
 } scratch_t;
 
 /* Steps 3-8 for one (batch b, window (wy, wx), head h): O = softmax(S) V in
@@ -123,15 +146,17 @@ static void unit_forward(const problem_t *p, int b, int wy, int wx, int h,
     const int M = p->M, N = M * M, d = p->d, r = p->rank;
     const double scale = 1.0 / sqrt((double)d);
 
-    /* Step 3: gather the window's N tokens from the rolled map. */
+    /* Step 3: gather the window's N tokens from the rolled map (a pad
+     * position gets zero vectors; it is masked below and never stored). */
     for (int i = 0; i < M; ++i)
         for (int j = 0; j < M; ++j) {
             int t = i * M + j;
-            size_t off = rolled_token_offset(p, b, wy * M + i, wx * M + j, h);
+            int64_t off = rolled_token_offset(p, b, wy * M + i, wx * M + j, h);
+            w->off[t] = off;
             for (int c = 0; c < d; ++c) {
-                w->q[(size_t)t * d + c] = read_elem(p->q, p->dtype, off + c);
-                w->k[(size_t)t * d + c] = read_elem(p->k, p->dtype, off + c);
-                w->v[(size_t)t * d + c] = read_elem(p->v, p->dtype, off + c);
+                w->q[(size_t)t * d + c] = off < 0 ? 0.0 : read_elem(p->q, p->dtype, (size_t)off + c);
+                w->k[(size_t)t * d + c] = off < 0 ? 0.0 : read_elem(p->k, p->dtype, (size_t)off + c);
+                w->v[(size_t)t * d + c] = off < 0 ? 0.0 : read_elem(p->v, p->dtype, (size_t)off + c);
             }
         }
 
@@ -164,19 +189,29 @@ static void unit_forward(const problem_t *p, int b, int wy, int wx, int h,
             w->s[(size_t)a * N + c] = sc;
         }
 
-    /* Step 6: additive -inf mask between different wrap regions. */
+    /* Step 6: additive -inf mask between different wrap regions, and on
+     * every pad key. */
     for (int a = 0; a < N; ++a) {
         int la = wrap_label(p, wy * M + a / M, wx * M + a % M);
         for (int c = 0; c < N; ++c) {
             int lc = wrap_label(p, wy * M + c / M, wx * M + c % M);
             if (la != lc)
                 w->s[(size_t)a * N + c] = -INFINITY;
+            if (w->off[c] < 0)
+                w->s[(size_t)a * N + c] = -INFINITY;
         }
     }
 
-    /* Step 7: row softmax (max subtracted, exp, divided by the sum). */
+    /* Step 7: row softmax (max subtracted, exp, divided by the sum).  A pad
+     * row has no output: its probabilities are zero (so nothing flows from it
+     * in the backward) and step 8 marks its output NaN. */
     for (int a = 0; a < N; ++a) {
         double *row = w->s + (size_t)a * N;
+        if (w->off[a] < 0) {
+            for (int c = 0; c < N; ++c)
+                row[c] = 0.0;
+            continue;
+        }
         double mx = -INFINITY;
         for (int c = 0; c < N; ++c)
             if (row[c] > mx)
@@ -196,14 +231,14 @@ static void unit_forward(const problem_t *p, int b, int wy, int wx, int h,
             double acc = 0.0;
             for (int c = 0; c < N; ++c)
                 acc += w->s[(size_t)a * N + c] * w->v[(size_t)c * d + e];
-            out[(size_t)a * d + e] = acc;
+            out[(size_t)a * d + e] = w->off[a] < 0 ? NAN : acc;
         }
 }
 
 /* Units are numbered u = ((b * nWy + wy) * nWx + wx) * heads + h. */
 static void unit_coords(const problem_t *p, int64_t u, int *b, int *wy, int *wx, int *h)
 {
-    int nWy = p->H / p->M, nWx = p->W / p->M;
+    int nWy = p->Hp / p->M, nWx = p->Wp / p->M;
     *h = (int)(u % p->heads);
     u /= p->heads;
     *wx = (int)(u % nWx);
@@ -232,8 +267,9 @@ static void *worker(void *arg)
     w.k = malloc(N * d * sizeof(double));
     w.v = malloc(N * d * sizeof(double));
     w.s = malloc(N * N * sizeof(double));
+    w.off = malloc(N * sizeof(int64_t));
     double *o = malloc(N * d * sizeof(double));
-    if (!w.q || !w.k || !w.v || !w.s || !o) {
+    if (!w.q || !w.k || !w.v || !w.s || !w.off || !o) {
         __atomic_store_n(&job->failed, 1, __ATOMIC_RELAXED);
         goto done;
     }
@@ -248,11 +284,12 @@ static void *worker(void *arg)
         unit_forward(p, b, wy, wx, h, &w, dst);
         if (job->out_map) {
             /* Step 9: write back through the inverse roll, i.e. to the same
-             * original position each token was gathered from. */
+             * original position each token was gathered from (pads: nowhere). */
             for (int i = 0; i < p->M; ++i)
                 for (int j = 0; j < p->M; ++j) {
-                    size_t off = rolled_token_offset(p, b, wy * p->M + i, wx * p->M + j, h);
-                    memcpy(job->out_map + off, dst + ((size_t)i * p->M + j) * d, d * sizeof(double));
+                    int64_t off = rolled_token_offset(p, b, wy * p->M + i, wx * p->M + j, h);
+                    if (off >= 0)
+                        memcpy(job->out_map + off, dst + ((size_t)i * p->M + j) * d, d * sizeof(double));
                 }
         }
     }
@@ -261,6 +298,7 @@ done:
     free(w.k);
     free(w.v);
     free(w.s);
+    free(w.off);
     free(o);
     return NULL;
 }
@@ -273,7 +311,7 @@ static int check_problem(const problem_t *p)
         return -1;
     if (p->B <= 0 || p->H <= 0 || p->W <= 0 || p->M <= 0 || p->heads <= 0)
         return -1;
-    if (p->H % p->M || p->W % p->M || p->shift < 0 || p->shift >= p->M)
+    if (p->shift < 0 || p->shift >= p->M)
         return -1;
     if (p->d <= 0 || p->d % 4)
         return -1;
@@ -330,24 +368,25 @@ int oracle_fwd(const void *q, const void *k, const void *v, int dtype,
                int B, int H, int W, int M, int shift, int heads, int d, int rank,
                double *out_map, int nthreads, double mem_budget_bytes)
 {
-    problem_t p = {q, k, v, dtype, theta, bias, B, H, W, M, shift, heads, d, rank};
+    problem_t p = make_problem(q, k, v, dtype, theta, bias, B, H, W, M, shift, heads, d, rank);
     if (check_problem(&p) || !out_map)
         return -1;
-    int64_t n = (int64_t)B * (H / M) * (W / M) * heads;
+    int64_t n = (int64_t)B * (p.Hp / M) * (p.Wp / M) * heads;
     return run(&p, NULL, n, NULL, out_map, nthreads, mem_budget_bytes);
 }
 
-/* Selected units; out_units [n_units][M*M][d] fp64 in window order p = i*M + j. */
+/* Selected units; out_units [n_units][M*M][d] fp64 in window order p = i*M + j
+ * (NaN rows at pad positions). */
 int oracle_fwd_units(const void *q, const void *k, const void *v, int dtype,
                      const float *theta, const void *bias,
                      int B, int H, int W, int M, int shift, int heads, int d, int rank,
                      const int64_t *units, int64_t n_units,
                      double *out_units, int nthreads, double mem_budget_bytes)
 {
-    problem_t p = {q, k, v, dtype, theta, bias, B, H, W, M, shift, heads, d, rank};
+    problem_t p = make_problem(q, k, v, dtype, theta, bias, B, H, W, M, shift, heads, d, rank);
     if (check_problem(&p) || !units || !out_units)
         return -1;
-    int64_t total = (int64_t)B * (H / M) * (W / M) * heads;
+    int64_t total = (int64_t)B * (p.Hp / M) * (p.Wp / M) * heads;
     for (int64_t n = 0; n < n_units; ++n)
         if (units[n] < 0 || units[n] >= total)
             return -1;
@@ -364,14 +403,16 @@ int oracle_rope(const double *vec, int d, double i, double j, const float *theta
     return 0;
 }
 
-/* Original (row, col) of rolled-window token p of window (wy, wx). */
+/* Original (row, col) of rolled-window token p of window (wy, wx), in the
+ * padded map; returns 1 when that position is padding, 0 for a real token. */
 int oracle_token_origin(int H, int W, int M, int shift, int wy, int wx, int p, int *y, int *x)
 {
     if (M <= 0 || p < 0 || p >= M * M || !y || !x)
         return -1;
-    *y = (wy * M + p / M + shift) % H;
-    *x = (wx * M + p % M + shift) % W;
-    return 0;
+    const int Hp = (H + M - 1) / M * M, Wp = (W + M - 1) / M * M;
+    *y = (wy * M + p / M + shift) % Hp;
+    *x = (wx * M + p % M + shift) % Wp;
+    return (*y >= H || *x >= W) ? 1 : 0;
 }
 
 /* ---- backward ---------------------------------------------------------------
@@ -410,14 +451,19 @@ static void unit_backward(const problem_t *p, int b, int wy, int wx, int h, cons
     const int M = p->M, N = M * M, d = p->d, r = p->rank;
     const double scale = 1.0 / sqrt((double)p->d);  /* the forward's d^-1/2 */
 
-    /* dO of the unit's rows, from the tokens' original positions */
+    /* dO of the unit's rows, from the tokens' original positions (zero at
+     * pad rows, which have no output) */
     for (int t = 0; t < N; ++t) {
-        size_t off = rolled_token_offset(p, b, wy * M + t / M, wx * M + t % M, h);
-        memcpy(g_o + (size_t)t * d, dout + off, (size_t)d * sizeof(double));
+        if (w->off[t] < 0)
+            memset(g_o + (size_t)t * d, 0, (size_t)d * sizeof(double));
+        else
+            memcpy(g_o + (size_t)t * d, dout + w->off[t], (size_t)d * sizeof(double));
     }
     /* dV, scattered straight to the map */
     for (int c = 0; c < N; ++c) {
-        size_t off = rolled_token_offset(p, b, wy * M + c / M, wx * M + c % M, h);
+        const int64_t off = w->off[c];
+        if (off < 0)
+            continue;
         for (int e = 0; e < d; ++e) {
             double acc = 0.0;
             for (int a = 0; a < N; ++a)
@@ -487,9 +533,10 @@ static void unit_backward(const problem_t *p, int b, int wy, int wx, int h, cons
             rope_rotate(gq, d, -i, -j, th);
             rope_rotate(gk, d, -i, -j, th);
         }
-        size_t off = rolled_token_offset(p, b, wy * M + t / M, wx * M + t % M, h);
-        memcpy(dq + off, gq, (size_t)d * sizeof(double));
-        memcpy(dk + off, gk, (size_t)d * sizeof(double));
+        if (w->off[t] >= 0) {
+            memcpy(dq + w->off[t], gq, (size_t)d * sizeof(double));
+            memcpy(dk + w->off[t], gk, (size_t)d * sizeof(double));
+        }
     }
 }
 
@@ -504,12 +551,13 @@ static void *bwd_worker(void *arg)
     w.k = malloc(N * d * sizeof(double));
     w.v = malloc(N * d * sizeof(double));
     w.s = malloc(N * N * sizeof(double));
+    w.off = malloc(N * sizeof(int64_t));
     double *o = malloc(N * d * sizeof(double));
     double *g_o = malloc(N * d * sizeof(double)), *g_s = malloc(N * N * sizeof(double));
     double *g_q = malloc(N * d * sizeof(double)), *g_k = malloc(N * d * sizeof(double));
     double *dth = job->dtheta ? calloc(nth, sizeof(double)) : NULL;
     double *dbi = job->dbias ? calloc(nbias > 0 ? nbias : 1, sizeof(double)) : NULL;
-    if (!w.q || !w.k || !w.v || !w.s || !o || !g_o || !g_s || !g_q || !g_k || (job->dtheta && !dth) ||
+    if (!w.q || !w.k || !w.v || !w.s || !w.off || !o || !g_o || !g_s || !g_q || !g_k || (job->dtheta && !dth) ||
         (job->dbias && !dbi)) {
         __atomic_store_n(&job->failed, 1, __ATOMIC_RELAXED);
         goto done;
@@ -538,6 +586,7 @@ done:
     free(w.k);
     free(w.v);
     free(w.s);
+    free(w.off);
     free(o);
     free(g_o);
     free(g_s);
@@ -558,7 +607,7 @@ int oracle_bwd(const void *q, const void *k, const void *v, int dtype,
                const double *dout, double *dq, double *dk, double *dv, double *dtheta, double *dbias,
                int nthreads)
 {
-    problem_t p = {q, k, v, dtype, theta, bias, B, H, W, M, shift, heads, d, rank};
+    problem_t p = make_problem(q, k, v, dtype, theta, bias, B, H, W, M, shift, heads, d, rank);
     if (check_problem(&p) || !dout || !dq || !dk || !dv)
         return -1;
     if ((dtheta != NULL && theta == NULL) || (dbias != NULL && bias == NULL))
@@ -568,7 +617,7 @@ int oracle_bwd(const void *q, const void *k, const void *v, int dtype,
         memset(dtheta, 0, (size_t)heads * (d / 4) * sizeof(double));
     if (dbias)
         memset(dbias, 0, (size_t)heads * 2 * N * rank * sizeof(double));
-    int64_t n_units = (int64_t)B * (H / M) * (W / M) * heads;
+    int64_t n_units = (int64_t)B * (p.Hp / M) * (p.Wp / M) * heads;
     long ncpu = sysconf(_SC_NPROCESSORS_ONLN);
     if (nthreads <= 0)
         nthreads = ncpu > 0 ? (int)ncpu : 1;

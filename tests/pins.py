@@ -73,16 +73,20 @@ def rotate_complex(x: np.ndarray, ycoord: np.ndarray, xcoord: np.ndarray, theta_
 def brute_global(q, k, v, M, s, theta=None, bias=None):
     """Masked global attention over all H*W tokens of each image and head.
 
-    Token (y, x) of the original map sits at rolled position ((y - s) mod H,
-    (x - s) mod W).  Two tokens may attend iff they fall in the same window of
-    the rolled map and carry the same Swin region id.  RoPE uses original
-    coordinates; the bias factors use the window-local position."""
+    The map's grid is padded to Hp x Wp, the multiples of M at or above H and
+    W (Swin pads before it rolls); only the H*W real tokens exist here.
+    Token (y, x) of the original map sits at rolled position ((y - s) mod Hp,
+    (x - s) mod Wp).  Two tokens may attend iff they fall in the same window
+    of the rolled grid and carry the same Swin region id of that grid.  RoPE
+    uses original coordinates; the bias factors use the window-local
+    position."""
     q, k, v = (storage_to_f64(a) for a in (q, k, v))
     B, H, W, heads, d = q.shape
+    Hp, Wp = -(-H // M) * M, -(-W // M) * M
     ys, xs = np.meshgrid(np.arange(H), np.arange(W), indexing="ij")
-    yr, xr = (ys - s) % H, (xs - s) % W
-    win = ((yr // M) * (W // M) + (xr // M)).ravel()
-    region = swin_region_labels(H, W, M, s)[yr, xr].ravel()
+    yr, xr = (ys - s) % Hp, (xs - s) % Wp
+    win = ((yr // M) * (Wp // M) + (xr // M)).ravel()
+    region = swin_region_labels(Hp, Wp, M, s)[yr, xr].ravel()
     allowed = (win[:, None] == win[None, :]) & (region[:, None] == region[None, :])
     plocal = ((yr % M) * M + (xr % M)).ravel()
     out = np.zeros_like(q)
@@ -228,6 +232,12 @@ def pin_brute_global(o):
         (2, 6, 6, 2, 4, 3, 1, "fp32", None, 4),
         (1, 8, 8, 2, 8, 4, 1, "bf16", "learned", 4),
         (1, 9, 6, 1, 8, 3, 2, "fp32", "learned", 0),
+        # maps that are not multiples of M: padded grid, pad positions hold no token
+        (1, 10, 7, 2, 8, 4, 2, "bf16", "learned", 0),
+        (2, 9, 13, 1, 8, 4, 0, "fp32", "learned", 0),
+        (1, 7, 5, 2, 4, 3, 1, "fp32", None, 4),
+        (1, 6, 14, 1, 8, 4, 3, "bf16", "standard", 0),
+        (1, 5, 5, 1, 8, 8, 4, "fp32", "learned", 0),
     ]
     for n, (B, H, W, heads, d, M, s, dt, rope, r) in enumerate(cases):
         q, k, v = _maps((B, H, W, heads, d), dt, f"pin-brute-{n}")
@@ -277,5 +287,30 @@ def pin_distinct_offsets(o, M=32, expected=3969):
     assert n == expected, f"{n} distinct offsets, expected {expected}"
 
 
+def pin_padding_closed_forms(o):
+    """Padding, by closed forms.  A 5 x 6 map at M = 4 pads to 8 x 8: rolled
+    window row 1 (no shift) holds only original row 4, so with Q = 0 each of
+    its outputs is the mean of V over that row's tokens of the same window
+    (the pad keys take no weight); constant V still gives the constant; and
+    the units' output marks pad positions NaN, real ones finite."""
+    B, H, W, heads, d, M = 1, 5, 6, 1, 4, 4
+    _, k, v = _maps((B, H, W, heads, d), "fp32", "pin-pad")
+    q = np.zeros_like(k)
+    out = o.fwd(q, k, v, M=M, shift=0)
+    vv = storage_to_f64(v)
+    _close(out[0, 4, 0:4, 0], np.broadcast_to(vv[0, 4, 0:4, 0].mean(0), (4, d)), 1e-13, "row-4 window mean")
+    _close(out[0, 4, 4:6, 0], np.broadcast_to(vv[0, 4, 4:6, 0].mean(0), (2, d)), 1e-13, "row-4 corner mean")
+    _close(out[0, 0:4, 4:6, 0], np.broadcast_to(vv[0, 0:4, 4:6, 0].reshape(8, d).mean(0), (4, 2, d)), 1e-13,
+           "right-edge window mean")
+    c = np.linspace(-1, 2, d).astype(np.float32)
+    cv = np.broadcast_to(c, v.shape).copy()
+    th = I.make_theta(heads, d, "learned", 4).numpy()
+    out = o.fwd(q + 1, k, cv, M=M, shift=3, theta=th)
+    _close(out, np.broadcast_to(c.astype(np.float64), out.shape), 1e-12, "constant V, padded")
+    units = o.fwd_units(q, k, v, [1 * 2 + 1], M=M, shift=0)   # window (1, 1): rows 4..7, cols 4..7
+    pad = np.array([(4 + p // M) >= H or (4 + p % M) >= W for p in range(M * M)])
+    assert np.all(np.isnan(units[0][pad])) and np.all(np.isfinite(units[0][~pad])), "pad rows NaN, real finite"
+
+
 ALL_PINS = [pin_rope_displacement, pin_theta_zero, pin_one_token_windows, pin_constant_v,
-            pin_zero_q_mean, pin_hand_worked, pin_brute_global, pin_bias_concat]
+            pin_zero_q_mean, pin_hand_worked, pin_brute_global, pin_bias_concat, pin_padding_closed_forms]

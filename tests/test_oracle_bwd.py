@@ -49,11 +49,13 @@ def fd_check(o, pr, name, grad, n_samples, seed):
         assert abs(fd - an) <= 2e-5 * scale, f"d{name}{idx}: finite difference {fd:.8f}, backward {an:.8f}"
 
 
-@pytest.mark.parametrize("shift,with_theta,with_bias", [(2, True, False), (0, True, True), (2, False, True),
-                                                        (1, True, True)])
-def test_gradients_match_finite_differences(shift, with_theta, with_bias):
+@pytest.mark.parametrize("shift,with_theta,with_bias,H,W", [(2, True, False, 8, 8), (0, True, True, 8, 8),
+                                                            (2, False, True, 8, 8), (1, True, True, 8, 8),
+                                                            (3, True, True, 7, 6), (0, True, False, 5, 9)])
+def test_gradients_match_finite_differences(shift, with_theta, with_bias, H, W):
+    """(the last two maps are not multiples of M = 4: the padded grid)"""
     o = oracle.oracle()
-    pr = problem(7 + shift, shift, with_theta, with_bias)
+    pr = problem(7 + shift, shift, with_theta, with_bias, H=H, W=W)
     dq, dk, dv, dtheta, dbias = o.bwd(pr["q"], pr["k"], pr["v"], pr["dout"], M=pr["M"], shift=shift,
                                       theta=pr["theta"], bias=pr["bias"])
     fd_check(o, pr, "q", dq, 48, 1)

@@ -20,11 +20,11 @@ MUTANTS = {
                               "double x0 = vec[2 * k + 1], x1 = vec[2 * k];")],
     "mask_dropped": [("if (la != lc)", "if (0)")],
     "mask_inverted": [("if (la != lc)", "if (la == lc && a != c)")],
-    "label_off_by_one": [("yr >= p->H - p->shift", "yr > p->H - p->shift")],
+    "label_off_by_one": [("yr >= p->Hp - p->shift", "yr > p->Hp - p->shift")],
     "scale_dropped": [("const double scale = 1.0 / sqrt((double)d);", "const double scale = 1.0;")],
     "roll_reversed": [
-        ("int y = (yr + p->shift) % p->H;", "int y = (yr - p->shift + p->H) % p->H;"),
-        ("int x = (xr + p->shift) % p->W;", "int x = (xr - p->shift + p->W) % p->W;"),
+        ("int y = (yr + p->shift) % p->Hp;", "int y = (yr - p->shift + p->Hp) % p->Hp;"),
+        ("int x = (xr + p->shift) % p->Wp;", "int x = (xr - p->shift + p->Wp) % p->Wp;"),
     ],
     "scores_transposed": [("dot += w->q[(size_t)a * d + e] * w->k[(size_t)c * d + e];",
                            "dot += w->q[(size_t)c * d + e] * w->k[(size_t)a * d + e];")],
@@ -38,9 +38,16 @@ MUTANTS = {
     "bias_scaled": [("sc += bd;", "sc += scale * bd;")],
     "bias_dropped": [("sc += bd;", "sc += 0.0 * bd;")],
     "scatter_unrolled": [(
-        "size_t off = rolled_token_offset(p, b, wy * p->M + i, wx * p->M + j, h);",
-        "size_t off = rolled_token_offset(p, b, (wy * p->M + i + p->H - p->shift) % p->H, "
-        "(wx * p->M + j + p->W - p->shift) % p->W, h);")],
+        "int64_t off = rolled_token_offset(p, b, wy * p->M + i, wx * p->M + j, h);\n                    if",
+        "int64_t off = rolled_token_offset(p, b, (wy * p->M + i + p->Hp - p->shift) % p->Hp, "
+        "(wx * p->M + j + p->Wp - p->shift) % p->Wp, h);\n                    if")],
+    # padding (maps that are not multiples of M)
+    "pad_keys_attended": [("            if (w->off[c] < 0)\n                w->s[(size_t)a * N + c] = -INFINITY;",
+                           "            if (0)\n                w->s[(size_t)a * N + c] = -INFINITY;")],
+    "roll_over_unpadded_map": [
+        ("int y = (yr + p->shift) % p->Hp;", "int y = (yr + p->shift) % p->H;"),
+        ("int x = (xr + p->shift) % p->Wp;", "int x = (xr + p->shift) % p->W;"),
+    ],
     "query_coords_global": [(
         "rope_rotate(w->q + (size_t)t * d, d, (double)i, (double)j, th);",
         "rope_rotate(w->q + (size_t)t * d, d, (double)(i + wy * M), (double)j, th);")],

@@ -47,6 +47,6 @@ def test_units_match_full_map(orc):
 def test_rejects_bad_problems(orc):
     q, k, v = pins._maps((1, 8, 8, 1, 8), "fp32", "reject")
     with pytest.raises(ValueError):
-        orc.fwd(q, k, v, M=3)            # 8 % 3 != 0
+        orc.fwd(q, k, v, M=0)            # windows need M >= 1
     with pytest.raises(ValueError):
         orc.fwd(q, k, v, M=4, shift=4)   # shift must be < M
