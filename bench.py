@@ -251,7 +251,8 @@ def oracle_sample_rate(w, target_s, base=0):
 # The metric is throughput against the window size M: besides the headline
 # workload, one line per sweep point (shift M/2, both head dims) and the dense
 # and SR calls, each timed with CUDA events over back-to-back calls.
-PER_M = [f"sweep_M{M}_d{d}_s{M // 2}" for M in (8, 16, 32, 64, 96) for d in (32, 64)] + ["dense", "sr"]
+PER_M = ([f"sweep_M{M}_d{d}_s{M // 2}" for M in (8, 16, 32, 64, 96) for d in (32, 64)]
+         + ["dense", "sr", "flashswin_M16", "flashswin_M32"])
 
 
 def per_m_table(dev, peaks, target_s=0.25):

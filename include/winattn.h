@@ -16,7 +16,13 @@
  *                + ( -inf if shift > 0 and L(p) != L(p') else 0 )
  *     o_p = sum_p' softmax_p'(z(p, .)) v_p'
  *
- *   and o_p is written back to the original position of token p.  R(i, j)
+ *   and o_p is written back to the original position of token p.  A map
+ *   whose sides are not multiples of M is padded at the bottom and right to
+ *   Hp x Wp, the next multiples of M, before the roll (H and W above read
+ *   Hp and Wp; Swin pads before its roll, and FlashSwin-T runs M = 16 and 32
+ *   on its 56 x 56 map, "FLASHSWIN" page, section "무엇과 다른가"); pad
+ *   positions hold no token: they are never attended to (-inf) and never
+ *   written, and nothing is copied.  R(i, j)
  *   is window-local 2D RoPE: pair (2k, 2k+1) of the first half of the head
  *   dim turns counter-clockwise by i * theta_h[k], pair (d/2 + 2k,
  *   d/2 + 2k + 1) of the second half by j * theta_h[k], k < d/4.  L is the
@@ -43,7 +49,7 @@ extern "C" {
 
 /* Return codes.  0 is success; every error is negative. */
 #define WINATTN_OK                  0
-#define WINATTN_ERR_ARG            -1  /* null pointer, non-positive size, H % M or W % M != 0,
+#define WINATTN_ERR_ARG            -1  /* null pointer, non-positive size, M > 256,
                                           shift outside [0, M), unsupported head dim d          */
 #define WINATTN_ERR_RANK           -2  /* rank > 0 without bias_feats, bias_feats without rank,
                                           or rank outside the supported set                    */
@@ -74,7 +80,8 @@ extern "C" {
  *               window-local p = i*M + j; or NULL when rank == 0.  16-byte
  *               aligned.  Read only.
  *   B, H_img, W_img, M, shift, heads, d, rank
- *               sizes: H_img % M == 0, W_img % M == 0, 0 <= shift < M,
+ *               sizes: any H_img, W_img >= 1 (padded to multiples of M as
+ *               above), 0 <= shift < M,
  *               d in {32, 64} for WINATTN_BF16, d in {16, 32, 64} for
  *               WINATTN_FP32; rank in {0, 16, 32}; M <= 256; the number of
  *               128-row query tiles must fit in a 31-bit grid.

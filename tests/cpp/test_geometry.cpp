@@ -49,7 +49,10 @@ static void check_fastdiv()
 static void check_problem(int B, int H, int W, int M, int s, int heads, int d)
 {
     const Geometry g = Geometry::make(B, H, W, M, s, heads, d, 0);
-    const int nWy = H / M, nWx = W / M, N = M * M;
+    // the grid is padded to multiples of M; pad positions hold no token
+    const int nWy = (H + M - 1) / M, nWx = (W + M - 1) / M, N = M * M;
+    const int Hp = nWy * M, Wp = nWx * M;
+    CHECK(g.Hp == Hp && g.Wp == Wp && g.padded == (Hp != H || Wp != W), "padded grid");
     const int U = N >= 128 ? 1 : 128 / N;
     CHECK(g.U == U, "U");
     // every (pack, tile, row) maps to the token plain arithmetic gives
@@ -69,10 +72,12 @@ static void check_problem(int B, int H, int W, int M, int s, int heads, int d)
                     const TokenRef tk = token_ref(g, w, p, h);
                     const int b = w / (nWy * nWx), wy = (w % (nWy * nWx)) / nWx, wx = w % nWx;
                     const int i = p / M, j = p % M;
-                    const int y = (wy * M + i + s) % H, x = (wx * M + j + s) % W;
-                    const long long off = ((((long long)b * H + y) * W + x) * heads + h) * d;
-                    const int label = s ? 2 * (wy * M + i >= H - s) + (wx * M + j >= W - s) : 0;
-                    CHECK(tk.offset == off && tk.i == i && tk.j == j && tk.label == label, "token_ref");
+                    const int y = (wy * M + i + s) % Hp, x = (wx * M + j + s) % Wp;
+                    const bool pad = y >= H || x >= W;
+                    const long long off = pad ? 0 : ((((long long)b * H + y) * W + x) * heads + h) * d;
+                    const int label = s ? 2 * (wy * M + i >= Hp - s) + (wx * M + j >= Wp - s) : 0;
+                    CHECK(tk.pad == pad && tk.offset == off && tk.i == i && tk.j == j && tk.label == label,
+                          "token_ref");
                     CHECK(window_wrapped(g, w) == (s > 0 && (wy == nWy - 1 || wx == nWx - 1)), "wrapped");
                 }
             }
@@ -100,6 +105,11 @@ int main()
     check_problem(1, 24, 24, 12, 6, 2, 32);
     check_problem(1, 64, 96, 32, 16, 3, 32);
     check_problem(1, 192, 96, 96, 48, 2, 64);
+    // padded grids
+    check_problem(2, 56, 56, 32, 16, 3, 32);
+    check_problem(1, 56, 56, 16, 8, 2, 32);
+    check_problem(2, 10, 13, 4, 2, 2, 32);
+    check_problem(1, 5, 7, 3, 1, 1, 64);
     if (failures) {
         std::printf("%d failures\n", failures);
         return 1;

@@ -60,10 +60,13 @@ def full_compare(w: I.Workload, shift: int, device="cuda", base: int = 0):
 
 
 def window_positions(H, W, M, shift, wy, wx):
+    """Original (y, x) of the window's tokens in window order, on the grid
+    padded to multiples of M, and which of them are real (not padding)."""
+    Hp, Wp = -(-H // M) * M, -(-W // M) * M
     p = np.arange(M * M)
-    y = (wy * M + p // M + shift) % H
-    x = (wx * M + p % M + shift) % W
-    return y, x
+    y = (wy * M + p // M + shift) % Hp
+    x = (wx * M + p % M + shift) % Wp
+    return y, x, (y < H) & (x < W)
 
 
 def sample_windows(nWy, nWx, rng, extra=2):
@@ -81,7 +84,7 @@ def sampled_compare(w: I.Workload, shift: int, images, heads=None, extra_windows
     out = run_gpu(*qkv, w.M, shift, theta, bias)
     assert torch.isfinite(out.float()).all().item(), "non-finite values in the output"
     rng = np.random.default_rng(seed)
-    nWy, nWx = w.H // w.M, w.W // w.M
+    nWy, nWx = -(-w.H // w.M), -(-w.W // w.M)
     heads = list(range(w.heads)) if heads is None else heads
     th = None if theta is None else theta.cpu().numpy()
     bs = I.to_storage_numpy(bias)
@@ -112,7 +115,13 @@ def sampled_compare(w: I.Workload, shift: int, images, heads=None, extra_windows
             locs = list(must.values()) + [locs[i] for i in rest[:extra]]
         ref = orc().fwd_units(*sub, units, M=w.M, shift=shift, theta=th, bias=bs)
         got_img = out[b].float().cpu().numpy().astype(np.float64)
-        got = np.stack([got_img[window_positions(w.H, w.W, w.M, shift, wy, wx) + (h,)]
-                        for (wy, wx, h) in locs])
+        got, keep = [], []
+        for (wy, wx, h) in locs:
+            y, x, real = window_positions(w.H, w.W, w.M, shift, wy, wx)
+            got.append(got_img[y[real], x[real], h])
+            keep.append(real)
+        # pad positions hold no token: compared rows are the real ones
+        got = np.concatenate(got)
+        ref = np.concatenate([r[k] for r, k in zip(ref, keep)])
         results.append(check(got, ref, w.dtype, f"{w.name} s{shift} image {b}"))
     return results

@@ -48,6 +48,7 @@ def test_check_args_accepts_valid(lib):
     assert chk(rank=16, bias=6 * A) == _lib.OK
     assert chk(dtype=_lib.FP32, d=16) == _lib.OK
     assert chk(M=1, shift=0) == _lib.OK
+    assert chk(M=3, shift=1) == _lib.OK   # 16 % 3 != 0: the grid is padded to 18 x 18
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -56,7 +57,6 @@ def test_check_args_accepts_valid(lib):
     (dict(B=0), _lib.ERR_ARG),
     (dict(heads=-1), _lib.ERR_ARG),
     (dict(M=0), _lib.ERR_ARG),
-    (dict(M=3), _lib.ERR_ARG),            # 16 % 3 != 0
     (dict(shift=8), _lib.ERR_ARG),        # shift must be < M
     (dict(shift=-1), _lib.ERR_ARG),
     (dict(d=48), _lib.ERR_ARG),           # bf16 head dims are 32 or 64
@@ -106,11 +106,13 @@ GENERIC, SMALL, LARGE, SIMT, PIPE = 0, 1, 2, 3, 4
     (2, 5, 5, 1, 0, 1, 32, 0, 128, 1, SMALL),        # one-token windows
     (1, 10, 10, 10, 0, 1, 32, 0, 1, 1, SMALL),       # 100 tokens: one ragged tile
     (1, 8, 8, 8, 0, 80, 32, 0, 2, 1, GENERIC),       # too many heads for a shared-memory RoPE table
+    (64, 56, 56, 32, 16, 3, 32, 0, 1, 8, LARGE),     # FlashSwin-T at M = 32: 56 padded to 64, pad keys masked
+    (2, 10, 13, 4, 2, 2, 32, 0, 8, 1, GENERIC),      # padded 12 x 16 grid of 16-token windows
 ])
 def test_launch_plan(lib, B, H, W, M, shift, heads, d, rank, U, tiles, kernel):
     rc, info = _lib.launch_info(B, H, W, M, shift, heads, d, rank, _lib.BF16)
     assert rc == _lib.OK
-    windows = B * (H // M) * (W // M)
+    windows = B * (-(-H // M)) * (-(-W // M))   # windows of the grid padded to multiples of M
     assert info["windows_per_tile"] == U
     assert info["kernel"] == kernel
     if kernel == LARGE:  # items are pairs of query tiles

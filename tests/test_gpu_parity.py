@@ -57,6 +57,14 @@ SMALL = [
     ("m96_s0_r16", 1, 96, 96, 96, 0, 2, 32, "bf16", None, 16),
     ("m8_s4_r32_rope", 2, 16, 16, 8, 4, 2, 32, "bf16", "learned", 32),
     ("m16_s8_d64_r16", 1, 32, 32, 16, 8, 1, 64, "bf16", "learned", 16),
+    # grids that are not multiples of M: padded, pad positions masked and never written
+    ("m32_s16_pad56", 1, 56, 56, 32, 16, 2, 32, "bf16", "learned", 0),
+    ("m32_s0_pad56", 1, 56, 56, 32, 0, 2, 32, "bf16", "standard", 0),
+    ("m16_s8_pad_d64", 1, 56, 40, 16, 8, 2, 64, "bf16", "learned", 0),
+    ("m4_s2_pad", 2, 10, 13, 4, 2, 2, 32, "bf16", "learned", 0),
+    ("m8_s4_pad20", 1, 20, 20, 8, 4, 2, 32, "bf16", "learned", 0),
+    ("m7_s3_pad_r16", 1, 10, 9, 7, 3, 2, 32, "bf16", None, 16),
+    ("fp32_m5_pad", 1, 12, 7, 5, 2, 2, 32, "fp32", "learned", 0),
     ("fp32_m8_d16", 1, 16, 16, 8, 4, 2, 16, "fp32", "learned", 0),
     ("fp32_m12_d64_r16", 1, 24, 24, 12, 6, 1, 64, "fp32", "learned", 16),
     ("fp32_m4_d32_r32", 2, 8, 8, 4, 2, 2, 32, "fp32", None, 32),
@@ -90,6 +98,15 @@ def test_dense_sampled(shift):
 def test_sr_rib_sampled():
     w = I.WORKLOADS["sr"]
     G.sampled_compare(w, 0, images=[w.B - 1], heads=[0, 5], extra_windows=0, max_units=6)
+
+
+@pytest.mark.parametrize("name", ["flashswin_M16", "flashswin_M32"])
+def test_flashswin_padded_sampled(name):
+    """FlashSwin-T's 56 x 56 map at M = 16 and 32 (padded to 64 x 64), full
+    size, sampled windows: every corner and seam window, which hold the pad
+    positions."""
+    w = I.WORKLOADS[name]
+    G.sampled_compare(w, w.shifts[0], images=[0, w.B - 1], extra_windows=2, max_units=12)
 
 
 SWEEP = [n for n in I.WORKLOADS if n.startswith("sweep_")]

@@ -171,6 +171,46 @@ struct LargeMaps {
     CUtensorMap k_full, k_half, v_full, v_half, w;
 };
 
+// Sets bits [start, start + len) of a 128-bit mask.
+__device__ __forceinline__ void set_bit_range(uint32_t (&mk)[4], int start, int len)
+{
+#pragma unroll
+    for (int wd = 0; wd < 4; ++wd) {
+        const int lo = max(start - 32 * wd, 0), hi = min(start + len - 32 * wd, 32);
+        if (hi > lo)
+            mk[wd] |= (hi - lo == 32 ? 0xFFFFFFFFu : ((1u << (hi - lo)) - 1u)) << lo;
+    }
+}
+
+// Real keys of key tile jt of window (wy, wx) on a padded grid, as a mask
+// over the tile's keys in box order (bit c = key c).  The tile's kr window
+// rows start at row y0 and never wrap inside the tile, so its real rows are
+// a prefix; in each row the real columns are a prefix of the box (two boxes
+// at the column seam: the far side starts at column 0).  Pad positions read
+// the TMA fill value and must take no weight.
+__device__ __forceinline__ void large_key_mask(const Geometry &g, int wy, int wx, int jt, int kr, int BN,
+                                               bool xwrap, uint32_t (&mk)[4])
+{
+    mk[0] = mk[1] = mk[2] = mk[3] = 0u;
+    int y0 = wy * g.M + jt * kr + g.shift;
+    if (y0 >= g.Hp)
+        y0 -= g.Hp;
+    const int vr = min(max(g.H - y0, 0), kr);
+    const int x0 = wx * g.M + g.shift;
+    if (!xwrap) {
+        const int pc = min(max(g.W - x0, 0), g.M);
+        for (int ri = 0; ri < vr; ++ri)
+            set_bit_range(mk, ri * g.M, pc);
+    } else {
+        const int hm = g.M >> 1;
+        const int pl = min(max(g.W - x0, 0), hm), pr = min(g.W, hm);
+        for (int ri = 0; ri < vr; ++ri) {
+            set_bit_range(mk, ri * hm, pl);
+            set_bit_range(mk, BN / 2 + ri * hm, pr);
+        }
+    }
+}
+
 // Epilogue of one query row of item ke: waits for the item's last P V, writes
 // O / l (bf16) to `dst` (the token's original position) and hands the O
 // buffer (ke % NOB) back to the P V issuer.
@@ -184,7 +224,7 @@ __device__ __forceinline__ bool large_epilogue_body(__nv_bfloat16 *dst_row, uint
     const uint32_t oe = obase + (ke % NOB) * 2 * D;
     const float inv = 1.f / le;
     const float2 i2 = make_float2(inv, inv);
-    uint4 *dst = reinterpret_cast<uint4 *>(dst_row);
+    uint4 *dst = reinterpret_cast<uint4 *>(dst_row);  // null for a pad row: loads only (warp-collective)
 #pragma unroll
     for (int ch = 0; ch < D / 16; ++ch) {
         float o[16];
@@ -200,7 +240,8 @@ __device__ __forceinline__ bool large_epilogue_body(__nv_bfloat16 *dst_row, uint
             u.y = pack_bf16x2(y[1].x, y[1].y);
             u.z = pack_bf16x2(y[2].x, y[2].y);
             u.w = pack_bf16x2(y[3].x, y[3].y);
-            dst[2 * ch + hh] = u;
+            if (dst)
+                dst[2 * ch + hh] = u;
         }
     }
     tc_fence_before_sync();
@@ -217,7 +258,10 @@ __device__ __noinline__ bool large_epilogue_call(__nv_bfloat16 *dst_row, uint32_
     return large_epilogue_body<D, NOB>(dst_row, obase, ke, le, o_last, t_free, abort_flag);
 }
 
-template <int D, int R, int BN>
+// PAD: the grid is padded (maps that are not multiples of M); the softmax
+// then masks pad keys per tile.  A separate instantiation, so that the
+// unpadded kernel's softmax carries none of it.
+template <int D, int R, int BN, bool PAD>
 __global__ void __launch_bounds__(kLargeThreads, 1)
     winattn_fwd_large_kernel(const __nv_bfloat16 *__restrict__ q, const float *__restrict__ theta,
                              const __nv_bfloat16 *__restrict__ bias, __nv_bfloat16 *__restrict__ out,
@@ -334,9 +378,11 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
                         }
                         const uint32_t sst = sbase + L::STAGES + s * L::STAGE;
                         mbar_arrive_expect_tx(&kv_full[s], bytes);
+                        // rows and columns past H, W (a padded grid) read the
+                        // fill value; they are masked in the softmax
                         int y0 = wy * M + jt * kr + g.shift;
-                        if (y0 >= g.H) y0 -= g.H;
-                        const int x0 = wx * M + g.shift;  // < W unless the window straddles the seam
+                        if (y0 >= g.Hp) y0 -= g.Hp;
+                        const int x0 = wx * M + g.shift;  // < Wp unless the window straddles the seam
                         const int c0 = h * D;
                         if (xwrap) {
                             const int x1 = 0;             // the seam's far side
@@ -582,11 +628,13 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
         constexpr int NCH = BN / 16;                           // 16-column chunks of S
         int c = 0;
         bool failed = false;
+        // off < 0: a pad row, nothing is stored
         auto epilogue = [&](int ke, int64_t off, float le) -> bool {
+            __nv_bfloat16 *dst = off < 0 ? nullptr : out + off;
             if constexpr (NOB == 2)
-                return large_epilogue_call<D, NOB>(out + off, obase, ke, le, &o_last[tile], &t_free[tile], abort_flag);
+                return large_epilogue_call<D, NOB>(dst, obase, ke, le, &o_last[tile], &t_free[tile], abort_flag);
             else
-                return large_epilogue_body<D, NOB>(out + off, obase, ke, le, &o_last[tile], &t_free[tile], abort_flag);
+                return large_epilogue_body<D, NOB>(dst, obase, ke, le, &o_last[tile], &t_free[tile], abort_flag);
         };
         // With two O buffers an item's epilogue runs after the first step of
         // the next item, when its last P V has long completed, instead of
@@ -631,6 +679,13 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
                     a0 = me_lx ? NCH / 2 : 0;
                     a1 = a0 + NCH / 2;
                 }
+                // a padded grid: pad keys of this tile (same for every row)
+                uint32_t mk[4] = {~0u, ~0u, ~0u, ~0u};
+                bool masked = false;
+                if constexpr (PAD) {
+                    large_key_mask(g, wy, wx, jt, kr, BN, xwrap, mk);
+                    masked = (mk[0] & mk[1] & mk[2] & (BN == 128 ? mk[3] : ~0u)) != ~0u;
+                }
                 // ---- pass 1: the row of S into registers (all loads in
                 // flight at once, one wait), then its max over the allowed
                 // columns (four independent max chains)
@@ -642,6 +697,14 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
 #pragma unroll
                 for (int ch = 1; ch < NC; ++ch)
                     reg_fence32(sv[ch]);
+                if (PAD && masked) {
+                    // pad keys: -inf scores, so they weigh nothing
+#pragma unroll
+                    for (int ch = 0; ch < NC; ++ch)
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            sv[ch][e] = ((mk[ch] >> e) & 1u) ? sv[ch][e] : 0xFF800000u;
+                }
                 float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
                 for (int ch = 0; ch < NC; ++ch) {
@@ -658,6 +721,8 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
                     }
                 }
                 const float mx = fmaxf(fmax3(mq[0], mq[1], mq[2]), mq[3]);
+                if (PAD && mx == -INFINITY)
+                    a0 = a1 = 0;  // nothing of this tile is left after the pad mask
                 float alpha = 1.f;
                 bool rescale = false;
                 if (mx > -INFINITY) {
@@ -738,9 +803,9 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
                 break;
             if constexpr (NOB == 2) {
                 pend_kk = kk;
-                pend_off = me.offset;
+                pend_off = me.pad ? -1 : me.offset;
                 pend_l = l;
-            } else if (!epilogue(kk, me.offset, l)) {
+            } else if (!epilogue(kk, me.pad ? -1 : me.offset, l)) {
                 failed = true;
                 break;
             }

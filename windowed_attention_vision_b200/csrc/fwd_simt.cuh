@@ -70,8 +70,10 @@ __global__ void __launch_bounds__(128)
     float qv[D + R];
     int qcode = 0xFFFF;
     TokenRef qt{};
-    if (qr.valid) {
+    if (qr.valid)
         qt = token_ref(g, qr.w, qr.p, it.h);
+    const bool qreal = qr.valid && !qt.pad;  // a pad row of a padded grid has no output
+    if (qreal) {
         qcode = (qr.slot << 2) | qt.label;
 #pragma unroll
         for (int e = 0; e < D; ++e)
@@ -106,8 +108,8 @@ __global__ void __launch_bounds__(128)
             float *vr = vs + t * D;
             if (kk < key_rows) {
                 const RowRef rr = tile_row(g, it.pack, kk / kTileRows, kk % kTileRows);
-                if (rr.valid) {
-                    const TokenRef tk = token_ref(g, rr.w, rr.p, it.h);
+                const TokenRef tk = rr.valid ? token_ref(g, rr.w, rr.p, it.h) : TokenRef{};
+                if (rr.valid && !tk.pad) {
                     code = (uint16_t)((rr.slot << 2) | tk.label);
                     float x[D];
 #pragma unroll
@@ -148,7 +150,7 @@ __global__ void __launch_bounds__(128)
             m = m_new;
         }
     }
-    if (qr.valid) {
+    if (qreal) {
         const float inv = 1.f / l;
 #pragma unroll
         for (int e = 0; e < D; ++e)

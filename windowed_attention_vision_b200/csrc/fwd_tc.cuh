@@ -154,8 +154,10 @@ __global__ void __launch_bounds__(128, 1)
     // ---- query row t
     const RowRef qr = tile_row(g, it.pack, it.tile, t);
     int qcode = 0xFFFF;  // matches no key code
-    if (qr.valid) {
-        const TokenRef tk = token_ref(g, qr.w, qr.p, it.h);
+    const TokenRef qtk = qr.valid ? token_ref(g, qr.w, qr.p, it.h) : TokenRef{};
+    const bool qreal = qr.valid && !qtk.pad;  // a pad row of a padded grid has no output
+    if (qreal) {
+        const TokenRef &tk = qtk;
         qcode = (qr.slot << 2) | tk.label;
         gather_rotate_store<D>(q + tk.offset, tab, tk.i, tk.j, scale, base + L::QC, t);
         if constexpr (R > 0)
@@ -181,8 +183,8 @@ __global__ void __launch_bounds__(128, 1)
         // ---- 1. gather K (rotated), w, V for key row t
         const RowRef kr = tile_row(g, it.pack, kv, t);
         uint16_t code = 0xFFFE;
-        if (kr.valid) {
-            const TokenRef tk = token_ref(g, kr.w, kr.p, it.h);
+        const TokenRef tk = kr.valid ? token_ref(g, kr.w, kr.p, it.h) : TokenRef{};
+        if (kr.valid && !tk.pad) {
             code = (uint16_t)((kr.slot << 2) | tk.label);
             gather_rotate_store<D>(k + tk.offset, tab, tk.i, tk.j, 1.f, base + L::KC, t);
             if constexpr (R > 0)
@@ -291,8 +293,8 @@ __global__ void __launch_bounds__(128, 1)
     }
 
     // ---- normalise and write back to the original (un-shifted) position
-    if (ok && qr.valid) {
-        const TokenRef tk = token_ref(g, qr.w, qr.p, it.h);
+    if (ok && qreal) {
+        const TokenRef &tk = qtk;
         const float inv = 1.f / l;
         uint4 *dst = reinterpret_cast<uint4 *>(out + tk.offset);
 #pragma unroll

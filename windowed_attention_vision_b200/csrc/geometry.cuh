@@ -8,6 +8,12 @@
 // so no rolled copy of the map is ever made, and the write-back goes to the
 // same original position (the inverse roll).
 //
+// A map whose sides are not multiples of M is padded at the bottom and right
+// to Hp x Wp (the next multiples of M), and the padded grid is rolled and cut
+// into windows (Swin pads before its roll); pad positions hold no token: they
+// are masked as keys and never written.  Nothing is copied: a pad position is
+// only a flag of the index math.
+//
 // Indices are 32-bit (the host rejects problems whose window or item counts
 // reach 2^31); divisions by the problem's runtime sizes use precomputed
 // multiply-shift reciprocals.
@@ -51,6 +57,8 @@ struct FastDiv {
 
 struct Geometry {
     int B, H, W, M, shift, heads, d, rank;
+    int Hp, Wp;        // H, W rounded up to multiples of M (the padded grid)
+    bool padded;       // Hp != H or Wp != W
     int nWy, nWx;      // windows per image along rows / columns
     int N;             // tokens per window, M*M
     int U;             // windows packed into one tile (>= 1; > 1 only when N <= 64)
@@ -64,8 +72,11 @@ struct Geometry {
     {
         Geometry g;
         g.B = B; g.H = H; g.W = W; g.M = M; g.shift = shift; g.heads = heads; g.d = d; g.rank = rank;
-        g.nWy = H / M;
-        g.nWx = W / M;
+        g.nWy = (H + M - 1) / M;
+        g.nWx = (W + M - 1) / M;
+        g.Hp = g.nWy * M;
+        g.Wp = g.nWx * M;
+        g.padded = g.Hp != H || g.Wp != W;
         g.N = M * M;
         g.U = g.N >= kTileRows ? 1 : kTileRows / g.N;
         g.n_tiles = g.U > 1 ? 1 : (g.N + kTileRows - 1) / kTileRows;
@@ -141,9 +152,10 @@ __host__ __device__ inline RowRef tile_row(const Geometry &g, int pack, int tile
 }
 
 struct TokenRef {
-    int64_t offset;  // element offset of the (token, head) d-vector in the map
+    int64_t offset;  // element offset of the (token, head) d-vector in the map (0 for a pad)
     int i, j;        // window-local row / column
     int label;       // wrap label: 2*[rolled row in last `shift` rows] + [rolled col in last `shift` cols]
+    bool pad;        // a pad position of the padded grid: no token
 };
 
 __host__ __device__ inline TokenRef token_ref(const Geometry &g, int w, int p, int h)
@@ -158,11 +170,12 @@ __host__ __device__ inline TokenRef token_ref(const Geometry &g, int w, int p, i
     const int yr = wy * g.M + t.i;
     const int xr = wx * g.M + t.j;
     int y = yr + g.shift;
-    if (y >= g.H) y -= g.H;
+    if (y >= g.Hp) y -= g.Hp;
     int x = xr + g.shift;
-    if (x >= g.W) x -= g.W;
-    t.label = g.shift ? 2 * (yr >= g.H - g.shift) + (xr >= g.W - g.shift) : 0;
-    t.offset = ((((int64_t)b * g.H + y) * g.W + x) * g.heads + h) * g.d;
+    if (x >= g.Wp) x -= g.Wp;
+    t.label = g.shift ? 2 * (yr >= g.Hp - g.shift) + (xr >= g.Wp - g.shift) : 0;
+    t.pad = y >= g.H || x >= g.W;
+    t.offset = t.pad ? 0 : ((((int64_t)b * g.H + y) * g.W + x) * g.heads + h) * g.d;
     return t;
 }
 

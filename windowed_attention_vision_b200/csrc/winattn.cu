@@ -40,7 +40,7 @@ int check_sizes(int B, int H, int W, int M, int shift, int heads, int d, int ran
         return WINATTN_ERR_DTYPE;
     if (B <= 0 || H <= 0 || W <= 0 || M <= 0 || heads <= 0 || M > kMaxM)
         return WINATTN_ERR_ARG;
-    if (H % M || W % M || shift < 0 || shift >= M)
+    if (shift < 0 || shift >= M)
         return WINATTN_ERR_ARG;
     if (dtype == WINATTN_BF16 && d != 32 && d != 64)
         return WINATTN_ERR_ARG;
@@ -222,6 +222,11 @@ KernelKind choose_kernel(const Geometry &g, int dtype)
 {
     if (dtype == WINATTN_FP32)
         return kSimt;
+    // the generic kernel resolves every token through the index math, pad
+    // positions of a padded grid included; of the specialised kernels only
+    // the large-window one masks pad keys
+    if (g.padded)
+        return kernel_enabled(kLarge) && large_ok(g) ? kLarge : kGeneric;
     if (kernel_enabled(kPipe) && pipe_ok(g) && (uint64_t)g.heads * g.M * (g.d / 4) * 8 <= kSmallTableMax &&
         pipe_smem(g) <= kMaxSmem)
         return kPipe;
@@ -395,25 +400,25 @@ bool encode_factor_map(CUtensorMap *m, const void *base, const Geometry &g, int 
 // Whether the built large-window kernel has exactly kLargeRegsLaunch
 // registers per thread: its warpgroups' setmaxnreg shares add up to the
 // launch's registers only then.  Looked up once per instantiation.
-template <int D, int R, int BN>
+template <int D, int R, int BN, bool PAD>
 bool large_regs_ok()
 {
     static const bool ok = [] {
         cudaFuncAttributes fa;
-        return cudaFuncGetAttributes(&fa, winattn_fwd_large_kernel<D, R, BN>) == cudaSuccess &&
+        return cudaFuncGetAttributes(&fa, winattn_fwd_large_kernel<D, R, BN, PAD>) == cudaSuccess &&
                fa.numRegs == (int)kLargeRegsLaunch;
     }();
     return ok;
 }
 
-template <int D, int R, int BN>
+template <int D, int R, int BN, bool PAD>
 int launch_large(const void *q, const void *k, const void *v, const float *theta, const void *bias, void *out,
                  const Geometry &g, cudaStream_t stream)
 {
     using T = __nv_bfloat16;
     // a build whose register count differs would wait forever in setmaxnreg:
     // its problems go to the generic tensor-core kernel instead
-    if (!large_regs_ok<D, R, BN>())
+    if (!large_regs_ok<D, R, BN, PAD>())
         return launch_tc<D, R>(q, k, v, theta, bias, out, g, stream);
     MapSet ms;
     const MapKey key = make_key(kLarge, g, k, v, bias, nullptr, nullptr);
@@ -430,8 +435,8 @@ int launch_large(const void *q, const void *k, const void *v, const float *theta
     static_assert(sizeof(LargeMaps) == 5 * sizeof(CUtensorMap), "LargeMaps is five maps");
     LargeMaps maps;
     std::memcpy(&maps, ms.m, sizeof maps);
-    auto kernel = winattn_fwd_large_kernel<D, R, BN>;
-    if (!smem_attr_once<winattn_fwd_large_kernel<D, R, BN>>())
+    auto kernel = winattn_fwd_large_kernel<D, R, BN, PAD>;
+    if (!smem_attr_once<winattn_fwd_large_kernel<D, R, BN, PAD>>())
         return WINATTN_ERR_CUDA;
     // all 512 TMEM columns per CTA: enough shared memory that no second CTA
     // is resident on the same SM
@@ -450,8 +455,10 @@ int launch_large_bn(const void *q, const void *k, const void *v, const float *th
                     const Geometry &g, cudaStream_t s)
 {
     if (large_tile_keys(g.M) == 96)
-        return launch_large<D, R, 96>(q, k, v, theta, bias, out, g, s);
-    return launch_large<D, R, 128>(q, k, v, theta, bias, out, g, s);
+        return g.padded ? launch_large<D, R, 96, true>(q, k, v, theta, bias, out, g, s)
+                        : launch_large<D, R, 96, false>(q, k, v, theta, bias, out, g, s);
+    return g.padded ? launch_large<D, R, 128, true>(q, k, v, theta, bias, out, g, s)
+                    : launch_large<D, R, 128, false>(q, k, v, theta, bias, out, g, s);
 }
 
 template <int D, int R, bool TMA>

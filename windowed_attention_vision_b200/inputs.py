@@ -57,7 +57,9 @@ class Workload:
 
     def flops(self) -> float:
         """Algorithmic FLOPs of one call: QK^T over d (+ rank) and PV over d,
-        every pair of each window counted (masked pairs included)."""
+        every pair of each window counted (masked pairs included; on a padded
+        grid, the pairs of real query tokens with every position of their
+        window, as the method computes whole windows)."""
         per_pair = 2 * (self.d + self.rank) + 2 * self.d
         return float(self.tokens) * self.heads * self.N * per_pair
 
@@ -83,6 +85,11 @@ WORKLOADS = {
     "swin": Workload("swin", 64, 56, 56, 8, (4,), 3, 32, "bf16", "learned"),
     "dense": Workload("dense", 16, 128, 128, 32, (0, 16), 3, 32, "bf16", "standard"),
     "sr": Workload("sr", 4, 192, 192, 96, (0,), 6, 32, "bf16", None, rank=16),
+    # FlashSwin-T's stage 1 with its larger windows (FLASHSWIN page, section
+    # "무엇과 다른가": M = 16 and 32 at patch 4 on the 56 x 56 map, which is
+    # not a multiple of either, so the grid is padded to 64 x 64)
+    "flashswin_M16": Workload("flashswin_M16", 64, 56, 56, 16, (8,), 3, 32, "bf16", "learned"),
+    "flashswin_M32": Workload("flashswin_M32", 64, 56, 56, 32, (16,), 3, 32, "bf16", "learned"),
 }
 for _M in (8, 16, 32, 64, 96):
     for _d in (32, 64):
