@@ -103,6 +103,75 @@ int winattn_fwd(const void *q, const void *k, const void *v,
                 void *out, void *stream);
 
 /*
+ * winattn_fwd_lse — winattn_fwd that also saves, for the backward pass, the
+ * log-sum-exp of every row's scores: lse[b][y][x][h] = log sum_p' exp z(p, p')
+ * over the allowed keys p' of token (y, x) of image b, head h (natural log,
+ * fp32, device, [B][H_img][W_img][heads], 4-byte aligned, must not overlap
+ * q, k, v or out; written for every token, never at pad positions).  The
+ * backward recomputes P = exp(z - lse) from it instead of storing any N x N
+ * matrix ("FLASHSWIN" page, section "무엇과 다른가": memory was what kept
+ * windows small in training).  Same arguments, results and errors as
+ * winattn_fwd otherwise (lse NULL: WINATTN_ERR_ARG).  Adds 4 bytes per token
+ * and head of writes.
+ */
+int winattn_fwd_lse(const void *q, const void *k, const void *v,
+                    const float *theta, const void *bias_feats,
+                    int B, int H_img, int W_img, int M, int shift,
+                    int heads, int d, int rank, int dtype,
+                    void *out, float *lse, void *stream);
+
+/*
+ * winattn_bwd — the backward pass: gradients of a scalar loss L with respect
+ * to q, k, v, the RoPE frequencies theta and the bias features, given
+ * dout = dL/dO, the forward's output `out` and its saved log-sum-exp `lse`
+ * (winattn_fwd_lse).  The FLASHSWIN page trains with learned frequencies
+ * theta = exp(omega) (section "어떻게 동작하나"; dL/domega = theta dL/dtheta)
+ * and names training memory as what kept windows small (section "무엇과
+ * 다른가"): no N x N matrix is stored, P is recomputed per tile as
+ * exp(z - lse).  With dS = P o (dP - rowsum(dO o O)), dP = dO V^T:
+ *   dv = P^T dO;  d(Rq) = d^-1/2 dS (Rk);  d(Rk) = d^-1/2 dS^T (Rq);
+ *   dq = R(i, j)^T d(Rq), dk likewise;  du = dS w, dw = dS^T u;
+ *   dtheta_k = sum over tokens of i (g_{2k+1} x~_{2k} - g_{2k} x~_{2k+1})
+ *              + j (same over the second half) for x~ = Rq, g = d(Rq) and
+ *              for x~ = Rk, g = d(Rk).
+ *
+ *   q, k, v, theta, bias_feats, sizes, dtype
+ *               as for winattn_fwd (dtype must be WINATTN_BF16).
+ *   out, dout   device, bf16 maps like q: the forward's output and dL/dO.
+ *   lse         device, fp32 [B][H_img][W_img][heads], from winattn_fwd_lse
+ *               with the same inputs.
+ *   dq, dk, dv  device, bf16 maps like q; caller-allocated, written for every
+ *               token; must not overlap each other or any input map.
+ *   dtheta      device, fp32 [heads][d/4], or NULL to skip (must be NULL
+ *               when theta is); overwritten (zeroed, then summed into).
+ *   dbias       device, fp32 [heads][2][M*M][rank] (du at index 0, dw at 1),
+ *               or NULL to skip (NULL when bias_feats is); 16-byte aligned;
+ *               overwritten.
+ *   workspace   device, at least winattn_bwd_workspace_bytes(...) bytes,
+ *               16-byte aligned (NULL allowed when that is 0): fp32 sums of
+ *               dQ over the key tiles of windows larger than one 128-row
+ *               tile.  Caller-owned; its contents on entry do not matter.
+ *
+ * Stream-ordered and asynchronous; allocates nothing.  theta, dbias and the
+ * workspace gradients are summed with fp32 atomics, so their last bits may
+ * vary from run to run; dq, dk, dv of windows of at most 128 tokens are
+ * written directly and are bit-reproducible.  Errors as winattn_fwd
+ * (WINATTN_ERR_DTYPE for fp32, WINATTN_ERR_SIZE for a short workspace,
+ * WINATTN_ERR_ALIAS for overlapping gradients).
+ */
+int winattn_bwd(const void *q, const void *k, const void *v,
+                const float *theta, const void *bias_feats,
+                const void *out, const void *dout, const float *lse,
+                int B, int H_img, int W_img, int M, int shift,
+                int heads, int d, int rank, int dtype,
+                void *dq, void *dk, void *dv, float *dtheta, float *dbias,
+                void *workspace, size_t workspace_bytes, void *stream);
+
+/* Device workspace bytes winattn_bwd needs (0 when every window fits one
+ * 128-row tile, M * M <= 128), or 0 for invalid sizes. */
+size_t winattn_bwd_workspace_bytes(int B, int H_img, int W_img, int M, int heads, int d);
+
+/*
  * winattn_check_args — the host-side argument checks of winattn_fwd alone:
  * returns the code winattn_fwd would return before enqueuing anything
  * (WINATTN_OK if the arguments are acceptable).  Touches no device and makes

@@ -54,6 +54,8 @@ def _bind(lib):
     vp, i32, i64, f64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double
     lib.oracle_fwd.argtypes = [vp, vp, vp, i32, vp, vp] + [i32] * 8 + [vp, i32, f64]
     lib.oracle_fwd.restype = i32
+    lib.oracle_fwd_lse.argtypes = [vp, vp, vp, i32, vp, vp] + [i32] * 8 + [vp, vp, i32, f64]
+    lib.oracle_fwd_lse.restype = i32
     lib.oracle_fwd_units.argtypes = [vp, vp, vp, i32, vp, vp] + [i32] * 8 + [vp, i64, vp, i32, f64]
     lib.oracle_fwd_units.restype = i32
     lib.oracle_rope.argtypes = [vp, i32, f64, f64, vp, vp]
@@ -116,6 +118,19 @@ class Oracle:
         if rc < 0:
             raise ValueError(f"oracle rejected the problem (code {rc})")
         return out
+
+    def fwd_lse(self, q, k, v, *, M, shift=0, theta=None, bias=None, nthreads=0, mem_budget=8e9):
+        """(O [B, H, W, heads, d], lse [B, H, W, heads]) in fp64: lse is each
+        row's log-sum-exp of its masked scores (natural log)."""
+        q, k, v, theta, bias, code, (B, H, W, heads, d, rank) = self._prep(q, k, v, theta, bias, M)
+        out = np.zeros((B, H, W, heads, d), dtype=np.float64)
+        lse = np.zeros((B, H, W, heads), dtype=np.float64)
+        rc = self.lib.oracle_fwd_lse(_ptr(q), _ptr(k), _ptr(v), code, _ptr(theta), _ptr(bias),
+                                     B, H, W, M, shift, heads, d, rank, _ptr(out), _ptr(lse), nthreads,
+                                     float(mem_budget))
+        if rc < 0:
+            raise ValueError(f"oracle rejected the problem (code {rc})")
+        return out, lse
 
     def fwd_units(self, q, k, v, units, *, M, shift=0, theta=None, bias=None,
                   nthreads=0, mem_budget=8e9) -> np.ndarray:

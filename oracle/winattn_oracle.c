@@ -136,6 +136,7 @@ static int wrap_label(const problem_t *p, int yr, int xr)
 typedef struct {
     double *q, *k, *v, *s; /* N x d, N x d, N x d, N x N */
     int64_t *off;          /* N: element offset of each window token, -1 for padding */
+    double *lse;           /* N: log-sum-exp of each row's masked scores (natural log) */
 } scratch_t;
 
 /* Steps 3-8 for one (batch b, window (wy, wx), head h): O = softmax(S) V in
@@ -223,6 +224,7 @@ static void unit_forward(const problem_t *p, int b, int wy, int wx, int h,
         }
         for (int c = 0; c < N; ++c)
             row[c] /= sum;
+        w->lse[a] = mx + log(sum);
     }
 
     /* Step 8: O = P V. */
@@ -253,6 +255,7 @@ typedef struct {
     int64_t n_units;
     double *out_units;     /* [n_units][N][d] or NULL */
     double *out_map;       /* [B][H][W][heads][d] or NULL (step 9 scatter) */
+    double *lse_map;       /* [B][H][W][heads] or NULL: each row's log-sum-exp, scattered like O */
     int64_t next;          /* shared work counter */
     int failed;
 } job_t;
@@ -268,8 +271,9 @@ static void *worker(void *arg)
     w.v = malloc(N * d * sizeof(double));
     w.s = malloc(N * N * sizeof(double));
     w.off = malloc(N * sizeof(int64_t));
+    w.lse = malloc(N * sizeof(double));
     double *o = malloc(N * d * sizeof(double));
-    if (!w.q || !w.k || !w.v || !w.s || !w.off || !o) {
+    if (!w.q || !w.k || !w.v || !w.s || !w.off || !w.lse || !o) {
         __atomic_store_n(&job->failed, 1, __ATOMIC_RELAXED);
         goto done;
     }
@@ -288,8 +292,11 @@ static void *worker(void *arg)
             for (int i = 0; i < p->M; ++i)
                 for (int j = 0; j < p->M; ++j) {
                     int64_t off = rolled_token_offset(p, b, wy * p->M + i, wx * p->M + j, h);
-                    if (off >= 0)
+                    if (off >= 0) {
                         memcpy(job->out_map + off, dst + ((size_t)i * p->M + j) * d, d * sizeof(double));
+                        if (job->lse_map)
+                            job->lse_map[off / (int64_t)d] = w.lse[i * p->M + j];
+                    }
                 }
         }
     }
@@ -299,6 +306,7 @@ done:
     free(w.v);
     free(w.s);
     free(w.off);
+    free(w.lse);
     free(o);
     return NULL;
 }
@@ -321,7 +329,7 @@ static int check_problem(const problem_t *p)
 }
 
 static int run(const problem_t *p, const int64_t *units, int64_t n_units,
-               double *out_units, double *out_map, int nthreads, double mem_budget_bytes)
+               double *out_units, double *out_map, double *lse_map, int nthreads, double mem_budget_bytes)
 {
     if (check_problem(p))
         return -1;
@@ -341,7 +349,7 @@ static int run(const problem_t *p, const int64_t *units, int64_t n_units,
     if (nthreads > n_units)
         nthreads = (int)n_units;
 
-    job_t job = {p, units, n_units, out_units, out_map, 0, 0};
+    job_t job = {p, units, n_units, out_units, out_map, lse_map, 0, 0};
     pthread_t *th = malloc(sizeof(pthread_t) * (size_t)nthreads);
     if (!th)
         return -2;
@@ -372,7 +380,22 @@ int oracle_fwd(const void *q, const void *k, const void *v, int dtype,
     if (check_problem(&p) || !out_map)
         return -1;
     int64_t n = (int64_t)B * (p.Hp / M) * (p.Wp / M) * heads;
-    return run(&p, NULL, n, NULL, out_map, nthreads, mem_budget_bytes);
+    return run(&p, NULL, n, NULL, out_map, NULL, nthreads, mem_budget_bytes);
+}
+
+/* As oracle_fwd, and also each row's log-sum-exp (natural log of the sum of
+ * exp of its masked scores, z = d^-1/2 q.k + u.w) into lse_map
+ * [B][H][W][heads] fp64. */
+int oracle_fwd_lse(const void *q, const void *k, const void *v, int dtype,
+                   const float *theta, const void *bias,
+                   int B, int H, int W, int M, int shift, int heads, int d, int rank,
+                   double *out_map, double *lse_map, int nthreads, double mem_budget_bytes)
+{
+    problem_t p = make_problem(q, k, v, dtype, theta, bias, B, H, W, M, shift, heads, d, rank);
+    if (check_problem(&p) || !out_map || !lse_map)
+        return -1;
+    int64_t n = (int64_t)B * (p.Hp / M) * (p.Wp / M) * heads;
+    return run(&p, NULL, n, NULL, out_map, lse_map, nthreads, mem_budget_bytes);
 }
 
 /* Selected units; out_units [n_units][M*M][d] fp64 in window order p = i*M + j
@@ -390,7 +413,7 @@ int oracle_fwd_units(const void *q, const void *k, const void *v, int dtype,
     for (int64_t n = 0; n < n_units; ++n)
         if (units[n] < 0 || units[n] >= total)
             return -1;
-    return run(&p, units, n_units, out_units, NULL, nthreads, mem_budget_bytes);
+    return run(&p, units, n_units, out_units, NULL, NULL, nthreads, mem_budget_bytes);
 }
 
 /* The rotation alone, for the displacement-identity checks: out = R(i, j) vec. */
@@ -552,12 +575,13 @@ static void *bwd_worker(void *arg)
     w.v = malloc(N * d * sizeof(double));
     w.s = malloc(N * N * sizeof(double));
     w.off = malloc(N * sizeof(int64_t));
+    w.lse = malloc(N * sizeof(double));
     double *o = malloc(N * d * sizeof(double));
     double *g_o = malloc(N * d * sizeof(double)), *g_s = malloc(N * N * sizeof(double));
     double *g_q = malloc(N * d * sizeof(double)), *g_k = malloc(N * d * sizeof(double));
     double *dth = job->dtheta ? calloc(nth, sizeof(double)) : NULL;
     double *dbi = job->dbias ? calloc(nbias > 0 ? nbias : 1, sizeof(double)) : NULL;
-    if (!w.q || !w.k || !w.v || !w.s || !w.off || !o || !g_o || !g_s || !g_q || !g_k || (job->dtheta && !dth) ||
+    if (!w.q || !w.k || !w.v || !w.s || !w.off || !w.lse || !o || !g_o || !g_s || !g_q || !g_k || (job->dtheta && !dth) ||
         (job->dbias && !dbi)) {
         __atomic_store_n(&job->failed, 1, __ATOMIC_RELAXED);
         goto done;
@@ -587,6 +611,7 @@ done:
     free(w.v);
     free(w.s);
     free(w.off);
+    free(w.lse);
     free(o);
     free(g_o);
     free(g_s);

@@ -125,3 +125,32 @@ def sampled_compare(w: I.Workload, shift: int, images, heads=None, extra_windows
         ref = np.concatenate([r[k] for r, k in zip(ref, keep)])
         results.append(check(got, ref, w.dtype, f"{w.name} s{shift} image {b}"))
     return results
+
+
+# Tolerance of the saved log-sum-exp: it moves by at most the largest error of
+# the row's scores (log-sum-exp is 1-Lipschitz in the max norm), and the bf16
+# scores carry the rounding of the rotated q and k (2^-9 relative each), at
+# most about 2^-8 |q||k| d^-1/2 ~ 2e-2 for N(0, 1) inputs at d = 32.
+LSE_TOL = {"fp32": dict(max_abs=1e-4), "bf16": dict(max_abs=3e-2, mean_abs=3e-3)}
+
+
+def lse_compare(w: I.Workload, shift: int, device="cuda", base: int = 0):
+    """Whole-map parity of O and of the saved log-sum-exp (winattn_fwd_lse)."""
+    (qkv,), theta, bias = I.make_inputs(w, "cpu", base)
+    dq, dk, dv = (t.to(device) for t in qkv)
+    lse = torch.full((w.B, w.H, w.W, w.heads), float("nan"), device=device)
+    out = wa.window_attention(dq, dk, dv, w.M, shift, theta=None if theta is None else theta.to(device),
+                              bias_feats=None if bias is None else bias.to(device), lse=lse)
+    torch.cuda.synchronize()
+    assert wa.device_status() == 0, "a bounded wait timed out"
+    ref, ref_lse = orc().fwd_lse(*(I.to_storage_numpy(t) for t in qkv), M=w.M, shift=shift,
+                                 theta=None if theta is None else theta.numpy(), bias=I.to_storage_numpy(bias))
+    check(as_f64(out), ref, w.dtype, f"{w.name} s{shift} (with lse)")
+    got = lse.double().cpu().numpy()
+    assert np.all(np.isfinite(got)), f"{w.name}: lse not written everywhere"
+    err = np.abs(got - ref_lse)
+    tol = LSE_TOL[w.dtype]
+    assert err.max() <= tol["max_abs"], f"{w.name} s{shift}: lse max-abs {err.max():.3e}"
+    if "mean_abs" in tol:
+        assert err.mean() <= tol["mean_abs"], f"{w.name} s{shift}: lse mean-abs {err.mean():.3e}"
+    return float(err.max())

@@ -70,7 +70,7 @@ def rotate_complex(x: np.ndarray, ycoord: np.ndarray, xcoord: np.ndarray, theta_
     return out
 
 
-def brute_global(q, k, v, M, s, theta=None, bias=None):
+def brute_global(q, k, v, M, s, theta=None, bias=None, with_lse=False):
     """Masked global attention over all H*W tokens of each image and head.
 
     The map's grid is padded to Hp x Wp, the multiples of M at or above H and
@@ -90,6 +90,7 @@ def brute_global(q, k, v, M, s, theta=None, bias=None):
     allowed = (win[:, None] == win[None, :]) & (region[:, None] == region[None, :])
     plocal = ((yr % M) * M + (xr % M)).ravel()
     out = np.zeros_like(q)
+    lse = np.zeros(q.shape[:4])
     for b in range(B):
         for h in range(heads):
             Q = q[b, :, :, h, :].reshape(H * W, d)
@@ -103,11 +104,13 @@ def brute_global(q, k, v, M, s, theta=None, bias=None):
                 bf = storage_to_f64(bias)
                 S = S + bf[h, 0][plocal] @ bf[h, 1][plocal].T
             S = np.where(allowed, S, -np.inf)
-            S = S - S.max(axis=1, keepdims=True)
-            P = np.exp(S)
-            P /= P.sum(axis=1, keepdims=True)
+            mx = S.max(axis=1, keepdims=True)
+            P = np.exp(S - mx)
+            tot = P.sum(axis=1, keepdims=True)
+            P /= tot
             out[b, :, :, h, :] = (P @ V).reshape(H, W, d)
-    return out
+            lse[b, :, :, h] = (mx + np.log(tot)).reshape(H, W)
+    return (out, lse) if with_lse else out
 
 
 def _close(a, b, tol=TOL, what=""):
@@ -249,6 +252,35 @@ def pin_brute_global(o):
         _close(got, ref, 1e-10, f"brute-force global case {n}")
 
 
+def pin_lse(o):
+    """The log-sum-exp the forward saves for the backward: equal to the
+    brute-force global one (masked scores over all real tokens, padded and
+    shifted grids included), and log(n) for Q = 0 without bias, where all n
+    allowed scores of a row are zero."""
+    cases = [(1, 8, 12, 2, 8, 4, 2, "bf16", "learned", 0), (1, 7, 5, 2, 4, 3, 1, "fp32", None, 4),
+             (2, 6, 9, 1, 8, 4, 0, "fp32", "learned", 0)]
+    for n, (B, H, W, heads, d, M, s, dt, rope, r) in enumerate(cases):
+        q, k, v = _maps((B, H, W, heads, d), dt, f"pin-lse-{n}")
+        th = I.make_theta(heads, d, rope, 31 + n)
+        th = None if th is None else th.numpy()
+        bias = I.to_storage_numpy(I.make_bias_feats(heads, M, r, dt, 37 + n)) if r else None
+        out, lse = o.fwd_lse(q, k, v, M=M, shift=s, theta=th, bias=bias)
+        ref_out, ref_lse = brute_global(q, k, v, M, s, th, bias, with_lse=True)
+        _close(out, ref_out, 1e-10, f"lse case {n}: output")
+        _close(lse, ref_lse, 1e-10, f"lse case {n}: log-sum-exp")
+    # zero queries: lse = log(size of the row's allowed set)
+    B, H, W, heads, d, M, s = 1, 8, 12, 1, 4, 4, 1
+    _, k, v = _maps((B, H, W, heads, d), "fp32", "pin-lse-q0")
+    _, lse = o.fwd_lse(np.zeros_like(k), k, v, M=M, shift=s)
+    reg = swin_region_labels(H, W, M, s)
+    for y in range(H):
+        for x in range(W):
+            yr, xr = (y - s) % H, (x - s) % W
+            n_allowed = sum(1 for y2 in range((yr // M) * M, (yr // M) * M + M)
+                            for x2 in range((xr // M) * M, (xr // M) * M + M) if reg[y2, x2] == reg[yr, xr])
+            assert abs(lse[0, y, x, 0] - math.log(n_allowed)) < 1e-13, f"zero-Q lse at ({y},{x})"
+
+
 def pin_bias_concat(o):
     """[Qc, Qp][Kc, Kp]^T = Qc Kc^T + Qp Kp^T: a problem with rank-r bias
     factors equals a bias-free problem of head dim d + r whose query rows are
@@ -313,4 +345,5 @@ def pin_padding_closed_forms(o):
 
 
 ALL_PINS = [pin_rope_displacement, pin_theta_zero, pin_one_token_windows, pin_constant_v,
-            pin_zero_q_mean, pin_hand_worked, pin_brute_global, pin_bias_concat, pin_padding_closed_forms]
+            pin_zero_q_mean, pin_hand_worked, pin_brute_global, pin_bias_concat, pin_padding_closed_forms,
+            pin_lse]

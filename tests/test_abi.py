@@ -159,3 +159,14 @@ def test_kernel_switch_routes_to_fallbacks(lib):
     # the generic and fp32 kernels have no switch
     assert _lib.set_kernel_enabled(_lib.KERNEL_GENERIC, False) == _lib.ERR_ARG
     assert _lib.set_kernel_enabled(_lib.KERNEL_SIMT, False) == _lib.ERR_ARG
+
+
+def test_bwd_workspace_bytes(lib):
+    # windows of at most one 128-row tile need none; larger ones an fp32 map
+    assert _lib.bwd_workspace_bytes(64, 56, 56, 8, 3, 32) == 0
+    assert _lib.bwd_workspace_bytes(1, 20, 20, 10, 2, 32) == 0
+    n = 16 * 128 * 128 * 3 * 32 * 4
+    assert _lib.bwd_workspace_bytes(16, 128, 128, 32, 3, 32) == (n + 255) // 256 * 256
+    assert _lib.bwd_workspace_bytes(1, 56, 56, 32, 3, 64) == (56 * 56 * 3 * 64 * 4 + 255) // 256 * 256
+    assert _lib.bwd_workspace_bytes(0, 8, 8, 4, 1, 32) == 0
+    assert _lib.bwd_workspace_bytes(1, 8, 8, 4, 1, 48) == 0

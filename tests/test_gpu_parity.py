@@ -209,3 +209,23 @@ def test_fallback_kernels(off, name, shift, serves):
     finally:
         for k in off:
             _lib.set_kernel_enabled(k, True)
+
+
+LSE_CASES = [
+    # name, B, H, W, M, shift, heads, d, dtype, rope, rank   (kernel that serves it)
+    ("swin", 64, 56, 56, 8, 4, 3, 32, "bf16", "learned", 0),            # pipelined 8 x 8
+    ("m8_s0_d64_lse", 2, 16, 24, 8, 0, 2, 64, "bf16", "standard", 0),   # pipelined, d = 64
+    ("m4_s2_lse", 2, 8, 12, 4, 2, 2, 32, "bf16", "learned", 0),         # generic (small kernel has no lse)
+    ("m12_s6_r16_lse", 1, 24, 24, 12, 6, 2, 32, "bf16", "learned", 16), # generic, ragged tiles, factors
+    ("m32_s16_lse", 2, 64, 64, 32, 16, 2, 32, "bf16", "learned", 0),    # large-window
+    ("m16_s0_d64_r16_lse", 1, 32, 48, 16, 0, 2, 64, "bf16", "learned", 16),
+    ("m32_s16_pad56_lse", 1, 56, 56, 32, 16, 2, 32, "bf16", "learned", 0),  # large-window, padded
+    ("fp32_lse", 1, 16, 16, 8, 4, 2, 32, "fp32", "learned", 0),         # fp32
+]
+
+
+@pytest.mark.parametrize("case", LSE_CASES, ids=[c[0] for c in LSE_CASES])
+def test_forward_saves_lse(case):
+    name, B, H, W, M, s, heads, d, dt, rope, r = case
+    w = I.Workload(name, B, H, W, M, (s,), heads, d, dt, rope, r)
+    G.lse_compare(w, s)

@@ -44,6 +44,7 @@ MUTANTS = {
     # padding (maps that are not multiples of M)
     "pad_keys_attended": [("            if (w->off[c] < 0)\n                w->s[(size_t)a * N + c] = -INFINITY;",
                            "            if (0)\n                w->s[(size_t)a * N + c] = -INFINITY;")],
+    "lse_without_max": [("w->lse[a] = mx + log(sum);", "w->lse[a] = log(sum);")],
     "roll_over_unpadded_map": [
         ("int y = (yr + p->shift) % p->Hp;", "int y = (yr + p->shift) % p->H;"),
         ("int x = (xr + p->shift) % p->Wp;", "int x = (xr + p->shift) % p->W;"),

@@ -14,7 +14,8 @@ import torch
 from . import _lib
 from ._lib import WinattnError
 
-__all__ = ["window_attention", "window_attention_host", "WinattnError", "device_status"]
+__all__ = ["window_attention", "window_attention_host", "window_attention_backward", "WinattnError",
+           "device_status"]
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -50,10 +51,11 @@ def _shape(q, k, v, theta, bias, M):
 
 def window_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, M: int, shift: int = 0,
                      theta: Optional[torch.Tensor] = None, bias_feats: Optional[torch.Tensor] = None,
-                     out: Optional[torch.Tensor] = None) -> torch.Tensor:
+                     out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Fused window attention on CUDA tensors [B, H, W, heads, d] (bf16 or fp32),
     enqueued on torch's current stream.  See include/winattn.h for the exact
-    operation."""
+    operation.  With ``lse`` (fp32 [B, H, W, heads]) each row's log-sum-exp is
+    saved there for the backward (winattn_fwd_lse)."""
     B, H, W, heads, d, rank = _shape(q, k, v, theta, bias_feats, M)
     for t in (q, k, v, theta, bias_feats):
         if t is not None and not t.is_cuda:
@@ -62,17 +64,54 @@ def window_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, M: int, 
         out = torch.empty_like(q)
     dev = q.device
     stream = torch.cuda.current_stream(dev).cuda_stream
+    if lse is not None and (lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, W, heads) or not lse.is_cuda
+                            or not lse.is_contiguous()):
+        raise WinattnError(_lib.ERR_ARG, "lse must be a contiguous fp32 CUDA tensor [B, H, W, heads]")
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(theta), _ptr(bias_feats), B, H, W, M, shift, heads, d, rank,
-            _dtype_code(q), _ptr(out), stream)
+            _dtype_code(q), _ptr(out))
+    call, what = (_lib.fwd, "winattn_fwd") if lse is None else (_lib.fwd_lse, "winattn_fwd_lse")
+    args = args + ((stream,) if lse is None else (_ptr(lse), stream))
     # the library works on the current device: switch only when q lives elsewhere
     if torch.cuda.current_device() == dev.index:
-        rc = _lib.fwd(*args)
+        rc = call(*args)
     else:
         with torch.cuda.device(dev):
-            rc = _lib.fwd(*args)
+            rc = call(*args)
     if rc != _lib.OK:
-        raise WinattnError(rc, "winattn_fwd")
+        raise WinattnError(rc, what)
     return out
+
+
+def window_attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+                              dout: torch.Tensor, lse: torch.Tensor, M: int, shift: int = 0,
+                              theta: Optional[torch.Tensor] = None, bias_feats: Optional[torch.Tensor] = None,
+                              workspace: Optional[torch.Tensor] = None):
+    """Gradients (dq, dk, dv, dtheta, dbias) of a loss given dout = dL/dO, the
+    forward's ``out`` and its saved ``lse`` (``window_attention(..., lse=...)``);
+    bf16 CUDA tensors, enqueued on torch's current stream (winattn_bwd).
+    dtheta is fp32 [heads, d/4] (None without theta), dbias fp32
+    [heads, 2, M*M, rank] (None without bias features)."""
+    B, H, W, heads, d, rank = _shape(q, k, v, theta, bias_feats, M)
+    for t in (out, dout):
+        if t.shape != q.shape or t.dtype != q.dtype or not t.is_contiguous():
+            raise WinattnError(_lib.ERR_ARG, "out and dout must be contiguous and shaped like q")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, W, heads) or not lse.is_contiguous():
+        raise WinattnError(_lib.ERR_ARG, "lse must be a contiguous fp32 tensor [B, H, W, heads]")
+    dev = q.device
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    dtheta = None if theta is None else torch.empty((heads, d // 4), dtype=torch.float32, device=dev)
+    dbias = None if bias_feats is None else torch.empty(tuple(bias_feats.shape), dtype=torch.float32, device=dev)
+    need = _lib.bwd_workspace_bytes(B, H, W, M, heads, d)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    with torch.cuda.device(dev):
+        rc = _lib.bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(theta), _ptr(bias_feats), _ptr(out), _ptr(dout), _ptr(lse),
+                      B, H, W, M, shift, heads, d, rank, _dtype_code(q), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dtheta),
+                      _ptr(dbias), _ptr(workspace), 0 if workspace is None else workspace.numel(), stream)
+    if rc != _lib.OK:
+        raise WinattnError(rc, "winattn_bwd")
+    return dq, dk, dv, dtheta, dbias
 
 
 def window_attention_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, M: int, shift: int = 0,

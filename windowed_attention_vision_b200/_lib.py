@@ -17,9 +17,10 @@ ERR_ARG, ERR_RANK, ERR_ALIGN, ERR_DTYPE, ERR_ARCH = -1, -2, -3, -4, -5
 ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_ALIAS, ERR_SIZE = -6, -7, -8, -9
 BF16, FP32 = 0, 1
 
-EXPORTS = ("winattn_fwd", "winattn_check_args", "winattn_fwd_host", "winattn_host_workspace_bytes",
+EXPORTS = ("winattn_fwd", "winattn_fwd_lse", "winattn_check_args", "winattn_fwd_host", "winattn_host_workspace_bytes",
            "winattn_strerror", "winattn_last_device_status", "winattn_launch_info", "winattn_fwd_host_static",
-           "winattn_selftest_wait_timeout", "winattn_set_kernel_enabled")
+           "winattn_selftest_wait_timeout", "winattn_set_kernel_enabled", "winattn_bwd",
+           "winattn_bwd_workspace_bytes")
 STATIC_WORKSPACE_BYTES = 32 << 20
 
 
@@ -44,6 +45,8 @@ def load(path: str = LIB_PATH):
     vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
     lib.winattn_fwd.argtypes = [vp, vp, vp, vp, vp] + [i32] * 9 + [vp, vp]
     lib.winattn_fwd.restype = i32
+    lib.winattn_fwd_lse.argtypes = [vp, vp, vp, vp, vp] + [i32] * 9 + [vp, vp, vp]
+    lib.winattn_fwd_lse.restype = i32
     lib.winattn_check_args.argtypes = [vp, vp, vp, vp, vp] + [i32] * 9 + [vp]
     lib.winattn_check_args.restype = i32
     lib.winattn_fwd_host.argtypes = [vp, vp, vp, vp, vp] + [i32] * 9 + [vp, vp, sz, vp]
@@ -60,6 +63,10 @@ def load(path: str = LIB_PATH):
     lib.winattn_launch_info.restype = i32
     lib.winattn_selftest_wait_timeout.argtypes = [vp]
     lib.winattn_selftest_wait_timeout.restype = i32
+    lib.winattn_bwd.argtypes = [vp] * 8 + [i32] * 9 + [vp] * 6 + [sz, vp]
+    lib.winattn_bwd.restype = i32
+    lib.winattn_bwd_workspace_bytes.argtypes = [i32] * 6
+    lib.winattn_bwd_workspace_bytes.restype = sz
     lib.winattn_set_kernel_enabled.argtypes = [i32, i32]
     lib.winattn_set_kernel_enabled.restype = i32
     _lib = lib
@@ -74,6 +81,23 @@ def fwd(q_ptr, k_ptr, v_ptr, theta_ptr, bias_ptr, B, H, W, M, shift, heads, d, r
         stream) -> int:
     return load().winattn_fwd(q_ptr, k_ptr, v_ptr, theta_ptr, bias_ptr, B, H, W, M, shift, heads, d, rank,
                               dtype, out_ptr, stream)
+
+
+def fwd_lse(q_ptr, k_ptr, v_ptr, theta_ptr, bias_ptr, B, H, W, M, shift, heads, d, rank, dtype, out_ptr, lse_ptr,
+            stream) -> int:
+    return load().winattn_fwd_lse(q_ptr, k_ptr, v_ptr, theta_ptr, bias_ptr, B, H, W, M, shift, heads, d, rank,
+                                  dtype, out_ptr, lse_ptr, stream)
+
+
+def bwd(q_ptr, k_ptr, v_ptr, theta_ptr, bias_ptr, out_ptr, dout_ptr, lse_ptr, B, H, W, M, shift, heads, d, rank,
+        dtype, dq_ptr, dk_ptr, dv_ptr, dtheta_ptr, dbias_ptr, ws_ptr, ws_bytes, stream) -> int:
+    return load().winattn_bwd(q_ptr, k_ptr, v_ptr, theta_ptr, bias_ptr, out_ptr, dout_ptr, lse_ptr, B, H, W, M, shift,
+                              heads, d, rank, dtype, dq_ptr, dk_ptr, dv_ptr, dtheta_ptr, dbias_ptr, ws_ptr, ws_bytes,
+                              stream)
+
+
+def bwd_workspace_bytes(B, H, W, M, heads, d) -> int:
+    return load().winattn_bwd_workspace_bytes(B, H, W, M, heads, d)
 
 
 def check_args(q_ptr, k_ptr, v_ptr, theta_ptr, bias_ptr, B, H, W, M, shift, heads, d, rank, dtype,

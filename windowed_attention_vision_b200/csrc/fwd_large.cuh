@@ -265,7 +265,8 @@ template <int D, int R, int BN, bool PAD>
 __global__ void __launch_bounds__(kLargeThreads, 1)
     winattn_fwd_large_kernel(const __nv_bfloat16 *__restrict__ q, const float *__restrict__ theta,
                              const __nv_bfloat16 *__restrict__ bias, __nv_bfloat16 *__restrict__ out,
-                             const Geometry g, const float scale, const __grid_constant__ LargeMaps maps)
+                             float *__restrict__ lse, const Geometry g, const float scale,
+                             const __grid_constant__ LargeMaps maps)
 {
     using L = LargeLayout<D, R, BN>;
     constexpr int NS = L::NS;
@@ -801,6 +802,9 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
             }
             if (failed)
                 break;
+            // log-sum-exp of the row's scores in natural units (m is in log2 units)
+            if (lse && !me.pad)
+                lse[me.offset / D] = (m + log2f(l)) * kLn2;
             if constexpr (NOB == 2) {
                 pend_kk = kk;
                 pend_off = me.pad ? -1 : me.offset;

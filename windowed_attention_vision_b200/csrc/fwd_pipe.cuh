@@ -89,7 +89,8 @@ struct PipeLayout {
     static constexpr int NO = D == 32 ? 2 : 1;
     static constexpr uint32_t OSTAGE = (MRING + NM * MSLOT + 1023) & ~1023u;
     static constexpr uint32_t OSUM = OSTAGE + NO * 256 * D;         // per TMEM buffer: row sum l, f32[4][128]
-    static constexpr uint32_t IJTAB = OSUM + kPipeBufs * 128 * 4;   // box row order: (i << 8 | j) u16[4][64]
+    static constexpr uint32_t OMAX = OSUM + kPipeBufs * 128 * 4;    // per TMEM buffer: row max (log2 units)
+    static constexpr uint32_t IJTAB = OMAX + kPipeBufs * 128 * 4;   // box row order: (i << 8 | j) u16[4][64]
     static constexpr uint32_t TABLE = IJTAB + 512;                  // RoPE (cos, sin) float4 [heads][8][D/8]
     static constexpr int kBars = 3 * NSQ + 2 * NSV + NM + 4 * kPipeBufs + 2;
     static __host__ __device__ uint32_t bars(int heads) { return TABLE + ((heads * 8 * (D / 4) * 8 + 15) & ~15u); }
@@ -105,7 +106,8 @@ __host__ __device__ inline bool pipe_ok(const Geometry &g)
 
 template <int D>
 __global__ void __launch_bounds__(kPipeThreads, 1)
-    winattn_fwd_pipe_kernel(const float *__restrict__ theta, __nv_bfloat16 *__restrict__ out, const Geometry g,
+    winattn_fwd_pipe_kernel(const float *__restrict__ theta, __nv_bfloat16 *__restrict__ out,
+                            float *__restrict__ lse, const Geometry g,
                             const float scale, const __grid_constant__ WindowMaps tm_q,
                             const __grid_constant__ WindowMaps tm_k, const __grid_constant__ WindowMaps tm_v,
                             const __grid_constant__ WindowMaps tm_o)
@@ -128,6 +130,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     uint16_t *ijtab = reinterpret_cast<uint16_t *>(base + L::IJTAB);
     float2 *table = reinterpret_cast<float2 *>(base + L::TABLE);
     float *osum = reinterpret_cast<float *>(base + L::OSUM);
+    float *omax = reinterpret_cast<float *>(base + L::OMAX);
     uint64_t *bars = reinterpret_cast<uint64_t *>(base + L::bars(g.heads));
     uint64_t *qk_full = bars, *ready = qk_full + NSQ, *qk_empty = ready + NSQ;
     uint64_t *v_full = qk_empty + NSQ, *v_empty = v_full + NSV, *meta_full = v_empty + NSV;
@@ -504,6 +507,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
             tmem_st16(tmem + lane_base + b * 128 + (1 - slot) * 32 + 16, zero);
             const float2 l2 = __fadd2_rn(lq[0], lq[1]);
             osum[b * 128 + row] = l2.x + l2.y;
+            omax[b * 128 + row] = -mneg;
             tmem_wait_st();
             tc_fence_before_sync();
             warp_arrive(&p_full[b]);
@@ -531,8 +535,27 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
             // after S of tile kk + 4, which needs this buffer back
             const int4 rec = lane < 2 ? reinterpret_cast<const int4 *>(base + L::MRING + m * L::MSLOT + 1024)[quarter * 2 + lane]
                                       : make_int4(0, 0, 0, -1);
-            const float inv = 1.f / osum[b * 128 + row];
+            const float lrow = osum[b * 128 + row];
+            const float inv = 1.f / lrow;
             const float2 i2 = make_float2(inv, inv);
+            if (lse) {
+                // the row's token from the warp's store record(s): the rows of
+                // a record's box in row-major order (box widths: 8 tokens for
+                // a half window of rows, 4 for a half of columns or a quadrant)
+                const int4 r0 = make_int4(__shfl_sync(~0u, rec.x, 0), __shfl_sync(~0u, rec.y, 0),
+                                          __shfl_sync(~0u, rec.z, 0), __shfl_sync(~0u, rec.w, 0));
+                const int4 r1 = make_int4(__shfl_sync(~0u, rec.x, 1), __shfl_sync(~0u, rec.y, 1),
+                                          __shfl_sync(~0u, rec.z, 1), __shfl_sync(~0u, rec.w, 1));
+                const bool quad = r0.w >= 0 && (r0.w & 3) == 3;
+                const int4 rr = quad && lane >= 16 ? r1 : r0;
+                const int ll = quad ? (lane & 15) : lane;
+                const int bw = (rr.w & 3) == 2 ? 8 : 4;
+                if (rr.w >= 0) {
+                    const int y = rr.y + ll / bw, x = rr.x + ll % bw, h = (rr.w >> 4) / D;
+                    lse[(((int64_t)rr.z * g.H + y) * g.W + x) * g.heads + h] =
+                        (omax[b * 128 + row] + log2f(lrow)) * kLn2;
+                }
+            }
             uint4 y[D / 8];
             // the buffer goes back to the S issuer as soon as O is in registers
 #pragma unroll

@@ -43,8 +43,8 @@ template <int D, int R>
 __global__ void __launch_bounds__(128)
     winattn_fwd_simt_kernel(const float *__restrict__ q, const float *__restrict__ k,
                             const float *__restrict__ v, const float *__restrict__ theta,
-                            const float *__restrict__ bias, float *__restrict__ out, const Geometry g,
-                            const float scale)
+                            const float *__restrict__ bias, float *__restrict__ out, float *__restrict__ lse,
+                            const Geometry g, const float scale)
 {
     using L = SimtLayout<D, R>;
     extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -152,6 +152,8 @@ __global__ void __launch_bounds__(128)
     }
     if (qreal) {
         const float inv = 1.f / l;
+        if (lse)
+            lse[qt.offset / D] = m + logf(l);
 #pragma unroll
         for (int e = 0; e < D; ++e)
             out[qt.offset + e] = o[e] * inv;

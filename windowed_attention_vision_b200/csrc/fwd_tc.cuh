@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(128, 1)
     winattn_fwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                           const __nv_bfloat16 *__restrict__ v, const float *__restrict__ theta,
                           const __nv_bfloat16 *__restrict__ bias, __nv_bfloat16 *__restrict__ out,
-                          const Geometry g, const float scale)
+                          float *__restrict__ lse, const Geometry g, const float scale)
 {
     using L = TcLayout<D, R>;
     extern __shared__ uint8_t smem_raw[];
@@ -296,6 +296,9 @@ __global__ void __launch_bounds__(128, 1)
     if (ok && qreal) {
         const TokenRef &tk = qtk;
         const float inv = 1.f / l;
+        // log-sum-exp of the row's scores in natural units (m is in log2 units)
+        if (lse)
+            lse[tk.offset / D] = (m + log2f(l)) * kLn2;
         uint4 *dst = reinterpret_cast<uint4 *>(out + tk.offset);
 #pragma unroll
         for (int c = 0; c < D / 8; ++c) {

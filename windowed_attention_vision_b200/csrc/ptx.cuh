@@ -14,6 +14,7 @@ namespace winattn {
 __device__ unsigned int g_status_word = 0;
 
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {

@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "../../include/winattn.h"
+#include "bwd_tc.cuh"
 #include "fwd_large.cuh"
 #include "fwd_pipe.cuh"
 #include "fwd_simt.cuh"
@@ -218,7 +219,7 @@ uint32_t small_smem(const Geometry &g)
 // Which kernel serves a problem: windows of <= 128 tokens go to the
 // persistent small-window kernel when its RoPE table and ring fit in shared
 // memory; fp32 goes to the SIMT kernel; everything else to the generic one.
-KernelKind choose_kernel(const Geometry &g, int dtype)
+KernelKind choose_kernel(const Geometry &g, int dtype, bool want_lse = false)
 {
     if (dtype == WINATTN_FP32)
         return kSimt;
@@ -230,8 +231,9 @@ KernelKind choose_kernel(const Geometry &g, int dtype)
     if (kernel_enabled(kPipe) && pipe_ok(g) && (uint64_t)g.heads * g.M * (g.d / 4) * 8 <= kSmallTableMax &&
         pipe_smem(g) <= kMaxSmem)
         return kPipe;
-    if (kernel_enabled(kSmall) && g.N <= kTileRows && (uint64_t)g.heads * g.M * (g.d / 4) * 8 <= kSmallTableMax &&
-        small_smem(g) <= kMaxSmem)
+    // (the small-window kernel does not write the log-sum-exp)
+    if (!want_lse && kernel_enabled(kSmall) && g.N <= kTileRows &&
+        (uint64_t)g.heads * g.M * (g.d / 4) * 8 <= kSmallTableMax && small_smem(g) <= kMaxSmem)
         return kSmall;
     if (kernel_enabled(kLarge) && large_ok(g))
         return kLarge;
@@ -287,12 +289,12 @@ int launch(int smem, const Geometry &g, cudaStream_t stream, auto... args)
 
 template <int D, int R>
 int launch_tc(const void *q, const void *k, const void *v, const float *theta, const void *bias, void *out,
-              const Geometry &g, cudaStream_t stream)
+              float *lse, const Geometry &g, cudaStream_t stream)
 {
     using T = __nv_bfloat16;
     return launch<winattn_fwd_tc_kernel<D, R>>((int)TcLayout<D, R>::bytes(g.M), g, stream,
                   static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), theta,
-                  static_cast<const T *>(bias), static_cast<T *>(out));
+                  static_cast<const T *>(bias), static_cast<T *>(out), lse);
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no
@@ -413,13 +415,13 @@ bool large_regs_ok()
 
 template <int D, int R, int BN, bool PAD>
 int launch_large(const void *q, const void *k, const void *v, const float *theta, const void *bias, void *out,
-                 const Geometry &g, cudaStream_t stream)
+                 float *lse, const Geometry &g, cudaStream_t stream)
 {
     using T = __nv_bfloat16;
     // a build whose register count differs would wait forever in setmaxnreg:
     // its problems go to the generic tensor-core kernel instead
     if (!large_regs_ok<D, R, BN, PAD>())
-        return launch_tc<D, R>(q, k, v, theta, bias, out, g, stream);
+        return launch_tc<D, R>(q, k, v, theta, bias, out, lse, g, stream);
     MapSet ms;
     const MapKey key = make_key(kLarge, g, k, v, bias, nullptr, nullptr);
     const bool ok = cached_maps(key, &ms, [&](MapSet *m) {
@@ -445,20 +447,20 @@ int launch_large(const void *q, const void *k, const void *v, const float *theta
     const int64_t items = g.wph * g.heads * (g.N / 256);
     const int64_t grid = items < sm_count() ? items : sm_count();
     kernel<<<(unsigned)grid, kLargeThreads, smem, stream>>>(static_cast<const T *>(q), theta,
-                                                           static_cast<const T *>(bias), static_cast<T *>(out), g,
-                                                           1.0f / std::sqrt((float)g.d), maps);
+                                                           static_cast<const T *>(bias), static_cast<T *>(out), lse,
+                                                           g, 1.0f / std::sqrt((float)g.d), maps);
     return cudaGetLastError() == cudaSuccess ? WINATTN_OK : WINATTN_ERR_CUDA;
 }
 
 template <int D, int R>
 int launch_large_bn(const void *q, const void *k, const void *v, const float *theta, const void *bias, void *out,
-                    const Geometry &g, cudaStream_t s)
+                    float *lse, const Geometry &g, cudaStream_t s)
 {
     if (large_tile_keys(g.M) == 96)
-        return g.padded ? launch_large<D, R, 96, true>(q, k, v, theta, bias, out, g, s)
-                        : launch_large<D, R, 96, false>(q, k, v, theta, bias, out, g, s);
-    return g.padded ? launch_large<D, R, 128, true>(q, k, v, theta, bias, out, g, s)
-                    : launch_large<D, R, 128, false>(q, k, v, theta, bias, out, g, s);
+        return g.padded ? launch_large<D, R, 96, true>(q, k, v, theta, bias, out, lse, g, s)
+                        : launch_large<D, R, 96, false>(q, k, v, theta, bias, out, lse, g, s);
+    return g.padded ? launch_large<D, R, 128, true>(q, k, v, theta, bias, out, lse, g, s)
+                    : launch_large<D, R, 128, false>(q, k, v, theta, bias, out, lse, g, s);
 }
 
 template <int D, int R, bool TMA>
@@ -506,8 +508,8 @@ int launch_small(const void *q, const void *k, const void *v, const float *theta
 }
 
 template <int D>
-int launch_pipe(const void *q, const void *k, const void *v, const float *theta, void *out, const Geometry &g,
-                cudaStream_t stream)
+int launch_pipe(const void *q, const void *k, const void *v, const float *theta, void *out, float *lse,
+                const Geometry &g, cudaStream_t stream)
 {
     static_assert(sizeof(WindowMaps) == 4 * sizeof(CUtensorMap), "WindowMaps is four maps");
     MapSet ms;
@@ -539,7 +541,7 @@ int launch_pipe(const void *q, const void *k, const void *v, const float *theta,
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const float scale = 1.0f / std::sqrt((float)g.d);
-    if (cudaLaunchKernelEx(&cfg, kernel, theta, static_cast<__nv_bfloat16 *>(out), g, scale, maps[0], maps[1],
+    if (cudaLaunchKernelEx(&cfg, kernel, theta, static_cast<__nv_bfloat16 *>(out), lse, g, scale, maps[0], maps[1],
                            maps[2], maps[3]) != cudaSuccess)
         return WINATTN_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? WINATTN_OK : WINATTN_ERR_CUDA;
@@ -547,19 +549,20 @@ int launch_pipe(const void *q, const void *k, const void *v, const float *theta,
 
 template <int D, int R>
 int launch_simt(const void *q, const void *k, const void *v, const float *theta, const void *bias, void *out,
-                const Geometry &g, cudaStream_t stream)
+                float *lse, const Geometry &g, cudaStream_t stream)
 {
     return launch<winattn_fwd_simt_kernel<D, R>>((int)SimtLayout<D, R>::bytes(g.M), g, stream,
                   static_cast<const float *>(q), static_cast<const float *>(k), static_cast<const float *>(v),
-                  theta, static_cast<const float *>(bias), static_cast<float *>(out));
+                  theta, static_cast<const float *>(bias), static_cast<float *>(out), lse);
 }
 
 int dispatch(const void *q, const void *k, const void *v, const float *theta, const void *bias, void *out,
-             const Geometry &g, int dtype, cudaStream_t s)
+             const Geometry &g, int dtype, cudaStream_t s, float *lse = nullptr)
 {
-    const KernelKind kind = choose_kernel(g, dtype);
+    const KernelKind kind = choose_kernel(g, dtype, lse != nullptr);
     if (kind == kPipe)
-        return g.d == 32 ? launch_pipe<32>(q, k, v, theta, out, g, s) : launch_pipe<64>(q, k, v, theta, out, g, s);
+        return g.d == 32 ? launch_pipe<32>(q, k, v, theta, out, lse, g, s)
+                         : launch_pipe<64>(q, k, v, theta, out, lse, g, s);
     if (kind == kSmall) {
         switch (g.d * 100 + g.rank) {
         case 3200: return launch_small<32, 0>(q, k, v, theta, bias, out, g, s);
@@ -571,33 +574,33 @@ int dispatch(const void *q, const void *k, const void *v, const float *theta, co
         }
     } else if (kind == kLarge) {
         switch (g.d * 100 + g.rank) {
-        case 3200: return launch_large_bn<32, 0>(q, k, v, theta, bias, out, g, s);
-        case 3216: return launch_large_bn<32, 16>(q, k, v, theta, bias, out, g, s);
-        case 3232: return launch_large_bn<32, 32>(q, k, v, theta, bias, out, g, s);
-        case 6400: return launch_large_bn<64, 0>(q, k, v, theta, bias, out, g, s);
-        case 6416: return launch_large_bn<64, 16>(q, k, v, theta, bias, out, g, s);
-        case 6432: return launch_large_bn<64, 32>(q, k, v, theta, bias, out, g, s);
+        case 3200: return launch_large_bn<32, 0>(q, k, v, theta, bias, out, lse, g, s);
+        case 3216: return launch_large_bn<32, 16>(q, k, v, theta, bias, out, lse, g, s);
+        case 3232: return launch_large_bn<32, 32>(q, k, v, theta, bias, out, lse, g, s);
+        case 6400: return launch_large_bn<64, 0>(q, k, v, theta, bias, out, lse, g, s);
+        case 6416: return launch_large_bn<64, 16>(q, k, v, theta, bias, out, lse, g, s);
+        case 6432: return launch_large_bn<64, 32>(q, k, v, theta, bias, out, lse, g, s);
         }
     } else if (kind == kGeneric) {
         switch (g.d * 100 + g.rank) {
-        case 3200: return launch_tc<32, 0>(q, k, v, theta, bias, out, g, s);
-        case 3216: return launch_tc<32, 16>(q, k, v, theta, bias, out, g, s);
-        case 3232: return launch_tc<32, 32>(q, k, v, theta, bias, out, g, s);
-        case 6400: return launch_tc<64, 0>(q, k, v, theta, bias, out, g, s);
-        case 6416: return launch_tc<64, 16>(q, k, v, theta, bias, out, g, s);
-        case 6432: return launch_tc<64, 32>(q, k, v, theta, bias, out, g, s);
+        case 3200: return launch_tc<32, 0>(q, k, v, theta, bias, out, lse, g, s);
+        case 3216: return launch_tc<32, 16>(q, k, v, theta, bias, out, lse, g, s);
+        case 3232: return launch_tc<32, 32>(q, k, v, theta, bias, out, lse, g, s);
+        case 6400: return launch_tc<64, 0>(q, k, v, theta, bias, out, lse, g, s);
+        case 6416: return launch_tc<64, 16>(q, k, v, theta, bias, out, lse, g, s);
+        case 6432: return launch_tc<64, 32>(q, k, v, theta, bias, out, lse, g, s);
         }
     } else {
         switch (g.d * 100 + g.rank) {
-        case 1600: return launch_simt<16, 0>(q, k, v, theta, bias, out, g, s);
-        case 1616: return launch_simt<16, 16>(q, k, v, theta, bias, out, g, s);
-        case 1632: return launch_simt<16, 32>(q, k, v, theta, bias, out, g, s);
-        case 3200: return launch_simt<32, 0>(q, k, v, theta, bias, out, g, s);
-        case 3216: return launch_simt<32, 16>(q, k, v, theta, bias, out, g, s);
-        case 3232: return launch_simt<32, 32>(q, k, v, theta, bias, out, g, s);
-        case 6400: return launch_simt<64, 0>(q, k, v, theta, bias, out, g, s);
-        case 6416: return launch_simt<64, 16>(q, k, v, theta, bias, out, g, s);
-        case 6432: return launch_simt<64, 32>(q, k, v, theta, bias, out, g, s);
+        case 1600: return launch_simt<16, 0>(q, k, v, theta, bias, out, lse, g, s);
+        case 1616: return launch_simt<16, 16>(q, k, v, theta, bias, out, lse, g, s);
+        case 1632: return launch_simt<16, 32>(q, k, v, theta, bias, out, lse, g, s);
+        case 3200: return launch_simt<32, 0>(q, k, v, theta, bias, out, lse, g, s);
+        case 3216: return launch_simt<32, 16>(q, k, v, theta, bias, out, lse, g, s);
+        case 3232: return launch_simt<32, 32>(q, k, v, theta, bias, out, lse, g, s);
+        case 6400: return launch_simt<64, 0>(q, k, v, theta, bias, out, lse, g, s);
+        case 6416: return launch_simt<64, 16>(q, k, v, theta, bias, out, lse, g, s);
+        case 6432: return launch_simt<64, 32>(q, k, v, theta, bias, out, lse, g, s);
         }
     }
     return WINATTN_ERR_ARG;
@@ -635,6 +638,56 @@ HostLanes *host_lanes()
         per_dev[dev] = h;
     }
     return per_dev[dev];
+}
+
+// ------------------------------------------------------------------ backward
+
+struct BwdArgs {
+    const void *q, *k, *v;
+    const float *theta;
+    const void *bias, *out, *dout;
+    const float *lse;
+    void *dq, *dk, *dv;
+    float *dtheta, *dbias, *dq_acc;
+};
+
+template <int D, int R>
+int launch_bwd(const BwdArgs &a, const Geometry &g, cudaStream_t s)
+{
+    using T = __nv_bfloat16;
+    const int smem = (int)BwdLayout<D, R>::bytes(g.M);
+    if (!smem_attr_once<winattn_bwd_tc_kernel<D, R>>())
+        return WINATTN_ERR_CUDA;
+    const float scale = 1.0f / std::sqrt((float)g.d);
+    winattn_bwd_tc_kernel<D, R><<<(unsigned)g.items, 128, smem, s>>>(
+        static_cast<const T *>(a.q), static_cast<const T *>(a.k), static_cast<const T *>(a.v), a.theta,
+        static_cast<const T *>(a.bias), static_cast<const T *>(a.out), static_cast<const T *>(a.dout), a.lse,
+        static_cast<T *>(a.dq), static_cast<T *>(a.dk), static_cast<T *>(a.dv), a.dtheta, a.dbias, a.dq_acc, g,
+        scale);
+    if (cudaGetLastError() != cudaSuccess)
+        return WINATTN_ERR_CUDA;
+    if (g.n_tiles > 1) {
+        const int64_t T_tok = (int64_t)g.B * g.H * g.W;
+        const dim3 grid((unsigned)((T_tok + 127) / 128), (unsigned)g.heads);
+        winattn_bwd_finalize_kernel<D><<<grid, 128, 0, s>>>(static_cast<const T *>(a.q), a.theta, a.dq_acc,
+                                                            static_cast<T *>(a.dq), a.dtheta, g, scale);
+        if (cudaGetLastError() != cudaSuccess)
+            return WINATTN_ERR_CUDA;
+    }
+    return WINATTN_OK;
+}
+
+int dispatch_bwd(const BwdArgs &a, const Geometry &g, cudaStream_t s)
+{
+    switch (g.d * 100 + g.rank) {
+    case 3200: return launch_bwd<32, 0>(a, g, s);
+    case 3216: return launch_bwd<32, 16>(a, g, s);
+    case 3232: return launch_bwd<32, 32>(a, g, s);
+    case 6400: return launch_bwd<64, 0>(a, g, s);
+    case 6416: return launch_bwd<64, 16>(a, g, s);
+    case 6432: return launch_bwd<64, 32>(a, g, s);
+    }
+    return WINATTN_ERR_ARG;
 }
 
 }  // namespace
@@ -676,6 +729,87 @@ int winattn_fwd(const void *q, const void *k, const void *v, const float *theta,
         return rc;
     const Geometry g = Geometry::make(B, H_img, W_img, M, shift, heads, d, rank);
     return dispatch(q, k, v, theta, bias_feats, out, g, dtype, static_cast<cudaStream_t>(stream));
+}
+
+size_t winattn_bwd_workspace_bytes(int B, int H_img, int W_img, int M, int heads, int d)
+{
+    if (B <= 0 || H_img <= 0 || W_img <= 0 || M <= 0 || M > kMaxM || heads <= 0 || (d != 32 && d != 64))
+        return 0;
+    // windows of more than one 128-row tile sum dQ over their key tiles in fp32
+    if ((int64_t)M * M <= kTileRows)
+        return 0;
+    return ((size_t)B * H_img * W_img * heads * d * 4 + 255) & ~size_t(255);
+}
+
+int winattn_bwd(const void *q, const void *k, const void *v, const float *theta, const void *bias_feats,
+                const void *out, const void *dout, const float *lse, int B, int H_img, int W_img, int M, int shift,
+                int heads, int d, int rank, int dtype, void *dq, void *dk, void *dv, float *dtheta, float *dbias,
+                void *workspace, size_t workspace_bytes, void *stream)
+{
+    int rc = check_sizes(B, H_img, W_img, M, shift, heads, d, rank, dtype);
+    if (rc != WINATTN_OK)
+        return rc;
+    if (dtype != WINATTN_BF16)
+        return WINATTN_ERR_DTYPE;
+    if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv)
+        return WINATTN_ERR_ARG;
+    if ((rank > 0) != (bias_feats != nullptr))
+        return WINATTN_ERR_RANK;
+    if ((dtheta && !theta) || (dbias && !bias_feats))
+        return WINATTN_ERR_ARG;
+    const void *maps[8] = {q, k, v, out, dout, dq, dk, dv};
+    for (const void *p : maps)
+        if (!aligned16(p))
+            return WINATTN_ERR_ALIGN;
+    if ((bias_feats && !aligned16(bias_feats)) || (dbias && !aligned16(dbias)) ||
+        (reinterpret_cast<uintptr_t>(theta) & 3u) || (reinterpret_cast<uintptr_t>(lse) & 3u) ||
+        (reinterpret_cast<uintptr_t>(dtheta) & 3u))
+        return WINATTN_ERR_ALIGN;
+    const size_t n = map_bytes(B, H_img, W_img, heads, d, dtype);
+    // the three gradients must not overlap one another or any input map
+    for (int o = 5; o < 8; ++o)
+        for (int i = 0; i < 8; ++i)
+            if (i != o && overlaps(maps[o], n, maps[i], n))
+                return WINATTN_ERR_ALIAS;
+    const size_t need = winattn_bwd_workspace_bytes(B, H_img, W_img, M, heads, d);
+    if (need && (!workspace || workspace_bytes < need))
+        return WINATTN_ERR_SIZE;
+    if (need && !aligned16(workspace))
+        return WINATTN_ERR_ALIGN;
+    rc = check_device();
+    if (rc != WINATTN_OK)
+        return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const Geometry g = Geometry::make(B, H_img, W_img, M, shift, heads, d, rank);
+    // the theta and bias-table gradients and the dQ sums are accumulated
+    if ((dtheta && cudaMemsetAsync(dtheta, 0, (size_t)heads * (d / 4) * 4, s) != cudaSuccess) ||
+        (dbias && cudaMemsetAsync(dbias, 0, (size_t)heads * 2 * g.N * rank * 4, s) != cudaSuccess) ||
+        (need && cudaMemsetAsync(workspace, 0, need, s) != cudaSuccess))
+        return WINATTN_ERR_CUDA;
+    BwdArgs a{q, k, v, theta, bias_feats, out, dout, lse, dq, dk, dv, dtheta, dbias,
+              need ? static_cast<float *>(workspace) : nullptr};
+    return dispatch_bwd(a, g, s);
+}
+
+int winattn_fwd_lse(const void *q, const void *k, const void *v, const float *theta, const void *bias_feats, int B,
+                    int H_img, int W_img, int M, int shift, int heads, int d, int rank, int dtype, void *out, float *lse,
+                    void *stream)
+{
+    int rc = winattn_check_args(q, k, v, theta, bias_feats, B, H_img, W_img, M, shift, heads, d, rank, dtype, out);
+    if (rc != WINATTN_OK)
+        return rc;
+    if (!lse)
+        return WINATTN_ERR_ARG;
+    if (reinterpret_cast<uintptr_t>(lse) & 3u)
+        return WINATTN_ERR_ALIGN;
+    const size_t n = map_bytes(B, H_img, W_img, heads, d, dtype), nl = (size_t)B * H_img * W_img * heads * 4;
+    if (overlaps(lse, nl, q, n) || overlaps(lse, nl, k, n) || overlaps(lse, nl, v, n) || overlaps(lse, nl, out, n))
+        return WINATTN_ERR_ALIAS;
+    rc = check_device();
+    if (rc != WINATTN_OK)
+        return rc;
+    const Geometry g = Geometry::make(B, H_img, W_img, M, shift, heads, d, rank);
+    return dispatch(q, k, v, theta, bias_feats, out, g, dtype, static_cast<cudaStream_t>(stream), lse);
 }
 
 size_t winattn_host_workspace_bytes(int B, int H_img, int W_img, int heads, int d, int dtype)
