@@ -56,6 +56,8 @@ def _bind(lib):
     lib.oracle_fwd.restype = i32
     lib.oracle_fwd_lse.argtypes = [vp, vp, vp, i32, vp, vp] + [i32] * 8 + [vp, vp, i32, f64]
     lib.oracle_fwd_lse.restype = i32
+    lib.oracle_fwd_sparse.argtypes = [vp, vp, vp, i32, vp, vp] + [i32] * 8 + [vp, i64, vp]
+    lib.oracle_fwd_sparse.restype = i32
     lib.oracle_fwd_units.argtypes = [vp, vp, vp, i32, vp, vp] + [i32] * 8 + [vp, i64, vp, i32, f64]
     lib.oracle_fwd_units.restype = i32
     lib.oracle_rope.argtypes = [vp, i32, f64, f64, vp, vp]
@@ -131,6 +133,22 @@ class Oracle:
         if rc < 0:
             raise ValueError(f"oracle rejected the problem (code {rc})")
         return out, lse
+
+    def fwd_sparse(self, q, k, v, o_lin, windows, *, M, shift=0, theta=None, bias=None) -> np.ndarray:
+        """The gated residual of HSMLA's two-path kernel: a copy of o_lin
+        [B, H, W, heads, d] where every token of the listed windows
+        (w = (b*nWy + wy)*nWx + wx, all heads) gets O_local - O_lin-local
+        added; fp64."""
+        q, k, v, theta, bias, code, (B, H, W, heads, d, rank) = self._prep(q, k, v, theta, bias, M)
+        out = np.array(o_lin, dtype=np.float64, copy=True, order="C")
+        if out.shape != q.shape:
+            raise ValueError("o_lin must have the shape of q")
+        windows = np.ascontiguousarray(windows, dtype=np.int32)
+        rc = self.lib.oracle_fwd_sparse(_ptr(q), _ptr(k), _ptr(v), code, _ptr(theta), _ptr(bias),
+                                        B, H, W, M, shift, heads, d, rank, _ptr(windows), len(windows), _ptr(out))
+        if rc < 0:
+            raise ValueError(f"oracle rejected the problem (code {rc})")
+        return out
 
     def fwd_units(self, q, k, v, units, *, M, shift=0, theta=None, bias=None,
                   nthreads=0, mem_budget=8e9) -> np.ndarray:

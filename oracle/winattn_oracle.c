@@ -44,6 +44,19 @@
  * forms, the displacement identity of the rotation, brute-force masked
  * global attention, Swin's slice-based region labels, planted mistakes).
  *
+ * The gated residual (oracle_fwd_sparse) follows "HSMLA: Hierarchical
+ * Softmax Multi-scale Linear Attention for Efficient Vision Transformers",
+ * section 2 (방법론), "Hierarchical Block-Level Gating" and "Two-Path
+ * Residual Kernel": every token keeps the global linear-attention output
+ * O_lin; only the gated blocks (here: windows) also run the local softmax
+ * attention, and add the residual O_local - O_lin-local, where O_lin-local is
+ * the linear attention (ReLU feature map, the EfficientViT-style kernel the
+ * page names) restricted to the same local keys.  Readings: the local keys
+ * of a token are its allowed set above (same window, same wrap label, real);
+ * O_lin-local uses the raw q, k (no rotation, no bias features), with
+ * O_lin-local = sum_p' relu(q).relu(k_p') v_p' / sum_p' relu(q).relu(k_p'),
+ * taken as 0 when that denominator is 0.
+ *
  * The backward (oracle_bwd) is the chain rule through the same steps: the
  * gradients of a scalar loss with respect to q, k, v, the RoPE frequencies
  * theta and the bias table, given the loss gradient dO at the output map.
@@ -414,6 +427,88 @@ int oracle_fwd_units(const void *q, const void *k, const void *v, int dtype,
         if (units[n] < 0 || units[n] >= total)
             return -1;
     return run(&p, units, n_units, out_units, NULL, NULL, nthreads, mem_budget_bytes);
+}
+
+/* The gated residual: out_map [B][H][W][heads][d] fp64 holds O_lin on entry;
+ * for every token of each listed window w = (b * nWy + wy) * nWx + wx (all
+ * heads), out += O_local - O_lin-local.  Windows may not repeat.  Plain
+ * loops, one window-head at a time. */
+int oracle_fwd_sparse(const void *q, const void *k, const void *v, int dtype,
+                      const float *theta, const void *bias,
+                      int B, int H, int W, int M, int shift, int heads, int d, int rank,
+                      const int32_t *windows, int64_t n_windows, double *out_map)
+{
+    problem_t p = make_problem(q, k, v, dtype, theta, bias, B, H, W, M, shift, heads, d, rank);
+    if (check_problem(&p) || !out_map || (n_windows > 0 && !windows) || d > 256)
+        return -1;
+    const int nWy = p.Hp / M, nWx = p.Wp / M;
+    const int64_t total = (int64_t)B * nWy * nWx;
+    for (int64_t n = 0; n < n_windows; ++n)
+        if (windows[n] < 0 || windows[n] >= total)
+            return -1;
+    const size_t N = (size_t)M * M;
+    scratch_t w;
+    w.q = malloc(N * d * sizeof(double));
+    w.k = malloc(N * d * sizeof(double));
+    w.v = malloc(N * d * sizeof(double));
+    w.s = malloc(N * N * sizeof(double));
+    w.off = malloc(N * sizeof(int64_t));
+    w.lse = malloc(N * sizeof(double));
+    double *o = malloc(N * d * sizeof(double));
+    double *kq = malloc(N * (size_t)d * 2 * sizeof(double));  /* relu(q), relu(k) of the raw rows */
+    int rc = 0;
+    if (!w.q || !w.k || !w.v || !w.s || !w.off || !w.lse || !o || !kq) {
+        rc = -2;
+        goto done;
+    }
+    for (int64_t n = 0; n < n_windows; ++n) {
+        const int wid = windows[n];
+        const int b = wid / (nWy * nWx), wy = (wid / nWx) % nWy, wx = wid % nWx;
+        for (int h = 0; h < heads; ++h) {
+            unit_forward(&p, b, wy, wx, h, &w, o);
+            /* the raw rows (unit_forward rotated q, k in place): re-read */
+            for (size_t t = 0; t < N; ++t)
+                for (int c = 0; c < d; ++c) {
+                    const int64_t off = w.off[t];
+                    const double qr = off < 0 ? 0.0 : read_elem(p.q, p.dtype, (size_t)off + c);
+                    const double kr = off < 0 ? 0.0 : read_elem(p.k, p.dtype, (size_t)off + c);
+                    kq[t * d + c] = qr > 0.0 ? qr : 0.0;
+                    kq[(N + t) * d + c] = kr > 0.0 ? kr : 0.0;
+                }
+            for (size_t a = 0; a < N; ++a) {
+                if (w.off[a] < 0)
+                    continue;
+                const int la = wrap_label(&p, wy * M + (int)a / M, wx * M + (int)a % M);
+                double den = 0.0;
+                double num[256];
+                for (int e = 0; e < d; ++e)
+                    num[e] = 0.0;
+                for (size_t c = 0; c < N; ++c) {
+                    if (w.off[c] < 0 || wrap_label(&p, wy * M + (int)c / M, wx * M + (int)c % M) != la)
+                        continue;
+                    double wgt = 0.0;
+                    for (int e = 0; e < d; ++e)
+                        wgt += kq[a * d + e] * kq[(N + c) * d + e];
+                    den += wgt;
+                    for (int e = 0; e < d; ++e)
+                        num[e] += wgt * w.v[c * d + e];
+                }
+                double *dst = out_map + w.off[a];
+                for (int e = 0; e < d; ++e)
+                    dst[e] += o[a * d + e] - (den > 0.0 ? num[e] / den : 0.0);
+            }
+        }
+    }
+done:
+    free(w.q);
+    free(w.k);
+    free(w.v);
+    free(w.s);
+    free(w.off);
+    free(w.lse);
+    free(o);
+    free(kq);
+    return rc;
 }
 
 /* The rotation alone, for the displacement-identity checks: out = R(i, j) vec. */

@@ -281,6 +281,66 @@ def pin_lse(o):
             assert abs(lse[0, y, x, 0] - math.log(n_allowed)) < 1e-13, f"zero-Q lse at ({y},{x})"
 
 
+def brute_sparse(q, k, v, o_lin, windows, M, s, theta=None, bias=None):
+    """HSMLA's gated residual written from the global formulation: softmax
+    part from brute_global, the local linear part as a masked matrix product
+    relu(Q) relu(K)^T over the same allowed pairs, added only to the tokens
+    of the listed windows of the rolled (padded) grid."""
+    B, H, W, heads, d = q.shape
+    Hp, Wp = -(-H // M) * M, -(-W // M) * M
+    soft = brute_global(q, k, v, M, s, theta, bias)
+    qf, kf, vf = (storage_to_f64(a) for a in (q, k, v))
+    ys, xs = np.meshgrid(np.arange(H), np.arange(W), indexing="ij")
+    yr, xr = (ys - s) % Hp, (xs - s) % Wp
+    win = ((yr // M) * (Wp // M) + (xr // M)).ravel()
+    region = swin_region_labels(Hp, Wp, M, s)[yr, xr].ravel()
+    allowed = (win[:, None] == win[None, :]) & (region[:, None] == region[None, :])
+    out = np.array(o_lin, dtype=np.float64, copy=True)
+    per_img = (Hp // M) * (Wp // M)
+    for b in range(B):
+        sel = np.isin(win, [w - b * per_img for w in windows if b * per_img <= w < (b + 1) * per_img])
+        for h in range(heads):
+            Q = np.maximum(qf[b, :, :, h].reshape(H * W, d), 0)
+            K = np.maximum(kf[b, :, :, h].reshape(H * W, d), 0)
+            V = vf[b, :, :, h].reshape(H * W, d)
+            L = np.where(allowed, Q @ K.T, 0.0)
+            den = L.sum(axis=1, keepdims=True)
+            lin = np.where(den > 0, (L @ V) / np.where(den > 0, den, 1.0), 0.0)
+            res = soft[b, :, :, h].reshape(H * W, d) - lin
+            o = out[b, :, :, h].reshape(H * W, d)
+            o[sel] += res[sel]
+            out[b, :, :, h] = o.reshape(H, W, d)
+    return out
+
+
+def pin_sparse_residual(o):
+    """The gated residual equals its global formulation on several shapes
+    (shifted, padded, with bias factors); windows that are not listed keep
+    O_lin bit for bit; with every window listed and the same constant
+    positive q and k everywhere, softmax and linear weights are both uniform,
+    so the residual vanishes and the output is O_lin."""
+    cases = [(2, 8, 12, 2, 8, 4, 2, "bf16", "learned", 0, [0, 3, 7, 9]),
+             (1, 10, 7, 1, 8, 4, 3, "fp32", None, 0, [1, 2, 5]),
+             (1, 8, 8, 2, 4, 4, 0, "bf16", None, 4, [0, 2, 3])]
+    for n, (B, H, W, heads, d, M, s, dt, rope, r, wins) in enumerate(cases):
+        q, k, v = _maps((B, H, W, heads, d), dt, f"pin-sparse-{n}")
+        th = I.make_theta(heads, d, rope, 41 + n)
+        th = None if th is None else th.numpy()
+        bias = I.to_storage_numpy(I.make_bias_feats(heads, M, r, dt, 43 + n)) if r else None
+        o_lin = np.random.default_rng(n).standard_normal((B, H, W, heads, d))
+        got = o.fwd_sparse(q, k, v, o_lin, wins, M=M, shift=s, theta=th, bias=bias)
+        ref = brute_sparse(q, k, v, o_lin, wins, M, s, th, bias)
+        _close(got, ref, 1e-10, f"sparse case {n}")
+        untouched = np.isclose(ref, o_lin, rtol=0, atol=0)
+        assert np.array_equal(got[untouched], o_lin[untouched]), "unlisted windows keep O_lin"
+    B, H, W, heads, d, M = 1, 8, 8, 1, 4, 4
+    c = np.full((B, H, W, heads, d), 0.5, np.float32)
+    _, _, v = _maps((B, H, W, heads, d), "fp32", "pin-sparse-const")
+    o_lin = np.random.default_rng(9).standard_normal((B, H, W, heads, d))
+    got = o.fwd_sparse(c, c, v, o_lin, [0, 1, 2, 3], M=M, shift=2)
+    _close(got, o_lin, 1e-12, "uniform weights: zero residual")
+
+
 def pin_bias_concat(o):
     """[Qc, Qp][Kc, Kp]^T = Qc Kc^T + Qp Kp^T: a problem with rank-r bias
     factors equals a bias-free problem of head dim d + r whose query rows are
@@ -346,4 +406,4 @@ def pin_padding_closed_forms(o):
 
 ALL_PINS = [pin_rope_displacement, pin_theta_zero, pin_one_token_windows, pin_constant_v,
             pin_zero_q_mean, pin_hand_worked, pin_brute_global, pin_bias_concat, pin_padding_closed_forms,
-            pin_lse]
+            pin_lse, pin_sparse_residual]

@@ -45,6 +45,11 @@ MUTANTS = {
     "pad_keys_attended": [("            if (w->off[c] < 0)\n                w->s[(size_t)a * N + c] = -INFINITY;",
                            "            if (0)\n                w->s[(size_t)a * N + c] = -INFINITY;")],
     "lse_without_max": [("w->lse[a] = mx + log(sum);", "w->lse[a] = log(sum);")],
+    "linear_without_relu": [("kq[t * d + c] = qr > 0.0 ? qr : 0.0;", "kq[t * d + c] = qr;")],
+    "residual_sign_flipped": [("dst[e] += o[a * d + e] - (den > 0.0 ? num[e] / den : 0.0);",
+                               "dst[e] += o[a * d + e] + (den > 0.0 ? num[e] / den : 0.0);")],
+    "linear_mask_dropped": [("if (w.off[c] < 0 || wrap_label(&p, wy * M + (int)c / M, wx * M + (int)c % M) != la)",
+                             "if (w.off[c] < 0)")],
     "roll_over_unpadded_map": [
         ("int y = (yr + p->shift) % p->Hp;", "int y = (yr + p->shift) % p->H;"),
         ("int x = (xr + p->shift) % p->Wp;", "int x = (xr + p->shift) % p->W;"),
