@@ -121,6 +121,42 @@ int winattn_fwd_lse(const void *q, const void *k, const void *v,
                     void *out, float *lse, void *stream);
 
 /*
+ * winattn_fwd_sparse — window attention on a list of gated windows only, as
+ * the residual refinement of a global linear attention ("HSMLA:
+ * Hierarchical Softmax Multi-scale Linear Attention for Efficient Vision
+ * Transformers", section 2, Hierarchical Block-Level Gating and Two-Path
+ * Residual Kernel): every token keeps the global linear-attention output
+ * O_lin, and the tokens of the gated windows add O_local - O_lin-local:
+ *
+ *   out_p <- out_p + o_p - ( sum_p' relu(q_p).relu(k_p') v_p' )
+ *                          / ( sum_p' relu(q_p).relu(k_p') )
+ *
+ * with o_p the window attention above and both sums over the allowed keys
+ * p' of p (same window, same wrap label, real tokens), on the raw q, k (no
+ * rotation, no bias features; the fraction is 0 when its denominator is 0).
+ *
+ *   q, k, v, theta, bias_feats, sizes  as for winattn_fwd; dtype WINATTN_BF16.
+ *   windows     device, int32 [n_windows], 4-byte aligned: window ids
+ *               w = (b * nWy + wy) * nWx + wx of the (padded) grid of windows
+ *               of the rolled map, nWy = ceil(H_img / M), nWx = ceil(W_img / M);
+ *               each id at most once (a repeated id adds its residual twice,
+ *               racing) and below B * nWy * nWx (not checked on the device:
+ *               an id out of range reads and writes outside the maps).
+ *   n_windows   0 .. B * nWy * nWx (0: nothing is enqueued).
+ *   out         device, bf16 map like q, holding O_lin on entry; updated in
+ *               place for the tokens of the listed windows, untouched
+ *               elsewhere.  Must not overlap q, k or v.
+ *
+ * Stream-ordered and asynchronous; allocates nothing.  Errors as winattn_fwd;
+ * WINATTN_ERR_DTYPE for fp32.
+ */
+int winattn_fwd_sparse(const void *q, const void *k, const void *v,
+                       const float *theta, const void *bias_feats,
+                       int B, int H_img, int W_img, int M, int shift,
+                       int heads, int d, int rank, int dtype,
+                       const int32_t *windows, int n_windows, void *out, void *stream);
+
+/*
  * winattn_bwd — the backward pass: gradients of a scalar loss L with respect
  * to q, k, v, the RoPE frequencies theta and the bias features, given
  * dout = dL/dO, the forward's output `out` and its saved log-sum-exp `lse`

@@ -14,8 +14,8 @@ import torch
 from . import _lib
 from ._lib import WinattnError
 
-__all__ = ["window_attention", "window_attention_host", "window_attention_backward", "WinattnError",
-           "device_status"]
+__all__ = ["window_attention", "window_attention_host", "window_attention_backward",
+           "window_attention_gated_residual", "WinattnError", "device_status"]
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -80,6 +80,28 @@ def window_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, M: int, 
     if rc != _lib.OK:
         raise WinattnError(rc, what)
     return out
+
+
+def window_attention_gated_residual(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o_lin: torch.Tensor,
+                                    windows: torch.Tensor, M: int, shift: int = 0,
+                                    theta: Optional[torch.Tensor] = None,
+                                    bias_feats: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """HSMLA's two-path residual on the gated windows (winattn_fwd_sparse):
+    ``o_lin`` (bf16, shaped like q) is updated in place for the tokens of the
+    listed windows (int32 CUDA tensor of window ids) and returned."""
+    B, H, W, heads, d, rank = _shape(q, k, v, theta, bias_feats, M)
+    if o_lin.shape != q.shape or o_lin.dtype != q.dtype or not o_lin.is_contiguous():
+        raise WinattnError(_lib.ERR_ARG, "o_lin must be contiguous and shaped like q")
+    if windows.dtype != torch.int32 or windows.dim() != 1 or not windows.is_contiguous():
+        raise WinattnError(_lib.ERR_ARG, "windows must be a contiguous int32 vector")
+    dev = q.device
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    with torch.cuda.device(dev):
+        rc = _lib.fwd_sparse(_ptr(q), _ptr(k), _ptr(v), _ptr(theta), _ptr(bias_feats), B, H, W, M, shift, heads, d,
+                             rank, _dtype_code(q), _ptr(windows), windows.numel(), _ptr(o_lin), stream)
+    if rc != _lib.OK:
+        raise WinattnError(rc, "winattn_fwd_sparse")
+    return o_lin
 
 
 def window_attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,

@@ -20,7 +20,7 @@ BF16, FP32 = 0, 1
 EXPORTS = ("winattn_fwd", "winattn_fwd_lse", "winattn_check_args", "winattn_fwd_host", "winattn_host_workspace_bytes",
            "winattn_strerror", "winattn_last_device_status", "winattn_launch_info", "winattn_fwd_host_static",
            "winattn_selftest_wait_timeout", "winattn_set_kernel_enabled", "winattn_bwd",
-           "winattn_bwd_workspace_bytes")
+           "winattn_bwd_workspace_bytes", "winattn_fwd_sparse")
 STATIC_WORKSPACE_BYTES = 32 << 20
 
 
@@ -67,6 +67,8 @@ def load(path: str = LIB_PATH):
     lib.winattn_bwd.restype = i32
     lib.winattn_bwd_workspace_bytes.argtypes = [i32] * 6
     lib.winattn_bwd_workspace_bytes.restype = sz
+    lib.winattn_fwd_sparse.argtypes = [vp] * 5 + [i32] * 9 + [vp, i32, vp, vp]
+    lib.winattn_fwd_sparse.restype = i32
     lib.winattn_set_kernel_enabled.argtypes = [i32, i32]
     lib.winattn_set_kernel_enabled.restype = i32
     _lib = lib
@@ -98,6 +100,12 @@ def bwd(q_ptr, k_ptr, v_ptr, theta_ptr, bias_ptr, out_ptr, dout_ptr, lse_ptr, B,
 
 def bwd_workspace_bytes(B, H, W, M, heads, d) -> int:
     return load().winattn_bwd_workspace_bytes(B, H, W, M, heads, d)
+
+
+def fwd_sparse(q_ptr, k_ptr, v_ptr, theta_ptr, bias_ptr, B, H, W, M, shift, heads, d, rank, dtype, win_ptr, n_win,
+               out_ptr, stream) -> int:
+    return load().winattn_fwd_sparse(q_ptr, k_ptr, v_ptr, theta_ptr, bias_ptr, B, H, W, M, shift, heads, d, rank,
+                                     dtype, win_ptr, n_win, out_ptr, stream)
 
 
 def check_args(q_ptr, k_ptr, v_ptr, theta_ptr, bias_ptr, B, H, W, M, shift, heads, d, rank, dtype,

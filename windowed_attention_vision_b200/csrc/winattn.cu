@@ -292,9 +292,13 @@ int launch_tc(const void *q, const void *k, const void *v, const float *theta, c
               float *lse, const Geometry &g, cudaStream_t stream)
 {
     using T = __nv_bfloat16;
-    return launch<winattn_fwd_tc_kernel<D, R>>((int)TcLayout<D, R>::bytes(g.M), g, stream,
-                  static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), theta,
-                  static_cast<const T *>(bias), static_cast<T *>(out), lse);
+    constexpr auto kernel = winattn_fwd_tc_kernel<D, R, false>;
+    if (!smem_attr_once<kernel>())
+        return WINATTN_ERR_CUDA;
+    kernel<<<(unsigned)g.items, kThreads, TcLayout<D, R>::bytes(g.M), stream>>>(
+        static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), theta,
+        static_cast<const T *>(bias), static_cast<T *>(out), lse, g, 1.0f / std::sqrt((float)g.d), nullptr, 0);
+    return cudaGetLastError() == cudaSuccess ? WINATTN_OK : WINATTN_ERR_CUDA;
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no
@@ -640,6 +644,38 @@ HostLanes *host_lanes()
     return per_dev[dev];
 }
 
+// ------------------------------------------------------------------ gated windows
+
+template <int D, int R>
+int launch_sparse(const void *q, const void *k, const void *v, const float *theta, const void *bias, void *out,
+                  const int32_t *windows, int n_windows, const Geometry &g, cudaStream_t stream)
+{
+    using T = __nv_bfloat16;
+    constexpr auto kernel = winattn_fwd_tc_kernel<D, R, true>;
+    if (!smem_attr_once<kernel>())
+        return WINATTN_ERR_CUDA;
+    const int64_t items = (int64_t)g.heads * ((n_windows + g.U - 1) / g.U) * g.n_tiles;
+    kernel<<<(unsigned)items, kThreads, TcLayout<D, R, true>::bytes(g.M), stream>>>(
+        static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), theta,
+        static_cast<const T *>(bias), static_cast<T *>(out), nullptr, g, 1.0f / std::sqrt((float)g.d), windows,
+        n_windows);
+    return cudaGetLastError() == cudaSuccess ? WINATTN_OK : WINATTN_ERR_CUDA;
+}
+
+int dispatch_sparse(const void *q, const void *k, const void *v, const float *theta, const void *bias, void *out,
+                    const int32_t *windows, int n_windows, const Geometry &g, cudaStream_t s)
+{
+    switch (g.d * 100 + g.rank) {
+    case 3200: return launch_sparse<32, 0>(q, k, v, theta, bias, out, windows, n_windows, g, s);
+    case 3216: return launch_sparse<32, 16>(q, k, v, theta, bias, out, windows, n_windows, g, s);
+    case 3232: return launch_sparse<32, 32>(q, k, v, theta, bias, out, windows, n_windows, g, s);
+    case 6400: return launch_sparse<64, 0>(q, k, v, theta, bias, out, windows, n_windows, g, s);
+    case 6416: return launch_sparse<64, 16>(q, k, v, theta, bias, out, windows, n_windows, g, s);
+    case 6432: return launch_sparse<64, 32>(q, k, v, theta, bias, out, windows, n_windows, g, s);
+    }
+    return WINATTN_ERR_ARG;
+}
+
 // ------------------------------------------------------------------ backward
 
 struct BwdArgs {
@@ -729,6 +765,31 @@ int winattn_fwd(const void *q, const void *k, const void *v, const float *theta,
         return rc;
     const Geometry g = Geometry::make(B, H_img, W_img, M, shift, heads, d, rank);
     return dispatch(q, k, v, theta, bias_feats, out, g, dtype, static_cast<cudaStream_t>(stream));
+}
+
+int winattn_fwd_sparse(const void *q, const void *k, const void *v, const float *theta, const void *bias_feats,
+                       int B, int H_img, int W_img, int M, int shift, int heads, int d, int rank, int dtype,
+                       const int32_t *windows, int n_windows, void *out, void *stream)
+{
+    // out holds O_lin and is updated in place: it may not alias q, k, v
+    int rc = winattn_check_args(q, k, v, theta, bias_feats, B, H_img, W_img, M, shift, heads, d, rank, dtype, out);
+    if (rc != WINATTN_OK)
+        return rc;
+    if (dtype != WINATTN_BF16)
+        return WINATTN_ERR_DTYPE;
+    if (n_windows < 0 || (n_windows > 0 && !windows))
+        return WINATTN_ERR_ARG;
+    if (reinterpret_cast<uintptr_t>(windows) & 3u)
+        return WINATTN_ERR_ALIGN;
+    if (n_windows == 0)
+        return WINATTN_OK;
+    rc = check_device();
+    if (rc != WINATTN_OK)
+        return rc;
+    const Geometry g = Geometry::make(B, H_img, W_img, M, shift, heads, d, rank);
+    if (n_windows > g.wph)
+        return WINATTN_ERR_ARG;  // windows may not repeat, so at most every window once
+    return dispatch_sparse(q, k, v, theta, bias_feats, out, windows, n_windows, g, static_cast<cudaStream_t>(stream));
 }
 
 size_t winattn_bwd_workspace_bytes(int B, int H_img, int W_img, int M, int heads, int d)
