@@ -58,6 +58,10 @@ def _bind(lib):
     lib.oracle_fwd_lse.restype = i32
     lib.oracle_fwd_sparse.argtypes = [vp, vp, vp, i32, vp, vp] + [i32] * 8 + [vp, i64, vp]
     lib.oracle_fwd_sparse.restype = i32
+    lib.oracle_rib_features.argtypes = [vp, vp, i32, i32, i32, vp]
+    lib.oracle_rib_features.restype = i32
+    lib.oracle_cla_gate.argtypes = [vp, vp, i32, vp, vp, vp, vp, i32, i32, i32, i32, vp]
+    lib.oracle_cla_gate.restype = i32
     lib.oracle_fwd_units.argtypes = [vp, vp, vp, i32, vp, vp] + [i32] * 8 + [vp, i64, vp, i32, f64]
     lib.oracle_fwd_units.restype = i32
     lib.oracle_rope.argtypes = [vp, i32, f64, f64, vp, vp]
@@ -182,6 +186,35 @@ class Oracle:
         if rc < 0:
             raise ValueError(f"oracle rejected the problem (code {rc})")
         return dq, dk, dv, dtheta, dbias
+
+    def rib_features(self, w1, w2, M) -> np.ndarray:
+        """Rank-r factor table [heads, 2, M*M, rank] fp64 from the MLP weights
+        w1 [heads, 2, 32, 64] and w2 [heads, 2, 64, rank] (fp32)."""
+        w1 = np.ascontiguousarray(w1, dtype=np.float32)
+        w2 = np.ascontiguousarray(w2, dtype=np.float32)
+        heads, rank = w1.shape[0], w2.shape[3]
+        if w1.shape != (heads, 2, 32, 64) or w2.shape != (heads, 2, 64, rank):
+            raise ValueError("w1 must be [heads, 2, 32, 64] and w2 [heads, 2, 64, rank]")
+        out = np.zeros((heads, 2, M * M, rank), dtype=np.float64)
+        if self.lib.oracle_rib_features(_ptr(w1), _ptr(w2), M, heads, rank, _ptr(out)):
+            raise ValueError("bad feature arguments")
+        return out
+
+    def cla_gate(self, x, o, dw, dw_b, pw, pw_b) -> np.ndarray:
+        """O * sigmoid(PW(DW3x3(x))) [B, H, W, C] fp64; x, o in storage form."""
+        x, o = np.ascontiguousarray(x), np.ascontiguousarray(o)
+        code = _dtype_code(x)
+        if _dtype_code(o) != code or x.shape != o.shape or x.ndim != 4:
+            raise ValueError("x and o must share one [B, H, W, C] shape and storage dtype")
+        B, H, W, C = x.shape
+        dw, dw_b, pw, pw_b = (np.ascontiguousarray(a, dtype=np.float32) for a in (dw, dw_b, pw, pw_b))
+        if dw.shape != (C, 3, 3) or dw_b.shape != (C,) or pw.shape != (C, C) or pw_b.shape != (C,):
+            raise ValueError("dw [C, 3, 3], dw_b [C], pw [C, C], pw_b [C]")
+        out = np.zeros((B, H, W, C), dtype=np.float64)
+        if self.lib.oracle_cla_gate(_ptr(x), _ptr(o), code, _ptr(dw), _ptr(dw_b), _ptr(pw), _ptr(pw_b), B, H, W, C,
+                                    _ptr(out)):
+            raise ValueError("bad gate arguments")
+        return out
 
     def rope(self, vec, i, j, theta_h) -> np.ndarray:
         """R(i, j) vec for one d-vector (window-local row i, column j)."""

@@ -57,6 +57,22 @@
  * O_lin-local = sum_p' relu(q).relu(k_p') v_p' / sum_p' relu(q).relu(k_p'),
  * taken as 0 when that denominator is 0.
  *
+ * The bias features themselves (oracle_rib_features) follow "Rank-Factorized
+ * Implicit Neural Bias", section 2.1: the 2D coordinate of each window
+ * position is mapped to Fourier features and a light MLP turns them into the
+ * rank-r query and key factors.  Readings (the page gives no sizes):
+ * coordinates c = 2 i / (M - 1) - 1 per axis (0 when M = 1); 8 octaves
+ * 2^k pi, features ordered [sin(2^k pi c_y)]_k, [cos(2^k pi c_y)]_k,
+ * [sin(2^k pi c_x)]_k, [cos(2^k pi c_x)]_k (32); one hidden layer of 64 with
+ * tanh, no biases; separate weights per head and per side (u, w).
+ *
+ * The convolutional local attention gate (oracle_cla_gate) follows the same
+ * page, section 2.2: a 3 x 3 depth-wise convolution and a 1 x 1 point-wise
+ * convolution of the block input, a sigmoid, and the attention output
+ * multiplied by that gate.  Readings: zero padding at the map border, one
+ * bias per channel after each convolution, the gate applied channel by
+ * channel to O of the same token.
+ *
  * The backward (oracle_bwd) is the chain rule through the same steps: the
  * gradients of a scalar loss with respect to q, k, v, the RoPE frequencies
  * theta and the bias table, given the loss gradient dO at the output map.
@@ -509,6 +525,90 @@ done:
     free(o);
     free(kq);
     return rc;
+}
+
+/* The rank-r factor table [heads][2][M*M][rank] (fp64) from the MLP weights
+ * w1 [heads][2][32][64] and w2 [heads][2][64][rank] (fp32). */
+int oracle_rib_features(const float *w1, const float *w2, int M, int heads, int rank, double *table)
+{
+    if (!w1 || !w2 || !table || M <= 0 || heads <= 0 || rank <= 0)
+        return -1;
+    const int N = M * M;
+    for (int h = 0; h < heads; ++h)
+        for (int side = 0; side < 2; ++side) {
+            const float *a = w1 + ((size_t)h * 2 + side) * 32 * 64;
+            const float *b = w2 + ((size_t)h * 2 + side) * 64 * rank;
+            for (int p = 0; p < N; ++p) {
+                const int i = p / M, j = p % M;
+                /* Fourier features of the window-local coordinate */
+                const double cy = M > 1 ? 2.0 * i / (M - 1) - 1.0 : 0.0;
+                const double cx = M > 1 ? 2.0 * j / (M - 1) - 1.0 : 0.0;
+                double f[32];
+                for (int k = 0; k < 8; ++k) {
+                    const double w = ldexp(acos(-1.0), k);  /* 2^k pi */
+                    f[k] = sin(w * cy);
+                    f[8 + k] = cos(w * cy);
+                    f[16 + k] = sin(w * cx);
+                    f[24 + k] = cos(w * cx);
+                }
+                /* the MLP: tanh(f w1) w2 */
+                double hid[64];
+                for (int c = 0; c < 64; ++c) {
+                    double acc = 0.0;
+                    for (int e = 0; e < 32; ++e)
+                        acc += f[e] * a[e * 64 + c];
+                    hid[c] = tanh(acc);
+                }
+                double *dst = table + (((size_t)h * 2 + side) * N + p) * rank;
+                for (int r = 0; r < rank; ++r) {
+                    double acc = 0.0;
+                    for (int c = 0; c < 64; ++c)
+                        acc += hid[c] * b[c * rank + r];
+                    dst[r] = acc;
+                }
+            }
+        }
+    return 0;
+}
+
+/* The gated attention output: out = O * sigmoid(PW(DW3x3(x))), all
+ * [B][H][W][C] fp64 (x and O as read from their storage dtype), dw
+ * [C][3][3], dw_b [C], pw [C_out][C_in], pw_b [C] fp32. */
+int oracle_cla_gate(const void *x, const void *o, int dtype, const float *dw, const float *dw_b, const float *pw,
+                    const float *pw_b, int B, int H, int W, int C, double *out)
+{
+    if (!x || !o || !dw || !dw_b || !pw || !pw_b || !out || B <= 0 || H <= 0 || W <= 0 || C <= 0)
+        return -1;
+    double *y = malloc((size_t)C * sizeof(double));
+    if (!y)
+        return -2;
+    for (int b = 0; b < B; ++b)
+        for (int r = 0; r < H; ++r)
+            for (int c = 0; c < W; ++c) {
+                /* depth-wise 3 x 3, zero outside the map */
+                for (int ch = 0; ch < C; ++ch) {
+                    double acc = dw_b[ch];
+                    for (int dy = -1; dy <= 1; ++dy)
+                        for (int dx = -1; dx <= 1; ++dx) {
+                            const int rr = r + dy, cc = c + dx;
+                            if (rr < 0 || rr >= H || cc < 0 || cc >= W)
+                                continue;
+                            acc += dw[ch * 9 + (dy + 1) * 3 + (dx + 1)] *
+                                   read_elem(x, dtype, (((size_t)b * H + rr) * W + cc) * C + ch);
+                        }
+                    y[ch] = acc;
+                }
+                /* point-wise 1 x 1, sigmoid, gate */
+                for (int co = 0; co < C; ++co) {
+                    double acc = pw_b[co];
+                    for (int ci = 0; ci < C; ++ci)
+                        acc += pw[(size_t)co * C + ci] * y[ci];
+                    const size_t idx = (((size_t)b * H + r) * W + c) * C + co;
+                    out[idx] = read_elem(o, dtype, idx) / (1.0 + exp(-acc));
+                }
+            }
+    free(y);
+    return 0;
 }
 
 /* The rotation alone, for the displacement-identity checks: out = R(i, j) vec. */

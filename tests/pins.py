@@ -341,6 +341,81 @@ def pin_sparse_residual(o):
     _close(got, o_lin, 1e-12, "uniform weights: zero residual")
 
 
+def _rib_weights(heads, rank, seed, scale=1.0):
+    rng = np.random.default_rng(seed)
+    w1 = (scale * rng.standard_normal((heads, 2, 32, 64)) / math.sqrt(32)).astype(np.float32)
+    w2 = (rng.standard_normal((heads, 2, 64, rank)) / math.sqrt(64)).astype(np.float32)
+    return w1, w2
+
+
+def pin_rib_features(o):
+    """The RIB factor MLP (RIB page, section 2.1) by closed forms and
+    symmetries of its Fourier features: at M = 1 every coordinate is 0 (sin 0,
+    cos 1); at M = 2 the coordinates are -1 and 1, where sin(2^k pi c) = 0 and
+    cos(2^k pi c) = -1 for k = 0, 1 after; with only cosine rows the table is
+    mirror-symmetric in each axis (cos is even), with only sine rows it is odd
+    under the point reflection (sin and tanh are odd); with only the row-axis
+    rows it does not depend on the column."""
+    heads, rank = 2, 16
+    w1, w2 = _rib_weights(heads, rank, 3)
+    f0 = np.concatenate([np.zeros(8), np.ones(8), np.zeros(8), np.ones(8)])
+    got = o.rib_features(w1, w2, 1)
+    for h in range(heads):
+        for s in range(2):
+            ref = np.tanh(f0 @ w1[h, s].astype(np.float64)) @ w2[h, s].astype(np.float64)
+            _close(got[h, s, 0], ref, 1e-12, "M = 1 closed form")
+    got = o.rib_features(w1, w2, 2)
+    cosv = np.array([-1.0] + [1.0] * 7)
+    for p in range(4):
+        f = np.concatenate([np.zeros(8), cosv, np.zeros(8), cosv])
+        for h in range(heads):
+            for s in range(2):
+                ref = np.tanh(f @ w1[h, s].astype(np.float64)) @ w2[h, s].astype(np.float64)
+                _close(got[h, s, p], ref, 1e-12, "M = 2 closed form")
+    M = 7
+    cos_only, sin_only, y_only = w1.copy(), w1.copy(), w1.copy()
+    cos_only[:, :, 0:8] = 0
+    cos_only[:, :, 16:24] = 0
+    sin_only[:, :, 8:16] = 0
+    sin_only[:, :, 24:32] = 0
+    y_only[:, :, 16:32] = 0
+    t = o.rib_features(cos_only, w2, M).reshape(heads, 2, M, M, rank)
+    _close(t, t[:, :, ::-1, :, :], 1e-12, "cosine rows: mirror in rows")
+    _close(t, t[:, :, :, ::-1, :], 1e-12, "cosine rows: mirror in columns")
+    t = o.rib_features(sin_only, w2, M).reshape(heads, 2, M, M, rank)
+    _close(t, -t[:, :, ::-1, ::-1, :], 1e-12, "sine rows: odd under point reflection")
+    t = o.rib_features(y_only, w2, M).reshape(heads, 2, M, M, rank)
+    _close(t, np.broadcast_to(t[:, :, :, :1, :], t.shape), 1e-12, "row-axis rows: no column dependence")
+
+
+def pin_cla_gate(o):
+    """The CLA gate (RIB page, section 2.2) against library routines: a
+    per-channel 2-D correlation with zero fill (scipy.signal.correlate2d),
+    a matrix product and the logistic function (scipy.special.expit); and
+    the closed form O * sigmoid(b) when the point-wise weights are zero."""
+    from scipy.signal import correlate2d
+    from scipy.special import expit
+    rng = np.random.default_rng(5)
+    B, H, W, C = 2, 5, 7, 8
+    x = I.to_storage_numpy(I.make_map((B, H, W, C), "bf16", 61))
+    ob = I.to_storage_numpy(I.make_map((B, H, W, C), "bf16", 62))
+    dw = rng.standard_normal((C, 3, 3)).astype(np.float32)
+    dw_b = rng.standard_normal(C).astype(np.float32)
+    pw = (rng.standard_normal((C, C)) / math.sqrt(C)).astype(np.float32)
+    pw_b = rng.standard_normal(C).astype(np.float32)
+    got = o.cla_gate(x, ob, dw, dw_b, pw, pw_b)
+    xf, of = storage_to_f64(x), storage_to_f64(ob)
+    y = np.zeros((B, H, W, C))
+    for b in range(B):
+        for c in range(C):
+            y[b, :, :, c] = correlate2d(xf[b, :, :, c], dw[c].astype(np.float64), mode="same",
+                                        boundary="fill") + dw_b[c]
+    ref = of * expit(y @ pw.T.astype(np.float64) + pw_b)
+    _close(got, ref, 1e-12, "gate against library routines")
+    got = o.cla_gate(x, ob, dw, dw_b, np.zeros_like(pw), pw_b)
+    _close(got, of * expit(pw_b.astype(np.float64)), 1e-12, "zero point-wise weights")
+
+
 def pin_bias_concat(o):
     """[Qc, Qp][Kc, Kp]^T = Qc Kc^T + Qp Kp^T: a problem with rank-r bias
     factors equals a bias-free problem of head dim d + r whose query rows are
@@ -406,4 +481,4 @@ def pin_padding_closed_forms(o):
 
 ALL_PINS = [pin_rope_displacement, pin_theta_zero, pin_one_token_windows, pin_constant_v,
             pin_zero_q_mean, pin_hand_worked, pin_brute_global, pin_bias_concat, pin_padding_closed_forms,
-            pin_lse, pin_sparse_residual]
+            pin_lse, pin_sparse_residual, pin_rib_features, pin_cla_gate]

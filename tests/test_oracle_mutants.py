@@ -50,6 +50,13 @@ MUTANTS = {
                                "dst[e] += o[a * d + e] + (den > 0.0 ? num[e] / den : 0.0);")],
     "linear_mask_dropped": [("if (w.off[c] < 0 || wrap_label(&p, wy * M + (int)c / M, wx * M + (int)c % M) != la)",
                              "if (w.off[c] < 0)")],
+    "rib_axes_swapped": [("f[k] = sin(w * cy);", "f[k] = sin(w * cx);"),
+                         ("f[8 + k] = cos(w * cy);", "f[8 + k] = cos(w * cx);")],
+    "rib_octave_off_by_one": [("const double w = ldexp(acos(-1.0), k);", "const double w = ldexp(acos(-1.0), k + 1);")],
+    "rib_no_tanh": [("hid[c] = tanh(acc);", "hid[c] = acc;")],
+    "cla_convolution_flipped": [("acc += dw[ch * 9 + (dy + 1) * 3 + (dx + 1)] *",
+                                 "acc += dw[ch * 9 + (1 - dy) * 3 + (1 - dx)] *")],
+    "cla_pointwise_transposed": [("acc += pw[(size_t)co * C + ci] * y[ci];", "acc += pw[(size_t)ci * C + co] * y[ci];")],
     "roll_over_unpadded_map": [
         ("int y = (yr + p->shift) % p->Hp;", "int y = (yr + p->shift) % p->H;"),
         ("int x = (xr + p->shift) % p->Wp;", "int x = (xr + p->shift) % p->W;"),
