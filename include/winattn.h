@@ -157,6 +157,62 @@ int winattn_fwd_sparse(const void *q, const void *k, const void *v,
                        const int32_t *windows, int n_windows, void *out, void *stream);
 
 /*
+ * winattn_rib_features — the rank-r bias factors of "Rank-Factorized
+ * Implicit Neural Bias: Scaling Super-Resolution Transformer with
+ * FlashAttention" (section 2.1) on the GPU: for every head, side (0 = u,
+ * queries; 1 = w, keys) and window position p = i*M + j, Fourier features of
+ * the window-local coordinate (c = 2 i / (M - 1) - 1 per axis, 0 when M = 1;
+ * [sin 2^k pi c_y]_k, [cos 2^k pi c_y]_k, [sin 2^k pi c_x]_k,
+ * [cos 2^k pi c_x]_k, k < 8) through tanh(f w1) w2.
+ *
+ *   w1     device fp32 [heads][2][32][64], 16-byte aligned.
+ *   w2     device fp32 [heads][2][64][rank], 16-byte aligned.
+ *   rank   16 or 32 (WINATTN_ERR_RANK otherwise); M <= 256.
+ *   table  device bf16 [heads][2][M*M][rank] (the bias_feats of winattn_fwd),
+ *          16-byte aligned; overwritten.
+ * Stream-ordered; allocates nothing.
+ */
+int winattn_rib_features(const float *w1, const float *w2, int M, int heads, int rank, void *table, void *stream);
+
+/*
+ * winattn_fwd_rib — winattn_fwd with rank-r bias features generated from the
+ * MLP weights in the same call: winattn_rib_features into `table` (caller
+ * owned, bf16 [heads][2][M*M][rank], 16-byte aligned, must not overlap the
+ * maps), then the attention reading it.  The table depends only on the
+ * window position and head, so it is built once per call (a few
+ * microseconds even at M = 96) and read by every window from L2, rather
+ * than recomputed by every CTA that loads a tile of it.  dtype WINATTN_BF16.
+ */
+int winattn_fwd_rib(const void *q, const void *k, const void *v, const float *theta,
+                    const float *w1, const float *w2,
+                    int B, int H_img, int W_img, int M, int shift,
+                    int heads, int d, int rank, int dtype,
+                    void *table, void *out, void *stream);
+
+/*
+ * winattn_cla_gate — the convolutional local attention gate of the same
+ * page (section 2.2): out = o * sigmoid(PW(DW3x3(x))) per token and channel,
+ * DW a depth-wise 3 x 3 convolution with zero padding and one bias per
+ * channel, PW a C x C point-wise convolution with bias.
+ *
+ *   x      device bf16 [B][H_img][W_img][C]: the block input the gate is
+ *          computed from.
+ *   o      device bf16, same shape: the attention output to gate.
+ *   dw     device fp32 [C][3][3];  dw_b  fp32 [C].
+ *   pw     device fp32 [C][C] (output channel major);  pw_b  fp32 [C].
+ *   C      16 .. 256, a multiple of 16 (heads * d of the attention).
+ *   out    device bf16, same shape; may be o itself (in place), must not
+ *          overlap x.
+ * One fused kernel: the depth-wise convolution in fp32 on the CUDA cores,
+ * rounded to bf16, the point-wise contraction on tcgen05 (fp32 accumulate),
+ * bias, sigmoid and product in the epilogue.  Stream-ordered; allocates
+ * nothing.
+ */
+int winattn_cla_gate(const void *x, const void *o, const float *dw, const float *dw_b,
+                     const float *pw, const float *pw_b, int B, int H_img, int W_img, int C, int dtype,
+                     void *out, void *stream);
+
+/*
  * winattn_bwd — the backward pass: gradients of a scalar loss L with respect
  * to q, k, v, the RoPE frequencies theta and the bias features, given
  * dout = dL/dO, the forward's output `out` and its saved log-sum-exp `lse`

@@ -15,7 +15,8 @@ from . import _lib
 from ._lib import WinattnError
 
 __all__ = ["window_attention", "window_attention_host", "window_attention_backward",
-           "window_attention_gated_residual", "WinattnError", "device_status"]
+           "window_attention_gated_residual", "rib_features", "window_attention_rib", "cla_gate", "WinattnError",
+           "device_status"]
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -102,6 +103,58 @@ def window_attention_gated_residual(q: torch.Tensor, k: torch.Tensor, v: torch.T
     if rc != _lib.OK:
         raise WinattnError(rc, "winattn_fwd_sparse")
     return o_lin
+
+
+def _call(fn, what, dev, *args):
+    with torch.cuda.device(dev):
+        rc = fn(*args, torch.cuda.current_stream(dev).cuda_stream)
+    if rc != _lib.OK:
+        raise WinattnError(rc, what)
+
+
+def rib_features(w1: torch.Tensor, w2: torch.Tensor, M: int, table: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The RIB factor table [heads, 2, M*M, rank] (bf16) from the MLP weights
+    w1 [heads, 2, 32, 64] and w2 [heads, 2, 64, rank] (fp32 CUDA tensors)."""
+    heads, rank = w1.shape[0], w2.shape[3]
+    if tuple(w1.shape) != (heads, 2, 32, 64) or tuple(w2.shape) != (heads, 2, 64, rank) or \
+            w1.dtype != torch.float32 or w2.dtype != torch.float32:
+        raise WinattnError(_lib.ERR_ARG, "w1 must be fp32 [heads, 2, 32, 64] and w2 fp32 [heads, 2, 64, rank]")
+    if table is None:
+        table = torch.empty((heads, 2, M * M, rank), dtype=torch.bfloat16, device=w1.device)
+    _call(_lib.rib_features, "winattn_rib_features", w1.device, _ptr(w1.contiguous()), _ptr(w2.contiguous()), M,
+          heads, rank, _ptr(table))
+    return table
+
+
+def window_attention_rib(q, k, v, M: int, shift: int, w1: torch.Tensor, w2: torch.Tensor,
+                         theta: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                         table: Optional[torch.Tensor] = None):
+    """Window attention whose rank-r bias features are generated from the RIB
+    MLP weights in the same call (winattn_fwd_rib); returns (out, table)."""
+    heads, rank = w1.shape[0], w2.shape[3]
+    B, H, W, hq, d = q.shape
+    if table is None:
+        table = torch.empty((heads, 2, M * M, rank), dtype=torch.bfloat16, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    _call(_lib.fwd_rib, "winattn_fwd_rib", q.device, _ptr(q), _ptr(k), _ptr(v), _ptr(theta), _ptr(w1), _ptr(w2), B,
+          H, W, M, shift, heads, d, rank, _dtype_code(q), _ptr(table), _ptr(out))
+    return out, table
+
+
+def cla_gate(x: torch.Tensor, o: torch.Tensor, dw: torch.Tensor, dw_b: torch.Tensor, pw: torch.Tensor,
+             pw_b: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """out = o * sigmoid(PW(DW3x3(x))) (winattn_cla_gate); x, o bf16 [B, H, W, C];
+    dw fp32 [C, 3, 3], dw_b [C], pw [C, C], pw_b [C].  out may be o."""
+    B, H, W, C = x.shape
+    if o.shape != x.shape or not x.is_contiguous() or not o.is_contiguous():
+        raise WinattnError(_lib.ERR_ARG, "x and o must be contiguous [B, H, W, C] tensors")
+    if out is None:
+        out = torch.empty_like(o)
+    _call(_lib.cla_gate, "winattn_cla_gate", x.device, _ptr(x), _ptr(o), _ptr(dw.contiguous()),
+          _ptr(dw_b.contiguous()), _ptr(pw.contiguous()), _ptr(pw_b.contiguous()), B, H, W, C, _dtype_code(x),
+          _ptr(out))
+    return out
 
 
 def window_attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,

@@ -20,7 +20,8 @@ BF16, FP32 = 0, 1
 EXPORTS = ("winattn_fwd", "winattn_fwd_lse", "winattn_check_args", "winattn_fwd_host", "winattn_host_workspace_bytes",
            "winattn_strerror", "winattn_last_device_status", "winattn_launch_info", "winattn_fwd_host_static",
            "winattn_selftest_wait_timeout", "winattn_set_kernel_enabled", "winattn_bwd",
-           "winattn_bwd_workspace_bytes", "winattn_fwd_sparse")
+           "winattn_bwd_workspace_bytes", "winattn_fwd_sparse", "winattn_rib_features", "winattn_fwd_rib",
+           "winattn_cla_gate")
 STATIC_WORKSPACE_BYTES = 32 << 20
 
 
@@ -69,6 +70,12 @@ def load(path: str = LIB_PATH):
     lib.winattn_bwd_workspace_bytes.restype = sz
     lib.winattn_fwd_sparse.argtypes = [vp] * 5 + [i32] * 9 + [vp, i32, vp, vp]
     lib.winattn_fwd_sparse.restype = i32
+    lib.winattn_rib_features.argtypes = [vp, vp, i32, i32, i32, vp, vp]
+    lib.winattn_rib_features.restype = i32
+    lib.winattn_fwd_rib.argtypes = [vp] * 6 + [i32] * 9 + [vp, vp, vp]
+    lib.winattn_fwd_rib.restype = i32
+    lib.winattn_cla_gate.argtypes = [vp] * 6 + [i32] * 5 + [vp, vp]
+    lib.winattn_cla_gate.restype = i32
     lib.winattn_set_kernel_enabled.argtypes = [i32, i32]
     lib.winattn_set_kernel_enabled.restype = i32
     _lib = lib
@@ -106,6 +113,21 @@ def fwd_sparse(q_ptr, k_ptr, v_ptr, theta_ptr, bias_ptr, B, H, W, M, shift, head
                out_ptr, stream) -> int:
     return load().winattn_fwd_sparse(q_ptr, k_ptr, v_ptr, theta_ptr, bias_ptr, B, H, W, M, shift, heads, d, rank,
                                      dtype, win_ptr, n_win, out_ptr, stream)
+
+
+def rib_features(w1_ptr, w2_ptr, M, heads, rank, table_ptr, stream) -> int:
+    return load().winattn_rib_features(w1_ptr, w2_ptr, M, heads, rank, table_ptr, stream)
+
+
+def fwd_rib(q_ptr, k_ptr, v_ptr, theta_ptr, w1_ptr, w2_ptr, B, H, W, M, shift, heads, d, rank, dtype, table_ptr,
+            out_ptr, stream) -> int:
+    return load().winattn_fwd_rib(q_ptr, k_ptr, v_ptr, theta_ptr, w1_ptr, w2_ptr, B, H, W, M, shift, heads, d, rank,
+                                  dtype, table_ptr, out_ptr, stream)
+
+
+def cla_gate(x_ptr, o_ptr, dw_ptr, dwb_ptr, pw_ptr, pwb_ptr, B, H, W, C, dtype, out_ptr, stream) -> int:
+    return load().winattn_cla_gate(x_ptr, o_ptr, dw_ptr, dwb_ptr, pw_ptr, pwb_ptr, B, H, W, C, dtype, out_ptr,
+                                   stream)
 
 
 def check_args(q_ptr, k_ptr, v_ptr, theta_ptr, bias_ptr, B, H, W, M, shift, heads, d, rank, dtype,

@@ -19,6 +19,7 @@
 #include "fwd_small.cuh"
 #include "fwd_tc.cuh"
 #include "geometry.cuh"
+#include "rib_cla.cuh"
 
 namespace winattn {
 
@@ -790,6 +791,78 @@ int winattn_fwd_sparse(const void *q, const void *k, const void *v, const float 
     if (n_windows > g.wph)
         return WINATTN_ERR_ARG;  // windows may not repeat, so at most every window once
     return dispatch_sparse(q, k, v, theta, bias_feats, out, windows, n_windows, g, static_cast<cudaStream_t>(stream));
+}
+
+int winattn_rib_features(const float *w1, const float *w2, int M, int heads, int rank, void *table, void *stream)
+{
+    if (!w1 || !w2 || !table || M <= 0 || M > kMaxM || heads <= 0)
+        return WINATTN_ERR_ARG;
+    if (rank != 16 && rank != 32)
+        return WINATTN_ERR_RANK;
+    if (!aligned16(table) || !aligned16(w1) || !aligned16(w2))
+        return WINATTN_ERR_ALIGN;
+    const int rc = check_device();
+    if (rc != WINATTN_OK)
+        return rc;
+    const dim3 grid((unsigned)((M * M + 127) / 128), (unsigned)(heads * 2));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    auto *t = static_cast<__nv_bfloat16 *>(table);
+    if (rank == 16)
+        winattn_rib_features_kernel<16><<<grid, 128, 0, s>>>(w1, w2, M, t);
+    else
+        winattn_rib_features_kernel<32><<<grid, 128, 0, s>>>(w1, w2, M, t);
+    return cudaGetLastError() == cudaSuccess ? WINATTN_OK : WINATTN_ERR_CUDA;
+}
+
+int winattn_fwd_rib(const void *q, const void *k, const void *v, const float *theta, const float *w1, const float *w2,
+                    int B, int H_img, int W_img, int M, int shift, int heads, int d, int rank, int dtype, void *table,
+                    void *out, void *stream)
+{
+    if (dtype != WINATTN_BF16)
+        return WINATTN_ERR_DTYPE;
+    if (!table)
+        return WINATTN_ERR_ARG;
+    // every argument of the attention is checked before the table is written
+    int rc = winattn_check_args(q, k, v, theta, table, B, H_img, W_img, M, shift, heads, d, rank, dtype, out);
+    if (rc != WINATTN_OK)
+        return rc;
+    const size_t nt = (size_t)heads * 2 * M * M * rank * 2, n = map_bytes(B, H_img, W_img, heads, d, dtype);
+    if (overlaps(table, nt, q, n) || overlaps(table, nt, k, n) || overlaps(table, nt, v, n) ||
+        overlaps(table, nt, out, n))
+        return WINATTN_ERR_ALIAS;
+    rc = winattn_rib_features(w1, w2, M, heads, rank, table, stream);
+    if (rc != WINATTN_OK)
+        return rc;
+    return winattn_fwd(q, k, v, theta, table, B, H_img, W_img, M, shift, heads, d, rank, dtype, out, stream);
+}
+
+int winattn_cla_gate(const void *x, const void *o, const float *dw, const float *dw_b, const float *pw,
+                     const float *pw_b, int B, int H_img, int W_img, int C, int dtype, void *out, void *stream)
+{
+    if (dtype != WINATTN_BF16)
+        return WINATTN_ERR_DTYPE;
+    if (!x || !o || !dw || !dw_b || !pw || !pw_b || !out || B <= 0 || H_img <= 0 || W_img <= 0)
+        return WINATTN_ERR_ARG;
+    if (C < 16 || C > 256 || C % 16)
+        return WINATTN_ERR_ARG;
+    if (!aligned16(x) || !aligned16(o) || !aligned16(out) || (reinterpret_cast<uintptr_t>(dw) & 3u) ||
+        (reinterpret_cast<uintptr_t>(dw_b) & 3u) || (reinterpret_cast<uintptr_t>(pw) & 3u) ||
+        (reinterpret_cast<uintptr_t>(pw_b) & 3u))
+        return WINATTN_ERR_ALIGN;
+    const size_t n = (size_t)B * H_img * W_img * C * 2;
+    if (overlaps(out, n, x, n) || (out != o && overlaps(out, n, o, n)))
+        return WINATTN_ERR_ALIAS;
+    const int rc = check_device();
+    if (rc != WINATTN_OK)
+        return rc;
+    if (!smem_attr_once<winattn_cla_gate_kernel>())
+        return WINATTN_ERR_CUDA;
+    const int64_t tiles = ((int64_t)B * H_img * W_img + 127) / 128;
+    const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+    winattn_cla_gate_kernel<<<grid, 128, GateLayout::bytes(C), static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(o), dw, dw_b, pw, pw_b, B, H_img,
+        W_img, C, static_cast<__nv_bfloat16 *>(out));
+    return cudaGetLastError() == cudaSuccess ? WINATTN_OK : WINATTN_ERR_CUDA;
 }
 
 size_t winattn_bwd_workspace_bytes(int B, int H_img, int W_img, int M, int heads, int d)
