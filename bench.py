@@ -301,6 +301,165 @@ def per_m_table(dev, peaks, target_s=0.25):
     return rows
 
 
+# The backward pass (winattn_bwd) on the training shapes: algorithmic bytes
+# read q, k, v, O, dO and the log-sum-exp once and write dq, dk, dv once;
+# algorithmic flops are the five contractions per pair of a window (S^T, dP^T,
+# dV, dK, dQ), masked pairs included.
+BWD = ["swin", "dense", "flashswin_M32"]
+
+
+def bwd_flops(w):
+    return float(w.tokens) * w.heads * w.N * (6 * (w.d + w.rank) + 4 * w.d)
+
+
+def bwd_bytes(w):
+    return 8.0 * w.tokens * w.heads * w.d * w.elt + 4.0 * w.tokens * w.heads
+
+
+def bwd_table(dev, peaks, target_s=0.25):
+    import torch
+
+    import windowed_attention_vision_b200 as wa
+    from windowed_attention_vision_b200 import inputs as I
+    stream = torch.cuda.current_stream(dev)
+    rows = []
+    for name in BWD:
+        w = I.WORKLOADS[name]
+        (qkv,), theta, bias = I.make_inputs(w, dev)
+        s = w.shifts[-1]
+        lse = torch.empty((w.B, w.H, w.W, w.heads), dtype=torch.float32, device=dev)
+        out = wa.window_attention(*qkv, w.M, s, theta=theta, bias_feats=bias, lse=lse)
+        dout = I.make_map(qkv[0].shape, "bf16", I.seed_for(w.name, "dout"), dev)
+
+        def one():
+            return wa.window_attention_backward(*qkv, out, dout, lse, w.M, s, theta=theta, bias_feats=bias)
+
+        one()
+        torch.cuda.synchronize(dev)
+        t0 = time.perf_counter()
+        one()
+        torch.cuda.synchronize(dev)
+        reps = int(max(3, min(100, target_s / max(time.perf_counter() - t0, 1e-5))))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            one()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        call_s = e0.elapsed_time(e1) / 1e3 / reps
+        flops, nbytes = bwd_flops(w), bwd_bytes(w)
+        ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+        if flops / nbytes < ridge:
+            bound, achieved, peak, unit = "hbm", nbytes / call_s / 1e9, peaks["hbm_gbs"], "GB/s"
+        else:
+            bound, achieved, peak, unit = "tensor", flops / call_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+        rows.append({"workload": name, "M": w.M, "d": w.d, "shift": s, "us_per_call": call_s * 1e6,
+                     "calls_timed": reps, "tflops": flops / call_s / 1e12, "tokens_per_s": w.tokens / call_s,
+                     "gbs": nbytes / call_s / 1e9, "bound": bound, "achieved": achieved, "peak": peak,
+                     "unit": unit, "frac": achieved / peak, "timing": "eager launches, CUDA events"})
+        del qkv, out, dout, lse
+        torch.cuda.empty_cache()
+    return rows
+
+
+def _time_calls(one, dev, target_s=0.25):
+    """Seconds per call of `one` (eager launches, CUDA events, after one
+    untimed call): enough calls to last about target_s."""
+    import torch
+    stream = torch.cuda.current_stream(dev)
+    one()
+    torch.cuda.synchronize(dev)
+    t0 = time.perf_counter()
+    one()
+    torch.cuda.synchronize(dev)
+    reps = int(max(3, min(200, target_s / max(time.perf_counter() - t0, 1e-5))))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    return e0.elapsed_time(e1) / 1e3 / reps, reps
+
+
+def _roof(flops, nbytes, call_s, peaks):
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if flops / nbytes < ridge:
+        return {"bound": "hbm", "achieved": nbytes / call_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": nbytes / call_s / 1e9 / peaks["hbm_gbs"]}
+    return {"bound": "tensor", "achieved": flops / call_s / 1e12, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": flops / call_s / 1e12 / peaks["bf16_tflops"]}
+
+
+def extras_table(dev, peaks):
+    """The rows around the attention: the gated-window residual (HSMLA) on
+    30% of the windows, the RIB factor table and the attention with factors
+    generated in the same call, and the CLA gate, each against its roofline
+    (algorithmic bytes / flops stated per row)."""
+    import math
+
+    import numpy as np
+    import torch
+
+    import windowed_attention_vision_b200 as wa
+    from windowed_attention_vision_b200 import inputs as I
+    rows = []
+    # gated residual: the listed windows' q, k, v read, out read and written;
+    # two contractions per path (softmax and linear) over their pairs
+    for name in ("swin", "dense"):
+        w = I.WORKLOADS[name]
+        (qkv,), theta, _ = I.make_inputs(w, dev)
+        nwin = w.B * (w.H // w.M) * (w.W // w.M)
+        wins = np.sort(np.random.default_rng(0).choice(nwin, int(round(0.3 * nwin)), replace=False))
+        wt = torch.from_numpy(wins.astype(np.int32)).to(dev)
+        frac = len(wins) / nwin
+        o_lin = torch.randn_like(qkv[0].float()).to(torch.bfloat16)
+        s = w.shifts[-1]
+        call_s, reps = _time_calls(lambda: wa.window_attention_gated_residual(*qkv, o_lin, wt, w.M, s, theta=theta),
+                                   dev)
+        flops, nbytes = 2 * w.flops() * frac, 5.0 * w.tokens * w.heads * w.d * 2 * frac
+        rows.append(dict({"row": "gated residual", "workload": name, "windows": f"{len(wins)} of {nwin}",
+                          "us_per_call": call_s * 1e6, "calls_timed": reps,
+                          "tokens_per_s": w.tokens * frac / call_s}, **_roof(flops, nbytes, call_s, peaks)))
+        del qkv, o_lin
+    # RIB factors (SR: M = 96, 6 heads, rank 16): the table alone, then the
+    # attention with the table generated in the same call
+    w = I.WORKLOADS["sr"]
+    g = torch.Generator().manual_seed(0)
+    w1 = (torch.randn((w.heads, 2, 32, 64), generator=g) / math.sqrt(32)).to(dev)
+    w2 = (torch.randn((w.heads, 2, 64, w.rank), generator=g) / math.sqrt(64)).to(dev)
+    table = torch.empty((w.heads, 2, w.N, w.rank), dtype=torch.bfloat16, device=dev)
+    call_s, reps = _time_calls(lambda: wa.rib_features(w1, w2, w.M, table), dev)
+    mlp_flops = w.heads * 2 * w.N * 2 * (32 * 64 + 64 * w.rank)
+    rows.append({"row": "RIB factor table", "workload": "sr (M 96, 6 heads, rank 16)", "us_per_call": call_s * 1e6,
+                 "calls_timed": reps, "mlp_gflops": mlp_flops / 1e9,
+                 "note": "fp32 CUDA-core MLP, once per call; a few microseconds next to the attention"})
+    (qkv,), _, _ = I.make_inputs(w, dev)
+    out = torch.empty_like(qkv[0])
+    call_s, reps = _time_calls(lambda: wa.window_attention_rib(*qkv, w.M, 0, w1, w2, out=out, table=table), dev)
+    rows.append(dict({"row": "attention with generated RIB factors", "workload": "sr", "us_per_call": call_s * 1e6,
+                      "calls_timed": reps, "tokens_per_s": w.tokens / call_s},
+                     **_roof(w.flops(), w.bytes(), call_s, peaks)))
+    del qkv, out
+    # CLA gate: x and O read once, out written once; 2 C^2 flops per token
+    for name, (B, H, W, C) in (("sr", (4, 192, 192, 192)), ("swin", (64, 56, 56, 96))):
+        x = torch.randn((B, H, W, C), device=dev).to(torch.bfloat16)
+        o = torch.randn_like(x)
+        dw = torch.randn((C, 3, 3), device=dev) / 3
+        dwb = torch.zeros(C, device=dev)
+        pw = torch.randn((C, C), device=dev) / math.sqrt(C)
+        pwb = torch.zeros(C, device=dev)
+        out = torch.empty_like(x)
+        call_s, reps = _time_calls(lambda: wa.cla_gate(x, o, dw, dwb, pw, pwb, out=out), dev)
+        T = B * H * W
+        rows.append(dict({"row": "CLA gate", "workload": f"{name} (B{B}, {H}x{W}, C {C})",
+                          "us_per_call": call_s * 1e6, "calls_timed": reps, "tokens_per_s": T / call_s},
+                         **_roof(2.0 * T * C * C, 3.0 * T * C * 2, call_s, peaks)))
+        del x, o, out
+    torch.cuda.empty_cache()
+    return rows
+
+
 def max_over_ranks(values, device):
     """Element-wise maximum of per-rank timings over all ranks (every rank
     calls it at the same point; the job is as slow as its slowest rank)."""
@@ -492,6 +651,8 @@ def run_ours(args):
                 "clocks": clocks.summary(), "e2e": e2e, "device_status": status}
         if not args.no_per_m:
             line["per_M"] = per_m_table(dev, peaks)
+            line["backward"] = bwd_table(dev, peaks)
+            line["extras"] = extras_table(dev, peaks)
         if world == 1 and not args.no_cpu_baseline:
             rate, sample, cores, _ = oracle_sample_rate(w, args.cpu_seconds)
             line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
