@@ -61,6 +61,9 @@ extern "C" {
 #define WINATTN_ERR_ALIAS          -8  /* out overlaps q, k or v                               */
 #define WINATTN_ERR_SIZE           -9  /* a size product overflows the kernel's index range,
                                           or a host workspace is too small                     */
+#define WINATTN_ERR_DEVICE_BOUNDS -10  /* debug builds (-DWINATTN_DEBUG) only: a kernel formed a
+                                          token index or TMA box origin outside the map (the
+                                          access was clamped into the map instead)            */
 
 /* Storage / arithmetic types of q, k, v, bias_feats and out. */
 #define WINATTN_BF16 0  /* bf16 storage; tensor-core QK^T and PV (bf16 in, fp32 accumulate),
@@ -342,7 +345,8 @@ const char *winattn_strerror(int code);
  * winattn_last_device_status — synchronises `stream`, then reads and clears
  * the current device's status word.  Returns WINATTN_OK when no kernel has
  * given up a bounded wait since the last read, WINATTN_ERR_DEVICE_TIMEOUT
- * when one has, or WINATTN_ERR_CUDA if the synchronisation failed.
+ * when one has, WINATTN_ERR_DEVICE_BOUNDS when a debug build found an index
+ * outside the map, or WINATTN_ERR_CUDA if the synchronisation failed.
  */
 int winattn_last_device_status(void *stream);
 

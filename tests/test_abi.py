@@ -77,7 +77,7 @@ def test_check_args_rejects(lib, kw, code):
 
 
 def test_strerror_covers_codes(lib):
-    for code in range(-9, 1):
+    for code in range(-10, 1):
         s = _lib.strerror(code)
         assert s and s != "unknown error code"
     assert _lib.strerror(-100) == "unknown error code"

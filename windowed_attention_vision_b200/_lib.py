@@ -10,11 +10,14 @@ import ctypes
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libwinattn.so")
+# WINATTN_LIB selects another build of the library, e.g. the bounds-checking
+# debug build (libwinattn_debug.so, made by build.build(debug=True))
+LIB_PATH = os.environ.get("WINATTN_LIB") or os.path.join(HERE, "libwinattn.so")
+DEBUG_LIB_PATH = os.path.join(HERE, "libwinattn_debug.so")
 
 OK = 0
 ERR_ARG, ERR_RANK, ERR_ALIGN, ERR_DTYPE, ERR_ARCH = -1, -2, -3, -4, -5
-ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_ALIAS, ERR_SIZE = -6, -7, -8, -9
+ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_ALIAS, ERR_SIZE, ERR_DEVICE_BOUNDS = -6, -7, -8, -9, -10
 BF16, FP32 = 0, 1
 
 EXPORTS = ("winattn_fwd", "winattn_fwd_lse", "winattn_check_args", "winattn_fwd_host", "winattn_host_workspace_bytes",
@@ -33,6 +36,7 @@ class WinattnError(RuntimeError):
 
 
 _lib = None
+loaded_path = None  # the library file this process loaded
 
 
 def load(path: str = LIB_PATH):
@@ -43,6 +47,8 @@ def load(path: str = LIB_PATH):
     if not os.path.exists(path):
         raise WinattnError(ERR_CUDA, f"CUDA library {path} is missing; run __graft_entry__.build()")
     lib = ctypes.CDLL(path)
+    global loaded_path
+    loaded_path = path
     vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
     lib.winattn_fwd.argtypes = [vp, vp, vp, vp, vp] + [i32] * 9 + [vp, vp]
     lib.winattn_fwd.restype = i32

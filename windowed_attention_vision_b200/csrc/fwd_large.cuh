@@ -383,8 +383,10 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
                         // fill value; they are masked in the softmax
                         int y0 = wy * M + jt * kr + g.shift;
                         if (y0 >= g.Hp) y0 -= g.Hp;
-                        const int x0 = wx * M + g.shift;  // < Wp unless the window straddles the seam
-                        const int c0 = h * D;
+                        int x0 = wx * M + g.shift;  // < Wp unless the window straddles the seam
+                        int c0 = h * D;
+                        // boxes of a padded grid may reach past H, W (fill), never past Hp, Wp
+                        debug_box(c0, x0, y0, b, D, g.heads * D, xwrap ? M / 2 : M, kr, g.Wp, g.Hp, g.B);
                         if (xwrap) {
                             const int x1 = 0;             // the seam's far side
                             const uint32_t half = (uint32_t)(BN / 2) * 2 * D;
@@ -400,6 +402,12 @@ __global__ void __launch_bounds__(kLargeThreads, 1)
                             tma_load_2d(sst + L::KB, &maps.w, 0, (h * 2 + 1) * N + jt * BN, &kv_full[s]);
                     }
                 }
+                // after an abort no consumer may take the stages armed last:
+                // wait (bounded) until their loads have landed, so none is
+                // still writing shared memory when the CTA exits
+                if (*abort_flag)
+                    for (int c2 = c > NS ? c - NS : 0; c2 < c; ++c2)
+                        mbar_wait(&kv_full[c2 % NS], (c2 / NS) & 1);
             }
         } else if (warp == 13) {
             // ============================================================ S issuer

@@ -219,6 +219,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         r.roff = (uint32_t)((my_slot * 64 + bi * (64 / nbox)) * 2 * D);
         r.c0 = it.h * D;
         r.go = true;
+        debug_box(r.c0, r.x0, r.y0, r.b, D, g.heads * D, (r.kind & 1) ? 4 : 8, (r.kind & 2) ? 4 : 8, g.W, g.H, g.B);
         return r;
     };
     auto valid_windows = [&](const Item &it) -> int {
@@ -230,7 +231,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         // ================================================================ Q/K loader
         // (starts right after the CTA barrier: the first tiles' DRAM latency
         // overlaps the RoPE warps' table setup)
-        for (int kk = 0; kk < count; ++kk) {
+        int kk = 0;
+        for (; kk < count; ++kk) {
             const int s = kk % NSQ;
             if (kk >= NSQ && !warp_wait(&qk_empty[s], ((kk / NSQ) - 1) & 1, abort_flag))
                 break;
@@ -246,9 +248,16 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
                 tma_load_4d(sst + L::KC + r.roff, pick_map(tm_k, r.kind), r.c0, r.x0, r.y0, r.b, &qk_full[s]);
             }
         }
+        // after an abort no consumer may take the stages armed last: wait
+        // (bounded) until their loads have landed before the CTA exits
+        if (*abort_flag && lane == 0)
+            for (int k2 = kk > NSQ ? kk - NSQ : 0; k2 < kk; ++k2)
+                mbar_wait(&qk_full[k2 % NSQ], (k2 / NSQ) & 1);
+        __syncwarp();
     } else if (warp == kPipeLoadWarp + 3) {
         // ================================================================ V loader
-        for (int kk = 0; kk < count; ++kk) {
+        int kk = 0;
+        for (; kk < count; ++kk) {
             const int s = kk % NSV;
             // once the tile's RoPE is done, V has about the S and softmax
             // time to arrive before P V needs it
@@ -275,6 +284,10 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
             if (r.go)
                 tma_load_4d(sst + r.roff, pick_map(tm_v, r.kind), r.c0, r.x0, r.y0, r.b, &v_full[s]);
         }
+        if (*abort_flag && lane == 0)
+            for (int k2 = kk > NSV ? kk - NSV : 0; k2 < kk; ++k2)
+                mbar_wait(&v_full[k2 % NSV], (k2 / NSV) & 1);
+        __syncwarp();
     } else if (warp == kPipeLoadWarp + 1) {
         // ================================================================ S issuer
         // S = Q K^T of each tile into TMEM buffer k % 4 as soon as its RoPE is
@@ -533,8 +546,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
             tc_fence_after_sync();
             // read before the buffer is released: the slot is rewritten only
             // after S of tile kk + 4, which needs this buffer back
-            const int4 rec = lane < 2 ? reinterpret_cast<const int4 *>(base + L::MRING + m * L::MSLOT + 1024)[quarter * 2 + lane]
-                                      : make_int4(0, 0, 0, -1);
+            int4 rec = lane < 2 ? reinterpret_cast<const int4 *>(base + L::MRING + m * L::MSLOT + 1024)[quarter * 2 + lane]
+                                : make_int4(0, 0, 0, -1);
             const float lrow = osum[b * 128 + row];
             const float inv = 1.f / lrow;
             const float2 i2 = make_float2(inv, inv);
@@ -587,6 +600,14 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (rec.w >= 0) {
+#ifdef WINATTN_DEBUG
+                {
+                    int c0 = rec.w >> 4, x0 = rec.x, y0 = rec.y, bb = rec.z;
+                    const int shp = rec.w & 3;
+                    debug_box(c0, x0, y0, bb, D, g.heads * D, shp == 2 ? 8 : 4, shp == 1 ? 8 : 4, g.W, g.H, g.B);
+                    rec = make_int4(x0, y0, bb, shp | (c0 << 4));
+                }
+#endif
                 const int shape = rec.w & 3;
                 const CUtensorMap *map = shape == 3 ? &tm_o.quarter : (shape == 1 ? &tm_o.xhalf : &tm_o.yhalf);
                 tma_store_4d(map, sbase + L::OSTAGE + e * 256 * D + (uint32_t)((quarter * 32 + lane * 16) * 2 * D),

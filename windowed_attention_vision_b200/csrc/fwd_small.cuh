@@ -328,10 +328,13 @@ __global__ void __launch_bounds__(SmallRoles<D>::kThreads, 1)
                     int x0 = wx * M + jx0 + g.shift;
                     if (x0 >= g.W) x0 -= g.W;
                     const uint32_t roff = (uint32_t)((my_slot * g.N + bi * (g.N / nbox)) * 2 * D);
-                    const int c0 = it.h * D;
-                    tma_load_4d(sst + L::QC + roff, pick_map(tm_q, kind), c0, x0, y0, b, &full[s]);
-                    tma_load_4d(sst + L::KC + roff, pick_map(tm_k, kind), c0, x0, y0, b, &full[s]);
-                    tma_load_4d(sst + L::VO + roff, pick_map(tm_v, kind), c0, x0, y0, b, &full[s]);
+                    int c0 = it.h * D;
+                    int bb = b;
+                    debug_box(c0, x0, y0, bb, D, g.heads * D, (kind & 1) ? hm : M, (kind & 2) ? hm : M, g.W, g.H,
+                              g.B);
+                    tma_load_4d(sst + L::QC + roff, pick_map(tm_q, kind), c0, x0, y0, bb, &full[s]);
+                    tma_load_4d(sst + L::KC + roff, pick_map(tm_k, kind), c0, x0, y0, bb, &full[s]);
+                    tma_load_4d(sst + L::VO + roff, pick_map(tm_v, kind), c0, x0, y0, bb, &full[s]);
                 }
             }
         }

@@ -27,6 +27,22 @@
 
 namespace winattn {
 
+#if defined(WINATTN_DEBUG) && defined(__CUDA_ARCH__)
+// Debug builds (-DWINATTN_DEBUG) check every index formed here and every TMA
+// box origin against the map; a violation sets kStatusBounds in the device
+// status word (read by winattn_last_device_status) and the access is clamped
+// into the map instead of trapping.
+extern __device__ unsigned int g_status_word;
+constexpr unsigned int kStatusBounds = 2u;
+__device__ __forceinline__ bool debug_in_range(int64_t v, int64_t lo, int64_t hi)
+{
+    if (v >= lo && v < hi)
+        return true;
+    atomicOr(&g_status_word, kStatusBounds);
+    return false;
+}
+#endif
+
 constexpr int kTileRows = 128;  // rows of a query tile / key tile (UMMA M and N)
 
 // Division by a fixed divisor d >= 1 for dividends n < 2^31: with
@@ -176,6 +192,16 @@ __host__ __device__ inline TokenRef token_ref(const Geometry &g, int w, int p, i
     t.label = g.shift ? 2 * (yr >= g.Hp - g.shift) + (xr >= g.Wp - g.shift) : 0;
     t.pad = y >= g.H || x >= g.W;
     t.offset = t.pad ? 0 : ((((int64_t)b * g.H + y) * g.W + x) * g.heads + h) * g.d;
+#if defined(WINATTN_DEBUG) && defined(__CUDA_ARCH__)
+    // the (b, y, x, h) the index math formed lies in the (padded) map, the
+    // window-local (i, j) in the window
+    if (!debug_in_range(b, 0, g.B) || !debug_in_range(y, 0, g.Hp) || !debug_in_range(x, 0, g.Wp) ||
+        !debug_in_range(h, 0, g.heads) || !debug_in_range(t.i, 0, g.M) || !debug_in_range(t.j, 0, g.M) ||
+        !debug_in_range(t.offset, 0, (int64_t)g.B * g.H * g.W * g.heads * g.d)) {
+        t.offset = 0;
+        t.pad = true;
+    }
+#endif
     return t;
 }
 

@@ -97,6 +97,25 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
 
 // ------------------------------------------------------------------ TMA
 
+// Debug builds: a box of bw x bh tokens at (c0, x0, y0, b) of a map with C
+// channels, W x H tokens (xlim, ylim: the extent the box may reach, the
+// padded grid for loads of padded problems) and B images must start on a
+// 16-byte channel boundary inside the map; otherwise the status word gets
+// its bounds bit and the origin is moved to (0, 0, 0, 0).
+__device__ __forceinline__ void debug_box(int &c0, int &x0, int &y0, int &b, int D, int C, int bw, int bh, int xlim,
+                                          int ylim, int B)
+{
+#ifdef WINATTN_DEBUG
+    if (c0 < 0 || (c0 & 7) || c0 + D > C || x0 < 0 || x0 + bw > xlim || y0 < 0 || y0 + bh > ylim || b < 0 ||
+        b >= B) {
+        atomicOr(&g_status_word, 2u);
+        c0 = x0 = y0 = b = 0;
+    }
+#else
+    (void)c0; (void)x0; (void)y0; (void)b; (void)D; (void)C; (void)bw; (void)bh; (void)xlim; (void)ylim; (void)B;
+#endif
+}
+
 // Tiled 4-D tensor load (no multicast) into this CTA's shared memory; the
 // bytes are counted on *bar.  The innermost coordinate c0 times the element
 // size must be a multiple of 16 bytes.

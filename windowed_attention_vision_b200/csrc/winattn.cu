@@ -1139,6 +1139,7 @@ const char *winattn_strerror(int code)
     case WINATTN_ERR_DEVICE_TIMEOUT: return "a bounded wait inside a kernel timed out";
     case WINATTN_ERR_ALIAS: return "out overlaps q, k or v";
     case WINATTN_ERR_SIZE: return "problem too large for the index range, or workspace too small";
+    case WINATTN_ERR_DEVICE_BOUNDS: return "a debug build found an index or TMA box outside the map";
     }
     return "unknown error code";
 }
@@ -1154,7 +1155,7 @@ int winattn_last_device_status(void *stream)
         const unsigned int zero = 0;
         if (cudaMemcpyToSymbol(g_status_word, &zero, sizeof zero) != cudaSuccess)
             return WINATTN_ERR_CUDA;
-        return WINATTN_ERR_DEVICE_TIMEOUT;
+        return (word & 1u) ? WINATTN_ERR_DEVICE_TIMEOUT : WINATTN_ERR_DEVICE_BOUNDS;
     }
     return WINATTN_OK;
 }
