@@ -7,9 +7,9 @@
 // the forward, no N x N matrix is ever stored: P is recomputed per tile as
 // exp(z - lse).
 //
-// One CTA of 128 threads owns one 128-row key tile of a window (or of a pack
-// of small windows); thread t owns key row t.  Per 128-row query tile of the
-// same window:
+// One CTA of 256 threads owns one 128-row key tile of a window (or of a pack
+// of small windows); two threads own key row t (see the kernel).  Per
+// 128-row query tile of the same window:
 //   1. gather: query row t rotated by window-local 2D RoPE in fp32, scaled by
 //      d^-1/2 and rounded to bf16 (with its factors u unscaled), dO row t,
 //      D_t = dO_t . O_t and the saved log-sum-exp;
@@ -55,8 +55,8 @@ struct BwdLayout {
     static constexpr uint32_t QI = DS + 32768;            // per query row: lse (log2 units), D, code
     static constexpr uint32_t TB = QI + 128 * 12;         // RoPE table [M][D/4] float2
     static __host__ __device__ uint32_t table_bytes(int M) { return (uint32_t)((M * (D / 4) * 8 + 15) & ~15); }
-    static __host__ __device__ uint32_t red(int M) { return TB + table_bytes(M); }            // f32 [4 warps][D/4]
-    static __host__ __device__ uint32_t bar(int M) { return red(M) + 4 * (D / 4) * 4; }       // u64
+    static __host__ __device__ uint32_t red(int M) { return TB + table_bytes(M); }            // f32 [8 warps][D/4]
+    static __host__ __device__ uint32_t bar(int M) { return red(M) + 8 * (D / 4) * 4; }       // u64
     static __host__ __device__ uint32_t tslot(int M) { return bar(M) + 8; }                   // u32
     static __host__ __device__ uint32_t bytes(int M) { return tslot(M) + 16 + 1024; }
 };
@@ -136,9 +136,9 @@ __device__ __forceinline__ void store_bf16_row(__nv_bfloat16 *dst, const float (
                            pack_bf16x2(x[8 * c + 4], x[8 * c + 5]), pack_bf16x2(x[8 * c + 6], x[8 * c + 7]));
 }
 
-// Sum of dth[k] over the CTA's 128 threads, added to dtheta[k] (one
-// reduction per frequency and CTA).
-template <int D>
+// Sum of dth[k] over the CTA's NW warps, added to dtheta[k] (one reduction
+// per frequency and CTA).
+template <int D, int NW>
 __device__ __forceinline__ void cta_add_dtheta(float (&dth)[D / 4], float *red_smem, float *dtheta_h)
 {
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
@@ -152,13 +152,94 @@ __device__ __forceinline__ void cta_add_dtheta(float (&dth)[D / 4], float *red_s
             red_smem[warp * (D / 4) + k] = v;
     }
     __syncthreads();
-    if (t < D / 4)
-        atomicAdd(dtheta_h + t, red_smem[t] + red_smem[D / 4 + t] + red_smem[2 * (D / 4) + t] +
-                                    red_smem[3 * (D / 4) + t]);
+    if (t < D / 4) {
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w)
+            sum += red_smem[w * (D / 4) + t];
+        atomicAdd(dtheta_h + t, sum);
+    }
 }
 
+// One half (dims [HALF * D/2, HALF * D/2 + D/2)) of a d-vector (bf16), in
+// fp32, rotated by R(i, j) when a table is given: the first half turns by
+// i theta_k, the second by j theta_k, k < D/4.
+template <int D>
+__device__ __forceinline__ void load_half_rotated(const __nv_bfloat16 *__restrict__ src, const float2 *table,
+                                                  int half, int i, int j, float (&x)[D / 2])
+{
+    const uint4 *s4 = reinterpret_cast<const uint4 *>(src + half * (D / 2));
+#pragma unroll
+    for (int c = 0; c < D / 16; ++c) {
+        const uint4 u = __ldg(s4 + c);
+        x[8 * c + 0] = bf16lo(u.x); x[8 * c + 1] = bf16hi(u.x);
+        x[8 * c + 2] = bf16lo(u.y); x[8 * c + 3] = bf16hi(u.y);
+        x[8 * c + 4] = bf16lo(u.z); x[8 * c + 5] = bf16hi(u.z);
+        x[8 * c + 6] = bf16lo(u.w); x[8 * c + 7] = bf16hi(u.w);
+    }
+    if (table) {
+        const int pos = half ? j : i;
+#pragma unroll
+        for (int k = 0; k < D / 4; ++k) {
+            const float2 r = table[pos * (D / 4) + k];
+            const float a0 = x[2 * k], a1 = x[2 * k + 1];
+            x[2 * k] = a0 * r.x - a1 * r.y;
+            x[2 * k + 1] = a0 * r.y + a1 * r.x;
+        }
+    }
+}
+
+// The gradient g = dL/d(R x) of one half of a rotated vector x~ (the half's
+// pairs all turn by pos theta_k, pos = i for the first half, j for the
+// second): adds pos (g1 x~0 - g0 x~1) to dth[k] and turns g back by
+// R(-pos theta_k) in place.
+template <int D>
+__device__ __forceinline__ void unrotate_half(float (&g)[D / 2], const float (&xr)[D / 2], const float2 *table, int pos,
+                                              float (&dth)[D / 4])
+{
+#pragma unroll
+    for (int k = 0; k < D / 4; ++k) {
+        const int a0 = 2 * k, a1 = 2 * k + 1;
+        dth[k] += (float)pos * (g[a1] * xr[a0] - g[a0] * xr[a1]);
+        const float2 r = table[pos * (D / 4) + k];
+        // R(-a) (g0, g1) = (g0 cos a + g1 sin a, -g0 sin a + g1 cos a)
+        const float y0 = g[a0] * r.x + g[a1] * r.y, y1 = g[a1] * r.x - g[a0] * r.y;
+        g[a0] = y0;
+        g[a1] = y1;
+    }
+}
+
+template <int N>
+__device__ __forceinline__ void store_bf16_vec(__nv_bfloat16 *dst, const float (&x)[N])
+{
+    uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+    for (int c = 0; c < N / 8; ++c)
+        d4[c] = make_uint4(pack_bf16x2(x[8 * c + 0], x[8 * c + 1]), pack_bf16x2(x[8 * c + 2], x[8 * c + 3]),
+                           pack_bf16x2(x[8 * c + 4], x[8 * c + 5]), pack_bf16x2(x[8 * c + 6], x[8 * c + 7]));
+}
+
+// N consecutive fp32 TMEM columns of this thread's lane (16 or 32).
+template <int N>
+__device__ __forceinline__ void tmem_ldn(uint32_t taddr, float (&v)[N])
+{
+    static_assert(N == 16 || N == 32, "16 or 32 columns");
+    if constexpr (N == 16)
+        tmem_ld16(taddr, v);
+    else
+        tmem_ld32(taddr, v);
+}
+
+constexpr int kBwdThreads = 256;
+
+// 256 threads: thread (half, t) with t = tid % 128 owns key row t (and query
+// row t of the current query tile); the two halves split the gathers (K~, w
+// | V; Q~, u | dO, D, lse), the query columns of the P / dS pass, and the two
+// halves of the head dim when gradients leave (the RoPE pairs of a half turn
+// by one coordinate, i or j).  Warps w and w + 4 share TMEM lane quarter
+// w % 4 and read different columns of it.
 template <int D, int R>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kBwdThreads)
     winattn_bwd_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                           const __nv_bfloat16 *__restrict__ v, const float *__restrict__ theta,
                           const __nv_bfloat16 *__restrict__ bias, const __nv_bfloat16 *__restrict__ o,
@@ -168,6 +249,7 @@ __global__ void __launch_bounds__(128)
                           float *__restrict__ dq_acc, const Geometry g, const float scale)
 {
     using L = BwdLayout<D, R>;
+    constexpr int DH = D / 2;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(base);
@@ -179,7 +261,8 @@ __global__ void __launch_bounds__(128)
     uint64_t *bar = reinterpret_cast<uint64_t *>(base + L::bar(g.M));
     uint32_t *tslot = reinterpret_cast<uint32_t *>(base + L::tslot(g.M));
 
-    const int t = threadIdx.x, warp = t >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int t = tid & 127, half = tid >> 7;
     // a single query tile per window: the gradient accumulators reuse the
     // S^T / dP^T columns (256 columns, two CTAs per SM); otherwise dV and dK~
     // live past column 256
@@ -192,14 +275,14 @@ __global__ void __launch_bounds__(128)
         tmem_alloc(tslot, ncols);
         tmem_relinquish();
     }
-    if (t == 0) {
+    if (tid == 0) {
         mbar_init(bar, 1);
         fence_mbar_init();
     }
     const Item it = decode_item(g, blockIdx.x);
     const int kt = it.tile;
     if (theta) {
-        for (int idx = t; idx < g.M * (D / 4); idx += blockDim.x) {
+        for (int idx = tid; idx < g.M * (D / 4); idx += kBwdThreads) {
             const int c = idx / (D / 4), kk = idx - c * (D / 4);
             float sn, cs;
             sincosf((float)c * __ldg(theta + it.h * (D / 4) + kk), &sn, &cs);
@@ -210,28 +293,33 @@ __global__ void __launch_bounds__(128)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *tslot;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const float2 *tab = theta ? table : nullptr;
     float dth[D / 4];
 #pragma unroll
     for (int e = 0; e < D / 4; ++e)
         dth[e] = 0.f;
 
-    // ---- key row t: K~ (rotated, bf16), w, V; its mask code
+    // ---- key row t: K~ (rotated, bf16) and w | V; its mask code
     const RowRef kr = tile_row(g, it.pack, kt, t);
     const TokenRef ktk = kr.valid ? token_ref(g, kr.w, kr.p, it.h) : TokenRef{};
     const bool kreal = kr.valid && !ktk.pad;
     const uint32_t kcode = kreal ? (uint32_t)((kr.slot << 2) | ktk.label) : 0xFFFEu;
-    if (kreal) {
-        gather_rotate_store<D>(k + ktk.offset, tab, ktk.i, ktk.j, 1.f, base + L::KT, t);
-        if constexpr (R > 0)
-            copy_row<R>(bias + (((int64_t)it.h * 2 + 1) * g.N + kr.p) * R, base + L::KB, t);
-        copy_row<D>(v + ktk.offset, base + L::VT, t);
+    if (half == 0) {
+        if (kreal) {
+            gather_rotate_store<D>(k + ktk.offset, tab, ktk.i, ktk.j, 1.f, base + L::KT, t);
+            if constexpr (R > 0)
+                copy_row<R>(bias + (((int64_t)it.h * 2 + 1) * g.N + kr.p) * R, base + L::KB, t);
+        } else {
+            zero_row<D>(base + L::KT, t);
+            if constexpr (R > 0)
+                zero_row<R>(base + L::KB, t);
+        }
     } else {
-        zero_row<D>(base + L::KT, t);
-        if constexpr (R > 0)
-            zero_row<R>(base + L::KB, t);
-        zero_row<D>(base + L::VT, t);
+        if (kreal)
+            copy_row<D>(v + ktk.offset, base + L::VT, t);
+        else
+            zero_row<D>(base + L::VT, t);
     }
 
     constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false);
@@ -244,14 +332,21 @@ __global__ void __launch_bounds__(128)
     bool ok = true;
 
     for (int qt = 0; qt < g.n_tiles && ok; ++qt) {
-        // ---- 1. query row t: Q~, u, dO, D = dO . O, lse, mask code
+        // ---- 1. query row t: Q~, u | dO, D = dO . O, lse, mask code
         const RowRef qr = tile_row(g, it.pack, qt, t);
         const TokenRef qtk = qr.valid ? token_ref(g, qr.w, qr.p, it.h) : TokenRef{};
         const bool qreal = qr.valid && !qtk.pad;
-        if (qreal) {
-            gather_rotate_store<D>(q + qtk.offset, tab, qtk.i, qtk.j, scale, base + L::QT, t);
-            if constexpr (R > 0)
-                copy_row<R>(bias + (((int64_t)it.h * 2 + 0) * g.N + qr.p) * R, base + L::QB, t);
+        if (half == 0) {
+            if (qreal) {
+                gather_rotate_store<D>(q + qtk.offset, tab, qtk.i, qtk.j, scale, base + L::QT, t);
+                if constexpr (R > 0)
+                    copy_row<R>(bias + (((int64_t)it.h * 2 + 0) * g.N + qr.p) * R, base + L::QB, t);
+            } else {
+                zero_row<D>(base + L::QT, t);
+                if constexpr (R > 0)
+                    zero_row<R>(base + L::QB, t);
+            }
+        } else if (qreal) {
             copy_row<D>(dout + qtk.offset, base + L::OT, t);
             const uint4 *o4 = reinterpret_cast<const uint4 *>(o + qtk.offset);
             const uint4 *g4 = reinterpret_cast<const uint4 *>(dout + qtk.offset);
@@ -267,9 +362,6 @@ __global__ void __launch_bounds__(128)
             q_lse[t] = __ldg(lse + qtk.offset / D) * kLog2e;
             q_code[t] = (uint32_t)((qr.slot << 2) | qtk.label);
         } else {
-            zero_row<D>(base + L::QT, t);
-            if constexpr (R > 0)
-                zero_row<R>(base + L::QB, t);
             zero_row<D>(base + L::OT, t);
             q_dd[t] = 0.f;
             q_lse[t] = 0.f;
@@ -280,7 +372,7 @@ __global__ void __launch_bounds__(128)
         __syncthreads();
 
         // ---- 2. S^T = K~ Q~^T, dP^T = V dO^T
-        if (t == 0) {
+        if (tid == 0) {
             tc_fence_after_sync();
 #pragma unroll
             for (int ks = 0; ks < D / 16; ++ks) {
@@ -310,9 +402,9 @@ __global__ void __launch_bounds__(128)
         }
         tc_fence_after_sync();
 
-        // ---- 3. P^T and dS^T of key row t, 32 queries at a time
+        // ---- 3. P^T and dS^T of key row t: this half's 64 queries, 32 at a time
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 2 * half; c < 2 * half + 2; ++c) {
             float s[32], dp[32];
             tmem_ld32(tmem + lane_off + cST + c * 32, s);
             tmem_ld32(tmem + lane_off + cDP + c * 32, dp);
@@ -347,7 +439,7 @@ __global__ void __launch_bounds__(128)
         __syncthreads();
 
         // ---- 4. dV += P^T dO, dK~ += dS^T Q~, dQ~ = dS K~
-        if (t == 0) {
+        if (tid == 0) {
             tc_fence_after_sync();
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
@@ -386,12 +478,10 @@ __global__ void __launch_bounds__(128)
         }
         tc_fence_after_sync();
 
-        // ---- 5. dQ~ of query row t (TMEM lane t)
+        // ---- 5. dQ~ of query row t (TMEM lane t): this half's head dims
         {
-            float gq[D];
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c)
-                tmem_ld32(tmem + lane_off + cDQ + c * 32, gq + c * 32);
+            float gq[DH];
+            tmem_ldn<DH>(tmem + lane_off + cDQ + half * DH, gq);
             float gu[R > 0 ? R : 1];
             if constexpr (R == 16)
                 tmem_ld16(tmem + lane_off + cDQ + D, gu);
@@ -399,25 +489,27 @@ __global__ void __launch_bounds__(128)
                 tmem_ld32(tmem + lane_off + cDQ + D, gu);
             if (qreal) {
                 if constexpr (R > 0) {
-                    float *du = dbias + (((int64_t)it.h * 2 + 0) * g.N + qr.p) * R;
+                    if (half == 0) {
+                        float *du = dbias + (((int64_t)it.h * 2 + 0) * g.N + qr.p) * R;
 #pragma unroll
-                    for (int e = 0; e < R; e += 4)
-                        red_add_v4(du + e, gu[e], gu[e + 1], gu[e + 2], gu[e + 3]);
+                        for (int e = 0; e < R; e += 4)
+                            red_add_v4(du + e, gu[e], gu[e + 1], gu[e + 2], gu[e + 3]);
+                    }
                 }
                 if (single) {
 #pragma unroll
-                    for (int e = 0; e < D; ++e)
+                    for (int e = 0; e < DH; ++e)
                         gq[e] *= scale;
                     if (tab) {
-                        float xr[D];
-                        load_rotated_f32<D>(q + qtk.offset, tab, qtk.i, qtk.j, xr);
-                        unrotate_grad<D>(gq, xr, tab, qtk.i, qtk.j, dth);
+                        float xr[DH];
+                        load_half_rotated<D>(q + qtk.offset, tab, half, qtk.i, qtk.j, xr);
+                        unrotate_half<D>(gq, xr, tab, half ? qtk.j : qtk.i, dth);
                     }
-                    store_bf16_row<D>(dq + qtk.offset, gq);
+                    store_bf16_vec<DH>(dq + qtk.offset + half * DH, gq);
                 } else {
-                    float *acc = dq_acc + qtk.offset;
+                    float *acc = dq_acc + qtk.offset + half * DH;
 #pragma unroll
-                    for (int e = 0; e < D; e += 4)
+                    for (int e = 0; e < DH; e += 4)
                         red_add_v4(acc + e, gq[e], gq[e + 1], gq[e + 2], gq[e + 3]);
                 }
             }
@@ -428,37 +520,36 @@ __global__ void __launch_bounds__(128)
         tc_fence_after_sync();
     }
 
-    // ---- dV, dK of key row t
+    // ---- dV, dK of key row t: this half's head dims
     if (ok) {
-        float gv[D], gk[D];
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-            tmem_ld32(tmem + lane_off + cDV + c * 32, gv + c * 32);
-            tmem_ld32(tmem + lane_off + cDK + c * 32, gk + c * 32);
-        }
+        float gv[DH], gk[DH];
+        tmem_ldn<DH>(tmem + lane_off + cDV + half * DH, gv);
+        tmem_ldn<DH>(tmem + lane_off + cDK + half * DH, gk);
         float gw[R > 0 ? R : 1];
         if constexpr (R == 16)
             tmem_ld16(tmem + lane_off + cDK + D, gw);
         if constexpr (R == 32)
             tmem_ld32(tmem + lane_off + cDK + D, gw);
         if (kreal) {
-            store_bf16_row<D>(dv + ktk.offset, gv);
+            store_bf16_vec<DH>(dv + ktk.offset + half * DH, gv);
             if (tab) {
-                float xr[D];
-                load_rotated_f32<D>(k + ktk.offset, tab, ktk.i, ktk.j, xr);
-                unrotate_grad<D>(gk, xr, tab, ktk.i, ktk.j, dth);
+                float xr[DH];
+                load_half_rotated<D>(k + ktk.offset, tab, half, ktk.i, ktk.j, xr);
+                unrotate_half<D>(gk, xr, tab, half ? ktk.j : ktk.i, dth);
             }
-            store_bf16_row<D>(dk + ktk.offset, gk);
+            store_bf16_vec<DH>(dk + ktk.offset + half * DH, gk);
             if constexpr (R > 0) {
-                float *dw = dbias + (((int64_t)it.h * 2 + 1) * g.N + kr.p) * R;
+                if (half == 0) {
+                    float *dw = dbias + (((int64_t)it.h * 2 + 1) * g.N + kr.p) * R;
 #pragma unroll
-                for (int e = 0; e < R; e += 4)
-                    red_add_v4(dw + e, gw[e], gw[e + 1], gw[e + 2], gw[e + 3]);
+                    for (int e = 0; e < R; e += 4)
+                        red_add_v4(dw + e, gw[e], gw[e + 1], gw[e + 2], gw[e + 3]);
+                }
             }
         }
         if (tab && dtheta)
-            cta_add_dtheta<D>(dth, red_smem, dtheta + it.h * (D / 4));
-    } else if (t == 0) {
+            cta_add_dtheta<D, kBwdThreads / 32>(dth, red_smem, dtheta + it.h * (D / 4));
+    } else if (tid == 0) {
         atomicOr(&g_status_word, 1u);
         // give an MMA that may still be in flight one more bounded chance to
         // land before its TMEM is released
@@ -547,7 +638,7 @@ __global__ void __launch_bounds__(128)
         store_bf16_row<D>(dq + off, gq);
     }
     if (theta && dtheta)
-        cta_add_dtheta<D>(dth, red_smem, dtheta + h * (D / 4));
+        cta_add_dtheta<D, 4>(dth, red_smem, dtheta + h * (D / 4));
 }
 
 }  // namespace winattn

@@ -98,9 +98,15 @@ struct GateLayout {
 
 // out = o * sigmoid(pw (dw3x3(x) + dw_b) + pw_b) per token and channel;
 // x, o, out bf16 [B][H][W][C] (out may be o); dw fp32 [C][3][3], dw_b [C],
-// pw fp32 [C_out][C_in], pw_b [C].  Persistent: grid <= the SM count, 128
-// threads, tile = 128 consecutive tokens of the row-major map.
-__global__ void __launch_bounds__(128, 1)
+// pw fp32 [C_out][C_in], pw_b [C].  Persistent: grid <= the SM count, tile =
+// 128 consecutive tokens of the row-major map.  512 threads: thread
+// (group, t) handles token t of the tile and the 16-channel atoms
+// a = group (mod 4), so that 16 warps hide the gather latency; warps w,
+// w + 4, w + 8, w + 12 share TMEM lane quarter w % 4 and read their own
+// atoms' columns of it.
+constexpr int kGateThreads = 512;
+
+__global__ void __launch_bounds__(kGateThreads, 1)
     winattn_cla_gate_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *o,
                             const float *__restrict__ dw, const float *__restrict__ dw_b,
                             const float *__restrict__ pw, const float *__restrict__ pw_b, int B, int H, int W, int C,
@@ -113,20 +119,21 @@ __global__ void __launch_bounds__(128, 1)
     float *s_dwb = s_dw + 9 * C, *s_pwb = s_dwb + C;
     uint64_t *bar = reinterpret_cast<uint64_t *>(base + GateLayout::bar_off(C));
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bar + 1);
-    const int t = threadIdx.x, warp = t >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int t = tid & 127, group = tid >> 7;  // token row of the tile, atom group
     const uint32_t ncols = C <= 32 ? 32u : (C <= 64 ? 64u : (C <= 128 ? 128u : 256u));
     if (warp == 0) {
         tmem_alloc(tslot, ncols);
         tmem_relinquish();
     }
-    if (t == 0) {
+    if (tid == 0) {
         mbar_init(bar, 1);
         fence_mbar_init();
     }
     // point-wise weights -> bf16 B operand: row co (output channel), 16-channel
     // input atoms of C_out rows x 32 bytes
     const int atoms = C / 16;
-    for (int idx = t; idx < C * atoms; idx += 128) {
+    for (int idx = tid; idx < C * atoms; idx += kGateThreads) {
         const int co = idx / atoms, a = idx - co * atoms;
         const float *src = pw + (size_t)co * C + a * 16;
         uint32_t pk[8];
@@ -137,9 +144,9 @@ __global__ void __launch_bounds__(128, 1)
         *reinterpret_cast<uint4 *>(dst + swz_offset(co, 0, 32)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         *reinterpret_cast<uint4 *>(dst + swz_offset(co, 1, 32)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
     }
-    for (int idx = t; idx < 9 * C; idx += 128)
+    for (int idx = tid; idx < 9 * C; idx += kGateThreads)
         s_dw[idx] = __ldg(dw + idx);
-    for (int idx = t; idx < C; idx += 128) {
+    for (int idx = tid; idx < C; idx += kGateThreads) {
         s_dwb[idx] = __ldg(dw_b + idx);
         s_pwb[idx] = __ldg(pw_b + idx);
     }
@@ -148,7 +155,7 @@ __global__ void __launch_bounds__(128, 1)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *tslot;
-    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    const uint32_t trow = tmem + ((uint32_t)((warp & 3) * 32) << 16);
     const uint32_t aoff = GateLayout::a_off(C);
     const uint32_t idesc = idesc_bf16_f32(128, C, false);
     const int64_t T = (int64_t)B * H * W;
@@ -165,7 +172,7 @@ __global__ void __launch_bounds__(128, 1)
             r = (int)((tok / W) % H);
             b = (int)(tok / ((int64_t)W * H));
         }
-        for (int a = 0; a < atoms; ++a) {
+        for (int a = group; a < atoms; a += 4) {
             float acc[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e)
@@ -202,7 +209,7 @@ __global__ void __launch_bounds__(128, 1)
         tc_fence_before_sync();
         __syncthreads();
         // ---- point-wise: G = A PW^T over 16-channel atoms
-        if (t == 0) {
+        if (tid == 0) {
             tc_fence_after_sync();
             for (int a = 0; a < atoms; ++a) {
                 const uint64_t ad = smem_desc(sbase + aoff + (uint32_t)a * 128 * 32, 16, 256, swizzle_code(32));
@@ -219,7 +226,8 @@ __global__ void __launch_bounds__(128, 1)
         }
         tc_fence_after_sync();
         // ---- epilogue: out = o * sigmoid(G + pw_b), 16 channels at a time
-        for (int a = 0; a < atoms; ++a) {
+        // (every lane of a warp runs the same atoms: the TMEM load is collective)
+        for (int a = group; a < atoms; a += 4) {
             float gv[16];
             tmem_ld16(trow + a * 16, gv);  // every lane: the load is warp-collective
             if (real) {
@@ -242,7 +250,7 @@ __global__ void __launch_bounds__(128, 1)
         tc_fence_before_sync();
         __syncthreads();
     }
-    if (!ok && t == 0) {
+    if (!ok && tid == 0) {
         atomicOr(&g_status_word, 1u);
         mbar_wait(bar, phase);
     }

@@ -696,7 +696,7 @@ int launch_bwd(const BwdArgs &a, const Geometry &g, cudaStream_t s)
     if (!smem_attr_once<winattn_bwd_tc_kernel<D, R>>())
         return WINATTN_ERR_CUDA;
     const float scale = 1.0f / std::sqrt((float)g.d);
-    winattn_bwd_tc_kernel<D, R><<<(unsigned)g.items, 128, smem, s>>>(
+    winattn_bwd_tc_kernel<D, R><<<(unsigned)g.items, kBwdThreads, smem, s>>>(
         static_cast<const T *>(a.q), static_cast<const T *>(a.k), static_cast<const T *>(a.v), a.theta,
         static_cast<const T *>(a.bias), static_cast<const T *>(a.out), static_cast<const T *>(a.dout), a.lse,
         static_cast<T *>(a.dq), static_cast<T *>(a.dk), static_cast<T *>(a.dv), a.dtheta, a.dbias, a.dq_acc, g,
@@ -859,7 +859,7 @@ int winattn_cla_gate(const void *x, const void *o, const float *dw, const float 
         return WINATTN_ERR_CUDA;
     const int64_t tiles = ((int64_t)B * H_img * W_img + 127) / 128;
     const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
-    winattn_cla_gate_kernel<<<grid, 128, GateLayout::bytes(C), static_cast<cudaStream_t>(stream)>>>(
+    winattn_cla_gate_kernel<<<grid, kGateThreads, GateLayout::bytes(C), static_cast<cudaStream_t>(stream)>>>(
         static_cast<const __nv_bfloat16 *>(x), static_cast<const __nv_bfloat16 *>(o), dw, dw_b, pw, pw_b, B, H_img,
         W_img, C, static_cast<__nv_bfloat16 *>(out));
     return cudaGetLastError() == cudaSuccess ? WINATTN_OK : WINATTN_ERR_CUDA;
