@@ -14,7 +14,7 @@ import torch
 from . import _lib
 from ._lib import WinattnError
 
-__all__ = ["window_attention", "window_attention_host", "window_attention_backward",
+__all__ = ["window_attention", "window_attention_host", "window_attention_backward", "window_attention_autograd",
            "window_attention_gated_residual", "rib_features", "window_attention_rib", "cla_gate", "WinattnError",
            "device_status"]
 
@@ -187,6 +187,39 @@ def window_attention_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     if rc != _lib.OK:
         raise WinattnError(rc, "winattn_bwd")
     return dq, dk, dv, dtheta, dbias
+
+
+class _WindowAttention(torch.autograd.Function):
+    """Forward through winattn_fwd_lse (saving each row's log-sum-exp),
+    backward through winattn_bwd: gradients for q, k, v, theta and the bias
+    features."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, theta, bias_feats, M, shift):
+        B, H, W, heads, d = q.shape
+        lse = torch.empty((B, H, W, heads), dtype=torch.float32, device=q.device)
+        out = window_attention(q, k, v, M, shift, theta=theta, bias_feats=bias_feats, lse=lse)
+        ctx.save_for_backward(q, k, v, theta, bias_feats, out, lse)
+        ctx.M, ctx.shift = M, shift
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, theta, bias, out, lse = ctx.saved_tensors
+        dq, dk, dv, dth, dbi = window_attention_backward(q, k, v, out, dout.contiguous(), lse, ctx.M, ctx.shift,
+                                                         theta=theta, bias_feats=bias)
+        if dbi is not None:
+            dbi = dbi.to(bias.dtype)
+        return dq, dk, dv, dth, dbi, None, None
+
+
+def window_attention_autograd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, M: int, shift: int = 0,
+                              theta: Optional[torch.Tensor] = None,
+                              bias_feats: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """window_attention as a differentiable torch op (bf16 CUDA tensors):
+    the learned frequencies theta (e.g. theta = omega.exp()) and the bias
+    features receive gradients too."""
+    return _WindowAttention.apply(q, k, v, theta, bias_feats, M, shift)
 
 
 def window_attention_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, M: int, shift: int = 0,
