@@ -35,7 +35,9 @@ _COMMON = [_CSRC + "ptx.cuh", _CSRC + "geometry.cuh", _CSRC + "waits.cuh"]
 # kernel id of winattn_launch_info -> (name used in profiles/, source files whose change voids a capture)
 KERNELS = {0: ("tc", [_CSRC + "fwd_tc.cuh"] + _COMMON), 1: ("small", [_CSRC + "fwd_small.cuh"] + _COMMON),
            2: ("large", [_CSRC + "fwd_large.cuh"] + _COMMON), 3: ("simt", [_CSRC + "fwd_simt.cuh"] + _COMMON),
-           4: ("pipe", [_CSRC + "fwd_pipe.cuh", _CSRC + "fwd_small.cuh"] + _COMMON)}
+           4: ("pipe", [_CSRC + "fwd_pipe.cuh", _CSRC + "fwd_small.cuh"] + _COMMON),
+           5: ("pipe16", [_CSRC + "fwd_pipe16.cuh", _CSRC + "fwd_pipe.cuh", _CSRC + "fwd_large.cuh",
+                          _CSRC + "fwd_small.cuh"] + _COMMON)}
 
 
 def parse():

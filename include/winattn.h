@@ -357,7 +357,7 @@ int winattn_last_device_status(void *stream);
  * dynamic shared memory bytes, windows packed per tile and the kernel chosen
  * (0 = generic tensor-core kernel, 1 = persistent small-window kernel,
  * 2 = persistent large-window kernel, 3 = fp32 SIMT kernel, 4 = pipelined
- * kernel for 8 x 8 windows).  Any output pointer may be NULL.  Makes no CUDA
+ * kernel for 8 x 8 windows, 5 = pipelined kernel for 16 x 16 windows).  Any output pointer may be NULL.  Makes no CUDA
  * call.  Returns the winattn_check_args code for the sizes (pointers are not
  * checked).
  */
@@ -381,7 +381,8 @@ int winattn_selftest_wait_timeout(void *stream);
 /*
  * winattn_set_kernel_enabled — process-wide switch of a specialised kernel
  * (the kernel ids of winattn_launch_info: 1 = persistent small-window,
- * 2 = persistent large-window, 4 = pipelined 8 x 8 kernel).  While a kernel is
+ * 2 = persistent large-window, 4 = pipelined 8 x 8 kernel, 5 = pipelined
+ * 16 x 16 kernel).  While a kernel is
  * disabled, winattn_fwd and winattn_launch_info route its problems to the
  * next kernel that serves them (in the end the generic tensor-core kernel,
  * which serves every bf16 problem); the results agree within the bf16

@@ -89,7 +89,7 @@ def test_host_workspace_bytes(lib):
     assert _lib.host_workspace_bytes(0, 16, 16, 2, 32, _lib.BF16) == 0
 
 
-GENERIC, SMALL, LARGE, SIMT, PIPE = 0, 1, 2, 3, 4
+GENERIC, SMALL, LARGE, SIMT, PIPE, PIPE16 = 0, 1, 2, 3, 4, 5
 
 
 @pytest.mark.parametrize("B,H,W,M,shift,heads,d,rank,U,tiles,kernel", [
@@ -98,6 +98,11 @@ GENERIC, SMALL, LARGE, SIMT, PIPE = 0, 1, 2, 3, 4
     (4, 32, 32, 8, 4, 4, 64, 0, 2, 1, PIPE),
     (4, 32, 32, 8, 3, 4, 32, 0, 2, 1, SMALL),        # shift 3: boxes are not whole swizzle atoms
     (4, 32, 32, 8, 4, 4, 32, 16, 2, 1, SMALL),       # rank-r factors
+    (4, 64, 64, 16, 8, 4, 32, 0, 1, 2, PIPE16),      # 256-token windows: two query tiles against one S
+    (2, 32, 48, 16, 0, 3, 64, 0, 1, 2, PIPE16),
+    (2, 32, 48, 16, 0, 16, 64, 0, 1, 2, LARGE),      # RoPE table of 16 heads: the 16 x 16 kernel has no room
+    (2, 32, 32, 16, 8, 2, 64, 16, 1, 2, GENERIC),    # rank-r factors at d = 64
+    (2, 32, 32, 16, 4, 2, 32, 0, 1, 2, GENERIC),     # shift 4: a query tile would straddle the row seam
     (16, 128, 128, 32, 0, 3, 32, 0, 1, 8, LARGE),    # 1024-token windows: 8 query tiles each
     (4, 192, 192, 96, 0, 6, 32, 16, 1, 72, LARGE),   # 9216-token windows
     (1, 48, 48, 24, 0, 1, 32, 0, 1, 5, GENERIC),     # 576 tokens: no whole-row key tiles
@@ -115,15 +120,16 @@ def test_launch_plan(lib, B, H, W, M, shift, heads, d, rank, U, tiles, kernel):
     windows = B * (-(-H // M)) * (-(-W // M))   # windows of the grid padded to multiples of M
     assert info["windows_per_tile"] == U
     assert info["kernel"] == kernel
-    if kernel == LARGE:  # items are pairs of query tiles
+    if kernel in (LARGE, PIPE16):  # items are pairs of query tiles
         assert info["work_items"] == heads * windows * tiles // 2
-        assert info["threads"] == 512 and info["grid"] == min(148, info["work_items"])
+        threads = 512 if kernel == LARGE else 768
+        assert info["threads"] == threads and info["grid"] == min(148, info["work_items"])
     else:
         assert info["work_items"] == heads * math.ceil(windows / U) * tiles
     if kernel == SMALL:
         groups = 4 if d == 32 else 3  # compute warpgroups, plus a loader warp
         assert info["threads"] == (4 * groups + 1) * 32 and info["grid"] == min(148, info["work_items"])
-    elif kernel == PIPE:  # RoPE x2, softmax x2, epilogue warpgroups, two loader and two MMA warps
+    elif kernel in (PIPE, PIPE16):  # RoPE x2, softmax x2, epilogue warpgroups, two loader and two MMA warps
         assert info["threads"] == 24 * 32 and info["grid"] == min(148, info["work_items"])
     elif kernel == GENERIC:
         assert info["threads"] == 128 and info["grid"] == info["work_items"]
@@ -141,9 +147,13 @@ def test_kernel_switch_routes_to_fallbacks(lib):
     is process-wide and returns its previous state."""
     dense = (16, 128, 128, 32, 16, 3, 32, 0, _lib.BF16)
     swin = (64, 56, 56, 8, 4, 3, 32, 0, _lib.BF16)
+    m16 = (4, 64, 64, 16, 8, 4, 32, 0, _lib.BF16)
     assert _lib.launch_info(*dense)[1]["kernel"] == _lib.KERNEL_LARGE
     assert _lib.launch_info(*swin)[1]["kernel"] == _lib.KERNEL_PIPE
+    assert _lib.launch_info(*m16)[1]["kernel"] == _lib.KERNEL_PIPE16
     try:
+        assert _lib.set_kernel_enabled(_lib.KERNEL_PIPE16, False) == 1
+        assert _lib.launch_info(*m16)[1]["kernel"] == _lib.KERNEL_LARGE
         assert _lib.set_kernel_enabled(_lib.KERNEL_LARGE, False) == 1
         assert _lib.launch_info(*dense)[1]["kernel"] == _lib.KERNEL_GENERIC
         assert _lib.set_kernel_enabled(_lib.KERNEL_PIPE, False) == 1
@@ -152,8 +162,9 @@ def test_kernel_switch_routes_to_fallbacks(lib):
         assert _lib.launch_info(*swin)[1]["kernel"] == _lib.KERNEL_GENERIC
         assert _lib.set_kernel_enabled(_lib.KERNEL_SMALL, False) == 0
     finally:
-        for k in (_lib.KERNEL_LARGE, _lib.KERNEL_PIPE, _lib.KERNEL_SMALL):
+        for k in (_lib.KERNEL_LARGE, _lib.KERNEL_PIPE, _lib.KERNEL_SMALL, _lib.KERNEL_PIPE16):
             _lib.set_kernel_enabled(k, True)
+    assert _lib.launch_info(*m16)[1]["kernel"] == _lib.KERNEL_PIPE16
     assert _lib.launch_info(*dense)[1]["kernel"] == _lib.KERNEL_LARGE
     assert _lib.launch_info(*swin)[1]["kernel"] == _lib.KERNEL_PIPE
     # the generic and fp32 kernels have no switch

@@ -41,7 +41,7 @@ SMALL = [
     ("m11_s5_d64_r16", 1, 22, 22, 11, 5, 2, 64, "bf16", "learned", 16),   # 121 tokens, small kernel
     ("m9_s4_r32", 2, 18, 9, 9, 4, 3, 32, "bf16", None, 32),
     ("m24_s0_r16", 1, 48, 48, 24, 0, 2, 32, "bf16", None, 16),      # bias factors, no RoPE
-    ("m16_s0_d32", 2, 32, 48, 16, 0, 2, 32, "bf16", "learned", 0),  # large-window kernel from here on
+    ("m16_s0_d32", 2, 32, 48, 16, 0, 2, 32, "bf16", "learned", 0),  # pipelined 16 x 16 kernel
     # several items per CTA: both O buffers of a query tile in turn, and the
     # epilogue of each item trailing the next item's first step
     ("m16_s8_d32_items", 8, 64, 64, 16, 8, 4, 32, "bf16", "learned", 0),
@@ -188,10 +188,12 @@ FALLBACKS = [
     ((_lib.KERNEL_LARGE,), "dense", 16, _lib.KERNEL_GENERIC),
     ((_lib.KERNEL_PIPE,), "swin", 4, _lib.KERNEL_SMALL),
     ((_lib.KERNEL_PIPE, _lib.KERNEL_SMALL), "swin", 4, _lib.KERNEL_GENERIC),
+    ((_lib.KERNEL_PIPE16,), "sweep_M16_d32_s8", 8, _lib.KERNEL_LARGE),
+    ((_lib.KERNEL_PIPE16,), "sweep_M16_d64_s8", 0, _lib.KERNEL_LARGE),
 ]
 
 
-@pytest.mark.parametrize("off,name,shift,serves", FALLBACKS, ids=["large-off", "pipe-off", "pipe-small-off"])
+@pytest.mark.parametrize("off,name,shift,serves", FALLBACKS, ids=["large-off", "pipe-off", "pipe-small-off", "pipe16-off-s8", "pipe16-off-d64-s0"])
 def test_fallback_kernels(off, name, shift, serves):
     """With specialised kernels switched off, their problems run on the next
     kernel that serves them (the path a build with an unexpected register
@@ -204,6 +206,8 @@ def test_fallback_kernels(off, name, shift, serves):
         assert rc == 0 and info["kernel"] == serves
         if w.name == "dense":
             G.sampled_compare(w, shift, images=[0, w.B - 1], extra_windows=2)
+        elif w.name.startswith("sweep_"):
+            G.sampled_compare(w, shift, images=[w.B - 1], heads=[0, w.heads - 1], extra_windows=1, max_units=16)
         else:
             G.full_compare(w, shift)
     finally:

@@ -166,7 +166,7 @@ def selftest_wait_timeout(stream) -> int:
     return load().winattn_selftest_wait_timeout(stream)
 
 
-KERNEL_GENERIC, KERNEL_SMALL, KERNEL_LARGE, KERNEL_SIMT, KERNEL_PIPE = 0, 1, 2, 3, 4
+KERNEL_GENERIC, KERNEL_SMALL, KERNEL_LARGE, KERNEL_SIMT, KERNEL_PIPE, KERNEL_PIPE16 = 0, 1, 2, 3, 4, 5
 
 
 def set_kernel_enabled(kernel: int, enabled: bool) -> int:

@@ -15,6 +15,7 @@
 #include "bwd_tc.cuh"
 #include "fwd_large.cuh"
 #include "fwd_pipe.cuh"
+#include "fwd_pipe16.cuh"
 #include "fwd_simt.cuh"
 #include "fwd_small.cuh"
 #include "fwd_tc.cuh"
@@ -92,12 +93,12 @@ int smem_bytes_for(const Geometry &g, int dtype)
 constexpr int kAssumedSMs = 148;          // B200; used only by winattn_launch_info
 constexpr uint32_t kMaxSmem = 227 * 1024;
 
-enum KernelKind { kGeneric = 0, kSmall = 1, kLarge = 2, kSimt = 3, kPipe = 4, kKinds = 5 };
+enum KernelKind { kGeneric = 0, kSmall = 1, kLarge = 2, kSimt = 3, kPipe = 4, kPipe16 = 5, kKinds = 6 };
 
 // Process-wide switches of the specialised kernels (winattn_set_kernel_enabled):
 // a disabled kind's problems go to the generic kernel.  The generic and SIMT
 // kernels cannot be disabled.
-std::atomic<int> g_kernel_enabled[kKinds] = {1, 1, 1, 1, 1};
+std::atomic<int> g_kernel_enabled[kKinds] = {1, 1, 1, 1, 1, 1};
 
 bool kernel_enabled(KernelKind k) { return g_kernel_enabled[k].load(std::memory_order_relaxed) != 0; }
 
@@ -204,6 +205,11 @@ uint32_t pipe_smem(const Geometry &g)
     return g.d == 32 ? PipeLayout<32>::bytes(g.heads) : PipeLayout<64>::bytes(g.heads);
 }
 
+uint32_t pipe16_smem(const Geometry &g)
+{
+    return g.d == 32 ? Pipe16Layout<32>::bytes(g.heads) : Pipe16Layout<64>::bytes(g.heads);
+}
+
 uint32_t small_smem(const Geometry &g)
 {
     switch (g.d * 100 + g.rank) {
@@ -232,6 +238,9 @@ KernelKind choose_kernel(const Geometry &g, int dtype, bool want_lse = false)
     if (kernel_enabled(kPipe) && pipe_ok(g) && (uint64_t)g.heads * g.M * (g.d / 4) * 8 <= kSmallTableMax &&
         pipe_smem(g) <= kMaxSmem)
         return kPipe;
+    // (the 16 x 16 pipelined kernel does not write the log-sum-exp)
+    if (!want_lse && kernel_enabled(kPipe16) && pipe16_ok(g) && pipe16_smem(g) <= kMaxSmem)
+        return kPipe16;
     // (the small-window kernel does not write the log-sum-exp)
     if (!want_lse && kernel_enabled(kSmall) && g.N <= kTileRows &&
         (uint64_t)g.heads * g.M * (g.d / 4) * 8 <= kSmallTableMax && small_smem(g) <= kMaxSmem)
@@ -552,6 +561,46 @@ int launch_pipe(const void *q, const void *k, const void *v, const float *theta,
     return cudaGetLastError() == cudaSuccess ? WINATTN_OK : WINATTN_ERR_CUDA;
 }
 
+template <int D>
+int launch_pipe16(const void *q, const void *k, const void *v, const float *theta, void *out, const Geometry &g,
+                  cudaStream_t stream)
+{
+    static_assert(sizeof(Pipe16StoreMaps) == 2 * sizeof(CUtensorMap), "two store maps");
+    MapSet ms;
+    const MapKey key = make_key(kPipe16, g, q, k, v, out, nullptr);
+    if (!cached_maps(key, &ms, [&](MapSet *m) {
+            WindowMaps *w = reinterpret_cast<WindowMaps *>(m->m);
+            return encode_window_maps(&w[0], q, g) && encode_window_maps(&w[1], k, g) &&
+                   encode_window_maps(&w[2], v, g) && encode_window_map(&m->m[12], out, g, 16, 2) &&
+                   encode_window_map(&m->m[13], out, g, 8, 4);
+        }))
+        return WINATTN_ERR_CUDA;
+    WindowMaps maps[3];
+    Pipe16StoreMaps om;
+    std::memcpy(maps, ms.m, sizeof maps);
+    std::memcpy(&om, &ms.m[12], sizeof om);
+    if (!smem_attr_once<winattn_fwd_pipe16_kernel<D>>())
+        return WINATTN_ERR_CUDA;
+    const int smem = (int)Pipe16Layout<D>::bytes(g.heads);
+    const int64_t items = g.wph * g.heads;
+    const int64_t grid = items < sm_count() ? items : sm_count();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kPipeThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const float scale = 1.0f / std::sqrt((float)g.d);
+    if (cudaLaunchKernelEx(&cfg, winattn_fwd_pipe16_kernel<D>, theta, g, scale, maps[0], maps[1], maps[2], om) !=
+        cudaSuccess)
+        return WINATTN_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? WINATTN_OK : WINATTN_ERR_CUDA;
+}
+
 template <int D, int R>
 int launch_simt(const void *q, const void *k, const void *v, const float *theta, const void *bias, void *out,
                 float *lse, const Geometry &g, cudaStream_t stream)
@@ -568,6 +617,8 @@ int dispatch(const void *q, const void *k, const void *v, const float *theta, co
     if (kind == kPipe)
         return g.d == 32 ? launch_pipe<32>(q, k, v, theta, out, lse, g, s)
                          : launch_pipe<64>(q, k, v, theta, out, lse, g, s);
+    if (kind == kPipe16)
+        return g.d == 32 ? launch_pipe16<32>(q, k, v, theta, out, g, s) : launch_pipe16<64>(q, k, v, theta, out, g, s);
     if (kind == kSmall) {
         switch (g.d * 100 + g.rank) {
         case 3200: return launch_small<32, 0>(q, k, v, theta, bias, out, g, s);
@@ -1182,6 +1233,12 @@ int winattn_launch_info(int B, int H_img, int W_img, int M, int shift, int heads
         if (grid) *grid = (int)(g.items < kAssumedSMs ? g.items : kAssumedSMs);
         if (threads) *threads = kPipeThreads;
         if (smem_bytes) *smem_bytes = (int)pipe_smem(g);
+    } else if (kind == kPipe16) {
+        const int64_t items = g.wph * g.heads;  // window-heads: two query tiles each
+        if (work_items) *work_items = items;
+        if (grid) *grid = (int)(items < kAssumedSMs ? items : kAssumedSMs);
+        if (threads) *threads = kPipeThreads;
+        if (smem_bytes) *smem_bytes = (int)pipe16_smem(g);
     } else if (kind == kSmall) {
         if (grid) *grid = (int)(g.items < kAssumedSMs ? g.items : kAssumedSMs);
         if (threads) *threads = g.d <= 32 ? SmallRoles<32>::kThreads : SmallRoles<64>::kThreads;
@@ -1205,7 +1262,7 @@ int winattn_selftest_wait_timeout(void *stream)
 
 int winattn_set_kernel_enabled(int kernel, int enabled)
 {
-    if (kernel != kSmall && kernel != kLarge && kernel != kPipe)
+    if (kernel != kSmall && kernel != kLarge && kernel != kPipe && kernel != kPipe16)
         return WINATTN_ERR_ARG;
     return g_kernel_enabled[kernel].exchange(enabled ? 1 : 0);
 }
