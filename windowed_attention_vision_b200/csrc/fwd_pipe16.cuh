@@ -28,7 +28,11 @@
 //   warps 8-15    two softmax warpgroups, one per query tile of an item:
 //                 exact max over the allowed granules, then exp2 (scale and
 //                 log2 e in one FFMA) and P as bf16 pairs over the consumed S
-//                 columns;
+//                 columns.  The exponentials of the two groups take turns
+//                 (group 0, group 1, group 0, ...): alone, a group's exp2 pass
+//                 has the SM's MUFU units to itself and runs in half the time,
+//                 while the other group waits for its S, takes its row max
+//                 or hands its P on;
 //   warps 16-19   epilogue: O / l as bf16 into a swizzled staging tile and TMA
 //                 box stores to the original, un-shifted positions.
 //
@@ -73,7 +77,7 @@ struct Pipe16Layout {
     static constexpr uint32_t QIJ = OSUM + kP16Bufs * 128 * 4;        // query rows: (i << 8 | j) u16[4 kinds][2][128]
     static constexpr uint32_t KIJ = QIJ + 4 * 2 * 128 * 2;            // key rows: u16[4 kinds][256]
     static constexpr uint32_t TABLE = KIJ + 4 * 256 * 2;              // RoPE (cos, sin) float4 [heads][16][D/8]
-    static constexpr int kBars = 3 * NSQ + 2 * NSV + NM + 4 * kP16Bufs + 2;
+    static constexpr int kBars = 3 * NSQ + 2 * NSV + NM + 4 * kP16Bufs + 2 + 2;
     static __host__ __device__ uint32_t bars(int heads) { return TABLE + (uint32_t)heads * 16 * (D / 8) * 16; }
     static __host__ __device__ uint32_t bytes(int heads) { return bars(heads) + kBars * 8 + 16 + 1024; }
 };
@@ -90,6 +94,22 @@ __host__ __device__ inline bool pipe16_ok(const Geometry &g)
 struct Pipe16StoreMaps {
     CUtensorMap o16x2, o8x4;
 };
+
+// P of 16 keys: exp2(s c2 - m) of each score in x[], summed into lq and
+// stored as 8 packed bf16 pairs at TMEM column `pcol`.
+__device__ __forceinline__ void exp_chunk16(const uint32_t (&x)[16], float2 cc, float2 mm, float2 (&lq)[2],
+                                            uint32_t pcol)
+{
+    uint32_t pk[8];
+#pragma unroll
+    for (int e = 0; e < 16; e += 2) {
+        const float2 z = __ffma2_rn(make_float2(__uint_as_float(x[e]), __uint_as_float(x[e + 1])), cc, mm);
+        const float2 p = make_float2(fast_exp2(z.x), fast_exp2(z.y));
+        lq[(e >> 1) & 1] = __fadd2_rn(lq[(e >> 1) & 1], p);
+        pk[e >> 1] = pack_bf16x2(p.x, p.y);
+    }
+    tmem_st8(pcol, pk);
+}
 
 template <int D>
 __global__ void __launch_bounds__(kPipeThreads, 1)
@@ -115,7 +135,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     uint64_t *qk_full = bars, *ready = qk_full + NSQ, *qk_empty = ready + NSQ;
     uint64_t *v_full = qk_empty + NSQ, *v_empty = v_full + NSV, *meta_full = v_empty + NSV;
     uint64_t *s_full = meta_full + NM, *p_full = s_full + NB, *o_full = p_full + NB, *t_free = o_full + NB;
-    uint64_t *fin = t_free + NB;
+    uint64_t *fin = t_free + NB, *turn = fin + 2;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + L::kBars);
     volatile uint32_t *abort_flag = tslot + 1;
 
@@ -148,6 +168,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         }
         mbar_init(&fin[0], 1);
         mbar_init(&fin[1], 1);
+        mbar_init(&turn[0], 4);             // one arrival per softmax warp of the other group
+        mbar_init(&turn[1], 4);
         *abort_flag = 0u;
         fence_mbar_init();
     }
@@ -427,6 +449,9 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         const float c2 = scale * kLog2e;
         const float2 cc = make_float2(c2, c2);
         const float ninf = -INFINITY;
+        // group 0 takes the first turn
+        if (grp == 1 && count > 0)
+            warp_arrive(&turn[0]);
         for (int kk = 0; kk < count; ++kk) {
             const int kt = 2 * kk + grp, b = kt % NB, m = kt % NM;
             if (!warp_wait(&s_full[b], (kt / NB) & 1, abort_flag))
@@ -459,34 +484,49 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
             }
             const float mneg = mx == ninf ? 0.f : -mx * c2;
             const float2 mm = make_float2(mneg, mneg);
-            // pass 2: P = exp2(s c2 - m) over the allowed granules, zeros
-            // elsewhere, packed over the consumed S columns
+            // this group's turn at the exponentials: phase kk of turn[grp]
+            if (!warp_wait(&turn[grp], kk & 1, abort_flag))
+                break;
+            // pass 2: P = exp2(s c2 - m) over the allowed granules in chunks
+            // of 16 keys, the load of chunk q + 1 in flight while chunk q is
+            // exponentiated; chunk q's P (8 packed columns) lands below every
+            // S column still to be read
+            int gl = 0, ng = 0;  // allowed granules, in order, 2 bits each
+#pragma unroll
+            for (int gi = 0; gi < 4; ++gi)
+                if ((gmask >> gi) & 1u)
+                    gl |= gi << (2 * ng++);
+            const int nq = 4 * ng;
+            auto chunk_col = [&](int q) { return ((gl >> (2 * (q >> 2))) & 3) * 64 + (q & 3) * 16; };
             float2 lq[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            uint32_t xa[16], xb[16];
+            tmem_ld16_issue(sreg + chunk_col(0), xa);
+            tmem_wait_ld16(xa);
+#pragma unroll 1
+            for (int q = 0; q < nq; q += 2) {
+                tmem_ld16_issue(sreg + chunk_col(q + 1), xb);  // nq is a multiple of 4
+                exp_chunk16(xa, cc, mm, lq, sreg + (chunk_col(q) >> 1));
+                tmem_wait_ld16(xb);
+                // (after the last pair: a spare load of chunk 0, never used)
+                tmem_ld16_issue(sreg + chunk_col(q + 2 < nq ? q + 2 : 0), xa);
+                exp_chunk16(xb, cc, mm, lq, sreg + (chunk_col(q + 1) >> 1));
+                tmem_wait_ld16(xa);
+            }
+            // zeros over the packed columns of the masked granules, once every
+            // S column has been read
 #pragma unroll 1
             for (int gi = 0; gi < 4; ++gi) {
-                const bool on = (gmask >> gi) & 1u;
+                if ((gmask >> gi) & 1u)
+                    continue;
+                uint32_t z[16];
 #pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    uint32_t pk[16];
-                    if (on) {
-                        float x[32];
-                        tmem_ld32(sreg + gi * 64 + h2 * 32, x);
-#pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            const float2 z = __ffma2_rn(make_float2(x[e], x[e + 1]), cc, mm);
-                            const float2 p = make_float2(fast_exp2(z.x), fast_exp2(z.y));
-                            lq[(e >> 1) & 1] = __fadd2_rn(lq[(e >> 1) & 1], p);
-                            pk[e >> 1] = pack_bf16x2(p.x, p.y);
-                        }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e)
-                            pk[e] = 0u;
-                    }
-                    // keys [64 gi + 32 h2, +32) -> packed columns [32 gi + 16 h2, +16)
-                    tmem_st16(sreg + gi * 32 + h2 * 16, pk);
-                }
+                for (int e = 0; e < 16; ++e)
+                    z[e] = 0u;
+                tmem_st16(sreg + gi * 32, z);
+                tmem_st16(sreg + gi * 32 + 16, z);
             }
+            // the other group's turn (group 1's last one is never taken)
+            warp_arrive(&turn[grp ^ 1]);
             const float2 l2 = __fadd2_rn(lq[0], lq[1]);
             osum[b * 128 + row] = l2.x + l2.y;
             tmem_wait_st();
