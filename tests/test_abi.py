@@ -122,14 +122,14 @@ def test_launch_plan(lib, B, H, W, M, shift, heads, d, rank, U, tiles, kernel):
     assert info["kernel"] == kernel
     if kernel in (LARGE, PIPE16):  # items are pairs of query tiles
         assert info["work_items"] == heads * windows * tiles // 2
-        threads = 512 if kernel == LARGE else 768
+        threads = 512 if kernel == LARGE else 1024  # the 16 x 16 kernel: RoPE x2, softmax x4, epilogue, 4 warps
         assert info["threads"] == threads and info["grid"] == min(148, info["work_items"])
     else:
         assert info["work_items"] == heads * math.ceil(windows / U) * tiles
     if kernel == SMALL:
         groups = 4 if d == 32 else 3  # compute warpgroups, plus a loader warp
         assert info["threads"] == (4 * groups + 1) * 32 and info["grid"] == min(148, info["work_items"])
-    elif kernel in (PIPE, PIPE16):  # RoPE x2, softmax x2, epilogue warpgroups, two loader and two MMA warps
+    elif kernel == PIPE:  # RoPE x2, softmax x2, epilogue warpgroups, two loader and two MMA warps
         assert info["threads"] == 24 * 32 and info["grid"] == min(148, info["work_items"])
     elif kernel == GENERIC:
         assert info["threads"] == 128 and info["grid"] == info["work_items"]

@@ -7,34 +7,43 @@
 // 8-15) against the whole window's 256 keys.  Because all keys of a window fit
 // one S of 128 x 256 fp32 (256 TMEM columns), each query tile takes one S
 // MMA and one softmax pass with the exact row max: no online rescale, no key
-// loop.  The roles follow the 8 x 8 kernel:
+// loop.  The roles (32 warps):
 //
-//   warp 20       Q/K loader: per item, the two query tiles' boxes and the
+//   warp 28       Q/K loader: per item, the two query tiles' boxes and the
 //                 window's K boxes (one, two or four per operand, by wrap
 //                 kind; the cyclic shift is box coordinates) into an
 //                 NSQ-stage ring;
-//   warp 23       V loader: the window's V boxes into an NSV-stage ring, once
+//   warp 31       V loader: the window's V boxes into an NSV-stage ring, once
 //                 the item's RoPE is done;
 //   warps 0-7     two RoPE warpgroups, alternate items: rotate the item's 256
 //                 query rows and 256 key rows in place in fp32, write each
 //                 query row's allowed 64-key granules and each epilogue warp's
 //                 store records;
-//   warp 21       S issuer: S = Q K^T of each query tile (M = 128, N = 256)
+//   warp 29       S issuer: S = Q K^T of each query tile (M = 128, N = 256)
 //                 into TMEM buffer (tile % 2); after both tiles of an item the
 //                 Q/K stage goes back to the loader;
-//   warp 22       P V issuer: O = P V (P from TMEM, 256 keys) into the same
-//                 buffer's columns 128 onwards; after both tiles the V stage
+//   warp 30       P V issuer: O = P V (P from TMEM, 256 keys) into the same
+//                 buffer's columns 192 onwards; after both tiles the V stage
 //                 goes back;
-//   warps 8-15    two softmax warpgroups, one per query tile of an item:
-//                 exact max over the allowed granules, then exp2 (scale and
-//                 log2 e in one FFMA) and P as bf16 pairs over the consumed S
-//                 columns.  The exponentials of the two groups take turns
-//                 (group 0, group 1, group 0, ...): alone, a group's exp2 pass
-//                 has the SM's MUFU units to itself and runs in half the time,
-//                 while the other group waits for its S, takes its row max
-//                 or hands its P on;
-//   warps 16-19   epilogue: O / l as bf16 into a swizzled staging tile and TMA
+//   warps 8-23    softmax, sixteen warps on every tile: warp (g, quarter)
+//                 takes the 64-key granule g of the 32 rows of TMEM lane
+//                 quarter `quarter`.  Each takes the max over its granule, the
+//                 four warps of a quarter exchange it through shared memory,
+//                 and each then writes exp2 (scale and log2 e in one FFMA) of
+//                 its granule as packed bf16 P over S columns it has read.
+//                 While they work on one buffer's tile, the other buffer's
+//                 tile goes through P V, the epilogue's read of O and the next
+//                 S, and four warps per SM sub-partition keep the MUFU units
+//                 busy;
+//   warps 24-27   epilogue: O / l as bf16 into a swizzled staging tile and TMA
 //                 box stores to the original, un-shifted positions.
+//
+// TMEM buffer b (256 columns) over one tile: S in columns 0-255; then P of
+// granule g (keys 64 g .. 64 g + 63, 32 packed columns) in columns 64 g .. 64 g
+// + 31 for g = 0, 1 and 64 g + 32 .. 64 g + 63 for g = 2, 3 (the last two
+// granules are exponentiated from their last chunk down, so each chunk's P
+// lands on S columns already read); O in columns 96 onwards (the gap between
+// granule 1's P and granule 2's, up to 64 columns).
 //
 // Wrap masks are structural: the key boxes of a window are its wrap-label
 // regions (halves at a seam, quadrants in the corner window), each a whole
@@ -53,6 +62,18 @@
 namespace winattn {
 
 constexpr int kP16Bufs = 2;  // TMEM buffers of 256 columns (one per query tile of an item)
+constexpr int kP16Rope = 2;                          // RoPE warpgroups (item k goes to group k % 2)
+constexpr int kP16SoftmaxWarp = 4 * kP16Rope;        // first softmax warp: two teams of eight
+constexpr int kP16EpiWarp = kP16SoftmaxWarp + 16;
+constexpr int kP16LoadWarp = kP16EpiWarp + 4;        // Q/K loader; S issuer, P V issuer and V loader follow
+constexpr int kP16Threads = (kP16LoadWarp + 4) * 32;
+constexpr uint32_t kP16O = 96;                      // TMEM column of O in a buffer
+
+// TMEM column (within a buffer) of the packed P of keys 16 c .. 16 c + 15.
+__host__ __device__ constexpr uint32_t p16_pcol(int c)
+{
+    return (uint32_t)((c >> 2) * 64 + ((c >> 2) >= 2 ? 32 : 0) + (c & 3) * 8);
+}
 
 template <int D>
 struct Pipe16Layout {
@@ -63,21 +84,21 @@ struct Pipe16Layout {
     // V ring, per item: values [256][D]
     static constexpr uint32_t V_STAGE = 512 * D;
     static constexpr int NSV = D == 32 ? 3 : 2;
-    // metadata ring, per query tile: allowed granules of each row (u32[128]),
-    // then the output TMA stores of each epilogue warp: int4 {x0, y0, image,
-    // box shape | head column << 4}; NM = 2 NSQ + 2 orders the writer of tile
-    // k + NM after the last reader of tile k
+    // metadata ring, per query tile: allowed granules of the rows of each lane
+    // quarter (u32[4]; a quarter's rows lie on one side of every seam), then
+    // at byte 64 the output TMA stores of each epilogue warp: int4 {x0, y0,
+    // image, box shape | head column << 4}; NM = 2 NSQ + 2 orders the writer
+    // of tile k + NM after the last reader of tile k
     static constexpr int NM = 2 * NSQ + 2;
-    static constexpr uint32_t MSLOT = 128 * 4 + 4 * 16;
+    static constexpr uint32_t MSLOT = 64 + 4 * 16;
     static constexpr uint32_t VRING = NSQ * QK_STAGE;
     static constexpr uint32_t MRING = VRING + NSV * V_STAGE;
     static constexpr int NO = D == 32 ? 2 : 1;
     static constexpr uint32_t OSTAGE = (MRING + NM * MSLOT + 1023) & ~1023u;
-    static constexpr uint32_t OSUM = OSTAGE + NO * 256 * D;           // per buffer: row sum l, f32[2][128]
-    static constexpr uint32_t QIJ = OSUM + kP16Bufs * 128 * 4;        // query rows: (i << 8 | j) u16[4 kinds][2][128]
-    static constexpr uint32_t KIJ = QIJ + 4 * 2 * 128 * 2;            // key rows: u16[4 kinds][256]
-    static constexpr uint32_t TABLE = KIJ + 4 * 256 * 2;              // RoPE (cos, sin) float4 [heads][16][D/8]
-    static constexpr int kBars = 3 * NSQ + 2 * NSV + NM + 4 * kP16Bufs + 2 + 2;
+    static constexpr uint32_t OSUM = OSTAGE + NO * 256 * D;           // partial row sums: f32[buffer][granule][128]
+    static constexpr uint32_t PMAX = OSUM + kP16Bufs * 4 * 128 * 4;   // partial row maxima: f32[buffer][granule][128]
+    static constexpr uint32_t TABLE = PMAX + kP16Bufs * 4 * 128 * 4;  // RoPE (cos, sin) float4 [heads][16][D/8]
+    static constexpr int kBars = 3 * NSQ + 2 * NSV + NM + 5 * kP16Bufs + 2;
     static __host__ __device__ uint32_t bars(int heads) { return TABLE + (uint32_t)heads * 16 * (D / 8) * 16; }
     static __host__ __device__ uint32_t bytes(int heads) { return bars(heads) + kBars * 8 + 16 + 1024; }
 };
@@ -112,7 +133,7 @@ __device__ __forceinline__ void exp_chunk16(const uint32_t (&x)[16], float2 cc, 
 }
 
 template <int D>
-__global__ void __launch_bounds__(kPipeThreads, 1)
+__global__ void __launch_bounds__(kP16Threads, 1)
     winattn_fwd_pipe16_kernel(const float *__restrict__ theta, const Geometry g, const float scale,
                               const __grid_constant__ WindowMaps tm_q, const __grid_constant__ WindowMaps tm_k,
                               const __grid_constant__ WindowMaps tm_v, const __grid_constant__ Pipe16StoreMaps tm_o)
@@ -122,20 +143,19 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     // Items alternate between the two RoPE groups, so an item's Q/K stage
     // (item % NSQ) must always fall to the same group; tiles alternate
     // between the softmax groups and share a metadata slot every NM tiles.
-    static_assert(NSQ % kPipeRope == 0, "a Q/K stage must always be consumed by the same RoPE group");
+    static_assert(NSQ % kP16Rope == 0, "a Q/K stage must always be consumed by the same RoPE group");
     static_assert(NM % 2 == 0 && NM == 2 * NSQ + 2, "metadata ring must order its writers after its readers");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(base);
-    uint16_t *qij = reinterpret_cast<uint16_t *>(base + L::QIJ);
-    uint16_t *kij = reinterpret_cast<uint16_t *>(base + L::KIJ);
     float4 *table4 = reinterpret_cast<float4 *>(base + L::TABLE);
     float *osum = reinterpret_cast<float *>(base + L::OSUM);
+    float *pmax = reinterpret_cast<float *>(base + L::PMAX);
     uint64_t *bars = reinterpret_cast<uint64_t *>(base + L::bars(g.heads));
     uint64_t *qk_full = bars, *ready = qk_full + NSQ, *qk_empty = ready + NSQ;
     uint64_t *v_full = qk_empty + NSQ, *v_empty = v_full + NSV, *meta_full = v_empty + NSV;
     uint64_t *s_full = meta_full + NM, *p_full = s_full + NB, *o_full = p_full + NB, *t_free = o_full + NB;
-    uint64_t *fin = t_free + NB, *turn = fin + 2;
+    uint64_t *max_ready = t_free + NB, *fin = max_ready + NB;
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + L::kBars);
     volatile uint32_t *abort_flag = tslot + 1;
 
@@ -162,20 +182,19 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
             mbar_init(&meta_full[m], 4);    // one arrival per RoPE warp
         for (int b = 0; b < NB; ++b) {
             mbar_init(&s_full[b], 1);
-            mbar_init(&p_full[b], 4);       // one arrival per softmax warp
+            mbar_init(&p_full[b], 16);      // one arrival per softmax warp
+            mbar_init(&max_ready[b], 16);   // the same
             mbar_init(&o_full[b], 1);
             mbar_init(&t_free[b], 4);       // one arrival per epilogue warp
         }
         mbar_init(&fin[0], 1);
         mbar_init(&fin[1], 1);
-        mbar_init(&turn[0], 4);             // one arrival per softmax warp of the other group
-        mbar_init(&turn[1], 4);
         *abort_flag = 0u;
         fence_mbar_init();
     }
-    if (warp == kPipeLoadWarp && lane < 8)
+    if (warp == kP16LoadWarp && lane < 8)
         tma_prefetch_map(pick_map(lane < 4 ? tm_q : tm_k, lane & 3));
-    if (warp == kPipeLoadWarp + 3 && lane < 4)
+    if (warp == kP16LoadWarp + 3 && lane < 4)
         tma_prefetch_map(pick_map(tm_v, lane));
     grid_launch_dependents();
     grid_dependency_wait();
@@ -192,7 +211,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     };
     auto wrap = [&](int v, int lim) { return v >= lim ? v - lim : v; };
 
-    if (warp == kPipeLoadWarp) {
+    if (warp == kP16LoadWarp) {
         // ================================================================ Q/K loader
         // lanes 0-3: query tile A's boxes, 4-7: tile B's, 8-11: the key boxes
         int kk = 0;
@@ -241,7 +260,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
             for (int k2 = kk > NSQ ? kk - NSQ : 0; k2 < kk; ++k2)
                 mbar_wait(&qk_full[k2 % NSQ], (k2 / NSQ) & 1);
         __syncwarp();
-    } else if (warp == kPipeLoadWarp + 3) {
+    } else if (warp == kP16LoadWarp + 3) {
         // ================================================================ V loader
         int kk = 0;
         for (; kk < count; ++kk) {
@@ -275,7 +294,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
             for (int k2 = kk > NSV ? kk - NSV : 0; k2 < kk; ++k2)
                 mbar_wait(&v_full[k2 % NSV], (k2 / NSV) & 1);
         __syncwarp();
-    } else if (warp == kPipeLoadWarp + 1) {
+    } else if (warp == kP16LoadWarp + 1) {
         // ================================================================ S issuer
         if (lane == 0) {
             constexpr uint32_t kIdescS = idesc_bf16_f32(128, 256, false);
@@ -306,7 +325,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
                 mbar_wait(&fin[0], 0);
             }
         }
-    } else if (warp == kPipeLoadWarp + 2) {
+    } else if (warp == kP16LoadWarp + 2) {
         // ================================================================ P V issuer
         if (lane == 0) {
             constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, true);
@@ -322,11 +341,12 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
                         break;
                     tc_fence_after_sync();
                     const uint32_t vst = sbase + L::VRING + s * L::V_STAGE;
-                    // 16 keys of V are 32 D bytes: +2 D in the start-address field
+                    // 16 keys of V are 32 D bytes: +2 D in the start-address field;
+                    // P of keys 16 ks .. 16 ks + 15 in 8 packed columns
                     const uint64_t vd = smem_desc(vst, 8192, 16 * D, swizzle_code(2 * D));
 #pragma unroll
                     for (int ks = 0; ks < 16; ++ks)
-                        umma_bf16_ts(tmem + b * 256 + 128, tmem + b * 256 + ks * 8, vd + (uint64_t)(2 * D * ks),
+                        umma_bf16_ts(tmem + b * 256 + kP16O, tmem + b * 256 + p16_pcol(ks), vd + (uint64_t)(2 * D * ks),
                                      kIdescPV, ks > 0);
                     umma_commit(&o_full[b]);
                 }
@@ -338,16 +358,14 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
                 mbar_wait(&fin[1], 0);
             }
         }
-    } else if (warp < kPipeSoftmaxWarp) {
+    } else if (warp < kP16SoftmaxWarp) {
         // ================================================================ RoPE groups
-        // the tables only these warps read: RoPE (cos, sin) of each head,
+        // the table only these warps read: RoPE (cos, sin) of each head,
         // table4[h][pos][k/2] = (cos k, cos k+1, sin k, sin k+1) of
-        // pos * theta_h[k], even k; the window-local (i, j) of each query row
-        // (per kind and query tile) and of each key row (per kind), in the
-        // order the boxes land
+        // pos * theta_h[k], even k
         if (theta) {
             float *tf = reinterpret_cast<float *>(table4);
-            for (int idx = t; idx < g.heads * 16 * (D / 4); idx += 32 * kPipeSoftmaxWarp) {
+            for (int idx = t; idx < g.heads * 16 * (D / 4); idx += 32 * kP16SoftmaxWarp) {
                 const int h = idx / (16 * (D / 4)), r = idx - h * 16 * (D / 4);
                 const int pos = r / (D / 4), kq = r - pos * (D / 4);
                 float sn, cs;
@@ -357,29 +375,10 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
                 e[2 + (kq & 1)] = sn;
             }
         }
-        for (int idx = t; idx < 4 * 2 * 128; idx += 32 * kPipeSoftmaxWarp) {
-            const int kind = idx >> 8, qh = (idx >> 7) & 1, r = idx & 127;
-            int i, j;
-            if (kind & 1) {  // two 8 x 8 boxes: columns 0-7, then 8-15
-                const int bx = r >> 6, rr = r & 63;
-                i = 8 * qh + (rr >> 3);
-                j = 8 * bx + (rr & 7);
-            } else {         // one 16 x 8 box, row-major
-                i = 8 * qh + (r >> 4);
-                j = r & 15;
-            }
-            qij[idx] = (uint16_t)((i << 8) | j);
-        }
-        for (int idx = t; idx < 4 * 256; idx += 32 * kPipeSoftmaxWarp) {
-            const int kind = idx >> 8, rp = idx & 255;
-            int i, j;
-            tma_row_coords(g, kind, rp, i, j);
-            kij[idx] = (uint16_t)((i << 8) | j);
-        }
-        named_bar_sync(1, 32 * kPipeSoftmaxWarp);
+        named_bar_sync(1, 32 * kP16SoftmaxWarp);
         const int grp = warp >> 2;
         const int row = t - 128 * grp;
-        for (int kk = grp; kk < count; kk += kPipeRope) {
+        for (int kk = grp; kk < count; kk += kP16Rope) {
             const int s = kk % NSQ;
             if (!warp_wait(&qk_full[s], (kk / NSQ) & 1, abort_flag))
                 break;
@@ -390,13 +389,32 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
             const int kind = window_kind(g, wy, wx);
             const float4 *tab = theta ? table4 + it.h * 16 * (D / 8) : nullptr;
             if (theta) {
+                // window-local (i, j) of each row, in the order the boxes land
                 for (int qh = 0; qh < 2; ++qh) {
-                    const uint32_t ij = qij[(kind * 2 + qh) * 128 + row];
-                    rotate_row_f2<D>(st + (qh ? L::QB : L::QA), row, tab, (int)(ij >> 8), (int)(ij & 0xFF), false, 1.f);
+                    int i, j;
+                    if (kind & 1) {  // two 8 x 8 boxes: columns 0-7, then 8-15
+                        i = 8 * qh + ((row & 63) >> 3);
+                        j = 8 * (row >> 6) + (row & 7);
+                    } else {         // one 16 x 8 box, row-major
+                        i = 8 * qh + (row >> 4);
+                        j = row & 15;
+                    }
+                    rotate_row_f2<D>(st + (qh ? L::QB : L::QA), row, tab, i, j, false, 1.f);
                 }
                 for (int kh = 0; kh < 2; ++kh) {
-                    const uint32_t ij = kij[kind * 256 + kh * 128 + row];
-                    rotate_row_f2<D>(st + L::KT, kh * 128 + row, tab, (int)(ij >> 8), (int)(ij & 0xFF), false, 1.f);
+                    const int rp = kh * 128 + row;
+                    int i, j;
+                    if (kind == 1) {         // two 8-wide, 16-high boxes, each row-major
+                        i = (rp & 127) >> 3;
+                        j = 8 * (rp >> 7) + (rp & 7);
+                    } else if (kind == 3) {  // four 8 x 8 quadrants, each row-major
+                        i = 8 * (rp >> 7) + ((rp & 63) >> 3);
+                        j = 8 * ((rp >> 6) & 1) + (rp & 7);
+                    } else {                 // one 16 x 16 box, or two 16 x 8 boxes stacked
+                        i = rp >> 4;
+                        j = rp & 15;
+                    }
+                    rotate_row_f2<D>(st + L::KT, rp, tab, i, j, false, 1.f);
                 }
             }
             // per query tile: this row's allowed 64-key granules, and the
@@ -413,8 +431,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
                     gm = qh ? 0xC : 0x3;
                 else
                     gm = 1u << (2 * qh + lx);
-                reinterpret_cast<uint32_t *>(ms)[row] = gm;
                 if ((row & 31) == 0) {
+                    reinterpret_cast<uint32_t *>(ms)[row >> 5] = gm;
                     // the store of epilogue warp q = row / 32: 2 window rows x
                     // 16 columns, or 4 rows x 8 columns on the column seam
                     const int qw = row >> 5;
@@ -429,7 +447,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
                         shape = 0;
                     }
                     const int y0 = wrap(wy * 16 + iy + g.shift, g.H), x0 = wrap(wx * 16 + jx + g.shift, g.W);
-                    reinterpret_cast<int4 *>(ms + 512)[qw] = make_int4(x0, y0, b, shape | (it.h * D) << 4);
+                    reinterpret_cast<int4 *>(ms + 64)[qw] = make_int4(x0, y0, b, shape | (it.h * D) << 4);
                 }
             }
             fence_proxy_async_smem();
@@ -440,41 +458,32 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
                 mbar_arrive(&meta_full[(2 * kk + 1) % NM]);
             }
         }
-    } else if (warp < kPipeEpiWarp) {
-        // ================================================================ softmax groups
-        // group qh takes query tile qh of every item (TMEM buffer qh)
-        const int grp = (warp - kPipeSoftmaxWarp) >> 2;
-        const int row = t - 32 * kPipeSoftmaxWarp - 128 * grp;
-        const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    } else if (warp < kP16EpiWarp) {
+        // ================================================================ softmax
+        // warp (gr, quarter) takes keys [64 gr, 64 gr + 64) of the rows of lane
+        // quarter `quarter`, for every tile
+        const int gr = (warp - kP16SoftmaxWarp) >> 2, quarter = warp & 3, row = quarter * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
         const float c2 = scale * kLog2e;
         const float2 cc = make_float2(c2, c2);
         const float ninf = -INFINITY;
-        // group 0 takes the first turn
-        if (grp == 1 && count > 0)
-            warp_arrive(&turn[0]);
-        for (int kk = 0; kk < count; ++kk) {
-            const int kt = 2 * kk + grp, b = kt % NB, m = kt % NM;
+        for (int kt = 0; kt < 2 * count; ++kt) {
+            const int b = kt % NB, m = kt % NM;
             if (!warp_wait(&s_full[b], (kt / NB) & 1, abort_flag))
                 break;
             if (!warp_wait(&meta_full[m], (kt / NM) & 1, abort_flag))
                 break;
             tc_fence_after_sync();
-            // the granules are the same for the 32 rows of a warp (a warp's rows
-            // lie on one side of every seam), and the TMEM loads below are
-            // warp-collective: branch on lane 0's mask
-            const uint32_t gmask = __shfl_sync(0xffffffffu,
-                reinterpret_cast<const uint32_t *>(base + L::MRING + m * L::MSLOT)[row], 0);
-            const uint32_t sreg = tmem + lane_base + b * 256;
-            // pass 1: the max over the allowed 64-key granules
+            const bool on = (reinterpret_cast<const uint32_t *>(base + L::MRING + m * L::MSLOT)[quarter] >> gr) & 1u;
+            const uint32_t sreg = tmem + lane_base + b * 256 + gr * 64;  // S of this granule
+            const uint32_t preg = tmem + lane_base + b * 256;
+            // pass 1: the max over this granule, if the rows may attend to it
             float mx = ninf;
-#pragma unroll 1
-            for (int gi = 0; gi < 4; ++gi) {
-                if (!((gmask >> gi) & 1u))
-                    continue;
+            if (on) {
 #pragma unroll
                 for (int h2 = 0; h2 < 2; ++h2) {
                     float x[32];
-                    tmem_ld32(sreg + gi * 64 + h2 * 32, x);
+                    tmem_ld32(sreg + h2 * 32, x);
                     float a = fmax3(x[0], x[1], x[2]);
 #pragma unroll
                     for (int e = 3; e < 31; e += 2)
@@ -482,58 +491,44 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
                     mx = fmax3(mx, a, x[31]);
                 }
             }
+            // exchange with the other three granules' warps of this quarter
+            float *pm = pmax + b * 4 * 128 + row;
+            pm[gr * 128] = mx;
+            warp_arrive(&max_ready[b]);
+            if (!warp_wait(&max_ready[b], (kt / NB) & 1, abort_flag))
+                break;
+            mx = fmaxf(fmaxf(pm[0], pm[128]), fmaxf(pm[256], pm[384]));
             const float mneg = mx == ninf ? 0.f : -mx * c2;
             const float2 mm = make_float2(mneg, mneg);
-            // this group's turn at the exponentials: phase kk of turn[grp]
-            if (!warp_wait(&turn[grp], kk & 1, abort_flag))
-                break;
-            // pass 2: P = exp2(s c2 - m) over the allowed granules in chunks
-            // of 16 keys, the load of chunk q + 1 in flight while chunk q is
-            // exponentiated; chunk q's P (8 packed columns) lands below every
-            // S column still to be read
-            int gl = 0, ng = 0;  // allowed granules, in order, 2 bits each
-#pragma unroll
-            for (int gi = 0; gi < 4; ++gi)
-                if ((gmask >> gi) & 1u)
-                    gl |= gi << (2 * ng++);
-            const int nq = 4 * ng;
-            auto chunk_col = [&](int q) { return ((gl >> (2 * (q >> 2))) & 3) * 64 + (q & 3) * 16; };
+            // pass 2: P = exp2(s c2 - m) in chunks of 16 keys, granules 0 and
+            // 1 from the first chunk up, 2 and 3 from the last down, so that
+            // chunk c's P (8 packed columns at p16_pcol) lands on S columns of
+            // this granule already read; zeros if the rows may not attend
             float2 lq[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-            uint32_t xa[16], xb[16];
-            tmem_ld16_issue(sreg + chunk_col(0), xa);
-            tmem_wait_ld16(xa);
+            if (on) {
 #pragma unroll 1
-            for (int q = 0; q < nq; q += 2) {
-                tmem_ld16_issue(sreg + chunk_col(q + 1), xb);  // nq is a multiple of 4
-                exp_chunk16(xa, cc, mm, lq, sreg + (chunk_col(q) >> 1));
-                tmem_wait_ld16(xb);
-                // (after the last pair: a spare load of chunk 0, never used)
-                tmem_ld16_issue(sreg + chunk_col(q + 2 < nq ? q + 2 : 0), xa);
-                exp_chunk16(xb, cc, mm, lq, sreg + (chunk_col(q + 1) >> 1));
-                tmem_wait_ld16(xa);
-            }
-            // zeros over the packed columns of the masked granules, once every
-            // S column has been read
-#pragma unroll 1
-            for (int gi = 0; gi < 4; ++gi) {
-                if ((gmask >> gi) & 1u)
-                    continue;
+                for (int q = 0; q < 4; ++q) {
+                    const int c = gr < 2 ? q : 3 - q;
+                    uint32_t xa[16];
+                    tmem_ld16_issue(sreg + c * 16, xa);
+                    tmem_wait_ld16(xa);
+                    exp_chunk16(xa, cc, mm, lq, preg + p16_pcol(4 * gr + c));
+                }
+            } else {
                 uint32_t z[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e)
                     z[e] = 0u;
-                tmem_st16(sreg + gi * 32, z);
-                tmem_st16(sreg + gi * 32 + 16, z);
+                tmem_st16(preg + p16_pcol(4 * gr), z);
+                tmem_st16(preg + p16_pcol(4 * gr) + 16, z);
             }
-            // the other group's turn (group 1's last one is never taken)
-            warp_arrive(&turn[grp ^ 1]);
             const float2 l2 = __fadd2_rn(lq[0], lq[1]);
-            osum[b * 128 + row] = l2.x + l2.y;
+            osum[(b * 4 + gr) * 128 + row] = l2.x + l2.y;
             tmem_wait_st();
             tc_fence_before_sync();
             warp_arrive(&p_full[b]);
         }
-    } else if (warp < kPipeLoadWarp) {
+    } else if (warp < kP16LoadWarp) {
         // ================================================================ epilogue
         const int quarter = warp & 3;
         const int row = quarter * 32 + lane;
@@ -541,19 +536,25 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         int kt = 0;
         for (; kt < 2 * count; ++kt) {
             const int b = kt % NB, e = kt % L::NO, m = kt % NM;
+            // (p_full: the row sums the softmax warps wrote before arriving)
             if (!warp_wait(&o_full[b], (kt / NB) & 1, abort_flag) ||
                 !warp_wait(&p_full[b], (kt / NB) & 1, abort_flag) ||
                 !warp_wait(&meta_full[m], (kt / NM) & 1, abort_flag))
                 break;
             tc_fence_after_sync();
-            const int4 rec = reinterpret_cast<const int4 *>(base + L::MRING + m * L::MSLOT + 512)[quarter];
-            const float inv = 1.f / osum[b * 128 + row];
+            const int4 rec = reinterpret_cast<const int4 *>(base + L::MRING + m * L::MSLOT + 64)[quarter];
+            const float *os = osum + b * 4 * 128 + row;
+            const float inv = 1.f / ((os[0] + os[128]) + (os[256] + os[384]));
             const float2 i2 = make_float2(inv, inv);
-            uint4 y[D / 8];
+            // this warp's staging rows have been read by its stores of tile kt - NO
+            if (kt >= L::NO)
+                bulk_wait_group_read<L::NO - 1>();
+            __syncwarp();
+            uint8_t *ost = base + L::OSTAGE + e * 256 * D;
 #pragma unroll
             for (int h2 = 0; h2 < D / 32; ++h2) {
                 float o[32];
-                tmem_ld32(tmem + lane_base + b * 256 + 128 + h2 * 32, o);
+                tmem_ld32(tmem + lane_base + b * 256 + kP16O + h2 * 32, o);
                 if (h2 == D / 32 - 1) {
                     tc_fence_before_sync();
                     warp_arrive(&t_free[b]);
@@ -564,18 +565,11 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
                         f[q] = __fmul2_rn(make_float2(o[8 * c + 2 * q], o[8 * c + 2 * q + 1]), i2);
-                    y[h2 * 4 + c] = make_uint4(pack_bf16x2(f[0].x, f[0].y), pack_bf16x2(f[1].x, f[1].y),
-                                               pack_bf16x2(f[2].x, f[2].y), pack_bf16x2(f[3].x, f[3].y));
+                    *reinterpret_cast<uint4 *>(ost + swz_offset(row, h2 * 4 + c, 2 * D)) =
+                        make_uint4(pack_bf16x2(f[0].x, f[0].y), pack_bf16x2(f[1].x, f[1].y),
+                                   pack_bf16x2(f[2].x, f[2].y), pack_bf16x2(f[3].x, f[3].y));
                 }
             }
-            // this warp's staging rows have been read by its stores of tile kt - NO
-            if (kt >= L::NO)
-                bulk_wait_group_read<L::NO - 1>();
-            __syncwarp();
-            uint8_t *ost = base + L::OSTAGE + e * 256 * D;
-#pragma unroll
-            for (int c = 0; c < D / 8; ++c)
-                *reinterpret_cast<uint4 *>(ost + swz_offset(row, c, 2 * D)) = y[c];
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {

@@ -586,7 +586,7 @@ int launch_pipe16(const void *q, const void *k, const void *v, const float *thet
     const int64_t grid = items < sm_count() ? items : sm_count();
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
-    cfg.blockDim = dim3(kPipeThreads);
+    cfg.blockDim = dim3(kP16Threads);
     cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -1237,7 +1237,7 @@ int winattn_launch_info(int B, int H_img, int W_img, int M, int shift, int heads
         const int64_t items = g.wph * g.heads;  // window-heads: two query tiles each
         if (work_items) *work_items = items;
         if (grid) *grid = (int)(items < kAssumedSMs ? items : kAssumedSMs);
-        if (threads) *threads = kPipeThreads;
+        if (threads) *threads = kP16Threads;
         if (smem_bytes) *smem_bytes = (int)pipe16_smem(g);
     } else if (kind == kSmall) {
         if (grid) *grid = (int)(g.items < kAssumedSMs ? g.items : kAssumedSMs);
