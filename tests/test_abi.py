@@ -112,6 +112,9 @@ GENERIC, SMALL, LARGE, SIMT, PIPE, PIPE16 = 0, 1, 2, 3, 4, 5
     (1, 10, 10, 10, 0, 1, 32, 0, 1, 1, SMALL),       # 100 tokens: one ragged tile
     (1, 8, 8, 8, 0, 80, 32, 0, 2, 1, GENERIC),       # too many heads for a shared-memory RoPE table
     (64, 56, 56, 32, 16, 3, 32, 0, 1, 8, LARGE),     # FlashSwin-T at M = 32: 56 padded to 64, pad keys masked
+    (64, 56, 56, 16, 8, 3, 32, 0, 1, 2, PIPE16),     # FlashSwin-T at M = 16: padded by half a window
+    (2, 40, 24, 16, 0, 2, 32, 0, 1, 2, PIPE16),      # the same without shift
+    (1, 36, 32, 16, 8, 2, 32, 0, 1, 2, LARGE),       # padded by 12 rows: pads split key granules
     (2, 10, 13, 4, 2, 2, 32, 0, 8, 1, GENERIC),      # padded 12 x 16 grid of 16-token windows
 ])
 def test_launch_plan(lib, B, H, W, M, shift, heads, d, rank, U, tiles, kernel):

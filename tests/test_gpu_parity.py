@@ -60,7 +60,10 @@ SMALL = [
     # grids that are not multiples of M: padded, pad positions masked and never written
     ("m32_s16_pad56", 1, 56, 56, 32, 16, 2, 32, "bf16", "learned", 0),
     ("m32_s0_pad56", 1, 56, 56, 32, 0, 2, 32, "bf16", "standard", 0),
-    ("m16_s8_pad_d64", 1, 56, 40, 16, 8, 2, 64, "bf16", "learned", 0),
+    ("m16_s8_pad_d64", 1, 56, 40, 16, 8, 2, 64, "bf16", "learned", 0),   # half-window pads: 16 x 16 kernel
+    ("m16_s0_pad_d32", 2, 40, 24, 16, 0, 2, 32, "bf16", "learned", 0),   # the same without shift
+    ("m16_s8_padw", 1, 32, 56, 16, 8, 3, 32, "bf16", "standard", 0),     # pad columns only
+    ("m16_s8_pad12", 1, 36, 32, 16, 8, 2, 32, "bf16", "learned", 0),     # 12 pad rows: large-window kernel
     ("m4_s2_pad", 2, 10, 13, 4, 2, 2, 32, "bf16", "learned", 0),
     ("m8_s4_pad20", 1, 20, 20, 8, 4, 2, 32, "bf16", "learned", 0),
     ("m7_s3_pad_r16", 1, 10, 9, 7, 3, 2, 32, "bf16", None, 16),
@@ -190,10 +193,12 @@ FALLBACKS = [
     ((_lib.KERNEL_PIPE, _lib.KERNEL_SMALL), "swin", 4, _lib.KERNEL_GENERIC),
     ((_lib.KERNEL_PIPE16,), "sweep_M16_d32_s8", 8, _lib.KERNEL_LARGE),
     ((_lib.KERNEL_PIPE16,), "sweep_M16_d64_s8", 0, _lib.KERNEL_LARGE),
+    ((_lib.KERNEL_PIPE16,), "flashswin_M16", 8, _lib.KERNEL_LARGE),
 ]
 
 
-@pytest.mark.parametrize("off,name,shift,serves", FALLBACKS, ids=["large-off", "pipe-off", "pipe-small-off", "pipe16-off-s8", "pipe16-off-d64-s0"])
+@pytest.mark.parametrize("off,name,shift,serves", FALLBACKS, ids=["large-off", "pipe-off", "pipe-small-off", "pipe16-off-s8", "pipe16-off-d64-s0",
+                              "pipe16-off-flashswin"])
 def test_fallback_kernels(off, name, shift, serves):
     """With specialised kernels switched off, their problems run on the next
     kernel that serves them (the path a build with an unexpected register
@@ -206,6 +211,8 @@ def test_fallback_kernels(off, name, shift, serves):
         assert rc == 0 and info["kernel"] == serves
         if w.name == "dense":
             G.sampled_compare(w, shift, images=[0, w.B - 1], extra_windows=2)
+        elif w.name.startswith("flashswin"):
+            G.sampled_compare(w, shift, images=[0, w.B - 1], extra_windows=2, max_units=12)
         elif w.name.startswith("sweep_"):
             G.sampled_compare(w, shift, images=[w.B - 1], heads=[0, w.heads - 1], extra_windows=1, max_units=16)
         else:

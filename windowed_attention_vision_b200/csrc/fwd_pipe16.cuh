@@ -48,6 +48,12 @@
 // Wrap masks are structural: the key boxes of a window are its wrap-label
 // regions (halves at a seam, quadrants in the corner window), each a whole
 // number of 64-key granules, and a query tile never straddles the row seam.
+// A map padded by half a window (H or W 8 short of a multiple of 16, as
+// FlashSwin-T's 56 x 56 at M = 16) has its pad positions in the last window
+// row and column, in exactly those halves: with shift 8 they are the halves
+// that wrap labels already separate, without shift the last window row and
+// column are split the same way.  Pad boxes load as zeros (out of the map)
+// and are never stored.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -87,8 +93,9 @@ struct Pipe16Layout {
     // metadata ring, per query tile: allowed granules of the rows of each lane
     // quarter (u32[4]; a quarter's rows lie on one side of every seam), then
     // at byte 64 the output TMA stores of each epilogue warp: int4 {x0, y0,
-    // image, box shape | head column << 4}; NM = 2 NSQ + 2 orders the writer
-    // of tile k + NM after the last reader of tile k
+    // image, box shape | head column << 4} (shape 0: 16 x 2 tokens, 1: 8 x 4,
+    // 2: pad positions, not stored); NM = 2 NSQ + 2 orders the writer of tile
+    // k + NM after the last reader of tile k
     static constexpr int NM = 2 * NSQ + 2;
     static constexpr uint32_t MSLOT = 64 + 4 * 16;
     static constexpr uint32_t VRING = NSQ * QK_STAGE;
@@ -104,10 +111,20 @@ struct Pipe16Layout {
 };
 
 // Shapes this kernel serves: bf16, 16 x 16 windows, no rank-r factors, shift
-// 0 or 8, a map that is a whole number of windows.
+// 0 or 8, a map that is a whole number of windows or padded by half a window.
 __host__ __device__ inline bool pipe16_ok(const Geometry &g)
 {
-    return g.M == 16 && g.rank == 0 && (g.shift == 0 || g.shift == 8) && !g.padded && (g.d == 32 || g.d == 64);
+    return g.M == 16 && g.rank == 0 && (g.shift == 0 || g.shift == 8) && (g.Hp - g.H == 0 || g.Hp - g.H == 8) &&
+           (g.Wp - g.W == 0 || g.Wp - g.W == 8) && (g.d == 32 || g.d == 64);
+}
+
+// Box layout of a window: bit 0 = split into column halves (the column wrap
+// seam, or pad columns), bit 1 = split into row halves (the row seam, or pad
+// rows); both only in the last window column / row.
+__device__ __forceinline__ int pipe16_kind(const Geometry &g, int wy, int wx)
+{
+    return (wx == g.nWx - 1 && (g.shift || g.Wp != g.W) ? 1 : 0) |
+           (wy == g.nWy - 1 && (g.shift || g.Hp != g.H) ? 2 : 0);
 }
 
 // Tensor maps of the output stores: boxes of 16 x 2 and 8 x 4 tokens (32 rows
@@ -222,7 +239,7 @@ __global__ void __launch_bounds__(kP16Threads, 1)
             const Item it = decode_item_head_minor(g, first + kk * stride);
             int b, wy, wx;
             window_of(it.pack, b, wy, wx);
-            const int kind = window_kind(g, wy, wx);
+            const int kind = pipe16_kind(g, wy, wx);
             const uint32_t sst = sbase + s * L::QK_STAGE;
             if (lane == 0)
                 mbar_arrive_expect_tx(&qk_full[s], (uint32_t)(L::QK_STAGE));
@@ -234,9 +251,9 @@ __global__ void __launch_bounds__(kP16Threads, 1)
                 const int qh = lane >> 2, bi = lane & 3;
                 const int nbox = (kind & 1) ? 2 : 1;
                 if (bi < nbox) {
-                    int y0 = wrap(wy * 16 + 8 * qh + g.shift, g.H);
-                    int x0 = wrap(wx * 16 + 8 * bi + g.shift, g.W);
-                    debug_box(c0, x0, y0, b, D, g.heads * D, nbox == 2 ? 8 : 16, 8, g.W, g.H, g.B);
+                    int y0 = wrap(wy * 16 + 8 * qh + g.shift, g.Hp);
+                    int x0 = wrap(wx * 16 + 8 * bi + g.shift, g.Wp);
+                    debug_box(c0, x0, y0, b, D, g.heads * D, nbox == 2 ? 8 : 16, 8, g.Wp, g.Hp, g.B);
                     tma_load_4d(sst + (qh ? L::QB : L::QA) + (uint32_t)(bi * 64 * 2 * D),
                                 pick_map(tm_q, nbox == 2 ? 3 : 2), c0, x0, y0, b, &qk_full[s]);
                 }
@@ -246,9 +263,9 @@ __global__ void __launch_bounds__(kP16Threads, 1)
                 if (bi < nbox) {
                     const int iy0 = (kind & 2) ? ((kind == 3 ? bi >> 1 : bi) * 8) : 0;
                     const int jx0 = (kind & 1) ? ((kind == 3 ? bi & 1 : bi) * 8) : 0;
-                    int y0 = wrap(wy * 16 + iy0 + g.shift, g.H);
-                    int x0 = wrap(wx * 16 + jx0 + g.shift, g.W);
-                    debug_box(c0, x0, y0, b, D, g.heads * D, (kind & 1) ? 8 : 16, (kind & 2) ? 8 : 16, g.W, g.H, g.B);
+                    int y0 = wrap(wy * 16 + iy0 + g.shift, g.Hp);
+                    int x0 = wrap(wx * 16 + jx0 + g.shift, g.Wp);
+                    debug_box(c0, x0, y0, b, D, g.heads * D, (kind & 1) ? 8 : 16, (kind & 2) ? 8 : 16, g.Wp, g.Hp, g.B);
                     tma_load_4d(sst + L::KT + (uint32_t)(bi * (256 / nbox) * 2 * D), pick_map(tm_k, kind), c0, x0, y0,
                                 b, &qk_full[s]);
                 }
@@ -273,7 +290,7 @@ __global__ void __launch_bounds__(kP16Threads, 1)
             const Item it = decode_item_head_minor(g, first + kk * stride);
             int b, wy, wx;
             window_of(it.pack, b, wy, wx);
-            const int kind = window_kind(g, wy, wx);
+            const int kind = pipe16_kind(g, wy, wx);
             if (lane == 0)
                 mbar_arrive_expect_tx(&v_full[s], (uint32_t)L::V_STAGE);
             __syncwarp();
@@ -282,10 +299,10 @@ __global__ void __launch_bounds__(kP16Threads, 1)
                 const int bi = lane;
                 const int iy0 = (kind & 2) ? ((kind == 3 ? bi >> 1 : bi) * 8) : 0;
                 const int jx0 = (kind & 1) ? ((kind == 3 ? bi & 1 : bi) * 8) : 0;
-                int y0 = wrap(wy * 16 + iy0 + g.shift, g.H);
-                int x0 = wrap(wx * 16 + jx0 + g.shift, g.W);
+                int y0 = wrap(wy * 16 + iy0 + g.shift, g.Hp);
+                int x0 = wrap(wx * 16 + jx0 + g.shift, g.Wp);
                 int c0 = it.h * D;
-                debug_box(c0, x0, y0, b, D, g.heads * D, (kind & 1) ? 8 : 16, (kind & 2) ? 8 : 16, g.W, g.H, g.B);
+                debug_box(c0, x0, y0, b, D, g.heads * D, (kind & 1) ? 8 : 16, (kind & 2) ? 8 : 16, g.Wp, g.Hp, g.B);
                 tma_load_4d(sbase + L::VRING + s * L::V_STAGE + (uint32_t)(bi * (256 / nbox) * 2 * D),
                             pick_map(tm_v, kind), c0, x0, y0, b, &v_full[s]);
             }
@@ -386,7 +403,7 @@ __global__ void __launch_bounds__(kP16Threads, 1)
             const Item it = decode_item_head_minor(g, first + kk * stride);
             int b, wy, wx;
             window_of(it.pack, b, wy, wx);
-            const int kind = window_kind(g, wy, wx);
+            const int kind = pipe16_kind(g, wy, wx);
             const float4 *tab = theta ? table4 + it.h * 16 * (D / 8) : nullptr;
             if (theta) {
                 // window-local (i, j) of each row, in the order the boxes land
@@ -446,7 +463,10 @@ __global__ void __launch_bounds__(kP16Threads, 1)
                         jx = 0;
                         shape = 0;
                     }
-                    const int y0 = wrap(wy * 16 + iy + g.shift, g.H), x0 = wrap(wx * 16 + jx + g.shift, g.W);
+                    const int y0 = wrap(wy * 16 + iy + g.shift, g.Hp), x0 = wrap(wx * 16 + jx + g.shift, g.Wp);
+                    // a box of pad positions (all of its tokens are) is not stored
+                    if (y0 >= g.H || x0 >= g.W)
+                        shape = 2;
                     reinterpret_cast<int4 *>(ms + 64)[qw] = make_int4(x0, y0, b, shape | (it.h * D) << 4);
                 }
             }
@@ -572,7 +592,7 @@ __global__ void __launch_bounds__(kP16Threads, 1)
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) {
+            if (lane == 0 && (rec.w & 15) != 2) {
                 int c0 = rec.w >> 4, x0 = rec.x, y0 = rec.y, bb = rec.z;
                 const int shape = rec.w & 15;
                 debug_box(c0, x0, y0, bb, D, g.heads * D, shape ? 8 : 16, shape ? 4 : 2, g.W, g.H, g.B);

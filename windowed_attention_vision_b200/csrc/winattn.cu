@@ -231,10 +231,14 @@ KernelKind choose_kernel(const Geometry &g, int dtype, bool want_lse = false)
     if (dtype == WINATTN_FP32)
         return kSimt;
     // the generic kernel resolves every token through the index math, pad
-    // positions of a padded grid included; of the specialised kernels only
-    // the large-window one masks pad keys
-    if (g.padded)
+    // positions of a padded grid included; of the specialised kernels the
+    // large-window one masks pad keys, and the 16 x 16 pipelined one serves
+    // pads of half a window (whole key granules and store boxes)
+    if (g.padded) {
+        if (!want_lse && kernel_enabled(kPipe16) && pipe16_ok(g) && pipe16_smem(g) <= kMaxSmem)
+            return kPipe16;
         return kernel_enabled(kLarge) && large_ok(g) ? kLarge : kGeneric;
+    }
     if (kernel_enabled(kPipe) && pipe_ok(g) && (uint64_t)g.heads * g.M * (g.d / 4) * 8 <= kSmallTableMax &&
         pipe_smem(g) <= kMaxSmem)
         return kPipe;
