@@ -228,6 +228,8 @@ LSE_CASES = [
     ("m8_s0_d64_lse", 2, 16, 24, 8, 0, 2, 64, "bf16", "standard", 0),   # pipelined, d = 64
     ("m4_s2_lse", 2, 8, 12, 4, 2, 2, 32, "bf16", "learned", 0),         # generic (small kernel has no lse)
     ("m12_s6_r16_lse", 1, 24, 24, 12, 6, 2, 32, "bf16", "learned", 16), # generic, ragged tiles, factors
+    ("m16_s8_lse", 2, 32, 48, 16, 8, 2, 32, "bf16", "learned", 0),     # pipelined 16 x 16
+    ("m16_s8_pad_d64_lse", 1, 56, 40, 16, 8, 2, 64, "bf16", "learned", 0),  # 16 x 16, half-window pads
     ("m32_s16_lse", 2, 64, 64, 32, 16, 2, 32, "bf16", "learned", 0),    # large-window
     ("m16_s0_d64_r16_lse", 1, 32, 48, 16, 0, 2, 64, "bf16", "learned", 16),
     ("m32_s16_pad56_lse", 1, 56, 56, 32, 16, 2, 32, "bf16", "learned", 0),  # large-window, padded

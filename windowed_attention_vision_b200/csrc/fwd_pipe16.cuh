@@ -112,6 +112,8 @@ struct Pipe16Layout {
 
 // Shapes this kernel serves: bf16, 16 x 16 windows, no rank-r factors, shift
 // 0 or 8, a map that is a whole number of windows or padded by half a window.
+// With `lse` it also writes each token's log-sum-exp (natural log of the sum
+// of exp(score) over the row), as the other forward kernels do.
 __host__ __device__ inline bool pipe16_ok(const Geometry &g)
 {
     return g.M == 16 && g.rank == 0 && (g.shift == 0 || g.shift == 8) && (g.Hp - g.H == 0 || g.Hp - g.H == 8) &&
@@ -151,7 +153,8 @@ __device__ __forceinline__ void exp_chunk16(const uint32_t (&x)[16], float2 cc, 
 
 template <int D>
 __global__ void __launch_bounds__(kP16Threads, 1)
-    winattn_fwd_pipe16_kernel(const float *__restrict__ theta, const Geometry g, const float scale,
+    winattn_fwd_pipe16_kernel(const float *__restrict__ theta, float *__restrict__ lse, const Geometry g,
+                              const float scale,
                               const __grid_constant__ WindowMaps tm_q, const __grid_constant__ WindowMaps tm_k,
                               const __grid_constant__ WindowMaps tm_v, const __grid_constant__ Pipe16StoreMaps tm_o)
 {
@@ -518,6 +521,11 @@ __global__ void __launch_bounds__(kP16Threads, 1)
             if (!warp_wait(&max_ready[b], (kt / NB) & 1, abort_flag))
                 break;
             mx = fmaxf(fmaxf(pm[0], pm[128]), fmaxf(pm[256], pm[384]));
+            // the row max for the epilogue's log-sum-exp: granule 0's slot
+            // takes the combined max (no larger than any partial it replaces
+            // for a warp still reading them, so their max is unchanged)
+            if (gr == 0)
+                pm[0] = mx;
             const float mneg = mx == ninf ? 0.f : -mx * c2;
             const float2 mm = make_float2(mneg, mneg);
             // pass 2: P = exp2(s c2 - m) in chunks of 16 keys, granules 0 and
@@ -564,7 +572,15 @@ __global__ void __launch_bounds__(kP16Threads, 1)
             tc_fence_after_sync();
             const int4 rec = reinterpret_cast<const int4 *>(base + L::MRING + m * L::MSLOT + 64)[quarter];
             const float *os = osum + b * 4 * 128 + row;
-            const float inv = 1.f / ((os[0] + os[128]) + (os[256] + os[384]));
+            const float lrow = (os[0] + os[128]) + (os[256] + os[384]);
+            const float inv = 1.f / lrow;
+            if (lse && (rec.w & 15) != 2) {
+                // this row's token: row `lane` of the warp's store box, row-major
+                const int bw = (rec.w & 15) ? 8 : 16;
+                const int y = rec.y + lane / bw, x = rec.x + lane % bw, h = (rec.w >> 4) / D;
+                lse[(((int64_t)rec.z * g.H + y) * g.W + x) * g.heads + h] =
+                    (pmax[b * 4 * 128 + row] * (scale * kLog2e) + log2f(lrow)) * kLn2;
+            }
             const float2 i2 = make_float2(inv, inv);
             // this warp's staging rows have been read by its stores of tile kt - NO
             if (kt >= L::NO)

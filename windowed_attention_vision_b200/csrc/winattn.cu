@@ -235,15 +235,14 @@ KernelKind choose_kernel(const Geometry &g, int dtype, bool want_lse = false)
     // large-window one masks pad keys, and the 16 x 16 pipelined one serves
     // pads of half a window (whole key granules and store boxes)
     if (g.padded) {
-        if (!want_lse && kernel_enabled(kPipe16) && pipe16_ok(g) && pipe16_smem(g) <= kMaxSmem)
+        if (kernel_enabled(kPipe16) && pipe16_ok(g) && pipe16_smem(g) <= kMaxSmem)
             return kPipe16;
         return kernel_enabled(kLarge) && large_ok(g) ? kLarge : kGeneric;
     }
     if (kernel_enabled(kPipe) && pipe_ok(g) && (uint64_t)g.heads * g.M * (g.d / 4) * 8 <= kSmallTableMax &&
         pipe_smem(g) <= kMaxSmem)
         return kPipe;
-    // (the 16 x 16 pipelined kernel does not write the log-sum-exp)
-    if (!want_lse && kernel_enabled(kPipe16) && pipe16_ok(g) && pipe16_smem(g) <= kMaxSmem)
+    if (kernel_enabled(kPipe16) && pipe16_ok(g) && pipe16_smem(g) <= kMaxSmem)
         return kPipe16;
     // (the small-window kernel does not write the log-sum-exp)
     if (!want_lse && kernel_enabled(kSmall) && g.N <= kTileRows &&
@@ -566,8 +565,8 @@ int launch_pipe(const void *q, const void *k, const void *v, const float *theta,
 }
 
 template <int D>
-int launch_pipe16(const void *q, const void *k, const void *v, const float *theta, void *out, const Geometry &g,
-                  cudaStream_t stream)
+int launch_pipe16(const void *q, const void *k, const void *v, const float *theta, void *out, float *lse,
+                  const Geometry &g, cudaStream_t stream)
 {
     static_assert(sizeof(Pipe16StoreMaps) == 2 * sizeof(CUtensorMap), "two store maps");
     MapSet ms;
@@ -599,7 +598,7 @@ int launch_pipe16(const void *q, const void *k, const void *v, const float *thet
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const float scale = 1.0f / std::sqrt((float)g.d);
-    if (cudaLaunchKernelEx(&cfg, winattn_fwd_pipe16_kernel<D>, theta, g, scale, maps[0], maps[1], maps[2], om) !=
+    if (cudaLaunchKernelEx(&cfg, winattn_fwd_pipe16_kernel<D>, theta, lse, g, scale, maps[0], maps[1], maps[2], om) !=
         cudaSuccess)
         return WINATTN_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? WINATTN_OK : WINATTN_ERR_CUDA;
@@ -622,7 +621,8 @@ int dispatch(const void *q, const void *k, const void *v, const float *theta, co
         return g.d == 32 ? launch_pipe<32>(q, k, v, theta, out, lse, g, s)
                          : launch_pipe<64>(q, k, v, theta, out, lse, g, s);
     if (kind == kPipe16)
-        return g.d == 32 ? launch_pipe16<32>(q, k, v, theta, out, g, s) : launch_pipe16<64>(q, k, v, theta, out, g, s);
+        return g.d == 32 ? launch_pipe16<32>(q, k, v, theta, out, lse, g, s)
+                         : launch_pipe16<64>(q, k, v, theta, out, lse, g, s);
     if (kind == kSmall) {
         switch (g.d * 100 + g.rank) {
         case 3200: return launch_small<32, 0>(q, k, v, theta, bias, out, g, s);
