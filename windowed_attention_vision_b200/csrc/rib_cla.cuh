@@ -115,7 +115,9 @@ __global__ void __launch_bounds__(kGateThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(base);
-    float *s_dw = reinterpret_cast<float *>(base + GateLayout::bias_off(C));  // [C][9], then dw_b, pw_b
+    // depth-wise weights [9 taps][C] (a tap's 16 channels of an atom are four
+    // float4 loads, the same address for every lane of a warp), then dw_b, pw_b
+    float *s_dw = reinterpret_cast<float *>(base + GateLayout::bias_off(C));
     float *s_dwb = s_dw + 9 * C, *s_pwb = s_dwb + C;
     uint64_t *bar = reinterpret_cast<uint64_t *>(base + GateLayout::bar_off(C));
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bar + 1);
@@ -144,8 +146,10 @@ __global__ void __launch_bounds__(kGateThreads, 1)
         *reinterpret_cast<uint4 *>(dst + swz_offset(co, 0, 32)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         *reinterpret_cast<uint4 *>(dst + swz_offset(co, 1, 32)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
     }
-    for (int idx = tid; idx < 9 * C; idx += kGateThreads)
-        s_dw[idx] = __ldg(dw + idx);
+    for (int idx = tid; idx < 9 * C; idx += kGateThreads) {
+        const int ch = idx / 9, tap = idx - ch * 9;
+        s_dw[tap * C + ch] = __ldg(dw + idx);
+    }
     for (int idx = tid; idx < C; idx += kGateThreads) {
         s_dwb[idx] = __ldg(dw_b + idx);
         s_pwb[idx] = __ldg(pw_b + idx);
@@ -190,10 +194,14 @@ __global__ void __launch_bounds__(kGateThreads, 1)
                         const uint4 u0 = __ldg(src), u1 = __ldg(src + 1);
                         const uint32_t wv[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
                         const int tap = (dy + 1) * 3 + (dx + 1);
+                        const float4 *wt = reinterpret_cast<const float4 *>(s_dw + tap * C + a * 16);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            acc[2 * e] = fmaf(s_dw[(a * 16 + 2 * e) * 9 + tap], bf16lo(wv[e]), acc[2 * e]);
-                            acc[2 * e + 1] = fmaf(s_dw[(a * 16 + 2 * e + 1) * 9 + tap], bf16hi(wv[e]), acc[2 * e + 1]);
+                        for (int e4 = 0; e4 < 4; ++e4) {
+                            const float4 wq = wt[e4];
+                            acc[4 * e4 + 0] = fmaf(wq.x, bf16lo(wv[2 * e4]), acc[4 * e4 + 0]);
+                            acc[4 * e4 + 1] = fmaf(wq.y, bf16hi(wv[2 * e4]), acc[4 * e4 + 1]);
+                            acc[4 * e4 + 2] = fmaf(wq.z, bf16lo(wv[2 * e4 + 1]), acc[4 * e4 + 2]);
+                            acc[4 * e4 + 3] = fmaf(wq.w, bf16hi(wv[2 * e4 + 1]), acc[4 * e4 + 3]);
                         }
                     }
             }
@@ -235,11 +243,16 @@ __global__ void __launch_bounds__(kGateThreads, 1)
                 const uint4 u0 = op[0], u1 = op[1];
                 const uint32_t ov[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
                 uint32_t pk[8];
+                const float4 *bq = reinterpret_cast<const float4 *>(s_pwb + a * 16);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float g0 = 1.f / (1.f + __expf(-(gv[2 * e] + s_pwb[a * 16 + 2 * e])));
-                    const float g1 = 1.f / (1.f + __expf(-(gv[2 * e + 1] + s_pwb[a * 16 + 2 * e + 1])));
-                    pk[e] = pack_bf16x2(bf16lo(ov[e]) * g0, bf16hi(ov[e]) * g1);
+                for (int e4 = 0; e4 < 4; ++e4) {
+                    const float4 bb = bq[e4];
+                    const float g0 = 1.f / (1.f + __expf(-(gv[4 * e4] + bb.x)));
+                    const float g1 = 1.f / (1.f + __expf(-(gv[4 * e4 + 1] + bb.y)));
+                    const float g2 = 1.f / (1.f + __expf(-(gv[4 * e4 + 2] + bb.z)));
+                    const float g3 = 1.f / (1.f + __expf(-(gv[4 * e4 + 3] + bb.w)));
+                    pk[2 * e4] = pack_bf16x2(bf16lo(ov[2 * e4]) * g0, bf16hi(ov[2 * e4]) * g1);
+                    pk[2 * e4 + 1] = pack_bf16x2(bf16lo(ov[2 * e4 + 1]) * g2, bf16hi(ov[2 * e4 + 1]) * g3);
                 }
                 uint4 *dp = reinterpret_cast<uint4 *>(out + tok * C + a * 16);
                 dp[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
