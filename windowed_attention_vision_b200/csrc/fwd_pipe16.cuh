@@ -1,5 +1,6 @@
 // Persistent, role-pipelined forward for 16 x 16 windows (256 tokens) without
-// rank-r factors, shift 0 or 8, on whole maps: FlashSwin-T's M = 16 ("FLASHSWIN"
+// rank-r factors, shift 0 or 8, on whole maps or maps padded by half a window,
+// optionally saving each row's log-sum-exp: FlashSwin-T's M = 16 ("FLASHSWIN"
 // page, section "무엇과 다른가": from M = 16 the fused kernel overtakes Swin),
 // and the M = 16 point of the window-size sweep.
 //
@@ -16,14 +17,14 @@
 //   warp 31       V loader: the window's V boxes into an NSV-stage ring, once
 //                 the item's RoPE is done;
 //   warps 0-7     two RoPE warpgroups, alternate items: rotate the item's 256
-//                 query rows and 256 key rows in place in fp32, write each
-//                 query row's allowed 64-key granules and each epilogue warp's
-//                 store records;
+//                 query rows and 256 key rows in place in fp32, write the
+//                 allowed 64-key granules of each TMEM lane quarter's rows
+//                 and each epilogue warp's store record;
 //   warp 29       S issuer: S = Q K^T of each query tile (M = 128, N = 256)
 //                 into TMEM buffer (tile % 2); after both tiles of an item the
 //                 Q/K stage goes back to the loader;
 //   warp 30       P V issuer: O = P V (P from TMEM, 256 keys) into the same
-//                 buffer's columns 192 onwards; after both tiles the V stage
+//                 buffer's columns 96 onwards; after both tiles the V stage
 //                 goes back;
 //   warps 8-23    softmax, sixteen warps on every tile: warp (g, quarter)
 //                 takes the 64-key granule g of the 32 rows of TMEM lane
@@ -69,7 +70,7 @@ namespace winattn {
 
 constexpr int kP16Bufs = 2;  // TMEM buffers of 256 columns (one per query tile of an item)
 constexpr int kP16Rope = 2;                          // RoPE warpgroups (item k goes to group k % 2)
-constexpr int kP16SoftmaxWarp = 4 * kP16Rope;        // first softmax warp: two teams of eight
+constexpr int kP16SoftmaxWarp = 4 * kP16Rope;        // first of the sixteen softmax warps
 constexpr int kP16EpiWarp = kP16SoftmaxWarp + 16;
 constexpr int kP16LoadWarp = kP16EpiWarp + 4;        // Q/K loader; S issuer, P V issuer and V loader follow
 constexpr int kP16Threads = (kP16LoadWarp + 4) * 32;
@@ -161,8 +162,8 @@ __global__ void __launch_bounds__(kP16Threads, 1)
     using L = Pipe16Layout<D>;
     constexpr int NSQ = L::NSQ, NSV = L::NSV, NM = L::NM, NB = kP16Bufs;
     // Items alternate between the two RoPE groups, so an item's Q/K stage
-    // (item % NSQ) must always fall to the same group; tiles alternate
-    // between the softmax groups and share a metadata slot every NM tiles.
+    // (item % NSQ) must always fall to the same group; query tiles share a
+    // metadata slot every NM tiles.
     static_assert(NSQ % kP16Rope == 0, "a Q/K stage must always be consumed by the same RoPE group");
     static_assert(NM % 2 == 0 && NM == 2 * NSQ + 2, "metadata ring must order its writers after its readers");
     extern __shared__ uint8_t smem_raw[];
