@@ -110,39 +110,50 @@ template <int D>
 __device__ __forceinline__ void rotate_row_f2(uint8_t *tile, int row, const float4 *table4, int i, int j,
                                               bool scale, float mul)
 {
+    // chunks in groups of G, every load of a group issued before its first
+    // store (the stores may alias later loads for all the compiler knows)
+    constexpr int NCK = D / 8, G = NCK < 4 ? NCK : 4;
 #pragma unroll
-    for (int c = 0; c < D / 8; ++c) {
-        const uint32_t off = swz_offset(row, c, 2 * D);
-        const uint4 u = *reinterpret_cast<const uint4 *>(tile + off);
-        float2 a01 = make_float2(bf16lo(u.x), bf16lo(u.y)), b01 = make_float2(bf16hi(u.x), bf16hi(u.y));
-        float2 a23 = make_float2(bf16lo(u.z), bf16lo(u.w)), b23 = make_float2(bf16hi(u.z), bf16hi(u.w));
-        if (table4) {
-            const bool second = 8 * c >= D / 2;
-            const float4 *tp = table4 + (second ? j : i) * (D / 8) + (second ? 2 * c - D / 8 : 2 * c);
-            const float4 r01 = tp[0], r23 = tp[1];
-            const float2 c01 = make_float2(r01.x, r01.y), s01 = make_float2(r01.z, r01.w);
-            const float2 c23 = make_float2(r23.x, r23.y), s23 = make_float2(r23.z, r23.w);
-            const float2 n01 = make_float2(-r01.z, -r01.w), n23 = make_float2(-r23.z, -r23.w);
-            float2 t = __ffma2_rn(b01, n01, __fmul2_rn(a01, c01));
-            b01 = __ffma2_rn(b01, c01, __fmul2_rn(a01, s01));
-            a01 = t;
-            t = __ffma2_rn(b23, n23, __fmul2_rn(a23, c23));
-            b23 = __ffma2_rn(b23, c23, __fmul2_rn(a23, s23));
-            a23 = t;
+    for (int c0 = 0; c0 < NCK; c0 += G) {
+        uint4 uu[G];
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+            uu[g] = *reinterpret_cast<const uint4 *>(tile + swz_offset(row, c0 + g, 2 * D));
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const int c = c0 + g;
+            const uint32_t off = swz_offset(row, c, 2 * D);
+            const uint4 u = uu[g];
+            float2 a01 = make_float2(bf16lo(u.x), bf16lo(u.y)), b01 = make_float2(bf16hi(u.x), bf16hi(u.y));
+            float2 a23 = make_float2(bf16lo(u.z), bf16lo(u.w)), b23 = make_float2(bf16hi(u.z), bf16hi(u.w));
+            if (table4) {
+                const bool second = 8 * c >= D / 2;
+                const float4 *tp = table4 + (second ? j : i) * (D / 8) + (second ? 2 * c - D / 8 : 2 * c);
+                const float4 r01 = tp[0], r23 = tp[1];
+                const float2 c01 = make_float2(r01.x, r01.y), s01 = make_float2(r01.z, r01.w);
+                const float2 c23 = make_float2(r23.x, r23.y), s23 = make_float2(r23.z, r23.w);
+                const float2 n01 = make_float2(-r01.z, -r01.w), n23 = make_float2(-r23.z, -r23.w);
+                float2 t = __ffma2_rn(b01, n01, __fmul2_rn(a01, c01));
+                b01 = __ffma2_rn(b01, c01, __fmul2_rn(a01, s01));
+                a01 = t;
+                t = __ffma2_rn(b23, n23, __fmul2_rn(a23, c23));
+                b23 = __ffma2_rn(b23, c23, __fmul2_rn(a23, s23));
+                a23 = t;
+            }
+            if (scale) {
+                const float2 m2 = make_float2(mul, mul);
+                a01 = __fmul2_rn(a01, m2);
+                b01 = __fmul2_rn(b01, m2);
+                a23 = __fmul2_rn(a23, m2);
+                b23 = __fmul2_rn(b23, m2);
+            }
+            uint4 o;
+            o.x = pack_bf16x2(a01.x, b01.x);
+            o.y = pack_bf16x2(a01.y, b01.y);
+            o.z = pack_bf16x2(a23.x, b23.x);
+            o.w = pack_bf16x2(a23.y, b23.y);
+            *reinterpret_cast<uint4 *>(tile + off) = o;
         }
-        if (scale) {
-            const float2 m2 = make_float2(mul, mul);
-            a01 = __fmul2_rn(a01, m2);
-            b01 = __fmul2_rn(b01, m2);
-            a23 = __fmul2_rn(a23, m2);
-            b23 = __fmul2_rn(b23, m2);
-        }
-        uint4 o;
-        o.x = pack_bf16x2(a01.x, b01.x);
-        o.y = pack_bf16x2(a01.y, b01.y);
-        o.z = pack_bf16x2(a23.x, b23.x);
-        o.w = pack_bf16x2(a23.y, b23.y);
-        *reinterpret_cast<uint4 *>(tile + off) = o;
     }
 }
 
